@@ -1,0 +1,207 @@
+/*
+ * gmm_fp8.h -- C-ABI of the B200 (sm_100a) FP8 grouped matmul library
+ * (libgmm_fp8.so): forward gmm, backward gmm wrt lhs (dlhs) and the transposed
+ * gmm wrt rhs (tgmm drhs) of Mixture-of-Experts expert MLPs.
+ *
+ * The operations (sources named by page title and section):
+ *   forward   out[m, :] = lhs[m, :] @ rhs[g(m)], rows sorted by expert and
+ *             partitioned by group_sizes ("FP8 Megablox for batch split",
+ *             maxtext PR #3770, Description; "Support quantization for
+ *             tokamax gmm v2", maxtext PR #4451, Description).
+ *   dlhs      dlhs[m, :] = dout[m, :] @ rhs[g(m)]^T, a gmm against the same
+ *             rhs with the transpose flag flipped (PR #4451, review thread on
+ *             ops.py).
+ *   drhs      dW[g] = lhs[rows of g]^T @ dout[rows of g], the transposed gmm
+ *             ("drhs_tgmm2", PR #4451, Description).
+ * FP8 recipe: lhs arrives unquantized and is quantized inside the call as
+ * clip(lhs / scale) to E4M3 with a static per-tensor [1, 1] scale or a dynamic
+ * per-block absmax scale, and results are multiplied back by the scales
+ * ("add static LHS scaling support for GMM v2 FWD", maxtext PR #4735, review
+ * threads on the LhsRef docstring and on inner_kernel).  rhs arrives already
+ * quantized with a per-channel scale of shape [G, N] (PR #3770 Description:
+ * weights quantized manually; PR #4451 review thread: a 2-D scale is per
+ * channel).  Gradients are quantized too (PR #3770 Description).
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers of the current CUDA device unless a
+ *    comment says otherwise.  The caller owns every buffer; the library never
+ *    allocates or frees device memory.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous on it; no call synchronizes except gmm_read_device_status.
+ *  - Matrices are row-major and dense (leading dimension = number of columns).
+ *  - Errors that the host can see (null pointers, bad sizes, misalignment,
+ *    a rule with no scale, a too-small workspace) return before anything is
+ *    launched.  Errors that only the device can see (bad group_sizes, an
+ *    unusable static scale, a wait that timed out) set bits in a status word
+ *    inside `ws`; read them with gmm_read_device_status.  Kernels clamp every
+ *    index, so bad group_sizes never cause an out-of-bounds access.
+ *  - Scales are fp32.  E4M3 codes are bytes (OCP E4M3: bias 7, no infinities,
+ *    largest finite 448).  Quantization: inv = fl32(1/s) (0 where s = 0),
+ *    code = E4M3 round-to-nearest-even of fl32(x * inv) saturated to +-448.
+ *    A dynamic scale is fl32(amax / 448) over a block of 128 values along the
+ *    contraction axis; a scale whose inverse overflows counts as 0.
+ *  - Shapes: K and N multiples of 128, all sizes positive, G <= 1024.
+ */
+#ifndef GMM_FP8_H
+#define GMM_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GMM_OK = 0,
+  GMM_ERR_INVALID_ARG = 1, /* null pointer, unknown enum, rule/dtype mismatch */
+  GMM_ERR_SHAPE = 2,       /* a size <= 0, or K/N not a multiple of 128 */
+  GMM_ERR_ALIGNMENT = 3,   /* a pointer not 16-byte aligned (TMA needs it) */
+  GMM_ERR_SCALE = 4,       /* device: static scale not finite or <= FLT_MIN */
+  GMM_ERR_UNSUPPORTED = 5, /* a valid request this build does not implement */
+  GMM_ERR_CUDA = 6,        /* a CUDA runtime call failed */
+  GMM_ERR_GROUP_SIZES = 7, /* device: a negative size or sum(group_sizes) > M */
+  GMM_ERR_TIMEOUT = 8,     /* device: a pipeline wait exceeded its time limit */
+  GMM_ERR_WORKSPACE = 9    /* ws is NULL or smaller than gmm_workspace_bytes */
+} gmm_status;
+
+typedef enum {
+  GMM_Q_NONE = 0,   /* no quantization: bf16 operands (the bf16 family) */
+  GMM_Q_STATIC = 1, /* per-tensor [1, 1] scale given by the caller */
+  GMM_Q_DYNAMIC = 2 /* per-block absmax scale, blocks of 128 along the contraction axis */
+} gmm_qrule;
+
+typedef enum { GMM_BF16 = 0, GMM_F32 = 1, GMM_E4M3 = 2 } gmm_dtype;
+
+typedef enum { GMM_OP_FWD = 0, GMM_OP_DLHS = 1, GMM_OP_DRHS = 2 } gmm_op;
+
+/* Device status bits (gmm_read_device_status, `bits_out`). */
+#define GMM_DEV_GROUP_SIZES 1u
+#define GMM_DEV_SCALE 2u
+#define GMM_DEV_TIMEOUT 4u
+
+/*
+ * An operand with its optional scale, after the pages' LhsRef / WeightsRef
+ * (PR #4735, review thread on the should_use_external_scale comment): the
+ * direction of the scale follows from the dtype.  An E4M3 operand is already
+ * quantized and `scale` dequantizes it (rhs: [G, N]).  A bf16 operand with
+ * rule STATIC is quantized inside the call with `scale` ([1, 1], one float);
+ * with rule DYNAMIC the call computes the scales itself (`scale` unused);
+ * with rule NONE it is used as bf16 (bf16 family; rhs must be bf16 too).
+ */
+typedef struct {
+  const void *data;
+  gmm_dtype dtype;
+  const float *scale;
+  gmm_qrule rule;
+} gmm_operand;
+
+/* Bytes of workspace that gmm_fwd (op FWD), gmm_dlhs (DLHS) or tgmm_drhs
+ * (DRHS) needs for these sizes; also enough for gmm_quantize with the same
+ * operand.  Returns 0 for invalid sizes. */
+size_t gmm_workspace_bytes(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G);
+
+/* Number of 128-row chunks a tgmm operand of `rows` rows and G groups can
+ * occupy at most: ceil(rows / 128) + G.  Sizes the axis-0 outputs below. */
+int64_t gmm_chunk_capacity(int64_t rows, int32_t G);
+
+/*
+ * Weight quantization (done once per weight update, outside the timed passes;
+ * PR #3770 Description: weights are quantized manually outside the kernel).
+ * w_bf16: [G, K, N] bf16.  scales: [G, N] fp32, s[g, n] = fl32(max_k |w| / 448).
+ * codes: E4M3 [G, K, N] when transpose_out == 0, else [G, N, K].
+ */
+gmm_status gmm_quantize_rhs(const void *w_bf16, int32_t G, int64_t K, int64_t N, int transpose_out,
+                            uint8_t *codes, float *scales, void *stream);
+
+/*
+ * Activation / gradient quantization, the step each pass runs first.  x_bf16
+ * is [rows, cols] bf16.
+ * axis == 1: blocks of 128 along each row (the forward lhs, the dlhs dout).
+ *   codes [rows, cols]; scales [cols/128, rows] (block-major) for DYNAMIC,
+ *   unused for STATIC.  With col_scale != NULL ([G, cols]) the quantized
+ *   value is fl32(x[m, n] * col_scale[g(m), n]) and rows in no group are 0
+ *   (this folds the rhs scale into dout for dlhs); group_sizes is then needed.
+ * axis == 0: the tgmm operand.  Each group's rows are cut into 128-row chunks
+ *   starting at the group's first row; chunk j (over all groups, in group
+ *   order) gets one scale per column.  codes are stored transposed and
+ *   padded: [cols, 128 * gmm_chunk_capacity(rows, G)], chunk j in columns
+ *   [128 j, 128 j + 128), pad rows 0.  scales [gmm_chunk_capacity, cols]
+ *   (written for STATIC too, all equal to the static scale).
+ * rule: STATIC (static_scale = device pointer to one float) or DYNAMIC.
+ * ws: workspace of at least gmm_workspace_bytes(...) for the pass that
+ * consumes this operand.
+ */
+gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrule rule, int axis,
+                        const float *static_scale, const int32_t *group_sizes, int32_t G,
+                        const float *col_scale, uint8_t *codes, float *scales, void *ws, size_t ws_bytes,
+                        void *stream);
+
+/*
+ * Forward gmm.  lhs: bf16 [M, K] with rule STATIC / DYNAMIC (or NONE for the
+ * bf16 family).  rhs: E4M3 codes with scales [G, N] (or bf16 for the bf16
+ * family), [G, K, N] when transpose_rhs == 0, [G, N, K] when 1.
+ * group_sizes: device int32 [G]; rows are sorted by group.
+ * out: [M, N] of out_dtype (BF16 or F32):
+ *   out[m, n] = s_r[g, n] * sum_b s_l[m, b] * sum_{k in b} q_l[m, k] * q_r[g, k, n]
+ * Rows outside every group are written as 0.
+ */
+gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
+                   int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                   void *stream);
+
+/*
+ * Backward gmm wrt lhs.  dout: bf16 [M, N], always quantized with DYNAMIC
+ * 128-blocks along N after folding the rhs column scale in (dout.rule must be
+ * DYNAMIC, or NONE for the bf16 family).  rhs: the same buffer and layout as
+ * for gmm_fwd with the same transpose_rhs.  dlhs: [M, K] of out_dtype:
+ *   dlhs[m, k] = sum_b s_t[m, b] * sum_{n in b} q_t[m, n] * q_r[g, k, n],
+ *   q_t, s_t = quantize(fl32(dout[m, n] * s_r[g, n]))
+ */
+gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
+                    int64_t M, int64_t K, int64_t N, void *dlhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                    void *stream);
+
+/*
+ * Transposed gmm (weight gradient).  lhs: bf16 [M, K] with rule STATIC (the
+ * forward's static scale, giving the forward's codes) or DYNAMIC; dout: bf16
+ * [M, N], rule DYNAMIC (or both NONE for the bf16 family).  Both are
+ * quantized per 128-row chunk of each group (axis 0 above).
+ * drhs: [G, K, N] of out_dtype (F32 or BF16):
+ *   dW[g, k, n] = sum_c s_x[c, k] * s_d[c, n] * sum_{m in chunk c} q_x[m, k] * q_d[m, n]
+ * Empty groups get dW[g] = 0.
+ */
+gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_sizes, int32_t G, int64_t M,
+                     int64_t K, int64_t N, void *drhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/*
+ * Synchronizes `stream`, then reads the device status word that the last call
+ * using `ws` left.  *bits_out (may be NULL) receives the raw GMM_DEV_* bits.
+ * Returns GMM_OK, or the most severe device error: TIMEOUT, SCALE,
+ * GROUP_SIZES.  ws is a device pointer.
+ */
+gmm_status gmm_read_device_status(const void *ws, uint32_t *bits_out, void *stream);
+
+/*
+ * Self-test of the bounded waits: launches one block that waits on a barrier
+ * nothing ever arrives on, with a limit of `limit_ns` nanoseconds; the wait
+ * gives up, sets GMM_DEV_TIMEOUT in ws's status word and the kernel returns.
+ * Read the result with gmm_read_device_status.
+ */
+gmm_status gmm_selftest_timeout(void *ws, uint64_t limit_ns, void *stream);
+
+/* Time limit of every pipeline wait in the kernels (default 4e9 ns). */
+void gmm_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Static text for a status code. */
+const char *gmm_status_string(gmm_status s);
+
+/* Number of kernels the last successful call on this host thread launched. */
+int32_t gmm_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GMM_FP8_H */

@@ -6,8 +6,8 @@ The compute runs in the CUDA library ``libgmm_fp8.so`` (C-ABI declared in
 The library is loaded on first use and a missing library raises an error:
 there is no CPU fallback.
 """
-# populated once ops.py exists
-# from .ops import (  # noqa: F401
-#     GmmError, gmm_fwd, gmm_dlhs, tgmm_drhs, gmm_quantize, gmm_quantize_rhs, gmm_plan, gmm_workspace_bytes,
-#     gmm_read_device_status, gmm_status_string, QRule, DType,
-# )
+from .ops import (  # noqa: F401
+    DType, GmmError, QRule, gmm_chunk_capacity, gmm_dlhs, gmm_fwd, gmm_plan, gmm_quantize, gmm_quantize_rhs,
+    gmm_read_device_status, gmm_selftest_timeout, gmm_set_wait_limit_ns, gmm_status_string, gmm_workspace_bytes,
+    last_launch_count, tgmm_drhs, workspace,
+)

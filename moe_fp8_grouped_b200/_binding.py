@@ -1,0 +1,73 @@
+"""ctypes loader for libgmm_fp8.so: argument marshalling only.
+
+The library sits next to this file (built in-tree by ``build.py``).  Loading
+fails loudly when it is missing: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgmm_fp8.so")
+
+# enums of include/gmm_fp8.h
+GMM_OK = 0
+STATUS_NAMES = {0: "GMM_OK", 1: "GMM_ERR_INVALID_ARG", 2: "GMM_ERR_SHAPE", 3: "GMM_ERR_ALIGNMENT",
+                4: "GMM_ERR_SCALE", 5: "GMM_ERR_UNSUPPORTED", 6: "GMM_ERR_CUDA", 7: "GMM_ERR_GROUP_SIZES",
+                8: "GMM_ERR_TIMEOUT", 9: "GMM_ERR_WORKSPACE"}
+Q_NONE, Q_STATIC, Q_DYNAMIC = 0, 1, 2
+DT_BF16, DT_F32, DT_E4M3 = 0, 1, 2
+OP_FWD, OP_DLHS, OP_DRHS = 0, 1, 2
+DEV_GROUP_SIZES, DEV_SCALE, DEV_TIMEOUT = 1, 2, 4
+
+# every symbol include/gmm_fp8.h declares
+EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm_quantize", "gmm_fwd",
+           "gmm_dlhs", "tgmm_drhs", "gmm_read_device_status", "gmm_selftest_timeout", "gmm_set_wait_limit_ns",
+           "gmm_status_string", "gmm_last_launch_count"]
+
+
+class Operand(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int), ("scale", ctypes.c_void_p),
+                ("rule", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with moe_fp8_grouped_b200.build.build() "
+                           "(there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
+    st = ctypes.c_int
+    L.gmm_workspace_bytes.argtypes = [ctypes.c_int, i64, i64, i64, i32]
+    L.gmm_workspace_bytes.restype = sz
+    L.gmm_chunk_capacity.argtypes = [i64, i32]
+    L.gmm_chunk_capacity.restype = i64
+    L.gmm_quantize_rhs.argtypes = [vp, i32, i64, i64, ctypes.c_int, vp, vp, vp]
+    L.gmm_quantize_rhs.restype = st
+    L.gmm_quantize.argtypes = [vp, i64, i64, ctypes.c_int, ctypes.c_int, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    L.gmm_quantize.restype = st
+    L.gmm_fwd.argtypes = [Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp, sz, vp]
+    L.gmm_fwd.restype = st
+    L.gmm_dlhs.argtypes = L.gmm_fwd.argtypes
+    L.gmm_dlhs.restype = st
+    L.tgmm_drhs.argtypes = [Operand, Operand, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp, sz, vp]
+    L.tgmm_drhs.restype = st
+    L.gmm_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
+    L.gmm_read_device_status.restype = st
+    L.gmm_selftest_timeout.argtypes = [vp, u64, vp]
+    L.gmm_selftest_timeout.restype = st
+    L.gmm_set_wait_limit_ns.argtypes = [u64]
+    L.gmm_set_wait_limit_ns.restype = None
+    L.gmm_status_string.argtypes = [ctypes.c_int]
+    L.gmm_status_string.restype = ctypes.c_char_p
+    L.gmm_last_launch_count.argtypes = []
+    L.gmm_last_launch_count.restype = i32
+    _lib = L
+    return L

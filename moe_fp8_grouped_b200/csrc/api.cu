@@ -1,0 +1,432 @@
+// api.cu -- the extern "C" entry points declared in include/gmm_fp8.h:
+// argument validation, workspace carving, TMA tensor maps and launches.
+// Nothing here allocates device memory; every buffer is the caller's.
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace gmm {
+
+static uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+static thread_local int32_t g_launches = 0;
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int64_t chunk_capacity(int64_t rows, int32_t G) { return (rows + kBlk - 1) / kBlk + G; }
+
+WsLayout ws_layout(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G) {
+  WsLayout L{};
+  size_t o = sizeof(WsHeader);
+  L.plan_offs = o;
+  o += align256(sizeof(int) * (G + 1));
+  L.plan_tpre = o;
+  o += align256(sizeof(int) * (G + 1));
+  if (op == GMM_OP_FWD || op == GMM_OP_DLHS) {
+    const int64_t C = (op == GMM_OP_FWD) ? K : N;  // contraction of the row operand
+    L.codes_a = o;
+    o += align256(static_cast<size_t>(M) * C);
+    L.scales_a = o;
+    o += align256(sizeof(float) * static_cast<size_t>(M) * (C / kBlk));
+    L.codes_b = L.scales_b = 0;
+  } else {
+    // transposed, chunk-padded operands; sized for 2-byte elements so that the
+    // bf16 family fits as well
+    const int64_t cap = chunk_capacity(M, G);
+    L.codes_a = o;
+    o += align256(static_cast<size_t>(K) * kBlk * cap * 2);
+    L.codes_b = o;
+    o += align256(static_cast<size_t>(N) * kBlk * cap * 2);
+    L.scales_a = o;
+    o += align256(sizeof(float) * static_cast<size_t>(cap) * K);
+    L.scales_b = o;
+    o += align256(sizeof(float) * static_cast<size_t>(cap) * N);
+  }
+  L.total = o;
+  return L;
+}
+
+// ----------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major 2-D tensor [outer, inner] with a row pitch in bytes; box
+// [box_outer, box_inner] with the 128-byte swizzle (box_inner * elem = 128).
+static bool make_map(CUtensorMap *m, const void *base, int elem, uint64_t inner, uint64_t outer,
+                     uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, elem == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ validation
+
+static bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static gmm_status check_sizes(int64_t M, int64_t K, int64_t N, int32_t G) {
+  if (M <= 0 || K <= 0 || N <= 0 || G <= 0) return GMM_ERR_SHAPE;
+  if (K % kBlk || N % kBlk) return GMM_ERR_SHAPE;
+  if (G > kMaxGroups) return GMM_ERR_UNSUPPORTED;
+  // 32-bit tile coordinates and row indices
+  if (M > (1 << 24) || K > (1 << 20) || N > (1 << 20) || static_cast<int64_t>(G) * (K > N ? K : N) > INT_MAX)
+    return GMM_ERR_UNSUPPORTED;
+  return GMM_OK;
+}
+
+static gmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA; }
+
+struct WsPtrs {
+  uint32_t *status;
+  int *offs, *tpre;
+  uint8_t *codes_a, *codes_b;
+  float *scales_a, *scales_b;
+};
+
+static WsPtrs carve(void *ws, const WsLayout &L) {
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  WsPtrs P;
+  P.status = reinterpret_cast<uint32_t *>(w);
+  P.offs = reinterpret_cast<int *>(w + L.plan_offs);
+  P.tpre = reinterpret_cast<int *>(w + L.plan_tpre);
+  P.codes_a = w + L.codes_a;
+  P.codes_b = L.codes_b ? w + L.codes_b : nullptr;
+  P.scales_a = reinterpret_cast<float *>(w + L.scales_a);
+  P.scales_b = L.scales_b ? reinterpret_cast<float *>(w + L.scales_b) : nullptr;
+  return P;
+}
+
+// quantized (fp8) or bf16-family operand pair; returns the element size
+static gmm_status classify(const gmm_operand &x, const gmm_operand &w, bool w_is_rhs, int *elem) {
+  if (!x.data || !w.data) return GMM_ERR_INVALID_ARG;
+  if (x.rule == GMM_Q_NONE) {
+    if (x.dtype != GMM_BF16 || w.dtype != GMM_BF16) return GMM_ERR_INVALID_ARG;
+    if (!w_is_rhs && w.rule != GMM_Q_NONE) return GMM_ERR_INVALID_ARG;
+    *elem = 2;
+    return GMM_OK;
+  }
+  if (x.rule != GMM_Q_STATIC && x.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
+  if (x.dtype != GMM_BF16) return GMM_ERR_INVALID_ARG;
+  if (x.rule == GMM_Q_STATIC && !x.scale) return GMM_ERR_INVALID_ARG;  // a present rule must be applied
+  if (w_is_rhs) {
+    if (w.dtype != GMM_E4M3 || !w.scale) return GMM_ERR_INVALID_ARG;
+  } else {
+    if (w.dtype != GMM_BF16 || w.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
+  }
+  *elem = 1;
+  return GMM_OK;
+}
+
+}  // namespace gmm
+
+using namespace gmm;
+
+extern "C" {
+
+size_t gmm_workspace_bytes(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G) {
+  if (check_sizes(M, K, N, G) != GMM_OK) return 0;
+  if (op != GMM_OP_FWD && op != GMM_OP_DLHS && op != GMM_OP_DRHS) return 0;
+  return ws_layout(op, M, K, N, G).total;
+}
+
+int64_t gmm_chunk_capacity(int64_t rows, int32_t G) { return chunk_capacity(rows, G); }
+
+const char *gmm_status_string(gmm_status s) {
+  switch (s) {
+    case GMM_OK: return "ok";
+    case GMM_ERR_INVALID_ARG: return "invalid argument";
+    case GMM_ERR_SHAPE: return "invalid shape (sizes must be positive, K and N multiples of 128)";
+    case GMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case GMM_ERR_SCALE: return "static scale not finite or not above FLT_MIN";
+    case GMM_ERR_UNSUPPORTED: return "unsupported size";
+    case GMM_ERR_CUDA: return "CUDA runtime error";
+    case GMM_ERR_GROUP_SIZES: return "group_sizes negative or summing past M";
+    case GMM_ERR_TIMEOUT: return "a device wait timed out";
+    case GMM_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int32_t gmm_last_launch_count(void) { return g_launches; }
+
+void gmm_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns = limit_ns ? limit_ns : kDefaultWaitLimitNs; }
+
+gmm_status gmm_quantize_rhs(const void *w_bf16, int32_t G, int64_t K, int64_t N, int transpose_out,
+                            uint8_t *codes, float *scales, void *stream) {
+  g_launches = 0;
+  if (!w_bf16 || !codes || !scales) return GMM_ERR_INVALID_ARG;
+  gmm_status s = check_sizes(1, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!al16(w_bf16) || !al16(codes) || !al16(scales)) return GMM_ERR_ALIGNMENT;
+  s = cuda_status(launch_quant_rhs(w_bf16, G, K, N, transpose_out != 0, codes, scales,
+                                   static_cast<cudaStream_t>(stream)));
+  if (s == GMM_OK) g_launches = 3;
+  return s;
+}
+
+gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrule rule, int axis,
+                        const float *static_scale, const int32_t *group_sizes, int32_t G, const float *col_scale,
+                        uint8_t *codes, float *scales, void *ws, size_t ws_bytes, void *stream) {
+  g_launches = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!x_bf16 || !codes) return GMM_ERR_INVALID_ARG;
+  if (rule != GMM_Q_STATIC && rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
+  if (rule == GMM_Q_STATIC && !static_scale) return GMM_ERR_INVALID_ARG;
+  if (rule == GMM_Q_DYNAMIC && !scales) return GMM_ERR_INVALID_ARG;
+  if (axis != 0 && axis != 1) return GMM_ERR_INVALID_ARG;
+  if ((axis == 0 || col_scale) && !group_sizes) return GMM_ERR_INVALID_ARG;
+  if (axis == 0 && !scales) return GMM_ERR_INVALID_ARG;
+  if (col_scale && rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
+  const int32_t Gq = group_sizes ? G : 1;
+  gmm_status s = check_sizes(rows, cols, cols, Gq);
+  if (s != GMM_OK) return s;
+  if (!al16(x_bf16) || !al16(codes) || (scales && !al16(scales)) || (col_scale && !al16(col_scale)))
+    return GMM_ERR_ALIGNMENT;
+  // the plan and status live in the first part of any pass's workspace
+  const WsLayout L = ws_layout(GMM_OP_FWD, 1, kBlk, kBlk, Gq);
+  if (!ws || ws_bytes < L.codes_a) return GMM_ERR_WORKSPACE;
+  WsPtrs P = carve(ws, L);
+  int n = 0;
+  if (group_sizes) {
+    s = cuda_status(launch_plan(group_sizes, Gq, rows, P.offs, P.tpre, P.status, st));
+    ++n;
+  } else {
+    s = cuda_status(cudaMemsetAsync(P.status, 0, sizeof(uint32_t), st));
+  }
+  if (s != GMM_OK) return s;
+  const bool dyn = rule == GMM_Q_DYNAMIC;
+  if (axis == 1)
+    s = cuda_status(launch_quant_rows(x_bf16, rows, cols, dyn, dyn ? nullptr : static_scale, col_scale, P.offs,
+                                      Gq, codes, scales, P.status, st));
+  else
+    s = cuda_status(launch_quant_chunks(x_bf16, rows, cols, dyn, dyn ? nullptr : static_scale, P.offs, P.tpre, Gq,
+                                        chunk_capacity(rows, Gq), codes, scales, false, P.status, st));
+  if (s == GMM_OK) g_launches = n + 1;
+  return s;
+}
+
+gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
+                   int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                   void *stream) {
+  g_launches = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gmm_status s = check_sizes(M, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!group_sizes || !out) return GMM_ERR_INVALID_ARG;
+  if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
+  int elem = 0;
+  if ((s = classify(lhs, rhs, true, &elem)) != GMM_OK) return s;
+  if (!al16(lhs.data) || !al16(rhs.data) || !al16(out) || !al16(ws) || (rhs.scale && !al16(rhs.scale)))
+    return GMM_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(GMM_OP_FWD, M, K, N, G);
+  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
+  WsPtrs P = carve(ws, L);
+  if ((s = cuda_status(launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st))) != GMM_OK) return s;
+  int n = 1;
+  const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
+  const void *A = lhs.data;
+  if (elem == 1) {
+    s = cuda_status(launch_quant_rows(lhs.data, M, K, dyn, dyn ? nullptr : lhs.scale, nullptr, P.offs, G, P.codes_a,
+                                      P.scales_a, P.status, st));
+    if (s != GMM_OK) return s;
+    ++n;
+    A = P.codes_a;
+  }
+  const bool bmn = transpose_rhs == 0;  // [G, K, N]: N contiguous = MN-major B
+  const uint32_t bke = 128 / elem;
+  CUtensorMap tmA, tmB;
+  if (!make_map(&tmA, A, elem, K, M, K * elem, bke, 128)) return GMM_ERR_CUDA;
+  const bool okB = bmn ? make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, bke)
+                       : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, 256);
+  if (!okB) return GMM_ERR_CUDA;
+  GemmParams p{};
+  p.mode = MODE_ROWS;
+  p.G = G;
+  p.M = static_cast<int>(M);
+  p.ncols = static_cast<int>(N);
+  p.kblocks = static_cast<int>(K / bke);
+  p.b_group_rows = static_cast<int>(bmn ? K : N);
+  p.offs = P.offs;
+  p.tpre = P.tpre;
+  p.row_scale = (elem == 1 && dyn) ? P.scales_a : nullptr;
+  p.row_scale_ld = M;
+  p.col_scale = elem == 1 ? rhs.scale : nullptr;
+  p.static_scale = (elem == 1 && !dyn) ? lhs.scale : nullptr;
+  p.out = out;
+  p.out_f32 = out_dtype == GMM_F32;
+  p.ld_out = N;
+  p.status = P.status;
+  p.wait_limit_ns = g_wait_limit_ns;
+  const GemmConfig cfg{elem, bmn, elem == 1 && dyn};
+  const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
+  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  if ((s = cuda_status(launch_gemm(cfg, tmA, tmB, p, grid, st))) != GMM_OK) return s;
+  g_launches = n + 1;
+  return GMM_OK;
+}
+
+gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
+                    int64_t M, int64_t K, int64_t N, void *dlhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                    void *stream) {
+  g_launches = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gmm_status s = check_sizes(M, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!group_sizes || !dlhs) return GMM_ERR_INVALID_ARG;
+  if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
+  int elem = 0;
+  if ((s = classify(dout, rhs, true, &elem)) != GMM_OK) return s;
+  if (elem == 1 && dout.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;  // gradients: dynamic blocks
+  if (!al16(dout.data) || !al16(rhs.data) || !al16(dlhs) || !al16(ws) || (rhs.scale && !al16(rhs.scale)))
+    return GMM_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(GMM_OP_DLHS, M, K, N, G);
+  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
+  WsPtrs P = carve(ws, L);
+  if ((s = cuda_status(launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st))) != GMM_OK) return s;
+  int n = 1;
+  const void *A = dout.data;
+  if (elem == 1) {
+    // t = fl32(dout * s_r[g(m), n]), dynamic 128-blocks along n
+    s = cuda_status(launch_quant_rows(dout.data, M, N, true, nullptr, rhs.scale, P.offs, G, P.codes_a, P.scales_a,
+                                      P.status, st));
+    if (s != GMM_OK) return s;
+    ++n;
+    A = P.codes_a;
+  }
+  const bool bmn = transpose_rhs != 0;  // [G, N, K]: K contiguous = MN-major B for dlhs
+  const uint32_t bke = 128 / elem;
+  CUtensorMap tmA, tmB;
+  if (!make_map(&tmA, A, elem, N, M, N * elem, bke, 128)) return GMM_ERR_CUDA;
+  const bool okB = bmn ? make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, bke)
+                       : make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, 256);
+  if (!okB) return GMM_ERR_CUDA;
+  GemmParams p{};
+  p.mode = MODE_ROWS;
+  p.G = G;
+  p.M = static_cast<int>(M);
+  p.ncols = static_cast<int>(K);
+  p.kblocks = static_cast<int>(N / bke);
+  p.b_group_rows = static_cast<int>(bmn ? N : K);
+  p.offs = P.offs;
+  p.tpre = P.tpre;
+  p.row_scale = elem == 1 ? P.scales_a : nullptr;
+  p.row_scale_ld = M;
+  p.col_scale = nullptr;
+  p.static_scale = nullptr;
+  p.out = dlhs;
+  p.out_f32 = out_dtype == GMM_F32;
+  p.ld_out = K;
+  p.status = P.status;
+  p.wait_limit_ns = g_wait_limit_ns;
+  const GemmConfig cfg{elem, bmn, elem == 1};
+  const int64_t items = ((M + 127) / 128 + G) * ((K + 255) / 256);
+  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  if ((s = cuda_status(launch_gemm(cfg, tmA, tmB, p, grid, st))) != GMM_OK) return s;
+  g_launches = n + 1;
+  return GMM_OK;
+}
+
+gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_sizes, int32_t G, int64_t M,
+                     int64_t K, int64_t N, void *drhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                     void *stream) {
+  g_launches = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gmm_status s = check_sizes(M, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!group_sizes || !drhs) return GMM_ERR_INVALID_ARG;
+  if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
+  int elem = 0;
+  if ((s = classify(lhs, dout, false, &elem)) != GMM_OK) return s;
+  if (!al16(lhs.data) || !al16(dout.data) || !al16(drhs) || !al16(ws)) return GMM_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(GMM_OP_DRHS, M, K, N, G);
+  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
+  WsPtrs P = carve(ws, L);
+  if ((s = cuda_status(launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st))) != GMM_OK) return s;
+  const int64_t cap = chunk_capacity(M, G);
+  const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
+  s = cuda_status(launch_quant_chunks(lhs.data, M, K, dyn, (elem == 1 && !dyn) ? lhs.scale : nullptr, P.offs,
+                                      P.tpre, G, cap, P.codes_a, P.scales_a, elem == 2, P.status, st));
+  if (s != GMM_OK) return s;
+  s = cuda_status(launch_quant_chunks(dout.data, M, N, true, nullptr, P.offs, P.tpre, G, cap, P.codes_b, P.scales_b,
+                                      elem == 2, P.status, st));
+  if (s != GMM_OK) return s;
+  const uint32_t bke = 128 / elem;
+  const uint64_t ldt = static_cast<uint64_t>(cap) * kBlk;  // elements per transposed row
+  CUtensorMap tmA, tmB;
+  if (!make_map(&tmA, P.codes_a, elem, ldt, K, ldt * elem, bke, 128)) return GMM_ERR_CUDA;
+  if (!make_map(&tmB, P.codes_b, elem, ldt, N, ldt * elem, bke, 256)) return GMM_ERR_CUDA;
+  GemmParams p{};
+  p.mode = MODE_TGMM;
+  p.G = G;
+  p.M = static_cast<int>(M);
+  p.ncols = static_cast<int>(N);
+  p.ktiles = static_cast<int>(K / kBlk);
+  p.stages_per_chunk = elem;
+  p.offs = P.offs;
+  p.tpre = P.tpre;
+  p.row_scale = P.scales_a;
+  p.row_scale_ld = K;
+  p.colblk_scale = P.scales_b;
+  p.colblk_ld = N;
+  p.out = drhs;
+  p.out_f32 = out_dtype == GMM_F32;
+  p.ld_out = N;
+  p.status = P.status;
+  p.wait_limit_ns = g_wait_limit_ns;
+  const GemmConfig cfg{elem, false, elem == 1};
+  const int64_t items = static_cast<int64_t>(G) * (K / kBlk) * ((N + 255) / 256);
+  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  if ((s = cuda_status(launch_gemm(cfg, tmA, tmB, p, grid, st))) != GMM_OK) return s;
+  g_launches = 4;
+  return GMM_OK;
+}
+
+gmm_status gmm_read_device_status(const void *ws, uint32_t *bits_out, void *stream) {
+  if (!ws) return GMM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t bits = 0;
+  if (cudaMemcpyAsync(&bits, ws, sizeof(bits), cudaMemcpyDeviceToHost, st) != cudaSuccess) return GMM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GMM_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  if (bits & GMM_DEV_TIMEOUT) return GMM_ERR_TIMEOUT;
+  if (bits & GMM_DEV_SCALE) return GMM_ERR_SCALE;
+  if (bits & GMM_DEV_GROUP_SIZES) return GMM_ERR_GROUP_SIZES;
+  return GMM_OK;
+}
+
+gmm_status gmm_selftest_timeout(void *ws, uint64_t limit_ns, void *stream) {
+  g_launches = 0;
+  if (!ws) return GMM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *status = static_cast<uint32_t *>(ws);
+  gmm_status s = cuda_status(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
+  if (s != GMM_OK) return s;
+  s = cuda_status(launch_timeout_selftest(status, limit_ns, st));
+  if (s == GMM_OK) g_launches = 1;
+  return s;
+}
+
+}  // extern "C"

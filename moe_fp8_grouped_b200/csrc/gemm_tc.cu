@@ -1,0 +1,461 @@
+// gemm_tc.cu -- persistent, warp-specialized grouped GEMM on the sm_100a
+// tensor cores (tcgen05), shared by the three passes:
+//
+//   forward gmm   rows = lhs rows of each group, contraction K, columns N
+//                 ("FP8 Megablox for batch split", maxtext PR #3770,
+//                 Description; "Support quantization for tokamax gmm v2",
+//                 maxtext PR #4451, Description)
+//   dlhs gmm      rows = dout rows, contraction N, columns K: the same rhs
+//                 read with the other major-ness (PR #4451, review thread on
+//                 ops.py: transpose_rhs flipped)
+//   tgmm drhs     rows = K, contraction = the rows of one group, columns N
+//                 ("drhs_tgmm2", PR #4451, Description)
+//
+// CTA layout (320 threads, one CTA per SM):
+//   warp 0     TMA producer: A tile 128 x 128 B, B tile 256 x 128 B per stage,
+//              4 stages in shared memory (128-byte swizzle)
+//   warp 1     TMEM allocator + MMA issuer: tcgen05.mma M=128 N=256, four
+//              32-byte K steps per stage, fp32 accumulators in TMEM, two
+//              256-column accumulator buffers
+//   warps 2-9  epilogue: tcgen05.ld, scale, store.  Warp w reads TMEM lanes
+//              32 (w % 4) .. +31 (rows) and column half (w - 2) / 4.
+//
+// Scaling ("add static LHS scaling support for GMM v2 FWD", maxtext PR
+// #4735, review thread on the LhsRef docstring: the result is multiplied back
+// by the scale):
+//   promote == false  one TMEM unit per tile; out = acc * s * col_scale
+//   promote == true   one TMEM unit per 128-long contraction block; the
+//                     epilogue accumulates acc += unit * row_scale (* the
+//                     block's column scale for tgmm) in registers.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gmm {
+
+constexpr int kBM = 128, kBN = 256;
+constexpr int kStages = 4;
+constexpr int kAStage = kBM * 128;  // bytes
+constexpr int kBStage = kBN * 128;
+constexpr int kThreads = 320;
+constexpr int kTmemCols = 512;
+
+constexpr size_t gemm_smem_bytes() {
+  return 1024                                    // alignment slack
+         + static_cast<size_t>(kStages) * (kAStage + kBStage)
+         + 16 * 8                                // mbarriers
+         + 16                                    // tmem slot, abort flag
+         + 2 * (kMaxGroups + 1) * sizeof(int);   // plan copy
+}
+
+struct Item {
+  int g, nt, kt, nblocks, r0, rend;
+};
+
+__device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const int *s_offs, const int *s_tpre,
+                                            int tn) {
+  Item t;
+  if (p.mode == MODE_ROWS) {
+    // items of group g: (tpre[g+1] - tpre[g]) m-tiles x tn n-tiles, m fastest
+    int lo = 0, hi = p.G + 1;  // first i with tpre[i] * tn > w
+    while (lo < hi) {
+      int mid = (lo + hi) >> 1;
+      if (s_tpre[mid] * tn > w) hi = mid;
+      else lo = mid + 1;
+    }
+    const int g = lo - 1;
+    const int mt_g = s_tpre[g + 1] - s_tpre[g];
+    const int local = w - s_tpre[g] * tn;
+    const int mt = local % mt_g;
+    t.g = g;
+    t.nt = local / mt_g;
+    t.kt = 0;
+    t.r0 = s_offs[g] + kBM * mt;
+    t.rend = min(s_offs[g + 1], t.r0 + kBM);
+    t.nblocks = p.kblocks;
+  } else {
+    const int per_g = p.ktiles * tn;
+    const int g = w / per_g, local = w % per_g;
+    t.g = g;
+    t.nt = local / p.ktiles;
+    t.kt = local % p.ktiles;
+    t.r0 = 0;
+    t.rend = 0;
+    t.nblocks = (s_tpre[g + 1] - s_tpre[g]) * p.stages_per_chunk;
+  }
+  return t;
+}
+
+template <int kElem>
+__device__ __forceinline__ void store32(void *out, int64_t off_elems, const float (&v)[32], int out_f32) {
+  if (out_f32) {
+    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + off_elems);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + off_elems);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * i + 2 * e], v[8 * i + 2 * e + 1]);
+        w[e] = *reinterpret_cast<uint32_t *>(&b);
+      }
+      dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+template <int kElem, bool kBMN, bool kPromote>
+__global__ void __launch_bounds__(kThreads, 1)
+    gmm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const GemmParams p) {
+  constexpr bool kF16 = (kElem == 2);
+  constexpr int kBKe = 128 / kElem;                 // contraction elements per stage
+  constexpr int kMmaK = 32 / kElem;                 // contraction elements per MMA
+  constexpr int kBBoxes = kBMN ? 2 * kElem : 1;     // TMA boxes per B stage
+  constexpr int kBBoxBytes = kBStage / kBBoxes;
+  constexpr uint32_t kIdesc = instr_desc(kF16, kBMN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + kStages * kAStage;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * kBStage);
+  uint64_t *full = bars;                 // [kStages] TMA -> MMA
+  uint64_t *empty = bars + kStages;      // [kStages] MMA -> TMA
+  uint64_t *tfull = bars + 2 * kStages;  // [2] MMA -> epilogue
+  uint64_t *tempty = tfull + 2;          // [2] epilogue -> MMA
+  uint64_t *drain = tempty + 2;          // MMA completion at exit
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *s_offs = reinterpret_cast<int *>(tmem_slot + 4);
+  int *s_tpre = s_offs + (kMaxGroups + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *reinterpret_cast<volatile int *>(tmem_slot + 2) = 0;  // never raised: exit drains ignore aborts
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i <= p.G; i += kThreads) {
+    s_offs[i] = p.offs[i];
+    s_tpre[i] = p.tpre[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  const int tn = (p.ncols + kBN - 1) / kBN;
+  const int total = (p.mode == MODE_ROWS) ? s_tpre[p.G] * tn : p.G * p.ktiles * tn;
+  const WaitCtl ctl{p.wait_limit_ns, abort_flag, p.status};
+  const WaitCtl ctl_drain{p.wait_limit_ns, reinterpret_cast<volatile int *>(tmem_slot + 2), p.status};
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+        const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+        for (int b = 0; b < t.nblocks; ++b, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, ctl)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kAStage + kBStage);
+          int ax, ay, bx, by;
+          if (p.mode == MODE_ROWS) {
+            ax = b * kBKe;
+            ay = t.r0;
+            if (kBMN) {
+              bx = t.nt * kBN;
+              by = t.g * p.b_group_rows + b * kBKe;
+            } else {
+              bx = b * kBKe;
+              by = t.g * p.b_group_rows + t.nt * kBN;
+            }
+          } else {
+            ax = s_tpre[t.g] * kBlk + b * kBKe;
+            ay = t.kt * kBM;
+            bx = ax;
+            by = t.nt * kBN;
+          }
+          tma_load_2d(sA + s * kAStage, &tmA, ax, ay, &full[s]);
+#pragma unroll
+          for (int h = 0; h < kBBoxes; ++h)
+            tma_load_2d(sB + s * kBStage + h * kBBoxBytes, &tmB, bx + (kBMN ? h * kBKe : 0), by, &full[s]);
+        }
+      }
+      // let every issued copy land before the CTA can exit
+      for (int i = (it > kStages ? it - kStages : 0); i < it; ++i)
+        mbar_wait(&full[i % kStages], (i / kStages) & 1, ctl_drain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int it = 0, u = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+        const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+        uint32_t buf = 0;
+        for (int b = 0; b < t.nblocks; ++b, ++it) {
+          const bool unit_start = kPromote || b == 0;
+          if (unit_start) {
+            buf = u & 1;
+            if (!mbar_wait(&tempty[buf], ((u >> 1) & 1) ^ 1, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          const int s = it % kStages;
+          if (!mbar_wait(&full[s], (it / kStages) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBStage);
+          const uint32_t d = tbase + buf * kBN;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
+                                        : smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&empty[s]);
+          if (kPromote || b == t.nblocks - 1) {
+            tc_commit(&tfull[buf]);
+            ++u;
+          }
+        }
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, ctl_drain);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
+    const float sstat = p.static_scale ? *p.static_scale : 1.0f;
+    const bool sstat_ok = isfinite(sstat) && sstat > 1.17549435e-38f;
+    int u = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+      const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+      const int col0 = t.nt * kBN + h * 128;
+      int64_t orow;
+      bool row_ok;
+      if (p.mode == MODE_ROWS) {
+        orow = t.r0 + row;
+        row_ok = orow < t.rend;
+      } else {
+        orow = static_cast<int64_t>(t.g) * p.ktiles * kBM + t.kt * kBM + row;
+        row_ok = true;
+      }
+      if (t.nblocks == 0) {  // empty group in tgmm: dW tile = 0
+        float z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (col0 + c * 32 < p.ncols) store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, z, p.out_f32);
+        continue;
+      }
+      if constexpr (kPromote) {
+        float acc[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+        for (int b = 0; b < t.nblocks; ++b) {
+          float rs;
+          const float *cs_base = nullptr;
+          if (p.mode == MODE_ROWS) {
+            const int64_t rr = min(static_cast<int64_t>(t.r0 + row), static_cast<int64_t>(p.M - 1));
+            rs = __ldg(p.row_scale + static_cast<int64_t>(b) * p.row_scale_ld + rr);
+          } else {
+            const int64_t ch = s_tpre[t.g] + b;
+            rs = __ldg(p.row_scale + ch * p.row_scale_ld + t.kt * kBM + row);
+            cs_base = p.colblk_scale + ch * p.colblk_ld + col0;
+          }
+          const uint32_t buf = u & 1;
+          if (!mbar_wait(&tfull[buf], (u >> 1) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tl + buf * kBN + c * 32, v);
+            tmem_wait_ld();
+            if (p.mode == MODE_ROWS) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(__uint_as_float(v[i]), rs, acc[c * 32 + i]);
+            } else {
+              // columns past ncols (a half tile when N % 256 == 128) are never
+              // stored; their scales are not read
+              const bool cols_ok = col0 + c * 32 < p.ncols;
+              const float4 *cs4 = reinterpret_cast<const float4 *>(cs_base + c * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 cs = cols_ok ? __ldg(cs4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                acc[c * 32 + 4 * i + 0] = fmaf(__uint_as_float(v[4 * i + 0]), rs * cs.x, acc[c * 32 + 4 * i + 0]);
+                acc[c * 32 + 4 * i + 1] = fmaf(__uint_as_float(v[4 * i + 1]), rs * cs.y, acc[c * 32 + 4 * i + 1]);
+                acc[c * 32 + 4 * i + 2] = fmaf(__uint_as_float(v[4 * i + 2]), rs * cs.z, acc[c * 32 + 4 * i + 2]);
+                acc[c * 32 + 4 * i + 3] = fmaf(__uint_as_float(v[4 * i + 3]), rs * cs.w, acc[c * 32 + 4 * i + 3]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+          ++u;
+        }
+        if (!ok) break;
+        if (row_ok) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (col0 + c * 32 >= p.ncols) continue;
+            float o[32];
+            if (p.col_scale) {
+              const float4 *cs4 = reinterpret_cast<const float4 *>(p.col_scale +
+                                                                   static_cast<int64_t>(t.g) * p.ncols + col0 + c * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 cs = __ldg(cs4 + i);
+                o[4 * i + 0] = acc[c * 32 + 4 * i + 0] * cs.x;
+                o[4 * i + 1] = acc[c * 32 + 4 * i + 1] * cs.y;
+                o[4 * i + 2] = acc[c * 32 + 4 * i + 2] * cs.z;
+                o[4 * i + 3] = acc[c * 32 + 4 * i + 3] * cs.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = acc[c * 32 + i];
+            }
+            store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32);
+          }
+        }
+      } else {
+        const uint32_t buf = u & 1;
+        if (!mbar_wait(&tfull[buf], (u >> 1) & 1, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float s0 = p.static_scale ? (sstat_ok ? sstat : 0.0f) : 1.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tl + buf * kBN + c * 32, v);
+          tmem_wait_ld();
+          if (!row_ok || col0 + c * 32 >= p.ncols) continue;
+          float o[32];
+          if (p.col_scale) {
+            const float4 *cs4 =
+                reinterpret_cast<const float4 *>(p.col_scale + static_cast<int64_t>(t.g) * p.ncols + col0 + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 cs = __ldg(cs4 + i);
+              o[4 * i + 0] = __uint_as_float(v[4 * i + 0]) * s0 * cs.x;
+              o[4 * i + 1] = __uint_as_float(v[4 * i + 1]) * s0 * cs.y;
+              o[4 * i + 2] = __uint_as_float(v[4 * i + 2]) * s0 * cs.z;
+              o[4 * i + 3] = __uint_as_float(v[4 * i + 3]) * s0 * cs.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(v[i]) * s0;
+          }
+          store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        ++u;
+      }
+    }
+    // rows outside every group are zero (row-ragged passes only)
+    if (p.mode == MODE_ROWS) {
+      const int esz = p.out_f32 ? 4 : 2;
+      const int64_t tail0 = s_offs[p.G];
+      const int64_t cpr = static_cast<int64_t>(p.ncols) * esz / 16;  // 16-byte chunks per row
+      const int64_t n = (static_cast<int64_t>(p.M) - tail0) * cpr;
+      const int et = threadIdx.x - 64;
+      for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + et; i < n; i += static_cast<int64_t>(gridDim.x) * 256) {
+        const int64_t r = tail0 + i / cpr, c = i % cpr;
+        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) + (r * p.ld_out) * esz + c * 16) =
+            make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+static int g_num_sms = 0;
+
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+template <int kElem, bool kBMN, bool kPromote>
+static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p, int grid,
+                               cudaStream_t st) {
+  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote>;
+  const size_t smem = gemm_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, st>>>(tmA, tmB, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
+                        int grid, cudaStream_t st) {
+  if (cfg.elem_bytes == 1) {
+    if (cfg.b_mn_major)
+      return cfg.promote ? launch_inst<1, true, true>(tmA, tmB, p, grid, st)
+                         : launch_inst<1, true, false>(tmA, tmB, p, grid, st);
+    return cfg.promote ? launch_inst<1, false, true>(tmA, tmB, p, grid, st)
+                       : launch_inst<1, false, false>(tmA, tmB, p, grid, st);
+  }
+  if (cfg.promote) return cudaErrorInvalidValue;
+  return cfg.b_mn_major ? launch_inst<2, true, false>(tmA, tmB, p, grid, st)
+                        : launch_inst<2, false, false>(tmA, tmB, p, grid, st);
+}
+
+}  // namespace gmm

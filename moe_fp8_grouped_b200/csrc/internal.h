@@ -1,0 +1,97 @@
+// internal.h -- declarations shared by the C-ABI layer (api.cu) and the
+// kernels (plan_quant.cu, gemm_tc.cu).  Not part of the public interface.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "gmm_fp8.h"
+
+namespace gmm {
+
+constexpr int kBlk = 128;         // quantization block / chunk length
+constexpr int kMaxGroups = 1024;  // groups handled per call
+constexpr uint64_t kDefaultWaitLimitNs = 4000000000ull;
+
+// Workspace: a 256-byte header (status word), the group plan, then the
+// quantized operands of the pass.
+struct WsHeader {
+  uint32_t status;  // GMM_DEV_* bits of the last call
+  uint32_t pad[63];
+};
+
+struct WsLayout {
+  size_t plan_offs;    // int32 [G + 1] row offsets (clamped)
+  size_t plan_tpre;    // int32 [G + 1] prefix of 128-row tiles / chunks per group
+  size_t codes_a;      // operand A codes
+  size_t codes_b;      // operand B codes (tgmm only)
+  size_t scales_a;     // fp32 scales of A
+  size_t scales_b;     // fp32 scales of B (tgmm only)
+  size_t total;
+};
+
+WsLayout ws_layout(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G);
+
+// Group plan: validates group_sizes, writes clamped offsets and the tile
+// prefix, and resets the status word to the group-size verdict.
+cudaError_t launch_plan(const int32_t *sizes, int G, int64_t M, int *offs, int *tpre, uint32_t *status,
+                        cudaStream_t st);
+
+// Row quantizer (axis 1).  static_scale != NULL selects the static rule;
+// col_scale != NULL folds col_scale[g(m), n] in (needs offs).
+cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dynamic, const float *static_scale,
+                              const float *col_scale, const int *offs, int G, uint8_t *codes, float *scales,
+                              uint32_t *status, cudaStream_t st);
+
+// Chunk quantizer (axis 0, tgmm operand), transposed + padded codes.
+// bf16_copy: write the bf16 values instead of codes (bf16 family packing).
+cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool dynamic, const float *static_scale,
+                                const int *offs, const int *tpre, int G, int64_t capacity, void *codes_t,
+                                float *scales, bool bf16_copy, uint32_t *status, cudaStream_t st);
+
+cudaError_t launch_quant_rhs(const void *w, int G, int64_t K, int64_t N, bool transpose_out, uint8_t *codes,
+                             float *scales, cudaStream_t st);
+
+cudaError_t launch_timeout_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t st);
+
+enum GemmMode { MODE_ROWS = 0, MODE_TGMM = 1 };
+
+struct GemmParams {
+  int mode;            // GemmMode
+  int G;
+  int M;               // rows of the row operand (MODE_ROWS) / of x (MODE_TGMM)
+  int ncols;           // output columns
+  int kblocks;         // MODE_ROWS: contraction stages (128 bytes of operand row each)
+  int ktiles;          // MODE_TGMM: 128-row tiles of the output (K / 128)
+  int b_group_rows;    // MODE_ROWS: rows per group in B's 2-D view
+  int stages_per_chunk;// MODE_TGMM: stages per 128-row chunk (1 fp8, 2 bf16)
+  const int *offs;     // [G + 1]
+  const int *tpre;     // [G + 1]
+  const float *row_scale;     // MODE_ROWS: [kblocks][M]; MODE_TGMM: [chunk][K]
+  int64_t row_scale_ld;
+  const float *colblk_scale;  // MODE_TGMM: [chunk][N]
+  int64_t colblk_ld;
+  const float *col_scale;     // [G][ncols] final per-column scale, or NULL
+  const float *static_scale;  // device scalar multiplied in at the end, or NULL
+  void *out;
+  int out_f32;
+  int64_t ld_out;
+  uint32_t *status;
+  uint64_t wait_limit_ns;
+};
+
+struct GemmConfig {
+  int elem_bytes;   // 1: E4M3 (kind::f8f6f4), 2: BF16 (kind::f16)
+  bool b_mn_major;  // B operand MN-major in shared memory
+  bool promote;     // one TMEM unit per contraction block, promoted in registers
+};
+
+int num_sms();
+
+cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        const GemmParams &p, int grid, cudaStream_t st);
+
+}  // namespace gmm

@@ -1,0 +1,459 @@
+// plan_quant.cu -- the group plan and the E4M3 quantizers.
+//
+// Quantization follows "add static LHS scaling support for GMM v2 FWD"
+// (maxtext PR #4735), review threads on the LhsRef docstring (lhs arrives
+// unquantized, qvalue = clip(lhs / scale)) and on inner_kernel (inverse scale
+// 0 where the scale is 0; lhs * inverse cast to the fp8 dtype): inv =
+// fl32(1/s), code = E4M3 round-to-nearest-even of fl32(x * inv), saturated to
+// +-448.  Every fp32 step is an explicit _rn intrinsic so that no FMA is
+// contracted and the codes are bit-identical to a plain IEEE evaluation.
+#include <cuda_bf16.h>
+#include <cfloat>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gmm {
+
+// ------------------------------------------------------------------ plan
+
+// One warp.  Lane l owns groups [l*per, (l+1)*per).  Negative sizes count as
+// 0; group g spans rows [min(P_g, M), min(P_g + s_g, M)) with P the prefix of
+// the non-negative sizes.  tpre is the prefix of ceil(rows / 128).
+__global__ void plan_kernel(const int32_t *__restrict__ sizes, int G, int64_t M, int *__restrict__ offs,
+                            int *__restrict__ tpre, uint32_t *__restrict__ status) {
+  const int lane = threadIdx.x;
+  const int per = (G + 31) / 32;
+  const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+  long long local = 0;
+  int bad = 0;
+  for (int g = g0; g < g1; ++g) {
+    int s = sizes[g];
+    if (s < 0) bad = 1;
+    local += s < 0 ? 0 : s;
+  }
+  long long incl = local;
+  for (int d = 1; d < 32; d <<= 1) {
+    long long v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  long long run = incl - local;  // exclusive prefix of this lane's first group
+  const long long total = __shfl_sync(0xffffffffu, incl, 31);
+  int tiles_local = 0;
+  for (int g = g0; g < g1; ++g) {
+    int s = sizes[g] < 0 ? 0 : sizes[g];
+    long long a = run < M ? run : M, b = run + s < M ? run + s : M;
+    tiles_local += static_cast<int>((b - a + kBlk - 1) / kBlk);
+    run += s;
+  }
+  int tincl = tiles_local;
+  for (int d = 1; d < 32; d <<= 1) {
+    int v = __shfl_up_sync(0xffffffffu, tincl, d);
+    if (lane >= d) tincl += v;
+  }
+  int trun = tincl - tiles_local;
+  run = incl - local;
+  for (int g = g0; g < g1; ++g) {
+    int s = sizes[g] < 0 ? 0 : sizes[g];
+    long long a = run < M ? run : M, b = run + s < M ? run + s : M;
+    offs[g] = static_cast<int>(a);
+    tpre[g] = trun;
+    trun += static_cast<int>((b - a + kBlk - 1) / kBlk);
+    run += s;
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 31) {
+    offs[G] = static_cast<int>(total < M ? total : M);
+    tpre[G] = tincl;
+  }
+  if (lane == 0) *status = (bad || total > M) ? GMM_DEV_GROUP_SIZES : 0u;
+}
+
+cudaError_t launch_plan(const int32_t *sizes, int G, int64_t M, int *offs, int *tpre, uint32_t *status,
+                        cudaStream_t st) {
+  plan_kernel<<<1, 32, 0, st>>>(sizes, G, M, offs, tpre, status);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- helpers
+
+__device__ __forceinline__ bool static_scale_ok(float s) { return isfinite(s) && s > FLT_MIN; }
+
+// Dynamic scale of a block: s = fl32(amax / 448), inv = fl32(1 / s), both 0
+// when s is 0 or when 1/s overflows.
+__device__ __forceinline__ void dyn_scale(float amax, float &s, float &inv) {
+  s = __fdiv_rn(amax, 448.0f);
+  inv = (s == 0.0f) ? 0.0f : __fdiv_rn(1.0f, s);
+  if (isinf(inv)) {
+    s = 0.0f;
+    inv = 0.0f;
+  }
+}
+
+__device__ __forceinline__ int group_of_row(const int *s_offs, int G, int64_t r) {
+  // first index i in [0, G] with offs[i] > r, minus one
+  int lo = 0, hi = G + 1;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (s_offs[mid] > r) hi = mid;
+    else lo = mid + 1;
+  }
+  int g = lo - 1;
+  return (g >= 0 && g < G && r < s_offs[g + 1]) ? g : -1;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&v)[8]) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+// ------------------------------------------------------ rows (axis 1)
+
+// A warp covers 256 consecutive values of one row: each half-warp one block
+// of 128, each lane 8 values (16 bytes).
+template <bool kDynamic, bool kColMult>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
+                                                         int64_t cols, const float *__restrict__ static_scale,
+                                                         const float *__restrict__ col_scale,
+                                                         const int *__restrict__ offs, int G,
+                                                         uint8_t *__restrict__ codes, float *__restrict__ scales,
+                                                         uint32_t *__restrict__ status) {
+  __shared__ int s_offs[kMaxGroups + 1];
+  if constexpr (kColMult) {
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) s_offs[i] = offs[i];
+    __syncthreads();
+  }
+  float inv_static = 0.0f;
+  if constexpr (!kDynamic) {
+    const float s = *static_scale;
+    const bool ok = static_scale_ok(s);
+    inv_static = ok ? __fdiv_rn(1.0f, s) : 0.0f;
+    if (!ok && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, GMM_DEV_SCALE);
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, hl = lane & 15;
+  const int64_t segs_per_row = (cols + 255) / 256;
+  const int64_t total = rows * segs_per_row;
+  for (int64_t seg = static_cast<int64_t>(blockIdx.x) * 8 + warp; seg < total;
+       seg += static_cast<int64_t>(gridDim.x) * 8) {
+    const int64_t r = seg / segs_per_row;
+    const int64_t cb = (seg % segs_per_row) * 256 + half * 128;  // block start
+    const int64_t c0 = cb + hl * 8;
+    const bool valid = cb < cols;
+    float v[8];
+    if (valid) {
+      uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + r * cols + c0));
+      bf16x8_to_f32(u, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+    if constexpr (kColMult) {
+      const int g = group_of_row(s_offs, G, r);
+      if (g < 0 || !valid) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+      } else {
+        const float4 *cs = reinterpret_cast<const float4 *>(col_scale + static_cast<int64_t>(g) * cols + c0);
+        float4 a = __ldg(cs), b = __ldg(cs + 1);
+        v[0] = __fmul_rn(v[0], a.x); v[1] = __fmul_rn(v[1], a.y);
+        v[2] = __fmul_rn(v[2], a.z); v[3] = __fmul_rn(v[3], a.w);
+        v[4] = __fmul_rn(v[4], b.x); v[5] = __fmul_rn(v[5], b.y);
+        v[6] = __fmul_rn(v[6], b.z); v[7] = __fmul_rn(v[7], b.w);
+      }
+    }
+    float s = 0.0f, inv;
+    if constexpr (kDynamic) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+      for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+      dyn_scale(amax, s, inv);
+    } else {
+      inv = inv_static;
+    }
+    if (valid) {
+      uint2 out;
+      out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
+              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
+      out.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv))) |
+              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
+      *reinterpret_cast<uint2 *>(codes + r * cols + c0) = out;
+      if (kDynamic && hl == 0) scales[(cb / kBlk) * rows + r] = s;
+    }
+  }
+}
+
+cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dynamic, const float *static_scale,
+                              const float *col_scale, const int *offs, int G, uint8_t *codes, float *scales,
+                              uint32_t *status, cudaStream_t st) {
+  const int64_t segs = rows * ((cols + 255) / 256);
+  int64_t blocks = (segs + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  if (dynamic && col_scale)
+    quant_rows_kernel<true, true><<<blocks, 256, 0, st>>>(xb, rows, cols, static_scale, col_scale, offs, G, codes,
+                                                          scales, status);
+  else if (dynamic)
+    quant_rows_kernel<true, false><<<blocks, 256, 0, st>>>(xb, rows, cols, static_scale, col_scale, offs, G,
+                                                           codes, scales, status);
+  else if (col_scale)
+    quant_rows_kernel<false, true><<<blocks, 256, 0, st>>>(xb, rows, cols, static_scale, col_scale, offs, G,
+                                                           codes, scales, status);
+  else
+    quant_rows_kernel<false, false><<<blocks, 256, 0, st>>>(xb, rows, cols, static_scale, col_scale, offs, G,
+                                                            codes, scales, status);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------- chunks (axis 0)
+
+// One CTA per (128-column slice, chunk).  The chunk's rows (at most 128, the
+// rest zero) are staged in shared memory; thread t owns column t % 128 and
+// rows [64 (t / 128), +64), and writes them as 64 contiguous bytes of the
+// transposed code matrix.
+template <bool kDynamic, bool kCopy>
+__global__ void __launch_bounds__(256) quant_chunks_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
+                                                           int64_t cols, const float *__restrict__ static_scale,
+                                                           const int *__restrict__ offs,
+                                                           const int *__restrict__ tpre, int G, void *codes_t,
+                                                           int64_t ld_t, float *__restrict__ scales,
+                                                           uint32_t *__restrict__ status) {
+  __shared__ __align__(16) __nv_bfloat16 tile[kBlk][kBlk + 8];
+  __shared__ float s_amax[2][kBlk];
+  __shared__ int s_info[3];
+  const int j = blockIdx.y;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kBlk;
+  if (threadIdx.x == 0) {
+    int g = -1;
+    if (j < tpre[G]) {
+      int lo = 0, hi = G + 1;  // first i with tpre[i] > j
+      while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (tpre[mid] > j) hi = mid;
+        else lo = mid + 1;
+      }
+      g = lo - 1;
+    }
+    s_info[0] = g;
+    if (g >= 0) {
+      const int r0 = offs[g] + kBlk * (j - tpre[g]);
+      s_info[1] = r0;
+      s_info[2] = min(r0 + kBlk, offs[g + 1]) - r0;
+    }
+  }
+  __syncthreads();
+  const int g = s_info[0];
+  if (g < 0) return;
+  const int r0 = s_info[1], nr = s_info[2];
+  for (int i = threadIdx.x; i < kBlk * 16; i += 256) {
+    const int rr = i >> 4, cc = (i & 15) * 8;
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (rr < nr) u = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc));
+    *reinterpret_cast<uint4 *>(&tile[rr][cc]) = u;
+  }
+  __syncthreads();
+  const int col = threadIdx.x & 127, h = threadIdx.x >> 7;
+  const int rb = 64 * h;
+  if constexpr (kCopy) {
+    // bf16 family: transposed bf16 copy, no scale
+    uint16_t *dst = static_cast<uint16_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j + rb;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint16_t lo = __bfloat16_as_ushort(tile[rb + q * 8 + 2 * e][col]);
+        const uint16_t hi = __bfloat16_as_ushort(tile[rb + q * 8 + 2 * e + 1][col]);
+        w[e] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+      }
+      *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return;
+  } else {
+    float s, inv;
+    if constexpr (kDynamic) {
+      float amax = 0.0f;
+      for (int r = rb; r < rb + 64; ++r) amax = fmaxf(amax, fabsf(__bfloat162float(tile[r][col])));
+      s_amax[h][col] = amax;
+      __syncthreads();
+      dyn_scale(fmaxf(s_amax[0][col], s_amax[1][col]), s, inv);
+    } else {
+      s = *static_scale;
+      const bool ok = static_scale_ok(s);
+      inv = ok ? __fdiv_rn(1.0f, s) : 0.0f;
+      if (!ok) s = 0.0f;
+      if (!ok && j == 0 && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, GMM_DEV_SCALE);
+    }
+    uint8_t *dst = static_cast<uint8_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j + rb;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = rb + q * 16 + e * 4;
+        const float a0 = __fmul_rn(__bfloat162float(tile[r][col]), inv);
+        const float a1 = __fmul_rn(__bfloat162float(tile[r + 1][col]), inv);
+        const float a2 = __fmul_rn(__bfloat162float(tile[r + 2][col]), inv);
+        const float a3 = __fmul_rn(__bfloat162float(tile[r + 3][col]), inv);
+        w[e] = static_cast<uint32_t>(cvt_e4m3x2(a0, a1)) | (static_cast<uint32_t>(cvt_e4m3x2(a2, a3)) << 16);
+      }
+      *reinterpret_cast<uint4 *>(dst + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (h == 0) scales[static_cast<int64_t>(j) * cols + c0 + col] = s;
+  }
+}
+
+cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool dynamic, const float *static_scale,
+                                const int *offs, const int *tpre, int G, int64_t capacity, void *codes_t,
+                                float *scales, bool bf16_copy, uint32_t *status, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(cols / kBlk), static_cast<unsigned>(capacity));
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  const int64_t ld_t = capacity * kBlk;
+  if (bf16_copy)
+    quant_chunks_kernel<false, true><<<grid, 256, 0, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t,
+                                                           ld_t, scales, status);
+  else if (dynamic)
+    quant_chunks_kernel<true, false><<<grid, 256, 0, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t,
+                                                           ld_t, scales, status);
+  else
+    quant_chunks_kernel<false, false><<<grid, 256, 0, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t,
+                                                            ld_t, scales, status);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ rhs (K7)
+
+// Column absmax of W[g, :, n] into amax_bits (fp32 bit patterns of values
+// >= 0 order like unsigned integers, so atomicMax on the bits is a max).
+__global__ void __launch_bounds__(256) rhs_amax_kernel(const __nv_bfloat16 *__restrict__ w, int64_t K, int64_t N,
+                                                       unsigned int *__restrict__ amax_bits) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int g = blockIdx.z;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * 128;
+  if (n >= N) return;
+  float m = 0.0f;
+  const int64_t k1 = min(k0 + 128, K);
+  for (int64_t k = k0; k < k1; ++k) m = fmaxf(m, fabsf(__bfloat162float(w[(g * K + k) * N + n])));
+  atomicMax(amax_bits + static_cast<int64_t>(g) * N + n, __float_as_uint(m));
+}
+
+// 128 x 128 tiles of W[g] (rows k, columns n): codes written row-wise
+// ([G, K, N]) or column-wise ([G, N, K]).
+template <bool kTranspose>
+__global__ void __launch_bounds__(256) rhs_codes_kernel(const __nv_bfloat16 *__restrict__ w, int64_t K, int64_t N,
+                                                        const unsigned int *__restrict__ amax_bits,
+                                                        uint8_t *__restrict__ codes) {
+  __shared__ __align__(16) __nv_bfloat16 tile[kBlk][kBlk + 8];
+  __shared__ float s_inv[kBlk];
+  const int g = blockIdx.z;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBlk, k0 = static_cast<int64_t>(blockIdx.y) * kBlk;
+  for (int i = threadIdx.x; i < kBlk * 16; i += 256) {
+    const int rr = i >> 4, cc = (i & 15) * 8;
+    *reinterpret_cast<uint4 *>(&tile[rr][cc]) =
+        __ldg(reinterpret_cast<const uint4 *>(w + (g * K + k0 + rr) * N + n0 + cc));
+  }
+  if (threadIdx.x < kBlk) {
+    float s, inv;
+    dyn_scale(__uint_as_float(amax_bits[static_cast<int64_t>(g) * N + n0 + threadIdx.x]), s, inv);
+    s_inv[threadIdx.x] = inv;
+  }
+  __syncthreads();
+  const int t = threadIdx.x & 127, h = threadIdx.x >> 7;
+  if constexpr (!kTranspose) {
+    // thread (row t, half h): 64 columns of row k0 + t
+    uint8_t *dst = codes + (g * K + k0 + t) * N + n0 + 64 * h;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t wv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = 64 * h + q * 16 + e * 4;
+        const float a0 = __fmul_rn(__bfloat162float(tile[t][c]), s_inv[c]);
+        const float a1 = __fmul_rn(__bfloat162float(tile[t][c + 1]), s_inv[c + 1]);
+        const float a2 = __fmul_rn(__bfloat162float(tile[t][c + 2]), s_inv[c + 2]);
+        const float a3 = __fmul_rn(__bfloat162float(tile[t][c + 3]), s_inv[c + 3]);
+        wv[e] = static_cast<uint32_t>(cvt_e4m3x2(a0, a1)) | (static_cast<uint32_t>(cvt_e4m3x2(a2, a3)) << 16);
+      }
+      *reinterpret_cast<uint4 *>(dst + q * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    }
+  } else {
+    // thread (column t, half h): 64 rows of column n0 + t
+    const float inv = s_inv[t];
+    uint8_t *dst = codes + (g * N + n0 + t) * K + k0 + 64 * h;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t wv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = 64 * h + q * 16 + e * 4;
+        const float a0 = __fmul_rn(__bfloat162float(tile[r][t]), inv);
+        const float a1 = __fmul_rn(__bfloat162float(tile[r + 1][t]), inv);
+        const float a2 = __fmul_rn(__bfloat162float(tile[r + 2][t]), inv);
+        const float a3 = __fmul_rn(__bfloat162float(tile[r + 3][t]), inv);
+        wv[e] = static_cast<uint32_t>(cvt_e4m3x2(a0, a1)) | (static_cast<uint32_t>(cvt_e4m3x2(a2, a3)) << 16);
+      }
+      *reinterpret_cast<uint4 *>(dst + q * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    }
+  }
+}
+
+// amax -> scale, in place.
+__global__ void rhs_scale_kernel(float *__restrict__ scales, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (i >= n) return;
+  float s, inv;
+  dyn_scale(scales[i], s, inv);
+  scales[i] = s;
+}
+
+cudaError_t launch_quant_rhs(const void *w, int G, int64_t K, int64_t N, bool transpose_out, uint8_t *codes,
+                             float *scales, cudaStream_t st) {
+  const __nv_bfloat16 *wb = static_cast<const __nv_bfloat16 *>(w);
+  cudaError_t e = cudaMemsetAsync(scales, 0, sizeof(float) * G * N, st);
+  if (e != cudaSuccess) return e;
+  rhs_amax_kernel<<<dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>((K + 127) / 128), G), 256,
+                    0, st>>>(wb, K, N, reinterpret_cast<unsigned int *>(scales));
+  dim3 grid(static_cast<unsigned>(N / kBlk), static_cast<unsigned>(K / kBlk), G);
+  if (transpose_out)
+    rhs_codes_kernel<true><<<grid, 256, 0, st>>>(wb, K, N, reinterpret_cast<unsigned int *>(scales), codes);
+  else
+    rhs_codes_kernel<false><<<grid, 256, 0, st>>>(wb, K, N, reinterpret_cast<unsigned int *>(scales), codes);
+  const int64_t n = static_cast<int64_t>(G) * N;
+  rhs_scale_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(scales, n);
+  return cudaGetLastError();
+}
+
+// -------------------------------------------------- bounded-wait self-test
+
+// Waits on a barrier that nothing arrives on; the bounded wait gives up after
+// limit_ns and records GMM_DEV_TIMEOUT.
+__global__ void timeout_selftest_kernel(uint32_t *status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtl ctl{limit_ns, &abort_flag, status};
+    mbar_wait(&bar, 0, ctl);  // phase 0 never completes
+  }
+}
+
+cudaError_t launch_timeout_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t st) {
+  timeout_selftest_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace gmm

@@ -1,0 +1,277 @@
+"""CUDA path vs the CPU oracle on small ragged cases (through the C-ABI).
+
+Codes and scales are compared bit for bit; pass outputs element by element
+within 2e-3 * sum|a*b| (plus bf16 output rounding).  Cases span several
+tiles, ragged tails, empty groups, unrouted rows, N not a multiple of the
+256-wide tile, both rhs layouts and both output dtypes.  Each pass is run on
+its own (the pages' review found a bug where one pass's flag leaked into
+another: "Support quantization for tokamax gmm v2", maxtext PR #4451, review
+thread on the dlhs selection).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_fp8_grouped_b200 as gm
+import oracle
+from moe_fp8_grouped_b200 import synth
+from parity import assert_close, check_guards, guarded, rule_code, untranspose_chunks
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": None,  # the tiny workload: G=8, M=256, K=512, N=512, group 3 empty
+    "ragged": (5, 700, 384, 640, [1, 129, 0, 300, 200]),  # 70 unrouted rows, N % 256 = 128
+    "g1": (1, 300, 256, 256, [300]),
+    "big_group": (2, 1100, 512, 256, [1000, 100]),
+}
+
+
+def case_inputs(name):
+    if CASES[name] is None:
+        return synth.make_inputs("tiny", seed=0)
+    G, M, K, N, sizes = CASES[name]
+    return synth.small_case(G, M, K, N, seed=7, sizes=sizes)
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch.device("cuda:0")
+
+
+def to_dev(inp, dev):
+    return (inp.lhs.to(dev), inp.w.to(dev), inp.dout.to(dev), inp.group_sizes.to(dev),
+            torch.tensor([inp.static_scale], dtype=torch.float32, device=dev))
+
+
+# ----------------------------------------------------------- quantizers
+
+@pytest.mark.parametrize("transpose", [False, True])
+def test_quantize_rhs_bitexact(dev, transpose):
+    inp = case_inputs("ragged")
+    codes, scales = gm.gmm_quantize_rhs(inp.w.to(dev), transpose_out=transpose)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    got = codes.cpu().numpy()
+    if transpose:
+        got = got.transpose(0, 2, 1)
+    assert np.array_equal(got, qr)
+    assert np.array_equal(scales.cpu().numpy(), sr)
+
+
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+def test_quantize_rows_bitexact(dev, rule):
+    inp = case_inputs("ragged")
+    x = inp.lhs.to(dev)
+    s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    codes, scales = gm.gmm_quantize(x, rule, axis=1, static_scale=s if rule == "static" else None)
+    qc, qs, _ = oracle.quantize_rows(inp.lhs, rule_code(rule), inp.static_scale)
+    assert np.array_equal(codes.cpu().numpy(), qc)
+    if rule == "dynamic":
+        assert np.array_equal(scales.cpu().numpy().T, qs)
+
+
+def test_quantize_rows_scaled_bitexact(dev):
+    inp = case_inputs("ragged")
+    _, sr = oracle.quantize_rhs(inp.w)
+    codes, scales = gm.gmm_quantize(inp.dout.to(dev), "dynamic", axis=1, group_sizes=inp.group_sizes.to(dev),
+                                    col_scale=torch.from_numpy(sr).to(dev))
+    qc, qs = oracle.quantize_rows_scaled(inp.dout, sr, inp.group_sizes)
+    assert np.array_equal(codes.cpu().numpy(), qc)
+    assert np.array_equal(scales.cpu().numpy().T, qs)
+
+
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("name", ["ragged", "tiny"])
+def test_quantize_chunks_bitexact(dev, rule, name):
+    inp = case_inputs(name)
+    M = inp.lhs.shape[0]
+    s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    codes_t, scales = gm.gmm_quantize(inp.lhs.to(dev), rule, axis=0, static_scale=s if rule == "static" else None,
+                                      group_sizes=inp.group_sizes.to(dev))
+    offs, _ = oracle.plan(inp.group_sizes, M)
+    got_c, got_s = untranspose_chunks(codes_t, scales, offs, M)
+    qc, qs = oracle.quantize_chunks(inp.lhs, rule_code(rule), inp.static_scale, inp.group_sizes)
+    assert np.array_equal(got_c, qc)
+    assert np.array_equal(got_s, qs)
+
+
+# ---------------------------------------------------------------- passes
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fwd(dev, name, rule, transpose, out_dtype):
+    inp = case_inputs(name)
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    M, N = lhs.shape[0], w.shape[2]
+    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
+    raw, out, pad, n = guarded((M, N), out_dtype)
+    gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=s if rule == "static" else None,
+               transpose_rhs=transpose, out=out)
+    assert gm.last_launch_count() == 3
+    torch.cuda.synchronize()
+    check_guards(raw, pad, n)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    ref, ab = oracle.gmm_fwd(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+    assert_close(out, ref, ab, f"fwd {name} {rule} t={transpose}")
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_dlhs(dev, name, transpose, out_dtype):
+    inp = case_inputs(name)
+    _, w, dout, gs, _ = to_dev(inp, dev)
+    M, K = inp.lhs.shape
+    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
+    raw, out, pad, n = guarded((M, K), out_dtype)
+    gm.gmm_dlhs(dout, codes, scales, gs, transpose_rhs=transpose, out=out)
+    torch.cuda.synchronize()
+    check_guards(raw, pad, n)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    ref, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
+    assert_close(out, ref, ab, f"dlhs {name} t={transpose}")
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_drhs(dev, name, rule, out_dtype):
+    inp = case_inputs(name)
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    G, K, N = w.shape
+    raw, out, pad, n = guarded((G, K, N), out_dtype)
+    gm.tgmm_drhs(lhs, dout, gs, rule=rule, static_scale=s if rule == "static" else None, out=out)
+    assert gm.last_launch_count() == 4
+    torch.cuda.synchronize()
+    check_guards(raw, pad, n)
+    ref, ab = oracle.tgmm_drhs(inp.lhs, rule_code(rule), inp.static_scale, inp.dout, inp.group_sizes)
+    assert_close(out, ref, ab, f"drhs {name} {rule}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_bf16_family(dev, name):
+    inp = case_inputs(name)
+    lhs, w, dout, gs, _ = to_dev(inp, dev)
+    f = gm.gmm_fwd(lhs, w, None, gs, rule="none", out_dtype=torch.float32)
+    ref, ab = oracle.gmm_fwd_bf16(inp.lhs, inp.w, inp.group_sizes)
+    assert_close(f, ref, ab, "bf16 fwd")
+    d = gm.gmm_dlhs(dout, w, None, gs, rule="none", out_dtype=torch.float32)
+    ref, ab = oracle.gmm_dlhs_bf16(inp.dout, inp.w, inp.group_sizes)
+    assert_close(d, ref, ab, "bf16 dlhs")
+    r = gm.tgmm_drhs(lhs, dout, gs, rule="none", out_dtype=torch.float32)
+    ref, ab = oracle.tgmm_drhs_bf16(inp.lhs, inp.dout, inp.group_sizes)
+    assert_close(r, ref, ab, "bf16 drhs")
+
+
+# ------------------------------------------------------------ identities
+
+def test_merged_gate_up_identity_gpu(dev):
+    """fwd(W0|W1) equals fwd(W0) | fwd(W1) bit for bit (each output column
+    sees the same K sequence); drhs likewise; dlhs adds up within tolerance."""
+    inp = synth.small_case(4, 600, 512, 512, seed=3, sizes=[200, 0, 250, 150])
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    c, sc = gm.gmm_quantize_rhs(w)
+    c0, s0 = gm.gmm_quantize_rhs(w[:, :, :256].contiguous())
+    c1, s1 = gm.gmm_quantize_rhs(w[:, :, 256:].contiguous())
+    for rule in ("static", "dynamic"):
+        kw = dict(rule=rule, static_scale=s if rule == "static" else None, out_dtype=torch.float32)
+        f = gm.gmm_fwd(lhs, c, sc, gs, **kw)
+        f0 = gm.gmm_fwd(lhs, c0, s0, gs, **kw)
+        f1 = gm.gmm_fwd(lhs, c1, s1, gs, **kw)
+        assert torch.equal(f, torch.cat([f0, f1], dim=1))
+        kw.pop("out_dtype")
+        r = gm.tgmm_drhs(lhs, dout, gs, **kw)
+        r0 = gm.tgmm_drhs(lhs, dout[:, :256].contiguous(), gs, **kw)
+        r1 = gm.tgmm_drhs(lhs, dout[:, 256:].contiguous(), gs, **kw)
+        assert torch.equal(r, torch.cat([r0, r1], dim=2))
+    d = gm.gmm_dlhs(dout, c, sc, gs, out_dtype=torch.float32)
+    d0 = gm.gmm_dlhs(dout[:, :256].contiguous(), c0, s0, gs, out_dtype=torch.float32)
+    d1 = gm.gmm_dlhs(dout[:, 256:].contiguous(), c1, s1, gs, out_dtype=torch.float32)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    _, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
+    assert np.all(np.abs((d - d0 - d1).cpu().numpy()) <= 2e-3 * ab)
+
+
+def test_passes_do_not_depend_on_each_other(dev):
+    """Each pass reads only its own inputs: a workspace left dirty by another
+    pass (or garbage) does not change the result."""
+    inp = case_inputs("ragged")
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    c, sc = gm.gmm_quantize_rhs(w)
+    G, K, N = w.shape
+    M = lhs.shape[0]
+    nbytes = max(gm.gmm_workspace_bytes(op, M, K, N, G) for op in (0, 1, 2))
+    clean = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    dirty = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device=dev)
+    a = gm.gmm_dlhs(dout, c, sc, gs, ws=clean, out_dtype=torch.float32)
+    b = gm.gmm_dlhs(dout, c, sc, gs, ws=dirty, out_dtype=torch.float32)
+    assert torch.equal(a, b)
+    a = gm.tgmm_drhs(lhs, dout, gs, rule="static", static_scale=s, ws=clean)
+    gm.gmm_fwd(lhs, c, sc, gs, rule="dynamic", ws=dirty)
+    b = gm.tgmm_drhs(lhs, dout, gs, rule="static", static_scale=s, ws=dirty)
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------- device status
+
+def test_group_sizes_past_M_are_clamped_and_reported(dev):
+    inp = synth.small_case(3, 300, 256, 256, seed=4, sizes=[100, 250, 50])
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    c, sc = gm.gmm_quantize_rhs(w)
+    ws = gm.workspace(gm.gmm_workspace_bytes(0, 300, 256, 256, 3), dev)
+    out = gm.gmm_fwd(lhs, c, sc, gs, rule="static", static_scale=s, ws=ws, out_dtype=torch.float32)
+    st, bits = gm.gmm_read_device_status(ws)
+    assert bits & 1 and st == 7  # GMM_ERR_GROUP_SIZES
+    qr, sr = oracle.quantize_rhs(inp.w)
+    ref, ab = oracle.gmm_fwd(inp.lhs, oracle.Q_STATIC, inp.static_scale, qr, sr, inp.group_sizes)
+    assert_close(out, ref, ab, "clamped fwd")
+    gs_neg = torch.tensor([100, -5, 50], dtype=torch.int32, device=dev)
+    gm.gmm_fwd(lhs, c, sc, gs_neg, rule="static", static_scale=s, ws=ws)
+    assert gm.gmm_read_device_status(ws)[0] == 7
+    gm.gmm_fwd(lhs, c, sc, torch.tensor([100, 100, 100], dtype=torch.int32, device=dev), rule="static",
+               static_scale=s, ws=ws)
+    assert gm.gmm_read_device_status(ws) == (0, 0)
+
+
+@pytest.mark.parametrize("bad", [0.0, float("inf"), float("nan"), -1.0])
+def test_unusable_static_scale_reports_and_outputs_zero(dev, bad):
+    inp = case_inputs("tiny")
+    lhs, w, _, gs, _ = to_dev(inp, dev)
+    c, sc = gm.gmm_quantize_rhs(w)
+    ws = gm.workspace(gm.gmm_workspace_bytes(0, 256, 512, 512, 8), dev)
+    out = gm.gmm_fwd(lhs, c, sc, gs, rule="static", static_scale=torch.tensor([bad], device=dev), ws=ws)
+    st, bits = gm.gmm_read_device_status(ws)
+    assert st == 4 and bits & 2  # GMM_ERR_SCALE
+    assert not out.float().abs().sum().item()
+
+
+def test_bounded_wait_gives_up_and_reports(dev):
+    ws = torch.zeros(1 << 16, dtype=torch.uint8, device=dev)
+    gm.gmm_selftest_timeout(ws, 50_000_000)  # 50 ms
+    st, bits = gm.gmm_read_device_status(ws)
+    assert st == 8 and bits & 4  # GMM_ERR_TIMEOUT
+    # the context is still usable
+    inp = case_inputs("g1")
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    c, sc = gm.gmm_quantize_rhs(w)
+    gm.gmm_fwd(lhs, c, sc, gs, rule="static", static_scale=s)
+    torch.cuda.synchronize()
+
+
+def test_host_errors_return_before_launch(dev):
+    inp = case_inputs("tiny")
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    c, sc = gm.gmm_quantize_rhs(w)
+    with pytest.raises(gm.GmmError) as e:
+        gm.gmm_fwd(lhs, c, sc, gs, rule="static", static_scale=None)  # a present rule must be applied
+    assert e.value.status == 1
+    with pytest.raises(gm.GmmError) as e:
+        gm.gmm_fwd(lhs, c, sc, gs, rule="static", static_scale=s, ws=torch.empty(16, dtype=torch.uint8,
+                                                                                  device=dev))
+    assert e.value.status == 9
+    with pytest.raises(gm.GmmError) as e:
+        gm.gmm_fwd(lhs[:, :500].contiguous(), c[:, :500].contiguous(), sc, gs, rule="static", static_scale=s)
+    assert e.value.status == 2
