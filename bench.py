@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 grouped matmul hot path on B200.
+
+One step = the three passes of one MoE expert-MLP layer on one batch:
+forward gmm (lhs quantized inside the call), dlhs gmm and tgmm drhs, on the
+Mixtral-like workload (G=8, M=16384 = 8192 tokens x top-2, K=4096,
+N=28672 = merged 2 x 14336, static per-tensor lhs scale, rhs pre-quantized
+E4M3 with per-(g, n) scales).  Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torchrun: N independent replicas (the path has no exchange
+step; each rank draws its own batch), weak scaling, time = max over ranks.
+--impl reference times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 grouped-GEMM TFLOP/s (fwd, dlhs, drhs) and % of B200 dense FP8 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+GEMM_SRC = os.path.join(ROOT, "moe_fp8_grouped_b200", "csrc", "gemm_tc.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="mixtral")
+    ap.add_argument("--m-override", type=int, default=None,
+                    help="fewer rows (same routing recipe), for profiler captures of a small case")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_of(w, extra=None):
+    cfg = {"workload": f"{w.name}: G={w.G} M={w.M} K={w.K} N={w.N}, lhs rule {w.rule}, fwd+dlhs+drhs",
+           "G": w.G, "M": w.M, "K": w.K, "N": w.N, "lhs_rule": w.rule, "routing": w.routing,
+           "out_dtypes": {"fwd": "bf16", "dlhs": "bf16", "drhs": "f32"},
+           "l2": "not flushed: inputs larger than L2 (rhs codes and dout exceed 126 MB)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    rows.append((float(p[1]), float(p[2]), float(p[3]), p[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------- our arm
+
+def traffic_record(kernel: str):
+    """DRAM bytes per launch from a committed ncu capture, or None when the
+    kernel source changed since the capture."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()[:16]
+        r = rec.get(kernel)
+        if r and r.get("gemm_src_sha256_16") == src_hash:
+            return r.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import moe_fp8_grouped_b200 as gm
+    from moe_fp8_grouped_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = synth.WORKLOADS[args.workload]
+    if args.m_override:
+        w = synth.with_rows(w, args.m_override)
+    inp = synth.make_inputs(w, seed=rank, device=str(dev))
+    gs = inp.group_sizes.to(dev)
+    rows_routed = int(inp.group_sizes.sum())
+    s_static = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    codes, rscales = gm.gmm_quantize_rhs(inp.w)  # weight quantization: outside the timed step
+    del inp.w
+    lhs, dout = inp.lhs, inp.dout
+    M, K, N, G = w.M, w.K, w.N, w.G
+    rule = w.rule
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    dl = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((G, K, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, N, G) for op in (0, 1, 2)), dtype=torch.uint8,
+                     device=dev)
+    sarg = s_static if rule == "static" else None
+    launches = [0]
+
+    def step(lhs_, dout_, codes_, rscales_, gs_):
+        gm.gmm_fwd(lhs_, codes_, rscales_, gs_, rule=rule, static_scale=sarg, out=out, ws=ws)
+        launches[0] += gm.last_launch_count()
+        gm.gmm_dlhs(dout_, codes_, rscales_, gs_, out=dl, ws=ws)
+        launches[0] += gm.last_launch_count()
+        gm.tgmm_drhs(lhs_, dout_, gs_, rule=rule, static_scale=sarg, out=dw, ws=ws)
+        launches[0] += gm.last_launch_count()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step(lhs, dout, codes, rscales, gs)
+    st, bits = gm.gmm_read_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} bits {bits} after warm-up")
+    barrier()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler start before the timed region
+    gm.profile_enable(True)
+    launches[0] = 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record()
+    for _ in range(args.steps):
+        step(lhs, dout, codes, rscales, gs)
+    e1.record()
+    barrier()
+    gm.profile_enable(False)
+    prof = gm.profile_collect()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    timed_launches = launches[0]
+
+    flops_pass = 2.0 * rows_routed * K * N
+    flops_step = 3 * flops_pass
+    value = world * flops_step * args.steps / (ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    fp8_peak_sustained = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    passes = {}
+    for name, key in (("fwd", "gemm_fwd"), ("dlhs", "gemm_dlhs"), ("drhs", "gemm_drhs")):
+        n, tot = prof.get(key, (0, 0.0))
+        if n:
+            avg = tot / n
+            passes[name] = {"gemm_ms": round(avg, 4), "gemm_tflops": round(flops_pass / (avg / 1e3) / 1e12, 1)}
+    total_prof = sum(t for _, t in prof.values())
+    kernels = {k: {"launches": n, "total_ms": round(t, 3), "share": round(t / total_prof, 4) if total_prof else None}
+               for k, (n, t) in sorted(prof.items())}
+    dom = max((k for k in prof if k.startswith("gemm_")), key=lambda k: prof[k][1])
+    dn, dt = prof[dom]
+    achieved = flops_pass / (dt / dn / 1e3) / 1e12
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": round(fp8_peak_sustained, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / fp8_peak_sustained, 4), "traffic": traffic_record(dom),
+                "peak_source": f"{peak_src} bf16 sustained cuBLAS x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)",
+                "algorithmic": f"2*sum(group_sizes)*K*N = {flops_pass:.4g} FLOP per launch"}
+
+    # end to end: pinned host buffers, copies inside the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        h_lhs, h_dout = lhs.cpu().pin_memory(), dout.cpu().pin_memory()
+        h_codes, h_rs, h_gs = codes.cpu().pin_memory(), rscales.cpu().pin_memory(), inp.group_sizes.pin_memory()
+        h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h_dl = torch.empty(dl.shape, dtype=dl.dtype, pin_memory=True)
+        h_dw = torch.empty(dw.shape, dtype=dw.dtype, pin_memory=True)
+        d_lhs, d_dout = torch.empty_like(lhs), torch.empty_like(dout)
+        d_codes, d_rs, d_gs = torch.empty_like(codes), torch.empty_like(rscales), torch.empty_like(gs)
+        h2d = sum(t.numel() * t.element_size() for t in (h_lhs, h_dout, h_codes, h_rs, h_gs))
+        d2h = sum(t.numel() * t.element_size() for t in (h_out, h_dl, h_dw))
+
+        def e2e_step():
+            d_lhs.copy_(h_lhs, non_blocking=True)
+            d_dout.copy_(h_dout, non_blocking=True)
+            d_codes.copy_(h_codes, non_blocking=True)
+            d_rs.copy_(h_rs, non_blocking=True)
+            d_gs.copy_(h_gs, non_blocking=True)
+            step(d_lhs, d_dout, d_codes, d_rs, d_gs)
+            h_out.copy_(out, non_blocking=True)
+            h_dl.copy_(dl, non_blocking=True)
+            h_dw.copy_(dw, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        f1.record()
+        barrier()
+        ems = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": round(world * flops_step * args.e2e_steps / (ems / 1e3) / 1e12, 2), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(ems / args.e2e_steps, 3),
+               "path": "pinned host -> device copies, gmm_fwd + gmm_dlhs + tgmm_drhs, device -> pinned host "
+                       "copies of out, dlhs and dW, all on one stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(w, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
+        "pct_fp8_peak": {"vs_nominal_4500": round(value / world / 4500.0 * 100, 2),
+                         "vs_measured_sustained": round(value / world / fp8_peak_sustained * 100, 2)},
+        "passes": passes, "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": timed_launches, "clocks": clk,
+    }
+    print(json.dumps(line))
+
+
+# ------------------------------------------------------ CPU (oracle) side
+
+_SAMPLE_CACHE = {}
+
+
+def _sample_group(w):
+    """One expert of the workload for the oracle sample: its row count and its
+    quantized weights (weight quantization is outside the timed passes)."""
+    if w.name not in _SAMPLE_CACHE:
+        import torch
+
+        import oracle
+        from moe_fp8_grouped_b200 import synth
+        gen = torch.Generator().manual_seed(0)
+        gs = synth.group_sizes(w, gen)
+        S = int(gs[[g for g in range(w.G) if int(gs[g]) > 0][0]])
+        W = (torch.randn((1, w.K, w.N), generator=gen) * 0.02).to(torch.bfloat16)
+        _SAMPLE_CACHE[w.name] = (S,) + tuple(oracle.quantize_rhs(W))
+    return _SAMPLE_CACHE[w.name]
+
+
+def cpu_baseline_sample(w, budget_s: float, seed: int = 0):
+    """Times the oracle on a bounded sample of the workload: batches of
+    forward rows, dlhs rows and drhs (g, k) rows until ~budget_s of wall time.
+    Returns TFLOP/s on the same FLOP count the GPU metric uses."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    S, qr, sr = _sample_group(w)
+    gen = torch.Generator().manual_seed(1000 + seed)
+    K, N = w.K, w.N
+    rule = oracle.Q_STATIC if w.rule == "static" else oracle.Q_DYNAMIC
+    s = 4.0 / 448.0
+    nt = oracle.num_threads()
+    S_drhs = min(S, 512)  # rows of the drhs sample group (bounded)
+    x_g = torch.randn((S_drhs, K), generator=gen).to(torch.bfloat16)
+    d_g = torch.randn((S_drhs, N), generator=gen).to(torch.bfloat16)
+    flops = 0.0
+    t_total = 0.0
+    batches = 0
+    while t_total < budget_s and batches < 1000:
+        rows = nt
+        lhs = torch.randn((rows, K), generator=gen).to(torch.bfloat16)
+        dout = torch.randn((rows, N), generator=gen).to(torch.bfloat16)
+        sizes = np.array([rows], np.int32)
+        t0 = time.perf_counter()
+        oracle.gmm_fwd(lhs, rule, s, qr, sr, sizes)
+        oracle.gmm_dlhs(dout, qr, sr, sizes)
+        oracle.tgmm_drhs(x_g, rule, s, d_g, np.array([S_drhs], np.int32), sel=list(range(nt)))
+        t_total += time.perf_counter() - t0
+        flops += 2.0 * rows * K * N * 2 + 2.0 * S_drhs * N * nt
+        batches += 1
+    return {"value": round(flops / t_total / 1e12, 6), "unit": UNIT, "cores": nt, "kind": "oracle",
+            "sample": f"{batches} batches of {nt} fwd rows + {nt} dlhs rows (K={K}, N={N}) + {nt} drhs (g,k) rows "
+                      f"over a {S_drhs}-row group; {t_total:.1f} s of oracle time; fp64 C loops, OpenMP over rows",
+            "seconds": round(t_total, 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return  # only rank 0 runs the CPU reference
+    from moe_fp8_grouped_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline_sample(w, per_step / 3)
+    vals, secs = [], 0.0
+    for i in range(args.steps):
+        r = cpu_baseline_sample(w, per_step / 3, seed=i)
+        vals.append(r["value"])
+        secs += r["seconds"]
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, {"parallelism": "CPU oracle on rank 0"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                         "sample": f"per step: {r['sample']}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -200,6 +200,24 @@ const char *gmm_status_string(gmm_status s);
 /* Number of kernels the last successful call on this host thread launched. */
 int32_t gmm_last_launch_count(void);
 
+/* Per-kernel timing for benchmarks.  While enabled, every kernel the library
+ * launches is bracketed by two CUDA events recorded on its stream (events
+ * come from a host-side pool; no device memory is allocated).  name is one of
+ * "plan", "quant_rows", "quant_chunks", "quant_rhs", "gemm_fwd", "gemm_dlhs",
+ * "gemm_drhs". */
+typedef struct {
+  const char *name;
+  int32_t launches;
+  double total_ms;
+} gmm_profile_entry;
+
+void gmm_profile_enable(int on);
+
+/* Synchronizes on the recorded events, aggregates them per kernel name into
+ * entries (at most max_entries), clears the record and returns the number of
+ * entries written. */
+int32_t gmm_profile_collect(gmm_profile_entry *entries, int32_t max_entries);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,12 +24,16 @@ DEV_GROUP_SIZES, DEV_SCALE, DEV_TIMEOUT = 1, 2, 4
 # every symbol include/gmm_fp8.h declares
 EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm_quantize", "gmm_fwd",
            "gmm_dlhs", "tgmm_drhs", "gmm_read_device_status", "gmm_selftest_timeout", "gmm_set_wait_limit_ns",
-           "gmm_status_string", "gmm_last_launch_count"]
+           "gmm_status_string", "gmm_last_launch_count", "gmm_profile_enable", "gmm_profile_collect"]
 
 
 class Operand(ctypes.Structure):
     _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int), ("scale", ctypes.c_void_p),
                 ("rule", ctypes.c_int)]
+
+
+class ProfileEntry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double)]
 
 
 _lib = None
@@ -69,5 +73,9 @@ def lib():
     L.gmm_status_string.restype = ctypes.c_char_p
     L.gmm_last_launch_count.argtypes = []
     L.gmm_last_launch_count.restype = i32
+    L.gmm_profile_enable.argtypes = [ctypes.c_int]
+    L.gmm_profile_enable.restype = None
+    L.gmm_profile_collect.argtypes = [ctypes.POINTER(ProfileEntry), i32]
+    L.gmm_profile_collect.restype = i32
     _lib = L
     return L

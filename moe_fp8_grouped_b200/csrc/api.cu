@@ -3,7 +3,10 @@
 // Nothing here allocates device memory; every buffer is the caller's.
 #include <climits>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "internal.h"
 
@@ -11,6 +14,41 @@ namespace gmm {
 
 static uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 static thread_local int32_t g_launches = 0;
+
+// ------------------------------------------------------------ profiling
+
+struct ProfRec {
+  const char *name;
+  cudaEvent_t a, b;
+};
+static std::mutex g_prof_mu;
+static bool g_prof_on = false;
+static std::vector<ProfRec> g_prof;
+static std::vector<cudaEvent_t> g_event_pool;
+
+static cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Runs one launch; when profiling is on, brackets it with events on `st`.
+template <class F>
+static cudaError_t prof(const char *name, cudaStream_t st, F &&launch) {
+  if (!g_prof_on) return launch();
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  ProfRec r{name, pool_event(), pool_event()};
+  cudaEventRecord(r.a, st);
+  cudaError_t e = launch();
+  cudaEventRecord(r.b, st);
+  g_prof.push_back(r);
+  return e;
+}
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -181,8 +219,10 @@ gmm_status gmm_quantize_rhs(const void *w_bf16, int32_t G, int64_t K, int64_t N,
   gmm_status s = check_sizes(1, K, N, G);
   if (s != GMM_OK) return s;
   if (!al16(w_bf16) || !al16(codes) || !al16(scales)) return GMM_ERR_ALIGNMENT;
-  s = cuda_status(launch_quant_rhs(w_bf16, G, K, N, transpose_out != 0, codes, scales,
-                                   static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = cuda_status(prof("quant_rhs", st, [&] {
+    return launch_quant_rhs(w_bf16, G, K, N, transpose_out != 0, codes, scales, st);
+  }));
   if (s == GMM_OK) g_launches = 3;
   return s;
 }
@@ -211,7 +251,7 @@ gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrul
   WsPtrs P = carve(ws, L);
   int n = 0;
   if (group_sizes) {
-    s = cuda_status(launch_plan(group_sizes, Gq, rows, P.offs, P.tpre, P.status, st));
+    s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, Gq, rows, P.offs, P.tpre, P.status, st); }));
     ++n;
   } else {
     s = cuda_status(cudaMemsetAsync(P.status, 0, sizeof(uint32_t), st));
@@ -219,11 +259,15 @@ gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrul
   if (s != GMM_OK) return s;
   const bool dyn = rule == GMM_Q_DYNAMIC;
   if (axis == 1)
-    s = cuda_status(launch_quant_rows(x_bf16, rows, cols, dyn, dyn ? nullptr : static_scale, col_scale, P.offs,
-                                      Gq, codes, scales, P.status, st));
+    s = cuda_status(prof("quant_rows", st, [&] {
+      return launch_quant_rows(x_bf16, rows, cols, dyn, dyn ? nullptr : static_scale, col_scale, P.offs, Gq, codes,
+                               scales, P.status, st);
+    }));
   else
-    s = cuda_status(launch_quant_chunks(x_bf16, rows, cols, dyn, dyn ? nullptr : static_scale, P.offs, P.tpre, Gq,
-                                        chunk_capacity(rows, Gq), codes, scales, false, P.status, st));
+    s = cuda_status(prof("quant_chunks", st, [&] {
+      return launch_quant_chunks(x_bf16, rows, cols, dyn, dyn ? nullptr : static_scale, P.offs, P.tpre, Gq,
+                                 chunk_capacity(rows, Gq), codes, scales, false, P.status, st);
+    }));
   if (s == GMM_OK) g_launches = n + 1;
   return s;
 }
@@ -244,13 +288,15 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   const WsLayout L = ws_layout(GMM_OP_FWD, M, K, N, G);
   if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
   WsPtrs P = carve(ws, L);
-  if ((s = cuda_status(launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st))) != GMM_OK) return s;
+  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
   int n = 1;
   const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
   const void *A = lhs.data;
   if (elem == 1) {
-    s = cuda_status(launch_quant_rows(lhs.data, M, K, dyn, dyn ? nullptr : lhs.scale, nullptr, P.offs, G, P.codes_a,
-                                      P.scales_a, P.status, st));
+    s = cuda_status(prof("quant_rows", st, [&] {
+      return launch_quant_rows(lhs.data, M, K, dyn, dyn ? nullptr : lhs.scale, nullptr, P.offs, G, P.codes_a,
+                               P.scales_a, P.status, st);
+    }));
     if (s != GMM_OK) return s;
     ++n;
     A = P.codes_a;
@@ -283,7 +329,8 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   const GemmConfig cfg{elem, bmn, elem == 1 && dyn};
   const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(launch_gemm(cfg, tmA, tmB, p, grid, st))) != GMM_OK) return s;
+  if ((s = cuda_status(prof("gemm_fwd", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
+    return s;
   g_launches = n + 1;
   return GMM_OK;
 }
@@ -305,13 +352,15 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   const WsLayout L = ws_layout(GMM_OP_DLHS, M, K, N, G);
   if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
   WsPtrs P = carve(ws, L);
-  if ((s = cuda_status(launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st))) != GMM_OK) return s;
+  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
   int n = 1;
   const void *A = dout.data;
   if (elem == 1) {
     // t = fl32(dout * s_r[g(m), n]), dynamic 128-blocks along n
-    s = cuda_status(launch_quant_rows(dout.data, M, N, true, nullptr, rhs.scale, P.offs, G, P.codes_a, P.scales_a,
-                                      P.status, st));
+    s = cuda_status(prof("quant_rows", st, [&] {
+      return launch_quant_rows(dout.data, M, N, true, nullptr, rhs.scale, P.offs, G, P.codes_a, P.scales_a,
+                               P.status, st);
+    }));
     if (s != GMM_OK) return s;
     ++n;
     A = P.codes_a;
@@ -344,7 +393,8 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   const GemmConfig cfg{elem, bmn, elem == 1};
   const int64_t items = ((M + 127) / 128 + G) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(launch_gemm(cfg, tmA, tmB, p, grid, st))) != GMM_OK) return s;
+  if ((s = cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
+    return s;
   g_launches = n + 1;
   return GMM_OK;
 }
@@ -364,14 +414,18 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   const WsLayout L = ws_layout(GMM_OP_DRHS, M, K, N, G);
   if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
   WsPtrs P = carve(ws, L);
-  if ((s = cuda_status(launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st))) != GMM_OK) return s;
+  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
   const int64_t cap = chunk_capacity(M, G);
   const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
-  s = cuda_status(launch_quant_chunks(lhs.data, M, K, dyn, (elem == 1 && !dyn) ? lhs.scale : nullptr, P.offs,
-                                      P.tpre, G, cap, P.codes_a, P.scales_a, elem == 2, P.status, st));
+  s = cuda_status(prof("quant_chunks", st, [&] {
+    return launch_quant_chunks(lhs.data, M, K, dyn, (elem == 1 && !dyn) ? lhs.scale : nullptr, P.offs, P.tpre, G,
+                               cap, P.codes_a, P.scales_a, elem == 2, P.status, st);
+  }));
   if (s != GMM_OK) return s;
-  s = cuda_status(launch_quant_chunks(dout.data, M, N, true, nullptr, P.offs, P.tpre, G, cap, P.codes_b, P.scales_b,
-                                      elem == 2, P.status, st));
+  s = cuda_status(prof("quant_chunks", st, [&] {
+    return launch_quant_chunks(dout.data, M, N, true, nullptr, P.offs, P.tpre, G, cap, P.codes_b, P.scales_b,
+                               elem == 2, P.status, st);
+  }));
   if (s != GMM_OK) return s;
   const uint32_t bke = 128 / elem;
   const uint64_t ldt = static_cast<uint64_t>(cap) * kBlk;  // elements per transposed row
@@ -399,7 +453,8 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   const GemmConfig cfg{elem, false, elem == 1};
   const int64_t items = static_cast<int64_t>(G) * (K / kBlk) * ((N + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(launch_gemm(cfg, tmA, tmB, p, grid, st))) != GMM_OK) return s;
+  if ((s = cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
+    return s;
   g_launches = 4;
   return GMM_OK;
 }
@@ -427,6 +482,38 @@ gmm_status gmm_selftest_timeout(void *ws, uint64_t limit_ns, void *stream) {
   s = cuda_status(launch_timeout_selftest(status, limit_ns, st));
   if (s == GMM_OK) g_launches = 1;
   return s;
+}
+
+void gmm_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+}
+
+int32_t gmm_profile_collect(gmm_profile_entry *entries, int32_t max_entries) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  // names point at string literals of this library, so they stay valid
+  std::map<std::string, std::pair<const char *, std::pair<int32_t, double>>> agg;
+  for (ProfRec &r : g_prof) {
+    float ms = 0.0f;
+    cudaEventSynchronize(r.b);
+    cudaEventElapsedTime(&ms, r.a, r.b);
+    auto &x = agg[r.name];
+    x.first = r.name;
+    x.second.first += 1;
+    x.second.second += ms;
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  int32_t n = 0;
+  for (auto &kv : agg) {
+    if (n >= max_entries) break;
+    entries[n].name = kv.second.first;
+    entries[n].launches = kv.second.second.first;
+    entries[n].total_ms = kv.second.second.second;
+    ++n;
+  }
+  return n;
 }
 
 }  // extern "C"

@@ -232,3 +232,15 @@ def gmm_plan(group_sizes: torch.Tensor, M: int):
     offs = torch.zeros(gs.numel() + 1, dtype=torch.int64)
     offs[1:] = torch.cumsum(gs, 0).clamp(max=M)
     return offs
+
+
+def profile_enable(on: bool = True):
+    """Bracket every library kernel launch with CUDA events (benchmarks)."""
+    B.lib().gmm_profile_enable(int(on))
+
+
+def profile_collect() -> dict:
+    """{kernel name: (launches, total ms)} since the last collect."""
+    arr = (B.ProfileEntry * 32)()
+    n = B.lib().gmm_profile_collect(arr, 32)
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}

@@ -64,6 +64,13 @@ WORKLOADS = {
 }
 
 
+def with_rows(w: Workload, M: int) -> Workload:
+    """The same workload with M rows (tokens scaled alike), e.g. a smaller
+    case of the same shape for profiler captures."""
+    tokens = M // w.topk if w.topk else 0
+    return dataclasses.replace(w, name=f"{w.name}_m{M}", M=M, tokens=tokens)
+
+
 def group_sizes(w: Workload, gen: torch.Generator) -> torch.Tensor:
     """int32 [G] row counts per expert, summing to M (CPU)."""
     G, M = w.G, w.M
