@@ -11,14 +11,15 @@
 //   tgmm drhs     rows = K, contraction = the rows of one group, columns N
 //                 ("drhs_tgmm2", PR #4451, Description)
 //
-// CTA layout (320 threads, one CTA per SM):
+// CTA layout (384 threads, one CTA per SM):
 //   warp 0     TMA producer: A tile 128 x 128 B, B tile 256 x 128 B per stage,
 //              4 stages in shared memory (128-byte swizzle)
 //   warp 1     TMEM allocator + MMA issuer: tcgen05.mma M=128 N=256, four
 //              32-byte K steps per stage, fp32 accumulators in TMEM, two
 //              256-column accumulator buffers
-//   warps 2-9  epilogue: tcgen05.ld, scale, store.  Warp w reads TMEM lanes
-//              32 (w % 4) .. +31 (rows) and column half (w - 2) / 4.
+//   warps 2-3  idle (they give their registers to the epilogue)
+//   warps 4-11 epilogue: tcgen05.ld, scale, store.  Warp w reads TMEM lanes
+//              32 (w % 4) .. +31 (rows) and column half (w - 4) / 4.
 //
 // Scaling ("add static LHS scaling support for GMM v2 FWD", maxtext PR
 // #4735, review thread on the LhsRef docstring: the result is multiplied back
@@ -38,14 +39,27 @@ constexpr int kBM = 128, kBN = 256;
 constexpr int kStages = 4;
 constexpr int kAStage = kBM * 128;  // bytes
 constexpr int kBStage = kBN * 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;     // 3 warpgroups: control, 2 x epilogue
+constexpr int kEpiWarp0 = 4;      // first epilogue warp
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 256;
 constexpr int kTmemCols = 512;
+// Register split (setmaxnreg): the control warpgroup gives registers to the
+// two epilogue warpgroups.  Sum must not exceed the launch allocation
+// (registers per thread at launch x 384); launch_inst checks it.
+// The promote variants keep 128 accumulators per thread and get the larger
+// epilogue share.
+template <bool kPromote>
+constexpr int regs_ctl() { return kPromote ? 40 : 72; }
+template <bool kPromote>
+constexpr int regs_epi() { return kPromote ? 232 : 216; }
 
 constexpr size_t gemm_smem_bytes() {
   return 1024                                    // alignment slack
          + static_cast<size_t>(kStages) * (kAStage + kBStage)
          + 16 * 8                                // mbarriers
-         + 16                                    // tmem slot, abort flag
+         + 16                                    // tmem slot, abort flags
+         + 3 * kBN * sizeof(float)               // column scale buffers
          + 2 * (kMaxGroups + 1) * sizeof(int);   // plan copy
 }
 
@@ -131,7 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *drain = tempty + 2;          // MMA completion at exit
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *s_offs = reinterpret_cast<int *>(tmem_slot + 4);
+  volatile int *no_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
+  float *s_cblk = reinterpret_cast<float *>(tmem_slot + 4);  // [2][256] per-block column scales (tgmm)
+  float *s_ctile = s_cblk + 2 * kBN;                          // [256] per-tile column scales
+  int *s_offs = reinterpret_cast<int *>(s_ctile + kBN);
   int *s_tpre = s_offs + (kMaxGroups + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,11 +160,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);
+      mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *reinterpret_cast<volatile int *>(tmem_slot + 2) = 0;  // never raised: exit drains ignore aborts
+    *no_abort = 0;  // never raised: the exit drains ignore aborts
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -170,11 +187,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tn = (p.ncols + kBN - 1) / kBN;
   const int total = (p.mode == MODE_ROWS) ? s_tpre[p.G] * tn : p.G * p.ktiles * tn;
   const WaitCtl ctl{p.wait_limit_ns, abort_flag, p.status};
-  const WaitCtl ctl_drain{p.wait_limit_ns, reinterpret_cast<volatile int *>(tmem_slot + 2), p.status};
+  const WaitCtl ctl_drain{p.wait_limit_ns, no_abort, p.status};
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp < 4) {
+    setmaxnreg_dec<regs_ctl<kPromote>()>();
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------- TMA producer
       int it = 0;
       bool ok = true;
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
@@ -212,58 +230,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       // let every issued copy land before the CTA can exit
       for (int i = (it > kStages ? it - kStages : 0); i < it; ++i)
         mbar_wait(&full[i % kStages], (i / kStages) & 1, ctl_drain);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      int it = 0, u = 0;
-      bool ok = true;
-      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-        const Item t = decode_item(w, p, s_offs, s_tpre, tn);
-        uint32_t buf = 0;
-        for (int b = 0; b < t.nblocks; ++b, ++it) {
-          const bool unit_start = kPromote || b == 0;
-          if (unit_start) {
-            buf = u & 1;
-            if (!mbar_wait(&tempty[buf], ((u >> 1) & 1) ^ 1, ctl)) {
+    } else if (warp == 1) {
+      // ----------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        int it = 0, u = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+          const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+          uint32_t buf = 0;
+          for (int b = 0; b < t.nblocks; ++b, ++it) {
+            const bool unit_start = kPromote || b == 0;
+            if (unit_start) {
+              buf = u & 1;
+              if (!mbar_wait(&tempty[buf], ((u >> 1) & 1) ^ 1, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            const int s = it % kStages;
+            if (!mbar_wait(&full[s], (it / kStages) & 1, ctl)) {
               ok = false;
               break;
             }
             tc_fence_after();
-          }
-          const int s = it % kStages;
-          if (!mbar_wait(&full[s], (it / kStages) & 1, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBStage);
-          const uint32_t d = tbase + buf * kBN;
+            const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBStage);
+            const uint32_t d = tbase + buf * kBN;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
-            const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
-                                        : smem_desc_sw128(b0 + kk * 32, 16, 1024);
-            tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
-          }
-          tc_commit(&empty[s]);
-          if (kPromote || b == t.nblocks - 1) {
-            tc_commit(&tfull[buf]);
-            ++u;
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+              const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
+                                          : smem_desc_sw128(b0 + kk * 32, 16, 1024);
+              tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
+            }
+            tc_commit(&empty[s]);
+            if (kPromote || b == t.nblocks - 1) {
+              tc_commit(&tfull[buf]);
+              ++u;
+            }
           }
         }
+        tc_commit(drain);
+        mbar_wait(drain, 0, ctl_drain);
       }
-      tc_commit(drain);
-      mbar_wait(drain, 0, ctl_drain);
+      __syncwarp();
     }
-    __syncwarp();
   } else {
-    // --------------------------------------------------------- epilogue
-    const int q = warp & 3, h = (warp - 2) >> 2;
+    setmaxnreg_inc<regs_epi<kPromote>()>();
+    // ---------------------------------------------------------- epilogue
+    const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
+    const int q = warp & 3, h = (warp - kEpiWarp0) >> 2;
     const int row = q * 32 + lane;
     const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
-    const float sstat = p.static_scale ? *p.static_scale : 1.0f;
-    const bool sstat_ok = isfinite(sstat) && sstat > 1.17549435e-38f;
+    float s_eff = 1.0f;
+    if (p.static_scale) {
+      const float v = *p.static_scale;
+      s_eff = (isfinite(v) && v > 1.17549435e-38f) ? v : 0.0f;
+    }
     int u = 0;
     bool ok = true;
     for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
@@ -287,47 +310,80 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (col0 + c * 32 < p.ncols) store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, z, p.out_f32);
         continue;
       }
+      // per-tile column scales (rhs s_r[g, n] of the forward pass)
+      if (p.col_scale) {
+        epi_bar();
+        const int n = t.nt * kBN + et;
+        s_ctile[et] = n < p.ncols ? __ldg(p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n) : 0.0f;
+        epi_bar();
+      }
       if constexpr (kPromote) {
-        float acc[128];
+        float2 acc[64];
 #pragma unroll
-        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-        for (int b = 0; b < t.nblocks; ++b) {
-          float rs;
-          const float *cs_base = nullptr;
-          if (p.mode == MODE_ROWS) {
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        const bool tg = p.mode == MODE_TGMM;
+        const int64_t ch0 = tg ? s_tpre[t.g] : 0;
+        // row scale of this thread's row for block b
+        auto row_scale_at = [&](int b) -> float {
+          if (!tg) {
             const int64_t rr = min(static_cast<int64_t>(t.r0 + row), static_cast<int64_t>(p.M - 1));
-            rs = __ldg(p.row_scale + static_cast<int64_t>(b) * p.row_scale_ld + rr);
-          } else {
-            const int64_t ch = s_tpre[t.g] + b;
-            rs = __ldg(p.row_scale + ch * p.row_scale_ld + t.kt * kBM + row);
-            cs_base = p.colblk_scale + ch * p.colblk_ld + col0;
+            return __ldg(p.row_scale + static_cast<int64_t>(b) * p.row_scale_ld + rr);
           }
+          return __ldg(p.row_scale + (ch0 + b) * p.row_scale_ld + t.kt * kBM + row);
+        };
+        auto col_block_scale = [&](int b) -> float {
+          const int n = t.nt * kBN + et;
+          return n < p.ncols ? __ldg(p.colblk_scale + (ch0 + b) * p.colblk_ld + n) : 0.0f;
+        };
+        const bool rconst = tg && p.static_scale != nullptr;  // static x: one scale for every chunk
+        if (tg) {
+          epi_bar();  // the previous tile's readers are done with slot 0
+          s_cblk[et] = col_block_scale(0);
+        }
+        float rs_next = rconst ? 1.0f : row_scale_at(0);
+        for (int b = 0; b < t.nblocks; ++b) {
+          const float rs = rs_next;
+          if (!rconst && b + 1 < t.nblocks) rs_next = row_scale_at(b + 1);
           const uint32_t buf = u & 1;
-          if (!mbar_wait(&tfull[buf], (u >> 1) & 1, ctl)) {
+          const bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
+          if (!epi_bar_and(got)) {
             ok = false;
             break;
           }
+          if (tg && b + 1 < t.nblocks) s_cblk[((b + 1) & 1) * kBN + et] = col_block_scale(b + 1);
           tc_fence_after();
+          const float *cb = s_cblk + (b & 1) * kBN + h * 128;
+          const float2 rs2 = make_float2(rs, rs);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tl + buf * kBN + c * 32, v);
+          for (int cp = 0; cp < 2; ++cp) {
+            uint32_t va[32], vb[32];
+            tmem_ld32(tl + buf * kBN + (2 * cp) * 32, va);
+            tmem_ld32(tl + buf * kBN + (2 * cp + 1) * 32, vb);
             tmem_wait_ld();
-            if (p.mode == MODE_ROWS) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(__uint_as_float(v[i]), rs, acc[c * 32 + i]);
-            } else {
-              // columns past ncols (a half tile when N % 256 == 128) are never
-              // stored; their scales are not read
-              const bool cols_ok = col0 + c * 32 < p.ncols;
-              const float4 *cs4 = reinterpret_cast<const float4 *>(cs_base + c * 32);
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t *v = half ? vb : va;
+              const int c = 2 * cp + half;
+              if (!tg) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float4 cs = cols_ok ? __ldg(cs4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-                acc[c * 32 + 4 * i + 0] = fmaf(__uint_as_float(v[4 * i + 0]), rs * cs.x, acc[c * 32 + 4 * i + 0]);
-                acc[c * 32 + 4 * i + 1] = fmaf(__uint_as_float(v[4 * i + 1]), rs * cs.y, acc[c * 32 + 4 * i + 1]);
-                acc[c * 32 + 4 * i + 2] = fmaf(__uint_as_float(v[4 * i + 2]), rs * cs.z, acc[c * 32 + 4 * i + 2]);
-                acc[c * 32 + 4 * i + 3] = fmaf(__uint_as_float(v[4 * i + 3]), rs * cs.w, acc[c * 32 + 4 * i + 3]);
+                for (int i = 0; i < 16; ++i)
+                  acc[c * 16 + i] = __ffma2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
+                                               rs2, acc[c * 16 + i]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 cs = *reinterpret_cast<const float4 *>(cb + c * 32 + 4 * i);
+                  float2 c01 = make_float2(cs.x, cs.y), c23 = make_float2(cs.z, cs.w);
+                  if (!rconst) {
+                    c01 = __fmul2_rn(c01, rs2);
+                    c23 = __fmul2_rn(c23, rs2);
+                  }
+                  acc[c * 16 + 2 * i] = __ffma2_rn(
+                      make_float2(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1])), c01, acc[c * 16 + 2 * i]);
+                  acc[c * 16 + 2 * i + 1] =
+                      __ffma2_rn(make_float2(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])), c23,
+                                 acc[c * 16 + 2 * i + 1]);
+                }
               }
             }
           }
@@ -338,59 +394,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (row_ok) {
+          const float fin = rconst ? s_eff : 1.0f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             if (col0 + c * 32 >= p.ncols) continue;
             float o[32];
-            if (p.col_scale) {
-              const float4 *cs4 = reinterpret_cast<const float4 *>(p.col_scale +
-                                                                   static_cast<int64_t>(t.g) * p.ncols + col0 + c * 32);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float4 cs = __ldg(cs4 + i);
-                o[4 * i + 0] = acc[c * 32 + 4 * i + 0] * cs.x;
-                o[4 * i + 1] = acc[c * 32 + 4 * i + 1] * cs.y;
-                o[4 * i + 2] = acc[c * 32 + 4 * i + 2] * cs.z;
-                o[4 * i + 3] = acc[c * 32 + 4 * i + 3] * cs.w;
+            for (int i = 0; i < 16; ++i) {
+              float2 a = acc[c * 16 + i];
+              if (p.col_scale) {
+                a.x *= s_ctile[h * 128 + c * 32 + 2 * i];
+                a.y *= s_ctile[h * 128 + c * 32 + 2 * i + 1];
               }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = acc[c * 32 + i];
+              o[2 * i] = a.x * fin;
+              o[2 * i + 1] = a.y * fin;
             }
             store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32);
           }
         }
       } else {
         const uint32_t buf = u & 1;
-        if (!mbar_wait(&tfull[buf], (u >> 1) & 1, ctl)) {
+        const bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
+        if (!epi_bar_and(got)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float s0 = p.static_scale ? (sstat_ok ? sstat : 0.0f) : 1.0f;
+        const float s0 = p.static_scale ? s_eff : 1.0f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tl + buf * kBN + c * 32, v);
+        for (int cp = 0; cp < 2; ++cp) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tl + buf * kBN + (2 * cp) * 32, va);
+          tmem_ld32(tl + buf * kBN + (2 * cp + 1) * 32, vb);
           tmem_wait_ld();
-          if (!row_ok || col0 + c * 32 >= p.ncols) continue;
-          float o[32];
-          if (p.col_scale) {
-            const float4 *cs4 =
-                reinterpret_cast<const float4 *>(p.col_scale + static_cast<int64_t>(t.g) * p.ncols + col0 + c * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 cs = __ldg(cs4 + i);
-              o[4 * i + 0] = __uint_as_float(v[4 * i + 0]) * s0 * cs.x;
-              o[4 * i + 1] = __uint_as_float(v[4 * i + 1]) * s0 * cs.y;
-              o[4 * i + 2] = __uint_as_float(v[4 * i + 2]) * s0 * cs.z;
-              o[4 * i + 3] = __uint_as_float(v[4 * i + 3]) * s0 * cs.w;
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t *v = half ? vb : va;
+            const int c = 2 * cp + half;
+            if (!row_ok || col0 + c * 32 >= p.ncols) continue;
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float cs = p.col_scale ? s_ctile[h * 128 + c * 32 + i] : 1.0f;
+              o[i] = __uint_as_float(v[i]) * s0 * cs;
             }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(v[i]) * s0;
+            store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32);
           }
-          store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32);
         }
         tc_fence_before();
         __syncwarp();
@@ -404,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t tail0 = s_offs[p.G];
       const int64_t cpr = static_cast<int64_t>(p.ncols) * esz / 16;  // 16-byte chunks per row
       const int64_t n = (static_cast<int64_t>(p.M) - tail0) * cpr;
-      const int et = threadIdx.x - 64;
-      for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + et; i < n; i += static_cast<int64_t>(gridDim.x) * 256) {
+      for (int64_t i = static_cast<int64_t>(blockIdx.x) * kEpiThreads + et; i < n;
+           i += static_cast<int64_t>(gridDim.x) * kEpiThreads) {
         const int64_t r = tail0 + i / cpr, c = i % cpr;
         *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) + (r * p.ld_out) * esz + c * 16) =
             make_uint4(0, 0, 0, 0);
@@ -438,7 +487,14 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
                                cudaStream_t st) {
   auto kern = gmm_tc_kernel<kElem, kBMN, kPromote>;
   const size_t smem = gemm_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  // setmaxnreg.inc waits for registers the CTA owns: never launch a split that
+  // does not fit the launch allocation
+  if (attr.numRegs * kThreads < regs_ctl<kPromote>() * 128 + regs_epi<kPromote>() * 256)
+    return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, st>>>(tmA, tmB, p);
   return cudaGetLastError();
