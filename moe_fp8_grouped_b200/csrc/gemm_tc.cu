@@ -101,23 +101,46 @@ __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const in
   return t;
 }
 
-template <int kElem>
-__device__ __forceinline__ void store32(void *out, int64_t off_elems, const float (&v)[32], int out_f32) {
+__device__ __forceinline__ void st_v8(void *dst, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                      uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(a0), "r"(a1), "r"(a2),
+               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&b);
+}
+
+// Stores 32 consecutive outputs of one row.  v8: the destination is 32-byte
+// aligned, so each instruction writes one full 32-byte sector.
+__device__ __forceinline__ void store32(void *out, int64_t off_elems, const float (&v)[32], int out_f32, bool v8) {
   if (out_f32) {
-    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + off_elems);
+    float *dst = static_cast<float *>(out) + off_elems;
+    if (v8) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int i = 0; i < 4; ++i)
+        st_v8(dst + 8 * i, __float_as_uint(v[8 * i]), __float_as_uint(v[8 * i + 1]), __float_as_uint(v[8 * i + 2]),
+              __float_as_uint(v[8 * i + 3]), __float_as_uint(v[8 * i + 4]), __float_as_uint(v[8 * i + 5]),
+              __float_as_uint(v[8 * i + 6]), __float_as_uint(v[8 * i + 7]));
+    } else {
+      float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
   } else {
-    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + off_elems);
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(out) + off_elems;
+    uint32_t w[16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t w[4];
+    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+    if (v8) {
+      st_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+      st_v8(dst + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+    } else {
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * i + 2 * e], v[8 * i + 2 * e + 1]);
-        w[e] = *reinterpret_cast<uint32_t *>(&b);
-      }
-      dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
     }
   }
 }
@@ -287,6 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float v = *p.static_scale;
       s_eff = (isfinite(v) && v > 1.17549435e-38f) ? v : 0.0f;
     }
+    const bool out_v8 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
     int u = 0;
     bool ok = true;
     for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
@@ -307,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) z[i] = 0.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          if (col0 + c * 32 < p.ncols) store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, z, p.out_f32);
+          if (col0 + c * 32 < p.ncols) store32(p.out, orow * p.ld_out + col0 + c * 32, z, p.out_f32, out_v8);
         continue;
       }
       // per-tile column scales (rhs s_r[g, n] of the forward pass)
@@ -409,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[2 * i] = a.x * fin;
               o[2 * i + 1] = a.y * fin;
             }
-            store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32);
+            store32(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32, out_v8);
           }
         }
       } else {
@@ -438,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float cs = p.col_scale ? s_ctile[h * 128 + c * 32 + i] : 1.0f;
               o[i] = __uint_as_float(v[i]) * s0 * cs;
             }
-            store32<kElem>(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32);
+            store32(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32, out_v8);
           }
         }
         tc_fence_before();

@@ -275,3 +275,30 @@ def test_host_errors_return_before_launch(dev):
     with pytest.raises(gm.GmmError) as e:
         gm.gmm_fwd(lhs[:, :500].contiguous(), c[:, :500].contiguous(), sc, gs, rule="static", static_scale=s)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_output_16_byte_aligned_only(dev, out_dtype):
+    """Outputs that are 16- but not 32-byte aligned take the 16-byte store path."""
+    inp = case_inputs("ragged")
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    G, K, N = w.shape
+    M = lhs.shape[0]
+    c, sc = gm.gmm_quantize_rhs(w)
+    esz = torch.tensor([], dtype=out_dtype).element_size()
+    for shape, fn, ref_fn in (
+        ((M, N), lambda o: gm.gmm_fwd(lhs, c, sc, gs, rule="static", static_scale=s, out=o),
+         lambda: oracle.gmm_fwd(inp.lhs, oracle.Q_STATIC, inp.static_scale, *oracle.quantize_rhs(inp.w),
+                                inp.group_sizes)),
+        ((G, K, N), lambda o: gm.tgmm_drhs(lhs, dout, gs, rule="dynamic", out=o),
+         lambda: oracle.tgmm_drhs(inp.lhs, oracle.Q_DYNAMIC, 0.0, inp.dout, inp.group_sizes)),
+    ):
+        n = int(np.prod(shape))
+        raw = torch.zeros(n * esz + 64, dtype=torch.uint8, device=dev)
+        base = raw.data_ptr()
+        off = (16 - base % 32) % 32 or 16  # 16 mod 32
+        out = raw[off: off + n * esz].view(out_dtype).view(*shape)
+        assert out.data_ptr() % 32 == 16
+        fn(out)
+        ref, ab = ref_fn()
+        assert_close(out, ref, ab, f"16B-aligned {shape}")
