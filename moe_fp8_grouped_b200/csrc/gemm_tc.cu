@@ -17,7 +17,9 @@
 //   warp 1     TMEM allocator + MMA issuer: tcgen05.mma M=128 N=256, four
 //              32-byte K steps per stage, fp32 accumulators in TMEM, two
 //              256-column accumulator buffers
-//   warps 2-3  idle (they give their registers to the epilogue)
+//   warp 2     scale loader: row / column scales of each TMEM unit into a
+//              shared-memory ring ahead of the epilogue
+//   warp 3     idle (gives its registers to the epilogue)
 //   warps 4-11 epilogue: tcgen05.ld, scale, store.  Warp w reads TMEM lanes
 //              32 (w % 4) .. +31 (rows) and column half (w - 4) / 4.
 //
@@ -44,6 +46,8 @@ constexpr int kEpiWarp0 = 4;      // first epilogue warp
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 256;
 constexpr int kTmemCols = 512;
+constexpr int kScaleSlots = 4;    // ring of per-unit scale slots (scale loader -> epilogue)
+constexpr int kNumBars = 24;      // mbarriers reserved in shared memory
 // Register split (setmaxnreg): the control warpgroup gives registers to the
 // two epilogue warpgroups.  Sum must not exceed the launch allocation
 // (registers per thread at launch x 384); launch_inst checks it.
@@ -57,9 +61,9 @@ constexpr int regs_epi() { return kPromote ? 232 : 216; }
 constexpr size_t gemm_smem_bytes() {
   return 1024                                    // alignment slack
          + static_cast<size_t>(kStages) * (kAStage + kBStage)
-         + 16 * 8                                // mbarriers
+         + kNumBars * 8                          // mbarriers
          + 16                                    // tmem slot, abort flags
-         + 3 * kBN * sizeof(float)               // column scale buffers
+         + kScaleSlots * (kBN + kBM) * sizeof(float)  // scale ring
          + 2 * (kMaxGroups + 1) * sizeof(int);   // plan copy
 }
 
@@ -161,20 +165,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sA = smem;
   uint8_t *sB = smem + kStages * kAStage;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * kBStage);
-  uint64_t *full = bars;                 // [kStages] TMA -> MMA
-  uint64_t *empty = bars + kStages;      // [kStages] MMA -> TMA
-  uint64_t *tfull = bars + 2 * kStages;  // [2] MMA -> epilogue
-  uint64_t *tempty = tfull + 2;          // [2] epilogue -> MMA
-  uint64_t *drain = tempty + 2;          // MMA completion at exit
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+  uint64_t *full = bars;                    // [kStages] TMA -> MMA
+  uint64_t *empty = bars + kStages;         // [kStages] MMA -> TMA
+  uint64_t *tfull = bars + 2 * kStages;     // [2] MMA -> epilogue
+  uint64_t *tempty = tfull + 2;             // [2] epilogue -> MMA
+  uint64_t *drain = tempty + 2;             // MMA completion at exit
+  uint64_t *sfull = drain + 1;              // [kScaleSlots] scale loader -> epilogue
+  uint64_t *sempty = sfull + kScaleSlots;   // [kScaleSlots] epilogue -> scale loader
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *no_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
-  float *s_cblk = reinterpret_cast<float *>(tmem_slot + 4);  // [2][256] per-block column scales (tgmm)
-  float *s_ctile = s_cblk + 2 * kBN;                          // [256] per-tile column scales
-  int *s_offs = reinterpret_cast<int *>(s_ctile + kBN);
+  float *s_scol = reinterpret_cast<float *>(tmem_slot + 4);  // [kScaleSlots][256] column scales per unit
+  float *s_srow = s_scol + kScaleSlots * kBN;                // [kScaleSlots][128] row scales per unit
+  int *s_offs = reinterpret_cast<int *>(s_srow + kScaleSlots * kBM);
   int *s_tpre = s_offs + (kMaxGroups + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Which scales each TMEM unit carries (the same decision in every role):
+  //   column scales: forward s_r[g, n] (every unit of a tile) or tgmm s_d[chunk, n]
+  //   row scales:    promoted row-ragged passes (s_l / s_t per 128-block),
+  //                  dynamic tgmm (s_x[chunk, k])
+  const bool tg = p.mode == MODE_TGMM;
+  const bool need_col = tg ? (p.colblk_scale != nullptr) : (p.col_scale != nullptr);
+  const bool need_row = kPromote && (tg ? p.static_scale == nullptr : true);
+  const bool use_ring = need_col || need_row;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -186,6 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kScaleSlots; ++i) {
+      mbar_init(&sfull[i], 32);
+      mbar_init(&sempty[i], kEpiWarps);
+    }
     *abort_flag = 0;
     *no_abort = 0;  // never raised: the exit drains ignore aborts
     fence_barrier_init();
@@ -297,6 +316,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(drain, 0, ctl_drain);
       }
       __syncwarp();
+    } else if (warp == 2 && use_ring) {
+      // --------------------------------------------------- scale loader
+      // Fills one ring slot per TMEM unit, in the order the epilogue consumes
+      // them, so that no global-memory latency sits on the epilogue's path.
+      int v = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+        const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+        const int units = kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0);
+        const int64_t ch0 = tg ? s_tpre[t.g] : 0;
+        for (int j = 0; j < units; ++j, ++v) {
+          const int slot = v % kScaleSlots;
+          bool got = true;
+          if (lane == 0) got = mbar_wait(&sempty[slot], ((v / kScaleSlots) & 1) ^ 1, ctl);
+          if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
+            ok = false;
+            break;
+          }
+          if (need_col) {
+            const int n = t.nt * kBN + 8 * lane;  // 8 columns per lane
+            float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+            if (n < p.ncols) {
+              const float *src = tg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
+                                    : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n;
+              c0 = __ldg(reinterpret_cast<const float4 *>(src));
+              c1 = __ldg(reinterpret_cast<const float4 *>(src) + 1);
+            }
+            float4 *dst = reinterpret_cast<float4 *>(s_scol + slot * kBN + 8 * lane);
+            dst[0] = c0;
+            dst[1] = c1;
+          }
+          if (need_row) {
+            float4 r;
+            if (tg) {
+              r = __ldg(reinterpret_cast<const float4 *>(p.row_scale + (ch0 + j) * p.row_scale_ld + t.kt * kBM +
+                                                         4 * lane));
+            } else {
+              const float *src = p.row_scale + static_cast<int64_t>(j) * p.row_scale_ld;
+              const int64_t last = p.M - 1;
+              const int64_t r0 = t.r0 + 4 * lane;
+              r.x = __ldg(src + min(r0, last));
+              r.y = __ldg(src + min(r0 + 1, last));
+              r.z = __ldg(src + min(r0 + 2, last));
+              r.w = __ldg(src + min(r0 + 3, last));
+            }
+            *reinterpret_cast<float4 *>(s_srow + slot * kBM + 4 * lane) = r;
+          }
+          mbar_arrive(&sfull[slot]);
+        }
+      }
     }
   } else {
     setmaxnreg_inc<regs_epi<kPromote>()>();
@@ -311,8 +380,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_eff = (isfinite(v) && v > 1.17549435e-38f) ? v : 0.0f;
     }
     const bool out_v8 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
-    int u = 0;
+    int u = 0;  // TMEM units consumed
+    int v = 0;  // scale slots consumed
     bool ok = true;
+    // waits for TMEM unit u (and its scale slot), then agrees with the other
+    // epilogue warps on whether to go on
+    auto wait_unit = [&](uint32_t buf, int slot) -> bool {
+      bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
+      if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kScaleSlots) & 1, ctl);
+      return epi_bar_and(got);
+    };
+    auto release_slot = [&](int slot) {
+      if (use_ring) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[slot]);
+        ++v;
+      }
+    };
     for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
       const Item t = decode_item(w, p, s_offs, s_tpre, tn);
       const int col0 = t.nt * kBN + h * 128;
@@ -334,50 +418,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (col0 + c * 32 < p.ncols) store32(p.out, orow * p.ld_out + col0 + c * 32, z, p.out_f32, out_v8);
         continue;
       }
-      // per-tile column scales (rhs s_r[g, n] of the forward pass)
-      if (p.col_scale) {
-        epi_bar();
-        const int n = t.nt * kBN + et;
-        s_ctile[et] = n < p.ncols ? __ldg(p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n) : 0.0f;
-        epi_bar();
-      }
       if constexpr (kPromote) {
         float2 acc[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-        const bool tg = p.mode == MODE_TGMM;
-        const int64_t ch0 = tg ? s_tpre[t.g] : 0;
-        // row scale of this thread's row for block b
-        auto row_scale_at = [&](int b) -> float {
-          if (!tg) {
-            const int64_t rr = min(static_cast<int64_t>(t.r0 + row), static_cast<int64_t>(p.M - 1));
-            return __ldg(p.row_scale + static_cast<int64_t>(b) * p.row_scale_ld + rr);
-          }
-          return __ldg(p.row_scale + (ch0 + b) * p.row_scale_ld + t.kt * kBM + row);
-        };
-        auto col_block_scale = [&](int b) -> float {
-          const int n = t.nt * kBN + et;
-          return n < p.ncols ? __ldg(p.colblk_scale + (ch0 + b) * p.colblk_ld + n) : 0.0f;
-        };
-        const bool rconst = tg && p.static_scale != nullptr;  // static x: one scale for every chunk
-        if (tg) {
-          epi_bar();  // the previous tile's readers are done with slot 0
-          s_cblk[et] = col_block_scale(0);
-        }
-        float rs_next = rconst ? 1.0f : row_scale_at(0);
+        int slot = 0;
         for (int b = 0; b < t.nblocks; ++b) {
-          const float rs = rs_next;
-          if (!rconst && b + 1 < t.nblocks) rs_next = row_scale_at(b + 1);
           const uint32_t buf = u & 1;
-          const bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
-          if (!epi_bar_and(got)) {
+          slot = v % kScaleSlots;
+          if (!wait_unit(buf, slot)) {
             ok = false;
             break;
           }
-          if (tg && b + 1 < t.nblocks) s_cblk[((b + 1) & 1) * kBN + et] = col_block_scale(b + 1);
           tc_fence_after();
-          const float *cb = s_cblk + (b & 1) * kBN + h * 128;
+          const float rs = need_row ? s_srow[slot * kBM + row] : 1.0f;
           const float2 rs2 = make_float2(rs, rs);
+          const float *cb = s_scol + slot * kBN + h * 128;
 #pragma unroll
           for (int cp = 0; cp < 2; ++cp) {
             uint32_t va[32], vb[32];
@@ -386,27 +442,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-              const uint32_t *v = half ? vb : va;
+              const uint32_t *vv = half ? vb : va;
               const int c = 2 * cp + half;
               if (!tg) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                  acc[c * 16 + i] = __ffma2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
-                                               rs2, acc[c * 16 + i]);
+                  acc[c * 16 + i] = __ffma2_rn(
+                      make_float2(__uint_as_float(vv[2 * i]), __uint_as_float(vv[2 * i + 1])), rs2, acc[c * 16 + i]);
               } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                   const float4 cs = *reinterpret_cast<const float4 *>(cb + c * 32 + 4 * i);
                   float2 c01 = make_float2(cs.x, cs.y), c23 = make_float2(cs.z, cs.w);
-                  if (!rconst) {
+                  if (need_row) {
                     c01 = __fmul2_rn(c01, rs2);
                     c23 = __fmul2_rn(c23, rs2);
                   }
                   acc[c * 16 + 2 * i] = __ffma2_rn(
-                      make_float2(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1])), c01, acc[c * 16 + 2 * i]);
-                  acc[c * 16 + 2 * i + 1] =
-                      __ffma2_rn(make_float2(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])), c23,
-                                 acc[c * 16 + 2 * i + 1]);
+                      make_float2(__uint_as_float(vv[4 * i]), __uint_as_float(vv[4 * i + 1])), c01,
+                      acc[c * 16 + 2 * i]);
+                  acc[c * 16 + 2 * i + 1] = __ffma2_rn(
+                      make_float2(__uint_as_float(vv[4 * i + 2]), __uint_as_float(vv[4 * i + 3])), c23,
+                      acc[c * 16 + 2 * i + 1]);
                 }
               }
             }
@@ -415,10 +472,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);
           ++u;
+          if (b + 1 < t.nblocks) release_slot(slot);  // the last slot is read again below
         }
         if (!ok) break;
         if (row_ok) {
-          const float fin = rconst ? s_eff : 1.0f;
+          // forward: the rhs column scale (in every unit's slot); static tgmm: s
+          const float fin = tg && p.static_scale ? s_eff : 1.0f;
+          const bool colmul = !tg && need_col;
+          const float *cf = s_scol + slot * kBN + h * 128;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             if (col0 + c * 32 >= p.ncols) continue;
@@ -426,9 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               float2 a = acc[c * 16 + i];
-              if (p.col_scale) {
-                a.x *= s_ctile[h * 128 + c * 32 + 2 * i];
-                a.y *= s_ctile[h * 128 + c * 32 + 2 * i + 1];
+              if (colmul) {
+                a.x *= cf[c * 32 + 2 * i];
+                a.y *= cf[c * 32 + 2 * i + 1];
               }
               o[2 * i] = a.x * fin;
               o[2 * i + 1] = a.y * fin;
@@ -436,15 +497,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             store32(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32, out_v8);
           }
         }
+        release_slot(slot);
       } else {
         const uint32_t buf = u & 1;
-        const bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
-        if (!epi_bar_and(got)) {
+        const int slot = v % kScaleSlots;
+        if (!wait_unit(buf, slot)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const float s0 = p.static_scale ? s_eff : 1.0f;
+        const float *cf = s_scol + slot * kBN + h * 128;
 #pragma unroll
         for (int cp = 0; cp < 2; ++cp) {
           uint32_t va[32], vb[32];
@@ -453,14 +516,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const uint32_t *v = half ? vb : va;
+            const uint32_t *vv = half ? vb : va;
             const int c = 2 * cp + half;
             if (!row_ok || col0 + c * 32 >= p.ncols) continue;
             float o[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float cs = p.col_scale ? s_ctile[h * 128 + c * 32 + i] : 1.0f;
-              o[i] = __uint_as_float(v[i]) * s0 * cs;
+              const float cs = need_col ? cf[c * 32 + i] : 1.0f;
+              o[i] = __uint_as_float(vv[i]) * s0 * cs;
             }
             store32(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32, out_v8);
           }
@@ -469,6 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++u;
+        release_slot(slot);
       }
     }
     // rows outside every group are zero (row-ragged passes only)

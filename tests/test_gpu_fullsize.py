@@ -1,0 +1,94 @@
+"""Full-size workloads on the GPU, checked on sampled outputs.
+
+Each workload runs at its real size through the same calls bench.py times
+(gmm_quantize_rhs once, then gmm_fwd, gmm_dlhs, tgmm_drhs with one shared
+workspace).  The oracle then recomputes sampled outputs one by one: a forward
+or dlhs row depends only on that row and its group's weights, and a drhs row
+(g, k) only on group g's rows, so each sample is an exact group-local
+sub-problem.  Weight codes and scales of the sampled groups are compared bit
+for bit; empty groups must give dW[g] = 0 exactly and unrouted rows 0.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_fp8_grouped_b200 as gm
+import oracle
+from moe_fp8_grouped_b200 import synth
+from parity import assert_close
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+WORKLOADS = ["mixtral", "dsv3_up", "dsv3_down", "ep_merged", "ep_separate", "ragged", "ragged_bf16"]
+
+
+def pick_groups(gs: np.ndarray, rng: np.random.Generator):
+    nz = np.flatnonzero(gs > 0)
+    picks = {int(nz[np.argmax(gs[nz])]), int(nz[np.argmin(gs[nz])]), int(rng.choice(nz))}
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_fullsize_sampled(name):
+    dev = torch.device("cuda:0")
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w, seed=0, device="cuda")
+    gs_h = inp.group_sizes.numpy().astype(np.int64)
+    gs = inp.group_sizes.to(dev)
+    M, K, N, G = w.M, w.K, w.N, w.G
+    bf16 = w.rule == "none"
+    rule = w.rule
+    s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    sarg = s if rule == "static" else None
+    ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, N, G) for op in (0, 1, 2)), dtype=torch.uint8, device=dev)
+    if bf16:
+        codes, scales = inp.w, None
+    else:
+        codes, scales = gm.gmm_quantize_rhs(inp.w)
+    out = gm.gmm_fwd(inp.lhs, codes, scales, gs, rule=rule, static_scale=sarg, ws=ws)
+    dl = gm.gmm_dlhs(inp.dout, codes, scales, gs, ws=ws, rule="none" if bf16 else "dynamic")
+    dw = gm.tgmm_drhs(inp.lhs, inp.dout, gs, rule=rule, static_scale=sarg, ws=ws)
+    st, bits = gm.gmm_read_device_status(ws)
+    assert st == 0, (st, bits)
+
+    offs = np.concatenate([[0], np.cumsum(gs_h)])
+    rng = np.random.default_rng(0)
+    groups = pick_groups(gs_h, rng)
+    qrule = {"static": oracle.Q_STATIC, "dynamic": oracle.Q_DYNAMIC, "none": None}[rule]
+    for g in groups:
+        a, b = int(offs[g]), int(offs[g + 1])
+        wg = inp.w[g:g + 1].cpu()
+        if not bf16:
+            qr, sr = oracle.quantize_rhs(wg)
+            assert np.array_equal(codes[g].cpu().numpy(), qr[0]), f"rhs codes of group {g}"
+            assert np.array_equal(scales[g].cpu().numpy(), sr[0]), f"rhs scales of group {g}"
+        rows = sorted({a, b - 1, int(rng.integers(a, b))})
+        one = np.array([len(rows)], np.int32)
+        lhs_r = inp.lhs[rows].cpu()
+        dout_r = inp.dout[rows].cpu()
+        if bf16:
+            ref, ab = oracle.gmm_fwd_bf16(lhs_r, wg, one)
+            assert_close(out[rows], ref, ab, f"{name} fwd g={g}")
+            ref, ab = oracle.gmm_dlhs_bf16(dout_r, wg, one)
+            assert_close(dl[rows], ref, ab, f"{name} dlhs g={g}")
+        else:
+            ref, ab = oracle.gmm_fwd(lhs_r, qrule, inp.static_scale, qr, sr, one)
+            assert_close(out[rows], ref, ab, f"{name} fwd g={g}")
+            ref, ab = oracle.gmm_dlhs(dout_r, qr, sr, one)
+            assert_close(dl[rows], ref, ab, f"{name} dlhs g={g}")
+        # drhs rows (g, k): the whole group is the sub-problem
+        ks = sorted({0, K - 1, int(rng.integers(0, K))})
+        x_g, d_g = inp.lhs[a:b].cpu(), inp.dout[a:b].cpu()
+        size = np.array([b - a], np.int32)
+        if bf16:
+            ref, ab = oracle.tgmm_drhs_bf16(x_g, d_g, size, sel=ks)
+        else:
+            ref, ab = oracle.tgmm_drhs(x_g, qrule, inp.static_scale, d_g, size, sel=ks)
+        assert_close(dw[g, ks], ref, ab, f"{name} drhs g={g}")
+    for g in np.flatnonzero(gs_h == 0)[:4]:
+        assert not torch.any(dw[int(g)] != 0), f"empty group {g} has nonzero dW"
+    tail = int(offs[-1])
+    if tail < M:
+        assert not torch.any(out[tail:] != 0) and not torch.any(dl[tail:] != 0)
+    del inp, codes, scales, out, dl, dw, ws
+    torch.cuda.empty_cache()
