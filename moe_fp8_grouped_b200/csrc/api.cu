@@ -441,10 +441,11 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   p.stages_per_chunk = elem;
   p.offs = P.offs;
   p.tpre = P.tpre;
-  p.row_scale = P.scales_a;
+  p.row_scale = elem == 1 ? P.scales_a : nullptr;  // the bf16 family has no scales
   p.row_scale_ld = K;
-  p.colblk_scale = P.scales_b;
+  p.colblk_scale = elem == 1 ? P.scales_b : nullptr;
   p.colblk_ld = N;
+  p.static_scale = (elem == 1 && !dyn) ? lhs.scale : nullptr;
   p.out = drhs;
   p.out_f32 = out_dtype == GMM_F32;
   p.ld_out = N;

@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   //   row scales:    promoted row-ragged passes (s_l / s_t per 128-block),
   //                  dynamic tgmm (s_x[chunk, k])
   const bool tg = p.mode == MODE_TGMM;
-  const bool need_col = tg ? (p.colblk_scale != nullptr) : (p.col_scale != nullptr);
+  const bool need_col = tg ? (kPromote && p.colblk_scale != nullptr) : (p.col_scale != nullptr);
   const bool need_row = kPromote && (tg ? p.static_scale == nullptr : true);
   const bool use_ring = need_col || need_row;
 
