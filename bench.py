@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--workload", default="mixtral")
     ap.add_argument("--m-override", type=int, default=None,
                     help="fewer rows (same routing recipe), for profiler captures of a small case")
+    ap.add_argument("--n-override", type=int, default=None,
+                    help="fewer output columns, for profiler captures of a small case")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -156,6 +158,8 @@ def run_ours(args):
     w = synth.WORKLOADS[args.workload]
     if args.m_override:
         w = synth.with_rows(w, args.m_override)
+    if args.n_override:
+        w = synth.with_cols(w, args.n_override)
     inp = synth.make_inputs(w, seed=rank, device=str(dev))
     gs = inp.group_sizes.to(dev)
     rows_routed = int(inp.group_sizes.sum())

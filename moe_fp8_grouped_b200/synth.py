@@ -71,6 +71,11 @@ def with_rows(w: Workload, M: int) -> Workload:
     return dataclasses.replace(w, name=f"{w.name}_m{M}", M=M, tokens=tokens)
 
 
+def with_cols(w: Workload, N: int) -> Workload:
+    """The same workload with N output columns."""
+    return dataclasses.replace(w, name=f"{w.name}_n{N}", N=N)
+
+
 def group_sizes(w: Workload, gen: torch.Generator) -> torch.Tensor:
     """int32 [G] row counts per expert, summing to M (CPU)."""
     G, M = w.G, w.M
