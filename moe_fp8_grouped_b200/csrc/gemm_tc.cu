@@ -383,19 +383,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int u = 0;  // TMEM units consumed
     int v = 0;  // scale slots consumed
     bool ok = true;
-    // Waits for TMEM unit u (and its scale slot).  Lane 0 waits and the warp
-    // shares its verdict, so the whole warp agrees (tcgen05.ld is warp-wide);
-    // warps never wait on one another.  After a timeout or an abort the warp
-    // stops waiting and only runs its loops out, touching no TMEM.
+    // waits for TMEM unit u (and its scale slot), then agrees with the other
+    // epilogue warps on whether to go on
     auto wait_unit = [&](uint32_t buf, int slot) -> bool {
-      bool got = ok;
-      if (lane == 0 && got) {
-        got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
-        if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kScaleSlots) & 1, ctl);
-      }
-      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-      ok = ok && got;
-      return got;
+      bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
+      if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kScaleSlots) & 1, ctl);
+      return epi_bar_and(got);
     };
     auto release_slot = [&](int slot) {
       if (use_ring) {
@@ -433,12 +426,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < t.nblocks; ++b) {
           const uint32_t buf = u & 1;
           slot = v % kScaleSlots;
-          if (wait_unit(buf, slot)) {
-            tc_fence_after();
-            const float rs = need_row ? s_srow[slot * kBM + row] : 1.0f;
-            const float2 rs2 = make_float2(rs, rs);
-            const float *cb = s_scol + slot * kBN + h * 128;
-            auto promote = [&](const uint32_t(&vv)[32], int c) {
+          if (!wait_unit(buf, slot)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float rs = need_row ? s_srow[slot * kBM + row] : 1.0f;
+          const float2 rs2 = make_float2(rs, rs);
+          const float *cb = s_scol + slot * kBN + h * 128;
+#pragma unroll
+          for (int cp = 0; cp < 2; ++cp) {
+            uint32_t va[32], vb[32];
+            tmem_ld32(tl + buf * kBN + (2 * cp) * 32, va);
+            tmem_ld32(tl + buf * kBN + (2 * cp + 1) * 32, vb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t *vv = half ? vb : va;
+              const int c = 2 * cp + half;
               if (!tg) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
@@ -461,27 +466,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                       acc[c * 16 + 2 * i + 1]);
                 }
               }
-            };
-            uint32_t va[32], vb[32];
-            tmem_ld32(tl + buf * kBN + 0 * 32, va);
-            tmem_ld32(tl + buf * kBN + 1 * 32, vb);
-            tmem_wait_ld();
-            promote(va, 0);
-            promote(vb, 1);
-            tmem_ld32(tl + buf * kBN + 2 * 32, va);
-            tmem_ld32(tl + buf * kBN + 3 * 32, vb);
-            tmem_wait_ld();
-            // the unit is in registers: hand the TMEM buffer back before the math
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-            promote(va, 2);
-            promote(vb, 3);
+            }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
           ++u;
           if (b + 1 < t.nblocks) release_slot(slot);  // the last slot is read again below
         }
-        if (row_ok && ok) {
+        if (!ok) break;
+        if (row_ok) {
           // forward: the rhs column scale (in every unit's slot); static tgmm: s
           const float fin = tg && p.static_scale ? s_eff : 1.0f;
           const bool colmul = !tg && need_col;
@@ -507,12 +501,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const uint32_t buf = u & 1;
         const int slot = v % kScaleSlots;
-        if (wait_unit(buf, slot)) {
-          tc_fence_after();
-          const float s0 = p.static_scale ? s_eff : 1.0f;
-          const float *cf = s_scol + slot * kBN + h * 128;
-          auto emit = [&](const uint32_t(&vv)[32], int c) {
-            if (!row_ok || col0 + c * 32 >= p.ncols) return;
+        if (!wait_unit(buf, slot)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float s0 = p.static_scale ? s_eff : 1.0f;
+        const float *cf = s_scol + slot * kBN + h * 128;
+#pragma unroll
+        for (int cp = 0; cp < 2; ++cp) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tl + buf * kBN + (2 * cp) * 32, va);
+          tmem_ld32(tl + buf * kBN + (2 * cp + 1) * 32, vb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t *vv = half ? vb : va;
+            const int c = 2 * cp + half;
+            if (!row_ok || col0 + c * 32 >= p.ncols) continue;
             float o[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -520,22 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[i] = __uint_as_float(vv[i]) * s0 * cs;
             }
             store32(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32, out_v8);
-          };
-          uint32_t va[32], vb[32];
-          tmem_ld32(tl + buf * kBN + 0 * 32, va);
-          tmem_ld32(tl + buf * kBN + 1 * 32, vb);
-          tmem_wait_ld();
-          emit(va, 0);
-          emit(vb, 1);
-          tmem_ld32(tl + buf * kBN + 2 * 32, va);
-          tmem_ld32(tl + buf * kBN + 3 * 32, vb);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
-          emit(va, 2);
-          emit(vb, 3);
+          }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
         ++u;
         release_slot(slot);
       }
