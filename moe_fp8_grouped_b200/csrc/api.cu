@@ -309,7 +309,6 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
                        : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, 256);
   if (!okB) return GMM_ERR_CUDA;
   GemmParams p{};
-  p.mode = MODE_ROWS;
   p.G = G;
   p.M = static_cast<int>(M);
   p.ncols = static_cast<int>(N);
@@ -326,7 +325,7 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   p.ld_out = N;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{elem, bmn, elem == 1 && dyn};
+  const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1 && dyn};
   const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   if ((s = cuda_status(prof("gemm_fwd", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
@@ -373,7 +372,6 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
                        : make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, 256);
   if (!okB) return GMM_ERR_CUDA;
   GemmParams p{};
-  p.mode = MODE_ROWS;
   p.G = G;
   p.M = static_cast<int>(M);
   p.ncols = static_cast<int>(K);
@@ -390,7 +388,7 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   p.ld_out = K;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{elem, bmn, elem == 1};
+  const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1};
   const int64_t items = ((M + 127) / 128 + G) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   if ((s = cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
@@ -429,30 +427,33 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   if (s != GMM_OK) return s;
   const uint32_t bke = 128 / elem;
   const uint64_t ldt = static_cast<uint64_t>(cap) * kBlk;  // elements per transposed row
+  // tile rows = dout columns n (A = dout^T chunks), tile columns = lhs columns
+  // k (B = lhs^T chunks); the epilogue writes dW[g, k, n]
   CUtensorMap tmA, tmB;
-  if (!make_map(&tmA, P.codes_a, elem, ldt, K, ldt * elem, bke, 128)) return GMM_ERR_CUDA;
-  if (!make_map(&tmB, P.codes_b, elem, ldt, N, ldt * elem, bke, 256)) return GMM_ERR_CUDA;
+  if (!make_map(&tmA, P.codes_b, elem, ldt, N, ldt * elem, bke, 128)) return GMM_ERR_CUDA;
+  if (!make_map(&tmB, P.codes_a, elem, ldt, K, ldt * elem, bke, 256)) return GMM_ERR_CUDA;
   GemmParams p{};
-  p.mode = MODE_TGMM;
   p.G = G;
   p.M = static_cast<int>(M);
-  p.ncols = static_cast<int>(N);
-  p.ktiles = static_cast<int>(K / kBlk);
+  p.ncols = static_cast<int>(K);
+  p.rtiles = static_cast<int>(N / kBlk);
   p.stages_per_chunk = elem;
   p.offs = P.offs;
   p.tpre = P.tpre;
-  p.row_scale = elem == 1 ? P.scales_a : nullptr;  // the bf16 family has no scales
-  p.row_scale_ld = K;
-  p.colblk_scale = elem == 1 ? P.scales_b : nullptr;
-  p.colblk_ld = N;
+  // fp8: dout chunk scales per tile row; lhs chunk scales per tile column
+  // (dynamic rule) or the static scale; the bf16 family has no scales
+  p.row_scale = elem == 1 ? P.scales_b : nullptr;
+  p.row_scale_ld = N;
+  p.colblk_scale = (elem == 1 && dyn) ? P.scales_a : nullptr;
+  p.colblk_ld = K;
   p.static_scale = (elem == 1 && !dyn) ? lhs.scale : nullptr;
   p.out = drhs;
   p.out_f32 = out_dtype == GMM_F32;
   p.ld_out = N;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{elem, false, elem == 1};
-  const int64_t items = static_cast<int64_t>(G) * (K / kBlk) * ((N + 255) / 256);
+  const GemmConfig cfg{MODE_TGMM, elem, false, elem == 1};
+  const int64_t items = static_cast<int64_t>(G) * (N / kBlk) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   if ((s = cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
     return s;

@@ -1,15 +1,18 @@
 // gemm_tc.cu -- persistent, warp-specialized grouped GEMM on the sm_100a
 // tensor cores (tcgen05), shared by the three passes:
 //
-//   forward gmm   rows = lhs rows of each group, contraction K, columns N
+//   forward gmm   tile rows = lhs rows of one group, contraction K, columns N
 //                 ("FP8 Megablox for batch split", maxtext PR #3770,
 //                 Description; "Support quantization for tokamax gmm v2",
 //                 maxtext PR #4451, Description)
-//   dlhs gmm      rows = dout rows, contraction N, columns K: the same rhs
-//                 read with the other major-ness (PR #4451, review thread on
-//                 ops.py: transpose_rhs flipped)
-//   tgmm drhs     rows = K, contraction = the rows of one group, columns N
-//                 ("drhs_tgmm2", PR #4451, Description)
+//   dlhs gmm      tile rows = dout rows, contraction N, columns K: the same
+//                 rhs read with the other major-ness (PR #4451, review thread
+//                 on ops.py: transpose_rhs flipped)
+//   tgmm drhs     tile rows = dout columns n, columns = lhs columns k,
+//                 contraction = the 128-row chunks of one group, written
+//                 transposed into dW[g, k, n] ("drhs_tgmm2", PR #4451,
+//                 Description).  With rows = n the dout chunk scale is one
+//                 number per accumulator row, like the row scale of dlhs.
 //
 // CTA layout (384 threads, one CTA per SM):
 //   warp 0     TMA producer: A tile 128 x 128 B, B tile 256 x 128 B per stage,
@@ -29,7 +32,7 @@
 //   promote == false  one TMEM unit per tile; out = acc * s * col_scale
 //   promote == true   one TMEM unit per 128-long contraction block; the
 //                     epilogue accumulates acc += unit * row_scale (* the
-//                     block's column scale for tgmm) in registers.
+//                     block's column scale for dynamic-lhs tgmm) in registers.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -67,15 +70,20 @@ constexpr size_t gemm_smem_bytes() {
          + 2 * (kMaxGroups + 1) * sizeof(int);   // plan copy
 }
 
+// One work item: tile row index rt (MODE_ROWS: rows r0 .. rend of group g;
+// MODE_TGMM: dout columns 128 rt ..), tile column index ct, and the number of
+// contraction stages.
 struct Item {
-  int g, nt, kt, nblocks, r0, rend;
+  int g, rt, ct, nblocks, r0, rend;
 };
 
+template <int kMode>
 __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const int *s_offs, const int *s_tpre,
                                             int tn) {
   Item t;
-  if (p.mode == MODE_ROWS) {
-    // items of group g: (tpre[g+1] - tpre[g]) m-tiles x tn n-tiles, m fastest
+  if constexpr (kMode == MODE_ROWS) {
+    // items of group g: (tpre[g+1] - tpre[g]) row tiles x tn column tiles,
+    // row tiles fastest
     int lo = 0, hi = p.G + 1;  // first i with tpre[i] * tn > w
     while (lo < hi) {
       int mid = (lo + hi) >> 1;
@@ -85,19 +93,20 @@ __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const in
     const int g = lo - 1;
     const int mt_g = s_tpre[g + 1] - s_tpre[g];
     const int local = w - s_tpre[g] * tn;
-    const int mt = local % mt_g;
     t.g = g;
-    t.nt = local / mt_g;
-    t.kt = 0;
-    t.r0 = s_offs[g] + kBM * mt;
+    t.rt = local % mt_g;
+    t.ct = local / mt_g;
+    t.r0 = s_offs[g] + kBM * t.rt;
     t.rend = min(s_offs[g + 1], t.r0 + kBM);
     t.nblocks = p.kblocks;
   } else {
-    const int per_g = p.ktiles * tn;
+    // items of group g: rtiles row tiles x tn column tiles, column tiles
+    // fastest (the group's lhs chunks stay in L2 across the row tiles)
+    const int per_g = p.rtiles * tn;
     const int g = w / per_g, local = w % per_g;
     t.g = g;
-    t.nt = local / p.ktiles;
-    t.kt = local % p.ktiles;
+    t.rt = local / tn;
+    t.ct = local % tn;
     t.r0 = 0;
     t.rend = 0;
     t.nblocks = (s_tpre[g + 1] - s_tpre[g]) * p.stages_per_chunk;
@@ -119,7 +128,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // Stores 32 consecutive outputs of one row.  v8: the destination is 32-byte
 // aligned, so each instruction writes one full 32-byte sector.
-__device__ __forceinline__ void store32(void *out, int64_t off_elems, const float (&v)[32], int out_f32, bool v8) {
+__device__ __forceinline__ void store_row32(void *out, int64_t off_elems, const float (&v)[32], int out_f32,
+                                            bool v8) {
   if (out_f32) {
     float *dst = static_cast<float *>(out) + off_elems;
     if (v8) {
@@ -149,11 +159,29 @@ __device__ __forceinline__ void store32(void *out, int64_t off_elems, const floa
   }
 }
 
-template <int kElem, bool kBMN, bool kPromote>
+// Stores 32 outputs of one tile row that are one column of the output
+// (dW[g, k0 + j, n] for j < 32, stride `pitch` elements).  The 32 lanes of a
+// warp hold 32 consecutive n, so each instruction writes 128 (f32) or 64
+// (bf16) contiguous bytes.
+__device__ __forceinline__ void store_col32(void *out, int64_t off_elems, int64_t pitch, const float (&v)[32],
+                                            int out_f32) {
+  if (out_f32) {
+    float *dst = static_cast<float *>(out) + off_elems;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) dst[j * pitch] = v[j];
+  } else {
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(out) + off_elems;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) dst[j * pitch] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+template <int kElem, bool kBMN, bool kPromote, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     gmm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const GemmParams p) {
   constexpr bool kF16 = (kElem == 2);
+  constexpr bool kTg = (kMode == MODE_TGMM);
   constexpr int kBKe = 128 / kElem;                 // contraction elements per stage
   constexpr int kMmaK = 32 / kElem;                 // contraction elements per MMA
   constexpr int kBBoxes = kBMN ? 2 * kElem : 1;     // TMA boxes per B stage
@@ -183,12 +211,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // Which scales each TMEM unit carries (the same decision in every role):
-  //   column scales: forward s_r[g, n] (every unit of a tile) or tgmm s_d[chunk, n]
-  //   row scales:    promoted row-ragged passes (s_l / s_t per 128-block),
-  //                  dynamic tgmm (s_x[chunk, k])
-  const bool tg = p.mode == MODE_TGMM;
-  const bool need_col = tg ? (kPromote && p.colblk_scale != nullptr) : (p.col_scale != nullptr);
-  const bool need_row = kPromote && (tg ? p.static_scale == nullptr : true);
+  //   column scales: forward s_r[g, n] (every unit of a tile); tgmm with a
+  //                  dynamic lhs rule: s_x[chunk, k]
+  //   row scales:    promoted row-ragged passes (s_l / s_t per 128-block);
+  //                  tgmm: s_d[chunk, n]
+  const bool need_col = kTg ? (kPromote && p.colblk_scale != nullptr) : (p.col_scale != nullptr);
+  const bool need_row = kPromote;
   const bool use_ring = need_col || need_row;
 
   if (threadIdx.x == 0) {
@@ -227,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_slot;
 
   const int tn = (p.ncols + kBN - 1) / kBN;
-  const int total = (p.mode == MODE_ROWS) ? s_tpre[p.G] * tn : p.G * p.ktiles * tn;
+  const int total = kTg ? p.G * p.rtiles * tn : s_tpre[p.G] * tn;
   const WaitCtl ctl{p.wait_limit_ns, abort_flag, p.status};
   const WaitCtl ctl_drain{p.wait_limit_ns, no_abort, p.status};
 
@@ -238,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-        const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+        const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
         for (int b = 0; b < t.nblocks; ++b, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, ctl)) {
@@ -247,21 +275,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&full[s], kAStage + kBStage);
           int ax, ay, bx, by;
-          if (p.mode == MODE_ROWS) {
+          if constexpr (!kTg) {
             ax = b * kBKe;
             ay = t.r0;
             if (kBMN) {
-              bx = t.nt * kBN;
+              bx = t.ct * kBN;
               by = t.g * p.b_group_rows + b * kBKe;
             } else {
               bx = b * kBKe;
-              by = t.g * p.b_group_rows + t.nt * kBN;
+              by = t.g * p.b_group_rows + t.ct * kBN;
             }
           } else {
-            ax = s_tpre[t.g] * kBlk + b * kBKe;
-            ay = t.kt * kBM;
+            ax = s_tpre[t.g] * kBlk + b * kBKe;  // the group's chunks in the transposed operands
+            ay = t.rt * kBM;                     // dout columns n
             bx = ax;
-            by = t.nt * kBN;
+            by = t.ct * kBN;                     // lhs columns k
           }
           tma_load_2d(sA + s * kAStage, &tmA, ax, ay, &full[s]);
 #pragma unroll
@@ -278,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0, u = 0;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-          const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+          const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
@@ -323,9 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int v = 0;
       bool ok = true;
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-        const Item t = decode_item(w, p, s_offs, s_tpre, tn);
+        const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
         const int units = kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0);
-        const int64_t ch0 = tg ? s_tpre[t.g] : 0;
+        const int64_t ch0 = kTg ? s_tpre[t.g] : 0;
         for (int j = 0; j < units; ++j, ++v) {
           const int slot = v % kScaleSlots;
           bool got = true;
@@ -335,11 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           if (need_col) {
-            const int n = t.nt * kBN + 8 * lane;  // 8 columns per lane
+            const int n = t.ct * kBN + 8 * lane;  // 8 columns per lane
             float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
             if (n < p.ncols) {
-              const float *src = tg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
-                                    : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n;
+              const float *src = kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
+                                     : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n;
               c0 = __ldg(reinterpret_cast<const float4 *>(src));
               c1 = __ldg(reinterpret_cast<const float4 *>(src) + 1);
             }
@@ -349,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (need_row) {
             float4 r;
-            if (tg) {
-              r = __ldg(reinterpret_cast<const float4 *>(p.row_scale + (ch0 + j) * p.row_scale_ld + t.kt * kBM +
+            if constexpr (kTg) {
+              r = __ldg(reinterpret_cast<const float4 *>(p.row_scale + (ch0 + j) * p.row_scale_ld + t.rt * kBM +
                                                          4 * lane));
             } else {
               const float *src = p.row_scale + static_cast<int64_t>(j) * p.row_scale_ld;
@@ -398,24 +426,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-      const Item t = decode_item(w, p, s_offs, s_tpre, tn);
-      const int col0 = t.nt * kBN + h * 128;
+      const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+      const int col0 = t.ct * kBN + h * 128;
       int64_t orow;
       bool row_ok;
-      if (p.mode == MODE_ROWS) {
+      if constexpr (!kTg) {
         orow = t.r0 + row;
         row_ok = orow < t.rend;
       } else {
-        orow = static_cast<int64_t>(t.g) * p.ktiles * kBM + t.kt * kBM + row;
+        orow = static_cast<int64_t>(t.rt) * kBM + row;  // n
         row_ok = true;
       }
+      // writes 32 tile columns starting at tile column col (a multiple of 32)
+      auto emit = [&](int col, const float(&o)[32]) {
+        if constexpr (!kTg) {
+          store_row32(p.out, orow * p.ld_out + col, o, p.out_f32, out_v8);
+        } else {
+          store_col32(p.out, (static_cast<int64_t>(t.g) * p.ncols + col) * p.ld_out + orow, p.ld_out, o,
+                      p.out_f32);
+        }
+      };
       if (t.nblocks == 0) {  // empty group in tgmm: dW tile = 0
         float z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          if (col0 + c * 32 < p.ncols) store32(p.out, orow * p.ld_out + col0 + c * 32, z, p.out_f32, out_v8);
+          if (col0 + c * 32 < p.ncols) emit(col0 + c * 32, z);
         continue;
       }
       if constexpr (kPromote) {
@@ -431,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const float rs = need_row ? s_srow[slot * kBM + row] : 1.0f;
+          const float rs = s_srow[slot * kBM + row];
           const float2 rs2 = make_float2(rs, rs);
           const float *cb = s_scol + slot * kBN + h * 128;
 #pragma unroll
@@ -444,20 +481,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int half = 0; half < 2; ++half) {
               const uint32_t *vv = half ? vb : va;
               const int c = 2 * cp + half;
-              if (!tg) {
+              if (!(kTg && need_col)) {
+                // one scale per accumulator row
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                  acc[c * 16 + i] = __ffma2_rn(
-                      make_float2(__uint_as_float(vv[2 * i]), __uint_as_float(vv[2 * i + 1])), rs2, acc[c * 16 + i]);
+                  acc[c * 16 + i] = __ffma2_rn(make_float2(__uint_as_float(vv[2 * i]), __uint_as_float(vv[2 * i + 1])),
+                                               rs2, acc[c * 16 + i]);
               } else {
+                // tgmm with a dynamic lhs rule: the lhs chunk scale varies
+                // along the columns k
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                   const float4 cs = *reinterpret_cast<const float4 *>(cb + c * 32 + 4 * i);
-                  float2 c01 = make_float2(cs.x, cs.y), c23 = make_float2(cs.z, cs.w);
-                  if (need_row) {
-                    c01 = __fmul2_rn(c01, rs2);
-                    c23 = __fmul2_rn(c23, rs2);
-                  }
+                  const float2 c01 = __fmul2_rn(make_float2(cs.x, cs.y), rs2);
+                  const float2 c23 = __fmul2_rn(make_float2(cs.z, cs.w), rs2);
                   acc[c * 16 + 2 * i] = __ffma2_rn(
                       make_float2(__uint_as_float(vv[4 * i]), __uint_as_float(vv[4 * i + 1])), c01,
                       acc[c * 16 + 2 * i]);
@@ -477,8 +514,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (row_ok) {
           // forward: the rhs column scale (in every unit's slot); static tgmm: s
-          const float fin = tg && p.static_scale ? s_eff : 1.0f;
-          const bool colmul = !tg && need_col;
+          const float fin = (kTg && p.static_scale) ? s_eff : 1.0f;
+          const bool colmul = !kTg && need_col;
           const float *cf = s_scol + slot * kBN + h * 128;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -494,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[2 * i] = a.x * fin;
               o[2 * i + 1] = a.y * fin;
             }
-            store32(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32, out_v8);
+            emit(col0 + c * 32, o);
           }
         }
         release_slot(slot);
@@ -525,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float cs = need_col ? cf[c * 32 + i] : 1.0f;
               o[i] = __uint_as_float(vv[i]) * s0 * cs;
             }
-            store32(p.out, orow * p.ld_out + col0 + c * 32, o, p.out_f32, out_v8);
+            emit(col0 + c * 32, o);
           }
         }
         tc_fence_before();
@@ -536,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // rows outside every group are zero (row-ragged passes only)
-    if (p.mode == MODE_ROWS) {
+    if constexpr (!kTg) {
       const int esz = p.out_f32 ? 4 : 2;
       const int64_t tail0 = s_offs[p.G];
       const int64_t cpr = static_cast<int64_t>(p.ncols) * esz / 16;  // 16-byte chunks per row
@@ -570,10 +607,10 @@ int num_sms() {
   return g_num_sms;
 }
 
-template <int kElem, bool kBMN, bool kPromote>
+template <int kElem, bool kBMN, bool kPromote, int kMode>
 static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p, int grid,
                                cudaStream_t st) {
-  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote>;
+  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode>;
   const size_t smem = gemm_smem_bytes();
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
@@ -590,16 +627,22 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
 
 cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                         int grid, cudaStream_t st) {
+  if (cfg.mode == MODE_TGMM) {
+    if (cfg.b_mn_major) return cudaErrorInvalidValue;
+    if (cfg.elem_bytes == 1 && cfg.promote) return launch_inst<1, false, true, MODE_TGMM>(tmA, tmB, p, grid, st);
+    if (cfg.elem_bytes == 2 && !cfg.promote) return launch_inst<2, false, false, MODE_TGMM>(tmA, tmB, p, grid, st);
+    return cudaErrorInvalidValue;
+  }
   if (cfg.elem_bytes == 1) {
     if (cfg.b_mn_major)
-      return cfg.promote ? launch_inst<1, true, true>(tmA, tmB, p, grid, st)
-                         : launch_inst<1, true, false>(tmA, tmB, p, grid, st);
-    return cfg.promote ? launch_inst<1, false, true>(tmA, tmB, p, grid, st)
-                       : launch_inst<1, false, false>(tmA, tmB, p, grid, st);
+      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS>(tmA, tmB, p, grid, st)
+                         : launch_inst<1, true, false, MODE_ROWS>(tmA, tmB, p, grid, st);
+    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS>(tmA, tmB, p, grid, st)
+                       : launch_inst<1, false, false, MODE_ROWS>(tmA, tmB, p, grid, st);
   }
   if (cfg.promote) return cudaErrorInvalidValue;
-  return cfg.b_mn_major ? launch_inst<2, true, false>(tmA, tmB, p, grid, st)
-                        : launch_inst<2, false, false>(tmA, tmB, p, grid, st);
+  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS>(tmA, tmB, p, grid, st)
+                        : launch_inst<2, false, false, MODE_ROWS>(tmA, tmB, p, grid, st);
 }
 
 }  // namespace gmm

@@ -59,31 +59,36 @@ cudaError_t launch_timeout_selftest(uint32_t *status, uint64_t limit_ns, cudaStr
 
 enum GemmMode { MODE_ROWS = 0, MODE_TGMM = 1 };
 
+// Tile space of one GEMM launch.  MODE_ROWS (forward, dlhs): tile rows are
+// 128-row slices of one group's rows, tile columns the output columns.
+// MODE_TGMM (drhs): tile rows are 128 dout columns n, tile columns 256 lhs
+// columns k, the contraction runs over the group's 128-row chunks, and the
+// result is written transposed into dW[g, k, n].
 struct GemmParams {
-  int mode;            // GemmMode
   int G;
   int M;               // rows of the row operand (MODE_ROWS) / of x (MODE_TGMM)
-  int ncols;           // output columns
+  int ncols;           // tile-space columns: N (forward), K (dlhs, tgmm)
   int kblocks;         // MODE_ROWS: contraction stages (128 bytes of operand row each)
-  int ktiles;          // MODE_TGMM: 128-row tiles of the output (K / 128)
+  int rtiles;          // MODE_TGMM: 128-row tiles (N / 128)
   int b_group_rows;    // MODE_ROWS: rows per group in B's 2-D view
   int stages_per_chunk;// MODE_TGMM: stages per 128-row chunk (1 fp8, 2 bf16)
   const int *offs;     // [G + 1]
   const int *tpre;     // [G + 1]
-  const float *row_scale;     // MODE_ROWS: [kblocks][M]; MODE_TGMM: [chunk][K]
+  const float *row_scale;     // MODE_ROWS: [kblocks][M]; MODE_TGMM: dout chunk scales [chunk][N]
   int64_t row_scale_ld;
-  const float *colblk_scale;  // MODE_TGMM: [chunk][N]
+  const float *colblk_scale;  // MODE_TGMM, dynamic x: lhs chunk scales [chunk][K]
   int64_t colblk_ld;
-  const float *col_scale;     // [G][ncols] final per-column scale, or NULL
+  const float *col_scale;     // MODE_ROWS: [G][ncols] final per-column scale, or NULL
   const float *static_scale;  // device scalar multiplied in at the end, or NULL
   void *out;
   int out_f32;
-  int64_t ld_out;
+  int64_t ld_out;             // MODE_ROWS: output row pitch; MODE_TGMM: N
   uint32_t *status;
   uint64_t wait_limit_ns;
 };
 
 struct GemmConfig {
+  int mode;         // GemmMode
   int elem_bytes;   // 1: E4M3 (kind::f8f6f4), 2: BF16 (kind::f16)
   bool b_mn_major;  // B operand MN-major in shared memory
   bool promote;     // one TMEM unit per contraction block, promoted in registers
