@@ -151,6 +151,29 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
                    void *stream);
 
 /*
+ * Forward gmm without a workspace argument, for callers that cannot allocate
+ * device memory: code that runs where cudaMalloc is not allowed (a host
+ * function enqueued on a stream), or that runs under a runtime which owns all
+ * device memory and forbids allocations after start-up (cudaMalloc would also
+ * synchronize the device).  The pages have no counterpart; it is a
+ * convenience of this library.
+ * Arguments and results are gmm_fwd's, minus ws and ws_bytes.  The scratch
+ * lives in one 32 MiB array of device memory inside the library, which every
+ * device holds, once the library is used on it, until the process exits.  A
+ * call whose gmm_workspace_bytes(GMM_OP_FWD, M, K, N, G) exceeds 32 MiB
+ * returns GMM_ERR_WORKSPACE before anything runs.  Nothing is allocated.
+ * The first call on a device looks up the array's device address; make that
+ * first call before any stream capture.  All calls share the array, which
+ * keeps the last call's contents (each call rewrites all it reads): calls
+ * whose kernels overlap on the GPU (concurrent streams) race, so serialize
+ * them.  Device-detected errors still clamp or zero as in gmm_fwd, but their
+ * status word is not readable through this entry point.
+ */
+gmm_status gmm_fwd_noalloc(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes,
+                           int32_t G, int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype,
+                           void *stream);
+
+/*
  * Backward gmm wrt lhs.  dout: bf16 [M, N], always quantized with DYNAMIC
  * 128-blocks along N after folding the rhs column scale in (dout.rule must be
  * DYNAMIC, or NONE for the bf16 family).  rhs: the same buffer and layout as
