@@ -49,8 +49,8 @@ constexpr int kEpiWarp0 = 4;      // first epilogue warp
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 256;
 constexpr int kTmemCols = 512;
-constexpr int kScaleSlots = 4;    // ring of per-unit scale slots (scale loader -> epilogue)
-constexpr int kNumBars = 24;      // mbarriers reserved in shared memory
+constexpr int kScaleSlots = 8;    // ring of per-unit scale slots (scale loader -> epilogue)
+constexpr int kNumBars = 32;      // mbarriers reserved in shared memory
 // Register split (setmaxnreg): the control warpgroup gives registers to the
 // two epilogue warpgroups.  Sum must not exceed the launch allocation
 // (registers per thread at launch x 384); launch_inst checks it.
@@ -362,38 +362,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          // cp.async straight into the slot: the loader never waits for the
+          // data, the slot's barrier completes when all 32 lanes' copies land
           if (need_col) {
-            const int n = t.ct * kBN + 8 * lane;  // 8 columns per lane
-            float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+            const int n = t.ct * kBN + 8 * lane;  // 8 columns per lane; columns >= ncols are never read
             if (n < p.ncols) {
               const float *src = kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
                                      : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n;
-              c0 = __ldg(reinterpret_cast<const float4 *>(src));
-              c1 = __ldg(reinterpret_cast<const float4 *>(src) + 1);
+              float *dst = s_scol + slot * kBN + 8 * lane;
+              cp_async_16(dst, src);
+              cp_async_16(dst + 4, src + 4);
             }
-            float4 *dst = reinterpret_cast<float4 *>(s_scol + slot * kBN + 8 * lane);
-            dst[0] = c0;
-            dst[1] = c1;
           }
           if (need_row) {
-            float4 r;
+            float *dst = s_srow + slot * kBM + 4 * lane;
             if constexpr (kTg) {
-              r = __ldg(reinterpret_cast<const float4 *>(p.row_scale + (ch0 + j) * p.row_scale_ld + t.rt * kBM +
-                                                         4 * lane));
+              cp_async_16(dst, p.row_scale + (ch0 + j) * p.row_scale_ld + t.rt * kBM + 4 * lane);
             } else {
               const float *src = p.row_scale + static_cast<int64_t>(j) * p.row_scale_ld;
               const int64_t last = p.M - 1;
               const int64_t r0 = t.r0 + 4 * lane;
-              r.x = __ldg(src + min(r0, last));
-              r.y = __ldg(src + min(r0 + 1, last));
-              r.z = __ldg(src + min(r0 + 2, last));
-              r.w = __ldg(src + min(r0 + 3, last));
+#pragma unroll
+              for (int e = 0; e < 4; ++e) cp_async_4(dst + e, src + min(r0 + e, last));
             }
-            *reinterpret_cast<float4 *>(s_srow + slot * kBM + 4 * lane) = r;
           }
-          mbar_arrive(&sfull[slot]);
+          cp_async_mbar_arrive(&sfull[slot]);
         }
       }
+      cp_async_wait_all();  // no copy in flight when the warp leaves
     }
   } else {
     setmaxnreg_inc<regs_epi<kPromote>()>();
