@@ -114,8 +114,12 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&v)[8]) {
 
 // ------------------------------------------------------ rows (axis 1)
 
-// A warp covers 256 consecutive values of one row: each half-warp one block
-// of 128, each lane 8 values (16 bytes).
+// A warp covers 256 consecutive values of one row per segment: each
+// half-warp one block of 128, each lane 8 values (16 bytes).  A warp takes
+// kSegs consecutive segments per step and issues all their loads first, so
+// that enough bytes are in flight to stream at HBM speed.
+constexpr int kSegs = 4;
+
 template <bool kDynamic, bool kColMult>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
                                                          int64_t cols, const float *__restrict__ static_scale,
@@ -139,53 +143,70 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *__
   const int half = lane >> 4, hl = lane & 15;
   const int64_t segs_per_row = (cols + 255) / 256;
   const int64_t total = rows * segs_per_row;
-  for (int64_t seg = static_cast<int64_t>(blockIdx.x) * 8 + warp; seg < total;
-       seg += static_cast<int64_t>(gridDim.x) * 8) {
-    const int64_t r = seg / segs_per_row;
-    const int64_t cb = (seg % segs_per_row) * 256 + half * 128;  // block start
-    const int64_t c0 = cb + hl * 8;
-    const bool valid = cb < cols;
-    float v[8];
-    if (valid) {
-      uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + r * cols + c0));
-      bf16x8_to_f32(u, v);
-    } else {
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * kSegs; base < total;
+       base += nwarps * kSegs) {
+    uint4 raw[kSegs];
+    float4 cs[kSegs][2];
+    int64_t r[kSegs], cb[kSegs];
+    bool valid[kSegs];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-    }
-    if constexpr (kColMult) {
-      const int g = group_of_row(s_offs, G, r);
-      if (g < 0 || !valid) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      } else {
-        const float4 *cs = reinterpret_cast<const float4 *>(col_scale + static_cast<int64_t>(g) * cols + c0);
-        float4 a = __ldg(cs), b = __ldg(cs + 1);
-        v[0] = __fmul_rn(v[0], a.x); v[1] = __fmul_rn(v[1], a.y);
-        v[2] = __fmul_rn(v[2], a.z); v[3] = __fmul_rn(v[3], a.w);
-        v[4] = __fmul_rn(v[4], b.x); v[5] = __fmul_rn(v[5], b.y);
-        v[6] = __fmul_rn(v[6], b.z); v[7] = __fmul_rn(v[7], b.w);
+    for (int u = 0; u < kSegs; ++u) {
+      const int64_t seg = base + u;
+      r[u] = seg / segs_per_row;
+      cb[u] = (seg % segs_per_row) * 256 + half * 128;
+      valid[u] = seg < total && cb[u] < cols;
+      raw[u] = valid[u] ? __ldg(reinterpret_cast<const uint4 *>(x + r[u] * cols + cb[u] + hl * 8))
+                        : make_uint4(0, 0, 0, 0);
+      if constexpr (kColMult) {
+        const int g = (seg < total) ? group_of_row(s_offs, G, r[u]) : -1;
+        if (g < 0) valid[u] = false;
+        if (valid[u]) {
+          const float4 *c = reinterpret_cast<const float4 *>(col_scale + static_cast<int64_t>(g) * cols + cb[u] +
+                                                             hl * 8);
+          cs[u][0] = __ldg(c);
+          cs[u][1] = __ldg(c + 1);
+        } else {
+          cs[u][0] = cs[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
     }
-    float s = 0.0f, inv;
-    if constexpr (kDynamic) {
-      float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int u = 0; u < kSegs; ++u) {
+      float v[8];
+      bf16x8_to_f32(raw[u], v);
+      if constexpr (kColMult) {
+        // t = fl32(dout * s_r[g(m), n]); rows in no group give t = 0
+        v[0] = __fmul_rn(v[0], cs[u][0].x); v[1] = __fmul_rn(v[1], cs[u][0].y);
+        v[2] = __fmul_rn(v[2], cs[u][0].z); v[3] = __fmul_rn(v[3], cs[u][0].w);
+        v[4] = __fmul_rn(v[4], cs[u][1].x); v[5] = __fmul_rn(v[5], cs[u][1].y);
+        v[6] = __fmul_rn(v[6], cs[u][1].z); v[7] = __fmul_rn(v[7], cs[u][1].w);
+        if (!valid[u]) {  // rows in no group: t = +0 exactly
 #pragma unroll
-      for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
-      dyn_scale(amax, s, inv);
-    } else {
-      inv = inv_static;
-    }
-    if (valid) {
-      uint2 out;
-      out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
-              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
-      out.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv))) |
-              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
-      *reinterpret_cast<uint2 *>(codes + r * cols + c0) = out;
-      if (kDynamic && hl == 0) scales[(cb / kBlk) * rows + r] = s;
+          for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+        }
+      }
+      float s = 0.0f, inv;
+      if constexpr (kDynamic) {
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+        for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+        dyn_scale(amax, s, inv);
+      } else {
+        inv = inv_static;
+      }
+      const bool in_range = base + u < total && cb[u] < cols;
+      if (in_range) {
+        uint2 out;
+        out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
+                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
+        out.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv))) |
+                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
+        *reinterpret_cast<uint2 *>(codes + r[u] * cols + cb[u] + hl * 8) = out;
+        if (kDynamic && hl == 0) scales[(cb[u] / kBlk) * rows + r[u]] = s;
+      }
     }
   }
 }
@@ -194,7 +215,7 @@ cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dy
                               const float *col_scale, const int *offs, int G, uint8_t *codes, float *scales,
                               uint32_t *status, cudaStream_t st) {
   const int64_t segs = rows * ((cols + 255) / 256);
-  int64_t blocks = (segs + 7) / 8;
+  int64_t blocks = (segs + 8 * kSegs - 1) / (8 * kSegs);
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
@@ -216,10 +237,14 @@ cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dy
 
 // ---------------------------------------------------- chunks (axis 0)
 
-// One CTA per (128-column slice, chunk).  The chunk's rows (at most 128, the
-// rest zero) are staged in shared memory; thread t owns column t % 128 and
-// rows [64 (t / 128), +64), and writes them as 64 contiguous bytes of the
-// transposed code matrix.
+// One CTA per (256-column slice, chunk).  The chunk's rows (at most 128, the
+// rest zero) are staged in shared memory; thread t owns column t: it takes the
+// column's absmax over the chunk and writes the column's 128 codes as one
+// 128-byte line of the transposed code matrix.
+constexpr int kChunkCols = 256;
+constexpr int kChunkPitch = kChunkCols + 8;  // bf16 per staged row (16-byte aligned rows)
+constexpr size_t kChunkSmem = static_cast<size_t>(kBlk) * kChunkPitch * sizeof(__nv_bfloat16);
+
 template <bool kDynamic, bool kCopy>
 __global__ void __launch_bounds__(256) quant_chunks_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
                                                            int64_t cols, const float *__restrict__ static_scale,
@@ -227,11 +252,11 @@ __global__ void __launch_bounds__(256) quant_chunks_kernel(const __nv_bfloat16 *
                                                            const int *__restrict__ tpre, int G, void *codes_t,
                                                            int64_t ld_t, float *__restrict__ scales,
                                                            uint32_t *__restrict__ status) {
-  __shared__ __align__(16) __nv_bfloat16 tile[kBlk][kBlk + 8];
-  __shared__ float s_amax[2][kBlk];
+  extern __shared__ __align__(16) uint8_t qsm[];
+  __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(qsm);  // [128][kChunkPitch]
   __shared__ int s_info[3];
   const int j = blockIdx.y;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kBlk;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kChunkCols;
   if (threadIdx.x == 0) {
     int g = -1;
     if (j < tpre[G]) {
@@ -254,38 +279,40 @@ __global__ void __launch_bounds__(256) quant_chunks_kernel(const __nv_bfloat16 *
   const int g = s_info[0];
   if (g < 0) return;
   const int r0 = s_info[1], nr = s_info[2];
-  for (int i = threadIdx.x; i < kBlk * 16; i += 256) {
-    const int rr = i >> 4, cc = (i & 15) * 8;
+  // 128 rows x 32 sixteen-byte pieces; rows past the chunk and columns past
+  // the matrix read as zero
+#pragma unroll 4
+  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 8); i += 256) {
+    const int rr = i >> 5, cc = (i & 31) * 8;
     uint4 u = make_uint4(0, 0, 0, 0);
-    if (rr < nr) u = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc));
-    *reinterpret_cast<uint4 *>(&tile[rr][cc]) = u;
+    if (rr < nr && c0 + cc < cols)
+      u = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc));
+    *reinterpret_cast<uint4 *>(tile + rr * kChunkPitch + cc) = u;
   }
   __syncthreads();
-  const int col = threadIdx.x & 127, h = threadIdx.x >> 7;
-  const int rb = 64 * h;
+  const int col = threadIdx.x;
+  if (c0 + col >= cols) return;
   if constexpr (kCopy) {
     // bf16 family: transposed bf16 copy, no scale
-    uint16_t *dst = static_cast<uint16_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j + rb;
+    uint16_t *dst = static_cast<uint16_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 16; ++q) {
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint16_t lo = __bfloat16_as_ushort(tile[rb + q * 8 + 2 * e][col]);
-        const uint16_t hi = __bfloat16_as_ushort(tile[rb + q * 8 + 2 * e + 1][col]);
+        const uint16_t lo = __bfloat16_as_ushort(tile[(q * 8 + 2 * e) * kChunkPitch + col]);
+        const uint16_t hi = __bfloat16_as_ushort(tile[(q * 8 + 2 * e + 1) * kChunkPitch + col]);
         w[e] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
       }
       *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    return;
   } else {
     float s, inv;
     if constexpr (kDynamic) {
       float amax = 0.0f;
-      for (int r = rb; r < rb + 64; ++r) amax = fmaxf(amax, fabsf(__bfloat162float(tile[r][col])));
-      s_amax[h][col] = amax;
-      __syncthreads();
-      dyn_scale(fmaxf(s_amax[0][col], s_amax[1][col]), s, inv);
+#pragma unroll 8
+      for (int r = 0; r < kBlk; ++r) amax = fmaxf(amax, fabsf(__bfloat162float(tile[r * kChunkPitch + col])));
+      dyn_scale(amax, s, inv);
     } else {
       s = *static_scale;
       const bool ok = static_scale_ok(s);
@@ -293,41 +320,51 @@ __global__ void __launch_bounds__(256) quant_chunks_kernel(const __nv_bfloat16 *
       if (!ok) s = 0.0f;
       if (!ok && j == 0 && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, GMM_DEV_SCALE);
     }
-    uint8_t *dst = static_cast<uint8_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j + rb;
+    uint8_t *dst = static_cast<uint8_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 8; ++q) {
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int r = rb + q * 16 + e * 4;
-        const float a0 = __fmul_rn(__bfloat162float(tile[r][col]), inv);
-        const float a1 = __fmul_rn(__bfloat162float(tile[r + 1][col]), inv);
-        const float a2 = __fmul_rn(__bfloat162float(tile[r + 2][col]), inv);
-        const float a3 = __fmul_rn(__bfloat162float(tile[r + 3][col]), inv);
+        const int r = q * 16 + e * 4;
+        const float a0 = __fmul_rn(__bfloat162float(tile[r * kChunkPitch + col]), inv);
+        const float a1 = __fmul_rn(__bfloat162float(tile[(r + 1) * kChunkPitch + col]), inv);
+        const float a2 = __fmul_rn(__bfloat162float(tile[(r + 2) * kChunkPitch + col]), inv);
+        const float a3 = __fmul_rn(__bfloat162float(tile[(r + 3) * kChunkPitch + col]), inv);
         w[e] = static_cast<uint32_t>(cvt_e4m3x2(a0, a1)) | (static_cast<uint32_t>(cvt_e4m3x2(a2, a3)) << 16);
       }
       *reinterpret_cast<uint4 *>(dst + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    if (h == 0) scales[static_cast<int64_t>(j) * cols + c0 + col] = s;
+    scales[static_cast<int64_t>(j) * cols + c0 + col] = s;
   }
+}
+
+template <bool kDynamic, bool kCopy>
+static cudaError_t launch_chunks_inst(dim3 grid, cudaStream_t st, const __nv_bfloat16 *xb, int64_t rows,
+                                      int64_t cols, const float *static_scale, const int *offs, const int *tpre,
+                                      int G, void *codes_t, int64_t ld_t, float *scales, uint32_t *status) {
+  auto kern = quant_chunks_kernel<kDynamic, kCopy>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kChunkSmem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 256, kChunkSmem, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t, scales, status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool dynamic, const float *static_scale,
                                 const int *offs, const int *tpre, int G, int64_t capacity, void *codes_t,
                                 float *scales, bool bf16_copy, uint32_t *status, cudaStream_t st) {
-  dim3 grid(static_cast<unsigned>(cols / kBlk), static_cast<unsigned>(capacity));
+  dim3 grid(static_cast<unsigned>((cols + kChunkCols - 1) / kChunkCols), static_cast<unsigned>(capacity));
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
   const int64_t ld_t = capacity * kBlk;
   if (bf16_copy)
-    quant_chunks_kernel<false, true><<<grid, 256, 0, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t,
-                                                           ld_t, scales, status);
-  else if (dynamic)
-    quant_chunks_kernel<true, false><<<grid, 256, 0, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t,
-                                                           ld_t, scales, status);
-  else
-    quant_chunks_kernel<false, false><<<grid, 256, 0, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t,
-                                                            ld_t, scales, status);
-  return cudaGetLastError();
+    return launch_chunks_inst<false, true>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t,
+                                           scales, status);
+  if (dynamic)
+    return launch_chunks_inst<true, false>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t,
+                                           scales, status);
+  return launch_chunks_inst<false, false>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t,
+                                          scales, status);
 }
 
 // ------------------------------------------------------------ rhs (K7)
