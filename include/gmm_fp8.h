@@ -139,7 +139,13 @@ gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrul
 
 /*
  * Forward gmm.  lhs: bf16 [M, K] with rule STATIC / DYNAMIC (or NONE for the
- * bf16 family).  rhs: E4M3 codes with scales [G, N] (or bf16 for the bf16
+ * bf16 family), quantized inside the call; or E4M3 codes [M, K] already
+ * quantized by the caller ("add static LHS scaling support for GMM v2 FWD",
+ * maxtext PR #4735, rebase commit text: activations quantized before the
+ * expert-parallel all-gather arrive as a pre-quantized array whose scale is
+ * re-applied after the matmul), with lhs.scale the static scale (rule STATIC,
+ * one float) or the block scales [K/128, M] (rule DYNAMIC, the layout
+ * gmm_quantize writes for axis 1); the quantize step is then skipped.  rhs: E4M3 codes with scales [G, N] (or bf16 for the bf16
  * family), [G, K, N] when transpose_rhs == 0, [G, N, K] when 1.
  * group_sizes: device int32 [G]; rows are sorted by group.
  * out: [M, N] of out_dtype (BF16 or F32):

@@ -167,7 +167,12 @@ static gmm_status classify(const gmm_operand &x, const gmm_operand &w, bool w_is
     return GMM_OK;
   }
   if (x.rule != GMM_Q_STATIC && x.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
-  if (x.dtype != GMM_BF16) return GMM_ERR_INVALID_ARG;
+  if (x.dtype == GMM_E4M3) {
+    // pre-quantized lhs (forward only): its scales come with it
+    if (!w_is_rhs || !x.scale) return GMM_ERR_INVALID_ARG;
+  } else if (x.dtype != GMM_BF16) {
+    return GMM_ERR_INVALID_ARG;
+  }
   if (x.rule == GMM_Q_STATIC && !x.scale) return GMM_ERR_INVALID_ARG;  // a present rule must be applied
   if (w_is_rhs) {
     if (w.dtype != GMM_E4M3 || !w.scale) return GMM_ERR_INVALID_ARG;
@@ -291,8 +296,9 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
   int n = 1;
   const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
+  const bool preq = lhs.dtype == GMM_E4M3;  // codes and scales supplied by the caller
   const void *A = lhs.data;
-  if (elem == 1) {
+  if (elem == 1 && !preq) {
     s = cuda_status(prof("quant_rows", st, [&] {
       return launch_quant_rows(lhs.data, M, K, dyn, dyn ? nullptr : lhs.scale, nullptr, P.offs, G, P.codes_a,
                                P.scales_a, P.status, st);
@@ -316,7 +322,7 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   p.b_group_rows = static_cast<int>(bmn ? K : N);
   p.offs = P.offs;
   p.tpre = P.tpre;
-  p.row_scale = (elem == 1 && dyn) ? P.scales_a : nullptr;
+  p.row_scale = (elem == 1 && dyn) ? (preq ? lhs.scale : P.scales_a) : nullptr;
   p.row_scale_ld = M;
   p.col_scale = elem == 1 ? rhs.scale : nullptr;
   p.static_scale = (elem == 1 && !dyn) ? lhs.scale : nullptr;
@@ -346,6 +352,7 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   int elem = 0;
   if ((s = classify(dout, rhs, true, &elem)) != GMM_OK) return s;
   if (elem == 1 && dout.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;  // gradients: dynamic blocks
+  if (dout.dtype != GMM_BF16) return GMM_ERR_INVALID_ARG;                   // the rhs scale is folded in
   if (!al16(dout.data) || !al16(rhs.data) || !al16(dlhs) || !al16(ws) || (rhs.scale && !al16(rhs.scale)))
     return GMM_ERR_ALIGNMENT;
   const WsLayout L = ws_layout(GMM_OP_DLHS, M, K, N, G);

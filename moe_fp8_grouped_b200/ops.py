@@ -134,10 +134,13 @@ def _operand(data, dtype_code, scale, rule):
 
 def gmm_fwd(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | None, group_sizes: torch.Tensor,
             rule="static", static_scale: torch.Tensor | None = None, transpose_rhs: bool = False,
-            out_dtype=torch.bfloat16, out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+            out_dtype=torch.bfloat16, out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+            lhs_scales: torch.Tensor | None = None):
     """Forward gmm: out[m] = lhs[m] @ rhs[g(m)] with lhs quantized inside the
     call (rule "static" with ``static_scale``, or "dynamic"); rule "none"
-    runs the bf16 family (rhs bf16, no scales)."""
+    runs the bf16 family (rhs bf16, no scales).  A uint8 / float8 ``lhs`` is
+    taken as already-quantized E4M3 codes: its scale is ``static_scale``
+    (static) or ``lhs_scales`` [K/128, M] (dynamic, as gmm_quantize writes)."""
     M, K = lhs.shape
     if transpose_rhs:
         G, N, K2 = rhs.shape
@@ -149,8 +152,12 @@ def gmm_fwd(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | Non
         out = torch.empty((M, N), dtype=out_dtype, device=lhs.device)
     if ws is None:
         ws = workspace(gmm_workspace_bytes(B.OP_FWD, M, K, N, G), lhs.device)
-    a = _operand(_dev(lhs, "lhs", torch.bfloat16), B.DT_BF16,
-                 _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None, r)
+    if lhs.dtype in (torch.uint8, torch.float8_e4m3fn):
+        sc = static_scale if r == B.Q_STATIC else lhs_scales
+        a = _operand(_dev(lhs, "lhs"), B.DT_E4M3, _dev(sc, "lhs scale", torch.float32) if sc is not None else None, r)
+    else:
+        a = _operand(_dev(lhs, "lhs", torch.bfloat16), B.DT_BF16,
+                     _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None, r)
     b = _operand(_dev(rhs, "rhs"), _TORCH_DT[rhs.dtype],
                  _dev(rhs_scales, "rhs_scales", torch.float32) if rhs_scales is not None else None, B.Q_NONE)
     st = B.lib().gmm_fwd(a, b, int(transpose_rhs), _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,

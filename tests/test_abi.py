@@ -79,7 +79,11 @@ def test_host_errors(L):
              None) == 3  # misaligned
     assert f(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, 1024, None) == 9  # workspace too small
     assert f(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, None, big, None) == 9  # no workspace
+    assert f(_op(FAKE, B.DT_E4M3, None, B.Q_DYNAMIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big,
+             None) == 1  # pre-quantized lhs without its scales
     d = L.gmm_dlhs
+    assert d(_op(FAKE, B.DT_E4M3, FAKE, B.Q_DYNAMIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big,
+             None) == 1  # dout must be bf16 (the rhs scale is folded in)
     assert d(_op(FAKE, B.DT_BF16, None, B.Q_STATIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big,
              None) == 1  # gradients are dynamic
     t = L.tgmm_drhs

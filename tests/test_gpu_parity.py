@@ -151,6 +151,28 @@ def test_drhs(dev, name, rule, out_dtype):
     assert_close(out, ref, ab, f"drhs {name} {rule}")
 
 
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("transpose", [False, True])
+def test_fwd_prequantized_lhs(dev, rule, transpose):
+    """lhs quantized before the call (for example ahead of an expert-parallel
+    all-gather): the forward takes the codes and scales as they are and gives
+    the same result as quantizing inside the call."""
+    inp = case_inputs("ragged")
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
+    sarg = s if rule == "static" else None
+    ql, sl = gm.gmm_quantize(lhs, rule, axis=1, static_scale=sarg)
+    inside = gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=sarg, transpose_rhs=transpose,
+                        out_dtype=torch.float32)
+    outside = gm.gmm_fwd(ql, codes, scales, gs, rule=rule, static_scale=sarg, lhs_scales=sl,
+                         transpose_rhs=transpose, out_dtype=torch.float32)
+    assert gm.last_launch_count() == 2  # plan + GEMM: no quantize step
+    assert torch.equal(inside, outside)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    ref, ab = oracle.gmm_fwd(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+    assert_close(outside, ref, ab, f"prequantized fwd {rule}")
+
+
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
 def test_bf16_family(dev, name):
     inp = case_inputs(name)
