@@ -79,6 +79,19 @@ def job_tflops(flops_per_step_per_rank: float, world: int, steps: int, ms: float
     return world * flops_per_step_per_rank * steps / (ms / 1e3) / 1e12
 
 
+def algorithmic_bytes(M, K, N, G, G_ne, rule):
+    """Bytes each pass must move: its inputs once and its outputs once (bf16
+    activations, E4M3 weights with fp32 [G, N] scales, dynamic block scales,
+    bf16 fwd / dlhs outputs, fp32 dW; bf16 weights for the bf16 family)."""
+    wb = 2 if rule == "none" else 1
+    wsc = 0 if rule == "none" else 4 * G * N
+    lsc = 4 * M * K // 128 if rule == "dynamic" else 0
+    gsc = 0 if rule == "none" else 4 * M * N // 128
+    return {"fwd": 2 * M * K + lsc + wb * G_ne * K * N + wsc + 2 * M * N,
+            "dlhs": 2 * M * N + gsc + wb * G_ne * K * N + wsc + 2 * M * K,
+            "drhs": 2 * M * K + 2 * M * N + 4 * G * K * N}
+
+
 def config_of(w, extra=None):
     cfg = {"workload": f"{w.name}: G={w.G} M={w.M} K={w.K} N={w.N}, lhs rule {w.rule}, fwd+dlhs+drhs",
            "G": w.G, "M": w.M, "K": w.K, "N": w.N, "lhs_rule": w.rule, "routing": w.routing,
@@ -171,7 +184,10 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    w = synth.WORKLOADS[args.workload]
+    # ep_separate: the EP-shrunk workload as two separate N=256 calls per pass
+    # (W0 and W1 apart) instead of one merged N=512 call
+    separate = args.workload == "ep_separate"
+    w = synth.WORKLOADS["ep_merged" if separate else args.workload]
     if args.m_override:
         w = synth.with_rows(w, args.m_override)
     if args.n_override:
@@ -179,27 +195,43 @@ def run_ours(args):
     inp = synth.make_inputs(w, seed=rank, device=str(dev))
     gs = inp.group_sizes.to(dev)
     rows_routed = int(inp.group_sizes.sum())
+    G_ne = int((inp.group_sizes > 0).sum())
     s_static = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
-    codes, rscales = gm.gmm_quantize_rhs(inp.w)  # weight quantization: outside the timed step
-    del inp.w
-    lhs, dout = inp.lhs, inp.dout
     M, K, N, G = w.M, w.K, w.N, w.G
     rule = w.rule
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    bf16_family = rule == "none"
+    parts = 2 if separate else 1
+    Np = N // parts
+    # weight quantization (or, for the bf16 family, nothing): outside the timed step
+    if bf16_family:
+        wparts = [(inp.w[:, :, i * Np:(i + 1) * Np].contiguous(), None) for i in range(parts)]
+    else:
+        wparts = [gm.gmm_quantize_rhs(inp.w[:, :, i * Np:(i + 1) * Np].contiguous()) for i in range(parts)]
+    codes, rscales = wparts[0]
+    del inp.w
+    lhs = inp.lhs
+    douts = [inp.dout[:, i * Np:(i + 1) * Np].contiguous() for i in range(parts)]
+    dout = douts[0]
+    del inp.dout
+    out = torch.empty((M, Np), dtype=torch.bfloat16, device=dev)
     dl = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    dw = torch.empty((G, K, N), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, N, G) for op in (0, 1, 2)), dtype=torch.uint8,
+    dw = torch.empty((G, K, Np), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, Np, G) for op in (0, 1, 2)), dtype=torch.uint8,
                      device=dev)
     sarg = s_static if rule == "static" else None
+    grule = "none" if bf16_family else "dynamic"
     launches = [0]
 
     def step(lhs_, dout_, codes_, rscales_, gs_):
-        gm.gmm_fwd(lhs_, codes_, rscales_, gs_, rule=rule, static_scale=sarg, out=out, ws=ws)
-        launches[0] += gm.last_launch_count()
-        gm.gmm_dlhs(dout_, codes_, rscales_, gs_, out=dl, ws=ws)
-        launches[0] += gm.last_launch_count()
-        gm.tgmm_drhs(lhs_, dout_, gs_, rule=rule, static_scale=sarg, out=dw, ws=ws)
-        launches[0] += gm.last_launch_count()
+        for i in range(parts):
+            c_, r_ = (codes_, rscales_) if i == 0 else wparts[i]
+            d_ = dout_ if i == 0 else douts[i]
+            gm.gmm_fwd(lhs_, c_, r_, gs_, rule=rule, static_scale=sarg, out=out, ws=ws)
+            launches[0] += gm.last_launch_count()
+            gm.gmm_dlhs(d_, c_, r_, gs_, out=dl, ws=ws, rule=grule)
+            launches[0] += gm.last_launch_count()
+            gm.tgmm_drhs(lhs_, d_, gs_, rule=rule, static_scale=sarg, out=dw, ws=ws)
+            launches[0] += gm.last_launch_count()
 
     def barrier():
         torch.cuda.synchronize()
@@ -232,36 +264,53 @@ def run_ours(args):
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     timed_launches = launches[0]
 
-    flops_pass = 2.0 * rows_routed * K * N
-    flops_step = 3 * flops_pass
+    flops_pass = 2.0 * rows_routed * K * Np  # one launch
+    flops_step = 3 * parts * flops_pass
     value = job_tflops(flops_step, world, args.steps, ms)
 
     peaks, peak_src = load_peaks()
-    fp8_peak_sustained = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    peak_tc = peaks["bf16_tflops_sustained"] * (1.0 if bf16_family else FP8_OVER_BF16)
+    peak_bw = peaks["hbm_gbs"]
+    bytes_pass = algorithmic_bytes(M, K, Np, G, G_ne, rule)
     passes = {}
     for name, key in (("fwd", "gemm_fwd"), ("dlhs", "gemm_dlhs"), ("drhs", "gemm_drhs")):
         n, tot = prof.get(key, (0, 0.0))
         if n:
             avg = tot / n
-            passes[name] = {"gemm_ms": round(avg, 4), "gemm_tflops": round(flops_pass / (avg / 1e3) / 1e12, 1)}
+            tfl = flops_pass / (avg / 1e3) / 1e12
+            gbs = bytes_pass[name] / (avg / 1e3) / 1e9
+            floor_ms = max(flops_pass / (peak_tc * 1e12), bytes_pass[name] / (peak_bw * 1e9)) * 1e3
+            passes[name] = {"gemm_ms": round(avg, 4), "gemm_tflops": round(tfl, 1), "gb_per_s": round(gbs, 1),
+                            "frac_tensor": round(tfl / peak_tc, 4), "frac_hbm": round(gbs / peak_bw, 4),
+                            "frac_roofline": round(floor_ms / avg, 4)}
     total_prof = sum(t for _, t in prof.values())
     kernels = {k: {"launches": n, "total_ms": round(t, 3), "share": round(t / total_prof, 4) if total_prof else None}
                for k, (n, t) in sorted(prof.items())}
     dom = max((k for k in prof if k.startswith("gemm_")), key=lambda k: prof[k][1])
     dn, dt = prof[dom]
-    achieved = flops_pass / (dt / dn / 1e3) / 1e12
-    roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": round(fp8_peak_sustained, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / fp8_peak_sustained, 4), "traffic": traffic_record(dom),
-                "peak_source": f"{peak_src} bf16 sustained cuBLAS x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)",
-                "algorithmic": f"2*sum(group_sizes)*K*N = {flops_pass:.4g} FLOP per launch"}
+    dname = dom.split("_")[1]
+    tc_bound = flops_pass / (peak_tc * 1e12) >= bytes_pass[dname] / (peak_bw * 1e9)  # seconds at each peak
+    if tc_bound:
+        achieved = flops_pass / (dt / dn / 1e3) / 1e12
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tc, 1),
+                    "unit": "TFLOP/s", "frac": round(achieved / peak_tc, 4),
+                    "peak_source": f"{peak_src} bf16 sustained cuBLAS" +
+                                   ("" if bf16_family else f" x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)"),
+                    "algorithmic": f"2*sum(group_sizes)*K*N = {flops_pass:.4g} FLOP per launch"}
+    else:
+        achieved = bytes_pass[dname] / (dt / dn / 1e3) / 1e9
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak_bw, 1),
+                    "unit": "GB/s", "frac": round(achieved / peak_bw, 4),
+                    "peak_source": f"{peak_src} HBM copy bandwidth",
+                    "algorithmic": f"{bytes_pass[dname]:.4g} bytes per launch (operands in, results out)"}
+    roofline["traffic"] = traffic_record(dom)
 
     # end to end: pinned host buffers, copies inside the timed region.  Steps
     # are pipelined over three streams (upload, compute, download) with two
     # device buffer sets, so step i's download overlaps step i+1's upload and
     # compute; every step still uploads its inputs and downloads its results.
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and parts == 1:
         h_lhs, h_dout = lhs.cpu().pin_memory(), dout.cpu().pin_memory()
         h_codes, h_rs, h_gs = codes.cpu().pin_memory(), rscales.cpu().pin_memory(), inp.group_sizes.pin_memory()
         h_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
@@ -300,7 +349,7 @@ def run_ours(args):
                     s_cmp.wait_event(down_done[b])  # download of step i-2 has read this output set
                 gm.gmm_fwd(a_lhs, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, out=o_out, ws=ws2[b])
                 launches[0] += gm.last_launch_count()
-                gm.gmm_dlhs(a_dout, a_codes, a_rs, a_gs, out=o_dl, ws=ws2[b])
+                gm.gmm_dlhs(a_dout, a_codes, a_rs, a_gs, out=o_dl, ws=ws2[b], rule=grule)
                 launches[0] += gm.last_launch_count()
                 gm.tgmm_drhs(a_lhs, a_dout, a_gs, rule=rule, static_scale=sarg, out=o_dw, ws=ws2[b])
                 launches[0] += gm.last_launch_count()
@@ -342,10 +391,15 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
-        "config": config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
-        "pct_fp8_peak": {"vs_nominal_4500": round(value / world / 4500.0 * 100, 2),
-                         "vs_measured_sustained": round(value / world / fp8_peak_sustained * 100, 2)},
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if bf16_family else "e4m3", "data": "synthetic",
+        "config": config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                                "calls_per_pass": parts,
+                                **({"workload": f"ep_separate: G={G} M={M} K={K}, two N={Np} calls per pass "
+                                                f"(W0, W1 apart), lhs rule {rule}, fwd+dlhs+drhs"}
+                                   if separate else {})}),
+        "pct_peak": {"vs_nominal": round(value / world / (2250.0 if bf16_family else 4500.0) * 100, 2),
+                     "vs_measured_sustained": round(value / world / peak_tc * 100, 2),
+                     "peak": "dense bf16" if bf16_family else "dense fp8"},
         "passes": passes, "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": timed_launches, "clocks": clk,
     }

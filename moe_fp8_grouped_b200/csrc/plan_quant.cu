@@ -114,10 +114,9 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&v)[8]) {
 
 // ------------------------------------------------------ rows (axis 1)
 
-// A warp covers 256 consecutive values of one row per segment: each
-// half-warp one block of 128, each lane 8 values (16 bytes).  A warp takes
-// kSegs consecutive segments per step and issues all their loads first, so
-// that enough bytes are in flight to stream at HBM speed.
+// A warp takes whole rows.  Within a row it covers 256 consecutive values
+// per segment (each half-warp one block of 128, each lane 8 values = 16
+// bytes) and kSegs segments per step, all loads issued first.
 constexpr int kSegs = 4;
 
 template <bool kDynamic, bool kColMult>
@@ -141,71 +140,74 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *__
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int half = lane >> 4, hl = lane & 15;
-  const int64_t segs_per_row = (cols + 255) / 256;
-  const int64_t total = rows * segs_per_row;
+  const int segs_per_row = static_cast<int>((cols + 255) / 256);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
-  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * kSegs; base < total;
-       base += nwarps * kSegs) {
-    uint4 raw[kSegs];
-    float4 cs[kSegs][2];
-    int64_t r[kSegs], cb[kSegs];
-    bool valid[kSegs];
-#pragma unroll
-    for (int u = 0; u < kSegs; ++u) {
-      const int64_t seg = base + u;
-      r[u] = seg / segs_per_row;
-      cb[u] = (seg % segs_per_row) * 256 + half * 128;
-      valid[u] = seg < total && cb[u] < cols;
-      raw[u] = valid[u] ? __ldg(reinterpret_cast<const uint4 *>(x + r[u] * cols + cb[u] + hl * 8))
-                        : make_uint4(0, 0, 0, 0);
-      if constexpr (kColMult) {
-        const int g = (seg < total) ? group_of_row(s_offs, G, r[u]) : -1;
-        if (g < 0) valid[u] = false;
-        if (valid[u]) {
-          const float4 *c = reinterpret_cast<const float4 *>(col_scale + static_cast<int64_t>(g) * cols + cb[u] +
-                                                             hl * 8);
-          cs[u][0] = __ldg(c);
-          cs[u][1] = __ldg(c + 1);
-        } else {
-          cs[u][0] = cs[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + warp; r < rows; r += nwarps) {
+    const __nv_bfloat16 *xr = x + r * cols;
+    uint8_t *cr = codes + r * cols;
+    const float *csr = nullptr;
+    bool row_in_group = true;
+    if constexpr (kColMult) {
+      const int g = group_of_row(s_offs, G, r);
+      row_in_group = g >= 0;
+      csr = col_scale + static_cast<int64_t>(g < 0 ? 0 : g) * cols;
     }
+    for (int sb = 0; sb < segs_per_row; sb += kSegs) {
+      uint4 raw[kSegs];
+      float4 cs[kSegs][2];
+      int cb[kSegs];
+      bool valid[kSegs];
 #pragma unroll
-    for (int u = 0; u < kSegs; ++u) {
-      float v[8];
-      bf16x8_to_f32(raw[u], v);
-      if constexpr (kColMult) {
-        // t = fl32(dout * s_r[g(m), n]); rows in no group give t = 0
-        v[0] = __fmul_rn(v[0], cs[u][0].x); v[1] = __fmul_rn(v[1], cs[u][0].y);
-        v[2] = __fmul_rn(v[2], cs[u][0].z); v[3] = __fmul_rn(v[3], cs[u][0].w);
-        v[4] = __fmul_rn(v[4], cs[u][1].x); v[5] = __fmul_rn(v[5], cs[u][1].y);
-        v[6] = __fmul_rn(v[6], cs[u][1].z); v[7] = __fmul_rn(v[7], cs[u][1].w);
-        if (!valid[u]) {  // rows in no group: t = +0 exactly
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+      for (int u = 0; u < kSegs; ++u) {
+        cb[u] = (sb + u) * 256 + half * 128;
+        valid[u] = sb + u < segs_per_row && cb[u] < cols;
+        raw[u] = valid[u] ? __ldg(reinterpret_cast<const uint4 *>(xr + cb[u] + hl * 8)) : make_uint4(0, 0, 0, 0);
+        if constexpr (kColMult) {
+          if (valid[u] && row_in_group) {
+            const float4 *c = reinterpret_cast<const float4 *>(csr + cb[u] + hl * 8);
+            cs[u][0] = __ldg(c);
+            cs[u][1] = __ldg(c + 1);
+          } else {
+            cs[u][0] = cs[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
       }
-      float s = 0.0f, inv;
-      if constexpr (kDynamic) {
-        float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      for (int u = 0; u < kSegs; ++u) {
+        if (sb + u >= segs_per_row) break;  // warp-uniform
+        float v[8];
+        bf16x8_to_f32(raw[u], v);
+        if constexpr (kColMult) {
+          // t = fl32(dout * s_r[g(m), n]); rows in no group give t = +0
+          v[0] = __fmul_rn(v[0], cs[u][0].x); v[1] = __fmul_rn(v[1], cs[u][0].y);
+          v[2] = __fmul_rn(v[2], cs[u][0].z); v[3] = __fmul_rn(v[3], cs[u][0].w);
+          v[4] = __fmul_rn(v[4], cs[u][1].x); v[5] = __fmul_rn(v[5], cs[u][1].y);
+          v[6] = __fmul_rn(v[6], cs[u][1].z); v[7] = __fmul_rn(v[7], cs[u][1].w);
+          if (!row_in_group) {
 #pragma unroll
-        for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
-        dyn_scale(amax, s, inv);
-      } else {
-        inv = inv_static;
-      }
-      const bool in_range = base + u < total && cb[u] < cols;
-      if (in_range) {
-        uint2 out;
-        out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
-                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
-        out.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv))) |
-                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
-        *reinterpret_cast<uint2 *>(codes + r[u] * cols + cb[u] + hl * 8) = out;
-        if (kDynamic && hl == 0) scales[(cb[u] / kBlk) * rows + r[u]] = s;
+            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+          }
+        }
+        float s = 0.0f, inv;
+        if constexpr (kDynamic) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+          for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+          dyn_scale(amax, s, inv);
+        } else {
+          inv = inv_static;
+        }
+        if (valid[u]) {
+          uint2 out;
+          out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
+                  (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
+          out.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv))) |
+                  (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
+          *reinterpret_cast<uint2 *>(cr + cb[u] + hl * 8) = out;
+          if (kDynamic && hl == 0) scales[static_cast<int64_t>(cb[u] / kBlk) * rows + r] = s;
+        }
       }
     }
   }
@@ -214,8 +216,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *__
 cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dynamic, const float *static_scale,
                               const float *col_scale, const int *offs, int G, uint8_t *codes, float *scales,
                               uint32_t *status, cudaStream_t st) {
-  const int64_t segs = rows * ((cols + 255) / 256);
-  int64_t blocks = (segs + 8 * kSegs - 1) / (8 * kSegs);
+  int64_t blocks = (rows + 7) / 8;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
@@ -237,21 +238,28 @@ cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dy
 
 // ---------------------------------------------------- chunks (axis 0)
 
-// One CTA per (256-column slice, chunk).  The chunk's rows (at most 128, the
-// rest zero) are staged in shared memory; thread t owns column t: it takes the
-// column's absmax over the chunk and writes the column's 128 codes as one
-// 128-byte line of the transposed code matrix.
+// One CTA of 128 threads per (256-column slice, chunk).  The chunk's rows (at
+// most 128, the rest zero) are staged in shared memory with cp.async; thread t
+// owns the adjacent columns 2t and 2t+1: it takes each column's absmax over the
+// chunk and writes each column's 128 codes as one 128-byte line of the
+// transposed code matrix.
 constexpr int kChunkCols = 256;
+constexpr int kChunkThreads = 128;
 constexpr int kChunkPitch = kChunkCols + 8;  // bf16 per staged row (16-byte aligned rows)
 constexpr size_t kChunkSmem = static_cast<size_t>(kBlk) * kChunkPitch * sizeof(__nv_bfloat16);
 
+__device__ __forceinline__ void cp_async_16_zfill(void *dst_smem, const void *src, bool in_range) {
+  // src-size 0 writes 16 zero bytes without reading
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)), "l"(src),
+               "r"(in_range ? 16 : 0)
+               : "memory");
+}
+
 template <bool kDynamic, bool kCopy>
-__global__ void __launch_bounds__(256) quant_chunks_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
-                                                           int64_t cols, const float *__restrict__ static_scale,
-                                                           const int *__restrict__ offs,
-                                                           const int *__restrict__ tpre, int G, void *codes_t,
-                                                           int64_t ld_t, float *__restrict__ scales,
-                                                           uint32_t *__restrict__ status) {
+__global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ static_scale,
+    const int *__restrict__ offs, const int *__restrict__ tpre, int G, void *codes_t, int64_t ld_t,
+    float *__restrict__ scales, uint32_t *__restrict__ status) {
   extern __shared__ __align__(16) uint8_t qsm[];
   __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(qsm);  // [128][kChunkPitch]
   __shared__ int s_info[3];
@@ -279,63 +287,78 @@ __global__ void __launch_bounds__(256) quant_chunks_kernel(const __nv_bfloat16 *
   const int g = s_info[0];
   if (g < 0) return;
   const int r0 = s_info[1], nr = s_info[2];
-  // 128 rows x 32 sixteen-byte pieces; rows past the chunk and columns past
-  // the matrix read as zero
-#pragma unroll 4
-  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 8); i += 256) {
+  // 128 rows x 32 sixteen-byte pieces, all in flight; rows past the chunk and
+  // columns past the matrix are zero-filled
+  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 8); i += kChunkThreads) {
     const int rr = i >> 5, cc = (i & 31) * 8;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (rr < nr && c0 + cc < cols)
-      u = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc));
-    *reinterpret_cast<uint4 *>(tile + rr * kChunkPitch + cc) = u;
+    const bool in = rr < nr && c0 + cc < cols;
+    const __nv_bfloat16 *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
+    cp_async_16_zfill(tile + rr * kChunkPitch + cc, src, in);
   }
+  cp_async_wait_all();
   __syncthreads();
-  const int col = threadIdx.x;
-  if (c0 + col >= cols) return;
+  const int col = 2 * threadIdx.x;  // and col + 1
+  if (c0 + col >= cols) return;     // cols is a multiple of 128: both columns are in or out
+  const uint32_t *t32 = reinterpret_cast<const uint32_t *>(tile);
+  auto pair = [&](int r) -> float2 {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t32[(r * kChunkPitch + col) >> 1]));
+  };
   if constexpr (kCopy) {
     // bf16 family: transposed bf16 copy, no scale
-    uint16_t *dst = static_cast<uint16_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
+    uint16_t *dst0 = static_cast<uint16_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
+    uint16_t *dst1 = dst0 + ld_t;
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
-      uint32_t w[4];
+      uint32_t w0[4], w1[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint16_t lo = __bfloat16_as_ushort(tile[(q * 8 + 2 * e) * kChunkPitch + col]);
-        const uint16_t hi = __bfloat16_as_ushort(tile[(q * 8 + 2 * e + 1) * kChunkPitch + col]);
-        w[e] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        const uint32_t a = t32[((q * 8 + 2 * e) * kChunkPitch + col) >> 1];
+        const uint32_t b = t32[((q * 8 + 2 * e + 1) * kChunkPitch + col) >> 1];
+        w0[e] = (a & 0xFFFFu) | (b << 16);
+        w1[e] = (a >> 16) | (b & 0xFFFF0000u);
       }
-      *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4 *>(dst0 + q * 8) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+      *reinterpret_cast<uint4 *>(dst1 + q * 8) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
     }
   } else {
-    float s, inv;
+    float s0, s1, inv0, inv1;
     if constexpr (kDynamic) {
-      float amax = 0.0f;
+      float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll 8
-      for (int r = 0; r < kBlk; ++r) amax = fmaxf(amax, fabsf(__bfloat162float(tile[r * kChunkPitch + col])));
-      dyn_scale(amax, s, inv);
+      for (int r = 0; r < kBlk; ++r) {
+        const float2 v = pair(r);
+        a0 = fmaxf(a0, fabsf(v.x));
+        a1 = fmaxf(a1, fabsf(v.y));
+      }
+      dyn_scale(a0, s0, inv0);
+      dyn_scale(a1, s1, inv1);
     } else {
-      s = *static_scale;
+      float s = *static_scale;
       const bool ok = static_scale_ok(s);
-      inv = ok ? __fdiv_rn(1.0f, s) : 0.0f;
+      const float inv = ok ? __fdiv_rn(1.0f, s) : 0.0f;
       if (!ok) s = 0.0f;
       if (!ok && j == 0 && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, GMM_DEV_SCALE);
+      s0 = s1 = s;
+      inv0 = inv1 = inv;
     }
-    uint8_t *dst = static_cast<uint8_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
+    uint8_t *dst0 = static_cast<uint8_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
+    uint8_t *dst1 = dst0 + ld_t;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      uint32_t w[4];
+      uint32_t w0[4], w1[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = q * 16 + e * 4;
-        const float a0 = __fmul_rn(__bfloat162float(tile[r * kChunkPitch + col]), inv);
-        const float a1 = __fmul_rn(__bfloat162float(tile[(r + 1) * kChunkPitch + col]), inv);
-        const float a2 = __fmul_rn(__bfloat162float(tile[(r + 2) * kChunkPitch + col]), inv);
-        const float a3 = __fmul_rn(__bfloat162float(tile[(r + 3) * kChunkPitch + col]), inv);
-        w[e] = static_cast<uint32_t>(cvt_e4m3x2(a0, a1)) | (static_cast<uint32_t>(cvt_e4m3x2(a2, a3)) << 16);
+        const float2 v0 = pair(r), v1 = pair(r + 1), v2 = pair(r + 2), v3 = pair(r + 3);
+        w0[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.x, inv0), __fmul_rn(v1.x, inv0))) |
+                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.x, inv0), __fmul_rn(v3.x, inv0))) << 16);
+        w1[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.y, inv1), __fmul_rn(v1.y, inv1))) |
+                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.y, inv1), __fmul_rn(v3.y, inv1))) << 16);
       }
-      *reinterpret_cast<uint4 *>(dst + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4 *>(dst0 + q * 16) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+      *reinterpret_cast<uint4 *>(dst1 + q * 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
     }
-    scales[static_cast<int64_t>(j) * cols + c0 + col] = s;
+    *reinterpret_cast<float2 *>(scales + static_cast<int64_t>(j) * cols + c0 + col) = make_float2(s0, s1);
   }
 }
 
@@ -347,7 +370,8 @@ static cudaError_t launch_chunks_inst(dim3 grid, cudaStream_t st, const __nv_bfl
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kChunkSmem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, 256, kChunkSmem, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t, scales, status);
+  kern<<<grid, kChunkThreads, kChunkSmem, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t, scales,
+                                                status);
   return cudaGetLastError();
 }
 
