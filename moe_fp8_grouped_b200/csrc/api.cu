@@ -121,6 +121,23 @@ static bool make_map(CUtensorMap *m, const void *base, int elem, uint64_t inner,
   return r == CUDA_SUCCESS;
 }
 
+// Output map for TMA stores: row-major [outer, inner] of f32 or bf16, no
+// swizzle, box [box_outer, box_inner].
+static bool make_out_map(CUtensorMap *m, const void *base, bool f32, uint64_t inner, uint64_t outer,
+                         uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t esz = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * esz};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------ validation
 
 static bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -334,7 +351,7 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1 && dyn};
   const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(prof("gemm_fwd", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
+  if ((s = cuda_status(prof("gemm_fwd", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
     return s;
   g_launches = n + 1;
   return GMM_OK;
@@ -398,7 +415,7 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1};
   const int64_t items = ((M + 127) / 128 + G) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
+  if ((s = cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
     return s;
   g_launches = n + 1;
   return GMM_OK;
@@ -439,6 +456,9 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, P.codes_b, elem, ldt, N, ldt * elem, bke, 128)) return GMM_ERR_CUDA;
   if (!make_map(&tmB, P.codes_a, elem, ldt, K, ldt * elem, bke, 256)) return GMM_ERR_CUDA;
+  CUtensorMap tmOut;  // dW as [G*K, N]: each epilogue warp stores 32 k-rows x 32 n
+  if (!make_out_map(&tmOut, drhs, out_dtype == GMM_F32, N, static_cast<uint64_t>(G) * K, 32, 32))
+    return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
   p.M = static_cast<int>(M);
@@ -462,7 +482,7 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   const GemmConfig cfg{MODE_TGMM, elem, false, elem == 1};
   const int64_t items = static_cast<int64_t>(G) * (N / kBlk) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, p, grid, st); }))) != GMM_OK)
+  if ((s = cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, p, grid, st); }))) != GMM_OK)
     return s;
   g_launches = 4;
   return GMM_OK;

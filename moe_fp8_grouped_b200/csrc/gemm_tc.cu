@@ -61,13 +61,21 @@ constexpr int regs_ctl() { return kPromote ? 40 : 72; }
 template <bool kPromote>
 constexpr int regs_epi() { return kPromote ? 232 : 216; }
 
+// tgmm keeps 3 pipeline stages and uses the freed shared memory to stage its
+// output for TMA stores (one 4 KB block per epilogue warp)
+template <int kMode>
+constexpr int stages_of() { return kMode == MODE_TGMM ? 3 : kStages; }
+constexpr int kStageOut = 4096;  // bytes of output staging per epilogue warp (tgmm)
+
+template <int kMode>
 constexpr size_t gemm_smem_bytes() {
   return 1024                                    // alignment slack
-         + static_cast<size_t>(kStages) * (kAStage + kBStage)
+         + static_cast<size_t>(stages_of<kMode>()) * (kAStage + kBStage)
          + kNumBars * 8                          // mbarriers
          + 16                                    // tmem slot, abort flags
          + kScaleSlots * (kBN + kBM) * sizeof(float)  // scale ring
-         + 2 * (kMaxGroups + 1) * sizeof(int);   // plan copy
+         + 2 * (kMaxGroups + 1) * sizeof(int)    // plan copy
+         + (kMode == MODE_TGMM ? 128 + kEpiWarps * kStageOut : 0);  // + alignment slack
 }
 
 // One work item: tile row index rt (MODE_ROWS: rows r0 .. rend of group g;
@@ -179,7 +187,7 @@ __device__ __forceinline__ void store_col32(void *out, int64_t off_elems, int64_
 template <int kElem, bool kBMN, bool kPromote, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     gmm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const GemmParams p) {
+                  const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   constexpr bool kF16 = (kElem == 2);
   constexpr bool kTg = (kMode == MODE_TGMM);
   constexpr int kBKe = 128 / kElem;                 // contraction elements per stage
@@ -187,15 +195,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBBoxes = kBMN ? 2 * kElem : 1;     // TMA boxes per B stage
   constexpr int kBBoxBytes = kBStage / kBBoxes;
   constexpr uint32_t kIdesc = instr_desc(kF16, kBMN);
+  constexpr int kSt = stages_of<kMode>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
-  uint8_t *sB = smem + kStages * kAStage;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * kBStage);
-  uint64_t *full = bars;                    // [kStages] TMA -> MMA
-  uint64_t *empty = bars + kStages;         // [kStages] MMA -> TMA
-  uint64_t *tfull = bars + 2 * kStages;     // [2] MMA -> epilogue
+  uint8_t *sB = smem + kSt * kAStage;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kSt * kBStage);
+  uint64_t *full = bars;                    // [kSt] TMA -> MMA
+  uint64_t *empty = bars + kSt;         // [kSt] MMA -> TMA
+  uint64_t *tfull = bars + 2 * kSt;     // [2] MMA -> epilogue
   uint64_t *tempty = tfull + 2;             // [2] epilogue -> MMA
   uint64_t *drain = tempty + 2;             // MMA completion at exit
   uint64_t *sfull = drain + 1;              // [kScaleSlots] scale loader -> epilogue
@@ -207,6 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *s_srow = s_scol + kScaleSlots * kBN;                // [kScaleSlots][128] row scales per unit
   int *s_offs = reinterpret_cast<int *>(s_srow + kScaleSlots * kBM);
   int *s_tpre = s_offs + (kMaxGroups + 1);
+  // tgmm output staging, 128-byte aligned (TMA store sources must be aligned)
+  uint8_t *s_stage_out =
+      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(s_tpre + (kMaxGroups + 1)) + 127) & ~uintptr_t(127));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -220,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool use_ring = need_col || need_row;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kSt; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -268,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
         const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
         for (int b = 0; b < t.nblocks; ++b, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, ctl)) {
+          const int s = it % kSt;
+          if (!mbar_wait(&empty[s], ((it / kSt) & 1) ^ 1, ctl)) {
             ok = false;
             break;
           }
@@ -298,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // let every issued copy land before the CTA can exit
-      for (int i = (it > kStages ? it - kStages : 0); i < it; ++i)
-        mbar_wait(&full[i % kStages], (i / kStages) & 1, ctl_drain);
+      for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
+        mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
     } else if (warp == 1) {
       // ----------------------------------------------------- MMA issuer
       if (lane == 0) {
@@ -318,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               tc_fence_after();
             }
-            const int s = it % kStages;
-            if (!mbar_wait(&full[s], (it / kStages) & 1, ctl)) {
+            const int s = it % kSt;
+            if (!mbar_wait(&full[s], (it / kSt) & 1, ctl)) {
               ok = false;
               break;
             }
@@ -438,8 +450,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (!kTg) {
           store_row32(p.out, orow * p.ld_out + col, o, p.out_f32, out_v8);
         } else {
-          store_col32(p.out, (static_cast<int64_t>(t.g) * p.ncols + col) * p.ld_out + orow, p.ld_out, o,
-                      p.out_f32);
+          // the warp's 32 x 32 block of dW[g, col .. col+31, n0 .. n0+31]:
+          // staged row-major (row k, 32 consecutive n) and written by one
+          // TMA store; the buffer is reused once the previous store read it
+          uint8_t *stg = s_stage_out + (warp - kEpiWarp0) * kStageOut;
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          if (p.out_f32) {
+            float *sf = reinterpret_cast<float *>(stg);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sf[j * 32 + lane] = o[j];
+          } else {
+            __nv_bfloat16 *sb = reinterpret_cast<__nv_bfloat16 *>(stg);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sb[j * 32 + lane] = __float2bfloat16_rn(o[j]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, t.rt * kBM + q * 32, t.g * p.ncols + col, stg);
+            bulk_commit();
+          }
         }
       };
       if (t.nblocks == 0) {  // empty group in tgmm: dW tile = 0
@@ -568,6 +599,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         release_slot(slot);
       }
     }
+    if constexpr (kTg) {
+      if (lane == 0) bulk_wait0();  // every dW store of this warp has landed
+      __syncwarp();
+    }
     // rows outside every group are zero (row-ragged passes only)
     if constexpr (!kTg) {
       const int esz = p.out_f32 ? 4 : 2;
@@ -604,10 +639,10 @@ int num_sms() {
 }
 
 template <int kElem, bool kBMN, bool kPromote, int kMode>
-static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p, int grid,
-                               cudaStream_t st) {
+static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
+                               const GemmParams &p, int grid, cudaStream_t st) {
   auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode>;
-  const size_t smem = gemm_smem_bytes();
+  const size_t smem = gemm_smem_bytes<kMode>();
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -617,28 +652,28 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
     return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(tmA, tmB, p);
+  kern<<<grid, kThreads, smem, st>>>(tmA, tmB, tmOut, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                        int grid, cudaStream_t st) {
+cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st) {
   if (cfg.mode == MODE_TGMM) {
     if (cfg.b_mn_major) return cudaErrorInvalidValue;
-    if (cfg.elem_bytes == 1 && cfg.promote) return launch_inst<1, false, true, MODE_TGMM>(tmA, tmB, p, grid, st);
-    if (cfg.elem_bytes == 2 && !cfg.promote) return launch_inst<2, false, false, MODE_TGMM>(tmA, tmB, p, grid, st);
+    if (cfg.elem_bytes == 1 && cfg.promote) return launch_inst<1, false, true, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
+    if (cfg.elem_bytes == 2 && !cfg.promote) return launch_inst<2, false, false, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
     return cudaErrorInvalidValue;
   }
   if (cfg.elem_bytes == 1) {
     if (cfg.b_mn_major)
-      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS>(tmA, tmB, p, grid, st)
-                         : launch_inst<1, true, false, MODE_ROWS>(tmA, tmB, p, grid, st);
-    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS>(tmA, tmB, p, grid, st)
-                       : launch_inst<1, false, false, MODE_ROWS>(tmA, tmB, p, grid, st);
+      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
+                         : launch_inst<1, true, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
+    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
+                       : launch_inst<1, false, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
   }
   if (cfg.promote) return cudaErrorInvalidValue;
-  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS>(tmA, tmB, p, grid, st)
-                        : launch_inst<2, false, false, MODE_ROWS>(tmA, tmB, p, grid, st);
+  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
+                        : launch_inst<2, false, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
 }
 
 }  // namespace gmm

@@ -96,7 +96,9 @@ struct GemmConfig {
 
 int num_sms();
 
+// tmOut: the output as a TMA tensor (MODE_TGMM: dW [G*K, N], box 32 x 32);
+// unused by MODE_ROWS.
 cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const GemmParams &p, int grid, cudaStream_t st);
+                        const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st);
 
 }  // namespace gmm
