@@ -65,7 +65,11 @@ constexpr int regs_epi() { return kPromote ? 232 : 216; }
 // output for TMA stores (one 4 KB block per epilogue warp)
 template <int kMode>
 constexpr int stages_of() { return kMode == MODE_TGMM ? 3 : kStages; }
-constexpr int kStageOut = 4096;  // bytes of output staging per epilogue warp (tgmm)
+constexpr int kStageOut = 4096;  // bytes of one output staging buffer (tgmm); two per epilogue warp
+
+// scale ring slots: tgmm keeps 4 to make room for its output staging
+template <int kMode>
+constexpr int ring_of() { return kMode == MODE_TGMM ? 4 : kScaleSlots; }
 
 template <int kMode>
 constexpr size_t gemm_smem_bytes() {
@@ -73,9 +77,9 @@ constexpr size_t gemm_smem_bytes() {
          + static_cast<size_t>(stages_of<kMode>()) * (kAStage + kBStage)
          + kNumBars * 8                          // mbarriers
          + 16                                    // tmem slot, abort flags
-         + kScaleSlots * (kBN + kBM) * sizeof(float)  // scale ring
+         + ring_of<kMode>() * (kBN + kBM) * sizeof(float)  // scale ring
          + 2 * (kMaxGroups + 1) * sizeof(int)    // plan copy
-         + (kMode == MODE_TGMM ? 128 + kEpiWarps * kStageOut : 0);  // + alignment slack
+         + (kMode == MODE_TGMM ? 128 + kEpiWarps * 2 * kStageOut : 0);  // + alignment slack
 }
 
 // One work item: tile row index rt (MODE_ROWS: rows r0 .. rend of group g;
@@ -196,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBBoxBytes = kBStage / kBBoxes;
   constexpr uint32_t kIdesc = instr_desc(kF16, kBMN);
   constexpr int kSt = stages_of<kMode>();
+  constexpr int kRing = ring_of<kMode>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -207,14 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *tfull = bars + 2 * kSt;     // [2] MMA -> epilogue
   uint64_t *tempty = tfull + 2;             // [2] epilogue -> MMA
   uint64_t *drain = tempty + 2;             // MMA completion at exit
-  uint64_t *sfull = drain + 1;              // [kScaleSlots] scale loader -> epilogue
-  uint64_t *sempty = sfull + kScaleSlots;   // [kScaleSlots] epilogue -> scale loader
+  uint64_t *sfull = drain + 1;              // [kRing] scale loader -> epilogue
+  uint64_t *sempty = sfull + kRing;   // [kRing] epilogue -> scale loader
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *no_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
-  float *s_scol = reinterpret_cast<float *>(tmem_slot + 4);  // [kScaleSlots][256] column scales per unit
-  float *s_srow = s_scol + kScaleSlots * kBN;                // [kScaleSlots][128] row scales per unit
-  int *s_offs = reinterpret_cast<int *>(s_srow + kScaleSlots * kBM);
+  float *s_scol = reinterpret_cast<float *>(tmem_slot + 4);  // [kRing][256] column scales per unit
+  float *s_srow = s_scol + kRing * kBN;                // [kRing][128] row scales per unit
+  int *s_offs = reinterpret_cast<int *>(s_srow + kRing * kBM);
   int *s_tpre = s_offs + (kMaxGroups + 1);
   // tgmm output staging, 128-byte aligned (TMA store sources must be aligned)
   uint8_t *s_stage_out =
@@ -241,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < kScaleSlots; ++i) {
+    for (int i = 0; i < kRing; ++i) {
       mbar_init(&sfull[i], 32);
       mbar_init(&sempty[i], kEpiWarps);
     }
@@ -367,9 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int units = kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0);
         const int64_t ch0 = kTg ? s_tpre[t.g] : 0;
         for (int j = 0; j < units; ++j, ++v) {
-          const int slot = v % kScaleSlots;
+          const int slot = v % kRing;
           bool got = true;
-          if (lane == 0) got = mbar_wait(&sempty[slot], ((v / kScaleSlots) & 1) ^ 1, ctl);
+          if (lane == 0) got = mbar_wait(&sempty[slot], ((v / kRing) & 1) ^ 1, ctl);
           if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
             ok = false;
             break;
@@ -416,6 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_eff = (isfinite(v) && v > 1.17549435e-38f) ? v : 0.0f;
     }
     const bool out_v8 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
+    const uint64_t evict_first = kTg ? l2_policy_evict_first() : 0;  // dW is written once: keep operands in L2
+    int nstore = 0;                                                     // tgmm stores issued by this warp
     int u = 0;  // TMEM units consumed
     int v = 0;  // scale slots consumed
     bool ok = true;
@@ -423,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // epilogue warps on whether to go on
     auto wait_unit = [&](uint32_t buf, int slot) -> bool {
       bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
-      if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kScaleSlots) & 1, ctl);
+      if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kRing) & 1, ctl);
       return epi_bar_and(got);
     };
     auto release_slot = [&](int slot) {
@@ -453,8 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the warp's 32 x 32 block of dW[g, col .. col+31, n0 .. n0+31]:
           // staged row-major (row k, 32 consecutive n) and written by one
           // TMA store; the buffer is reused once the previous store read it
-          uint8_t *stg = s_stage_out + (warp - kEpiWarp0) * kStageOut;
-          if (lane == 0) bulk_wait_read0();
+          uint8_t *stg = s_stage_out + ((warp - kEpiWarp0) * 2 + (nstore & 1)) * kStageOut;
+          ++nstore;
+          if (lane == 0) bulk_wait_read1();  // the store issued from this buffer two stores ago has read it
           __syncwarp();
           if (p.out_f32) {
             float *sf = reinterpret_cast<float *>(stg);
@@ -468,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmOut, t.rt * kBM + q * 32, t.g * p.ncols + col, stg);
+            tma_store_2d_hint(&tmOut, t.rt * kBM + q * 32, t.g * p.ncols + col, stg, evict_first);
             bulk_commit();
           }
         }
@@ -489,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int slot = 0;
         for (int b = 0; b < t.nblocks; ++b) {
           const uint32_t buf = u & 1;
-          slot = v % kScaleSlots;
+          slot = v % kRing;
           if (!wait_unit(buf, slot)) {
             ok = false;
             break;
@@ -564,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         release_slot(slot);
       } else {
         const uint32_t buf = u & 1;
-        const int slot = v % kScaleSlots;
+        const int slot = v % kRing;
         if (!wait_unit(buf, slot)) {
           ok = false;
           break;
