@@ -89,7 +89,9 @@ def algorithmic_bytes(M, K, N, G, G_ne, rule):
     gsc = 0 if rule == "none" else 4 * M * N // 128
     return {"fwd": 2 * M * K + lsc + wb * G_ne * K * N + wsc + 2 * M * N,
             "dlhs": 2 * M * N + gsc + wb * G_ne * K * N + wsc + 2 * M * K,
-            "drhs": 2 * M * K + 2 * M * N + 4 * G * K * N}
+            "drhs": 2 * M * K + 2 * M * N + 4 * G * K * N,
+            # merged gate|up forward with SwiGLU fused: the [M, N/2] bf16 result only
+            "fwd_swiglu": 2 * M * K + lsc + wb * G_ne * K * N + wsc + M * N}
 
 
 def config_of(w, extra=None):
@@ -304,6 +306,38 @@ def run_ours(args):
                     "peak_source": f"{peak_src} HBM copy bandwidth",
                     "algorithmic": f"{bytes_pass[dname]:.4g} bytes per launch (operands in, results out)"}
     roofline["traffic"] = traffic_record(dom)
+
+    # merged gate|up workloads: the forward with SwiGLU fused into its
+    # epilogue, timed on its own (not part of the step), with an L2 flush
+    # (a 256 MiB write) before each call
+    if w.merged and parts == 1:
+        sw_out = torch.empty((M, N // 2), dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+        def swiglu_call():
+            gm.gmm_fwd_swiglu(lhs, codes, rscales, gs, rule=rule, static_scale=sarg, out=sw_out, ws=ws)
+
+        for _ in range(3):
+            swiglu_call()
+        barrier()
+        gm.profile_enable(True)
+        for _ in range(min(args.steps, 20)):
+            flush.zero_()
+            swiglu_call()
+        barrier()
+        gm.profile_enable(False)
+        n, tot = gm.profile_collect().get("gemm_fwd_swiglu", (0, 0.0))
+        if n:
+            avg = tot / n
+            tfl = flops_pass / (avg / 1e3) / 1e12
+            gbs = bytes_pass["fwd_swiglu"] / (avg / 1e3) / 1e9
+            floor_ms = max(flops_pass / (peak_tc * 1e12), bytes_pass["fwd_swiglu"] / (peak_bw * 1e9)) * 1e3
+            passes["fwd_swiglu"] = {"gemm_ms": round(avg, 4), "gemm_tflops": round(tfl, 1),
+                                    "gb_per_s": round(gbs, 1), "frac_tensor": round(tfl / peak_tc, 4),
+                                    "frac_hbm": round(gbs / peak_bw, 4), "frac_roofline": round(floor_ms / avg, 4),
+                                    "note": "gmm_fwd_swiglu: out[M, N/2] = silu(gate) * up of the merged "
+                                            "product; timed apart from the step, L2 flushed per call"}
+        del sw_out, flush
 
     # end to end: pinned host buffers, copies inside the timed region.  Steps
     # are pipelined over three streams (upload, compute, download) with two

@@ -157,6 +157,24 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
                    void *stream);
 
 /*
+ * Forward gmm of the merged gate|up weights with the SwiGLU activation fused
+ * into its epilogue ("FP8 Megablox for batch split", maxtext PR #3770,
+ * Description (2): W0 and W1 are concatenated so that one gmm call covers
+ * both projections; SwiGLU is the activation they feed).  rhs is the merged
+ * buffer W = [W0 | W1] along N, exactly as for the merged gmm_fwd call, with
+ * N = 2F and F a multiple of 128.  Every other argument is gmm_fwd's.
+ * out: [M, F] of out_dtype:
+ *   out[m, j] = silu(h[m, j]) * h[m, F + j],  silu(z) = z / (1 + exp(-z)),
+ * where h = gmm_fwd(lhs, rhs) is the merged product, computed in fp32 and
+ * never written to memory.  Rows outside every group are 0.  N not a multiple
+ * of 256 returns GMM_ERR_SHAPE.  Workspace: gmm_workspace_bytes(GMM_OP_FWD,
+ * M, K, N, G) with the merged N.
+ */
+gmm_status gmm_fwd_swiglu(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes,
+                          int32_t G, int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws,
+                          size_t ws_bytes, void *stream);
+
+/*
  * Forward gmm without a workspace argument, for callers that cannot allocate
  * device memory: code that runs where cudaMalloc is not allowed (a host
  * function enqueued on a stream), or that runs under a runtime which owns all
@@ -195,7 +213,14 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
  * Transposed gmm (weight gradient).  lhs: bf16 [M, K] with rule STATIC (the
  * forward's static scale, giving the forward's codes) or DYNAMIC; dout: bf16
  * [M, N], rule DYNAMIC (or both NONE for the bf16 family).  Both are
- * quantized per 128-row chunk of each group (axis 0 above).
+ * quantized per 128-row chunk of each group (axis 0 above).  With the static
+ * rule lhs may instead be the E4M3 codes [M, K] the forward used (from
+ * gmm_quantize, axis 1, or passed to gmm_fwd pre-quantized) with lhs.scale
+ * the same static scale: the codes are only re-laid out, not quantized again
+ * ("add static LHS scaling support for GMM v2 FWD", maxtext PR #4735, rebase
+ * commit text: activations quantized once, ahead of the pass that uses them).
+ * A pre-quantized lhs with rule DYNAMIC returns GMM_ERR_INVALID_ARG (its
+ * blocks run along K, the tgmm's along rows).
  * drhs: [G, K, N] of out_dtype (F32 or BF16):
  *   dW[g, k, n] = sum_c s_x[c, k] * s_d[c, n] * sum_{m in chunk c} q_x[m, k] * q_d[m, n]
  * Empty groups get dW[g] = 0.

@@ -185,8 +185,9 @@ static gmm_status classify(const gmm_operand &x, const gmm_operand &w, bool w_is
   }
   if (x.rule != GMM_Q_STATIC && x.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
   if (x.dtype == GMM_E4M3) {
-    // pre-quantized lhs (forward only): its scales come with it
-    if (!w_is_rhs || !x.scale) return GMM_ERR_INVALID_ARG;
+    // pre-quantized lhs: its scales come with it (the forward takes either
+    // rule, the tgmm the static one only)
+    if (!x.scale || (!w_is_rhs && x.rule != GMM_Q_STATIC)) return GMM_ERR_INVALID_ARG;
   } else if (x.dtype != GMM_BF16) {
     return GMM_ERR_INVALID_ARG;
   }
@@ -294,13 +295,17 @@ gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrul
   return s;
 }
 
-gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
-                   int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
-                   void *stream) {
+}  // extern "C"
+
+// Forward pass shared by gmm_fwd (F == 0) and gmm_fwd_swiglu (F = N / 2).
+static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
+                           int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                           void *stream, int64_t F) {
   g_launches = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   gmm_status s = check_sizes(M, K, N, G);
   if (s != GMM_OK) return s;
+  if (F && N != 2 * F) return GMM_ERR_SHAPE;
   if (!group_sizes || !out) return GMM_ERR_INVALID_ARG;
   if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
   int elem = 0;
@@ -328,13 +333,16 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   const uint32_t bke = 128 / elem;
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, A, elem, K, M, K * elem, bke, 128)) return GMM_ERR_CUDA;
+  // SwiGLU tiles take the gate rows and the up rows of a K-major rhs as two
+  // 128-row boxes
   const bool okB = bmn ? make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, bke)
-                       : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, 256);
+                       : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, F ? 128 : 256);
   if (!okB) return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
   p.M = static_cast<int>(M);
   p.ncols = static_cast<int>(N);
+  p.swiglu_f = static_cast<int>(F);
   p.kblocks = static_cast<int>(K / bke);
   p.b_group_rows = static_cast<int>(bmn ? K : N);
   p.offs = P.offs;
@@ -345,16 +353,33 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
   p.static_scale = (elem == 1 && !dyn) ? lhs.scale : nullptr;
   p.out = out;
   p.out_f32 = out_dtype == GMM_F32;
-  p.ld_out = N;
+  p.ld_out = F ? F : N;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
   const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1 && dyn};
   const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(prof("gemm_fwd", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
+  if ((s = cuda_status(prof(F ? "gemm_fwd_swiglu" : "gemm_fwd", st,
+                            [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
     return s;
   g_launches = n + 1;
   return GMM_OK;
+}
+
+extern "C" {
+
+gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
+                   int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                   void *stream) {
+  return fwd_impl(lhs, rhs, transpose_rhs, group_sizes, G, M, K, N, out, out_dtype, ws, ws_bytes, stream, 0);
+}
+
+gmm_status gmm_fwd_swiglu(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes,
+                          int32_t G, int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws,
+                          size_t ws_bytes, void *stream) {
+  g_launches = 0;
+  if (N <= 0 || N % (2 * kBlk)) return GMM_ERR_SHAPE;
+  return fwd_impl(lhs, rhs, transpose_rhs, group_sizes, G, M, K, N, out, out_dtype, ws, ws_bytes, stream, N / 2);
 }
 
 gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
@@ -439,10 +464,15 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
   const int64_t cap = chunk_capacity(M, G);
   const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
-  s = cuda_status(prof("quant_chunks", st, [&] {
-    return launch_quant_chunks(lhs.data, M, K, dyn, (elem == 1 && !dyn) ? lhs.scale : nullptr, P.offs, P.tpre, G,
-                               cap, P.codes_a, P.scales_a, elem == 2, P.status, st);
-  }));
+  if (lhs.dtype == GMM_E4M3)  // static codes given: re-laid out only
+    s = cuda_status(prof("chunk_codes", st, [&] {
+      return launch_chunk_codes(static_cast<const uint8_t *>(lhs.data), M, K, P.offs, P.tpre, G, cap, P.codes_a, st);
+    }));
+  else
+    s = cuda_status(prof("quant_chunks", st, [&] {
+      return launch_quant_chunks(lhs.data, M, K, dyn, (elem == 1 && !dyn) ? lhs.scale : nullptr, P.offs, P.tpre, G,
+                                 cap, P.codes_a, P.scales_a, elem == 2, P.status, st);
+    }));
   if (s != GMM_OK) return s;
   s = cuda_status(prof("quant_chunks", st, [&] {
     return launch_quant_chunks(dout.data, M, N, true, nullptr, P.offs, P.tpre, G, cap, P.codes_b, P.scales_b,

@@ -33,6 +33,13 @@
 //   promote == true   one TMEM unit per 128-long contraction block; the
 //                     epilogue accumulates acc += unit * row_scale (* the
 //                     block's column scale for dynamic-lhs tgmm) in registers.
+//
+// SwiGLU (forward only, p.swiglu_f = F > 0): the rhs holds the gate and up
+// weights side by side, W = [W0 | W1] along N = 2F ("FP8 Megablox for batch
+// split", maxtext PR #3770, Description (2): the merged gating gmm).  A tile
+// takes 128 gate columns and the same 128 up columns (two B boxes), so one
+// thread holds matching gate and up results and writes silu(gate) * up into
+// out[M, F]; the 2F-wide product never reaches memory.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -88,6 +95,16 @@ constexpr size_t gemm_smem_bytes() {
 struct Item {
   int g, rt, ct, nblocks, r0, rend;
 };
+
+// Column of the (2-D view of the) rhs held by tile column c (0 .. 255) of
+// column tile ct: plain tiles are 256 consecutive columns; SwiGLU tiles are
+// gate columns 128 ct .. 128 ct + 127, then up columns F + 128 ct ..
+__device__ __forceinline__ int tile_col_n(int ct, int c, int F) {
+  return F ? (c < 128 ? 128 * ct + c : F + 128 * ct + (c - 128)) : kBN * ct + c;
+}
+
+// x * sigmoid(x); -0 for large negative x, where exp(-x) overflows
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 
 template <int kMode>
 __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const int *s_offs, const int *s_tpre,
@@ -309,9 +326,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             by = t.ct * kBN;                     // lhs columns k
           }
           tma_load_2d(sA + s * kAStage, &tmA, ax, ay, &full[s]);
+          if constexpr (kBMN) {
+            // boxes of 128 bytes along n (columns of W[g] in [K, N])
 #pragma unroll
-          for (int h = 0; h < kBBoxes; ++h)
-            tma_load_2d(sB + s * kBStage + h * kBBoxBytes, &tmB, bx + (kBMN ? h * kBKe : 0), by, &full[s]);
+            for (int h = 0; h < kBBoxes; ++h)
+              tma_load_2d(sB + s * kBStage + h * kBBoxBytes, &tmB, tile_col_n(t.ct, h * kBKe, p.swiglu_f), by,
+                          &full[s]);
+          } else if (!kTg && p.swiglu_f) {
+            // two boxes of 128 rows (n) of W[g] in [N, K]: gate rows, up rows
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tma_load_2d(sB + s * kBStage + h * (kBStage / 2), &tmB, bx,
+                          t.g * p.b_group_rows + tile_col_n(t.ct, h * 128, p.swiglu_f), &full[s]);
+          } else {
+            tma_load_2d(sB + s * kBStage, &tmB, bx, by, &full[s]);
+          }
         }
       }
       // let every issued copy land before the CTA can exit
@@ -382,7 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // cp.async straight into the slot: the loader never waits for the
           // data, the slot's barrier completes when all 32 lanes' copies land
           if (need_col) {
-            const int n = t.ct * kBN + 8 * lane;  // 8 columns per lane; columns >= ncols are never read
+            // 8 columns per lane (never straddling a gate / up boundary);
+            // columns >= ncols are never read
+            const int n = kTg ? t.ct * kBN + 8 * lane : tile_col_n(t.ct, 8 * lane, p.swiglu_f);
             if (n < p.ncols) {
               const float *src = kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
                                      : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n;
@@ -414,11 +445,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
     const int q = warp & 3, h = (warp - kEpiWarp0) >> 2;
     const int row = q * 32 + lane;
-    const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
+    const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);  // the warp's TMEM lanes
+    const bool sw = !kTg && p.swiglu_f > 0;
+    // tile column of the thread's 32-column chunk c (0 .. 3): the column half h
+    // of the tile, or for SwiGLU gate columns 64 h .. (c = 0, 1) and the
+    // matching up columns 128 + 64 h .. (c = 2, 3)
+    auto colt = [&](int c) -> int { return sw ? ((c & 2) ? 128 : 0) + h * 64 + (c & 1) * 32 : h * 128 + c * 32; };
     float s_eff = 1.0f;
     if (p.static_scale) {
       const float v = *p.static_scale;
       s_eff = (isfinite(v) && v > 1.17549435e-38f) ? v : 0.0f;
+      // reported here too for operands quantized before the call
+      if (s_eff == 0.0f && blockIdx.x == 0 && et == 0) atomicOr(p.status, GMM_DEV_SCALE);
     }
     const bool out_v8 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
     const uint64_t evict_first = kTg ? l2_policy_evict_first() : 0;  // dW is written once: keep operands in L2
@@ -426,12 +464,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int u = 0;  // TMEM units consumed
     int v = 0;  // scale slots consumed
     bool ok = true;
-    // waits for TMEM unit u (and its scale slot), then agrees with the other
-    // epilogue warps on whether to go on
+    // waits for TMEM unit u (and its scale slot); the decision is uniform
+    // within the warp.  Warps decide on their own: one that stops raises the
+    // abort flag, which ends every other warp's next wait, and no barrier
+    // among the epilogue warps is ever entered after that point.
     auto wait_unit = [&](uint32_t buf, int slot) -> bool {
       bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
       if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kRing) & 1, ctl);
-      return epi_bar_and(got);
+      return __all_sync(0xffffffffu, got);
     };
     auto release_slot = [&](int slot) {
       if (use_ring) {
@@ -505,12 +545,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float rs = s_srow[slot * kBM + row];
           const float2 rs2 = make_float2(rs, rs);
-          const float *cb = s_scol + slot * kBN + h * 128;
+          const float *cs = s_scol + slot * kBN;
 #pragma unroll
           for (int cp = 0; cp < 2; ++cp) {
+            // chunks 2 cp, 2 cp + 1 (compile-time accumulator indices)
             uint32_t va[32], vb[32];
-            tmem_ld32(tl + buf * kBN + (2 * cp) * 32, va);
-            tmem_ld32(tl + buf * kBN + (2 * cp + 1) * 32, vb);
+            tmem_ld32(tl + buf * kBN + colt(2 * cp), va);
+            tmem_ld32(tl + buf * kBN + colt(2 * cp + 1), vb);
             tmem_wait_ld();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -527,9 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // along the columns k
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                  const float4 cs = *reinterpret_cast<const float4 *>(cb + c * 32 + 4 * i);
-                  const float2 c01 = __fmul2_rn(make_float2(cs.x, cs.y), rs2);
-                  const float2 c23 = __fmul2_rn(make_float2(cs.z, cs.w), rs2);
+                  const float4 c4 = *reinterpret_cast<const float4 *>(cs + colt(c) + 4 * i);
+                  const float2 c01 = __fmul2_rn(make_float2(c4.x, c4.y), rs2);
+                  const float2 c23 = __fmul2_rn(make_float2(c4.z, c4.w), rs2);
                   acc[c * 16 + 2 * i] = __ffma2_rn(
                       make_float2(__uint_as_float(vv[4 * i]), __uint_as_float(vv[4 * i + 1])), c01,
                       acc[c * 16 + 2 * i]);
@@ -551,22 +592,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           // forward: the rhs column scale (in every unit's slot); static tgmm: s
           const float fin = (kTg && p.static_scale) ? s_eff : 1.0f;
           const bool colmul = !kTg && need_col;
-          const float *cf = s_scol + slot * kBN + h * 128;
+          const float *cf = s_scol + slot * kBN;
+          if (sw) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (col0 + c * 32 >= p.ncols) continue;
-            float o[32];
+            for (int c = 0; c < 2; ++c) {
+              const float *fg = cf + colt(c), *fu = cf + colt(c + 2);
+              float o[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float2 a = acc[c * 16 + i];
-              if (colmul) {
-                a.x *= cf[c * 32 + 2 * i];
-                a.y *= cf[c * 32 + 2 * i + 1];
+              for (int i = 0; i < 16; ++i) {
+                const float2 a = acc[c * 16 + i], b2 = acc[(c + 2) * 16 + i];
+                o[2 * i] = silu(a.x * fg[2 * i]) * (b2.x * fu[2 * i]);
+                o[2 * i + 1] = silu(a.y * fg[2 * i + 1]) * (b2.y * fu[2 * i + 1]);
               }
-              o[2 * i] = a.x * fin;
-              o[2 * i + 1] = a.y * fin;
+              emit(t.ct * 128 + h * 64 + c * 32, o);
             }
-            emit(col0 + c * 32, o);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int col = t.ct * kBN + colt(c);
+              if (col >= p.ncols) continue;
+              float o[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float2 a = acc[c * 16 + i];
+                if (colmul) {
+                  a.x *= cf[colt(c) + 2 * i];
+                  a.y *= cf[colt(c) + 2 * i + 1];
+                }
+                o[2 * i] = a.x * fin;
+                o[2 * i + 1] = a.y * fin;
+              }
+              emit(col, o);
+            }
           }
         }
         release_slot(slot);
@@ -579,25 +636,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const float s0 = p.static_scale ? s_eff : 1.0f;
-        const float *cf = s_scol + slot * kBN + h * 128;
+        const float *cf = s_scol + slot * kBN;
 #pragma unroll
         for (int cp = 0; cp < 2; ++cp) {
+          const int ca = sw ? cp : 2 * cp, cb = sw ? cp + 2 : 2 * cp + 1;
           uint32_t va[32], vb[32];
-          tmem_ld32(tl + buf * kBN + (2 * cp) * 32, va);
-          tmem_ld32(tl + buf * kBN + (2 * cp + 1) * 32, vb);
+          tmem_ld32(tl + buf * kBN + colt(ca), va);
+          tmem_ld32(tl + buf * kBN + colt(cb), vb);
           tmem_wait_ld();
+          if (sw) {
+            if (row_ok) {
+              const float *fg = cf + colt(ca), *fu = cf + colt(cb);
+              float o[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float gs = need_col ? fg[i] : 1.0f, us = need_col ? fu[i] : 1.0f;
+                o[i] = silu(__uint_as_float(va[i]) * s0 * gs) * (__uint_as_float(vb[i]) * s0 * us);
+              }
+              emit(t.ct * 128 + h * 64 + cp * 32, o);
+            }
+            continue;
+          }
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const uint32_t *vv = half ? vb : va;
-            const int c = 2 * cp + half;
-            if (!row_ok || col0 + c * 32 >= p.ncols) continue;
+            const int c = half ? cb : ca;
+            const int col = t.ct * kBN + colt(c);
+            if (!row_ok || col >= p.ncols) continue;
             float o[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float cs = need_col ? cf[c * 32 + i] : 1.0f;
-              o[i] = __uint_as_float(vv[i]) * s0 * cs;
+              const float cs1 = need_col ? cf[colt(c) + i] : 1.0f;
+              o[i] = __uint_as_float(vv[i]) * s0 * cs1;
             }
-            emit(col0 + c * 32, o);
+            emit(col, o);
           }
         }
         tc_fence_before();
@@ -615,7 +687,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (!kTg) {
       const int esz = p.out_f32 ? 4 : 2;
       const int64_t tail0 = s_offs[p.G];
-      const int64_t cpr = static_cast<int64_t>(p.ncols) * esz / 16;  // 16-byte chunks per row
+      const int64_t out_w = sw ? p.swiglu_f : p.ncols;           // output columns
+      const int64_t cpr = out_w * esz / 16;                      // 16-byte chunks per row
       const int64_t n = (static_cast<int64_t>(p.M) - tail0) * cpr;
       for (int64_t i = static_cast<int64_t>(blockIdx.x) * kEpiThreads + et; i < n;
            i += static_cast<int64_t>(gridDim.x) * kEpiThreads) {

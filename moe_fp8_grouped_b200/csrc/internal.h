@@ -52,6 +52,11 @@ cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool 
                                 const int *offs, const int *tpre, int G, int64_t capacity, void *codes_t,
                                 float *scales, bool bf16_copy, uint32_t *status, cudaStream_t st);
 
+// Already-quantized E4M3 rows [rows, cols] into the chunk layout of
+// launch_quant_chunks (codes only).
+cudaError_t launch_chunk_codes(const uint8_t *codes, int64_t rows, int64_t cols, const int *offs, const int *tpre,
+                               int G, int64_t capacity, uint8_t *codes_t, cudaStream_t st);
+
 cudaError_t launch_quant_rhs(const void *w, int G, int64_t K, int64_t N, bool transpose_out, uint8_t *codes,
                              float *scales, cudaStream_t st);
 
@@ -83,6 +88,9 @@ struct GemmParams {
   void *out;
   int out_f32;
   int64_t ld_out;             // MODE_ROWS: output row pitch; MODE_TGMM: N
+  int swiglu_f;               // MODE_ROWS forward: F > 0 fuses SwiGLU over the merged
+                              // columns [0, F) gate | [F, 2F) up and writes [M, F];
+                              // 0 writes the plain product
   uint32_t *status;
   uint64_t wait_limit_ns;
 };

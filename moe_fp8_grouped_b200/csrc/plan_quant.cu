@@ -255,6 +255,22 @@ __device__ __forceinline__ void cp_async_16_zfill(void *dst_smem, const void *sr
                : "memory");
 }
 
+// Chunk j (over all groups, in group order): first row r0 and row count nr;
+// false when j is past the last chunk.
+__device__ __forceinline__ bool find_chunk(int j, const int *offs, const int *tpre, int G, int &r0, int &nr) {
+  if (j >= tpre[G]) return false;
+  int lo = 0, hi = G + 1;  // first i with tpre[i] > j
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (tpre[mid] > j) hi = mid;
+    else lo = mid + 1;
+  }
+  const int g = lo - 1;
+  r0 = offs[g] + kBlk * (j - tpre[g]);
+  nr = min(r0 + kBlk, offs[g + 1]) - r0;
+  return true;
+}
+
 template <bool kDynamic, bool kCopy>
 __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
     const __nv_bfloat16 *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ static_scale,
@@ -265,27 +281,9 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
   __shared__ int s_info[3];
   const int j = blockIdx.y;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kChunkCols;
-  if (threadIdx.x == 0) {
-    int g = -1;
-    if (j < tpre[G]) {
-      int lo = 0, hi = G + 1;  // first i with tpre[i] > j
-      while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if (tpre[mid] > j) hi = mid;
-        else lo = mid + 1;
-      }
-      g = lo - 1;
-    }
-    s_info[0] = g;
-    if (g >= 0) {
-      const int r0 = offs[g] + kBlk * (j - tpre[g]);
-      s_info[1] = r0;
-      s_info[2] = min(r0 + kBlk, offs[g + 1]) - r0;
-    }
-  }
+  if (threadIdx.x == 0) s_info[0] = find_chunk(j, offs, tpre, G, s_info[1], s_info[2]) ? 1 : 0;
   __syncthreads();
-  const int g = s_info[0];
-  if (g < 0) return;
+  if (!s_info[0]) return;
   const int r0 = s_info[1], nr = s_info[2];
   // 128 rows x 32 sixteen-byte pieces, all in flight; rows past the chunk and
   // columns past the matrix are zero-filled
@@ -389,6 +387,59 @@ cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool 
                                            scales, status);
   return launch_chunks_inst<false, false>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t,
                                           scales, status);
+}
+
+// Already-quantized E4M3 lhs (static rule): its codes laid out as the chunk
+// quantizer lays out the codes it makes (transposed, padded, zero pad rows),
+// bytes copied unchanged.  Same CTA shape as quant_chunks_kernel.
+constexpr int kCodePitch = kChunkCols + 16;  // bytes per staged row (16-byte aligned rows)
+
+__global__ void __launch_bounds__(kChunkThreads) chunk_codes_kernel(const uint8_t *__restrict__ x, int64_t cols,
+                                                                    const int *__restrict__ offs,
+                                                                    const int *__restrict__ tpre, int G,
+                                                                    uint8_t *__restrict__ codes_t, int64_t ld_t) {
+  __shared__ __align__(16) uint8_t tile[kBlk * kCodePitch];
+  __shared__ int s_info[3];
+  const int j = blockIdx.y;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kChunkCols;
+  if (threadIdx.x == 0) s_info[0] = find_chunk(j, offs, tpre, G, s_info[1], s_info[2]) ? 1 : 0;
+  __syncthreads();
+  if (!s_info[0]) return;
+  const int r0 = s_info[1], nr = s_info[2];
+  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 16); i += kChunkThreads) {
+    const int rr = i >> 4, cc = (i & 15) * 16;
+    const bool in = rr < nr && c0 + cc < cols;
+    const uint8_t *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
+    cp_async_16_zfill(tile + rr * kCodePitch + cc, src, in);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int col = 2 * threadIdx.x;  // and col + 1
+  if (c0 + col >= cols) return;     // cols is a multiple of 128: both columns are in or out
+  uint8_t *dst0 = codes_t + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
+  uint8_t *dst1 = dst0 + ld_t;
+  auto pair = [&](int r) -> uint32_t { return *reinterpret_cast<const uint16_t *>(tile + r * kCodePitch + col); };
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint32_t w0[4], w1[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = q * 16 + e * 4;
+      const uint32_t a = pair(r), b = pair(r + 1), c = pair(r + 2), d = pair(r + 3);
+      w0[e] = (a & 0xFFu) | ((b & 0xFFu) << 8) | ((c & 0xFFu) << 16) | ((d & 0xFFu) << 24);
+      w1[e] = (a >> 8) | ((b >> 8) << 8) | ((c >> 8) << 16) | ((d >> 8) << 24);
+    }
+    *reinterpret_cast<uint4 *>(dst0 + q * 16) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    *reinterpret_cast<uint4 *>(dst1 + q * 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  }
+}
+
+cudaError_t launch_chunk_codes(const uint8_t *codes, int64_t rows, int64_t cols, const int *offs, const int *tpre,
+                               int G, int64_t capacity, uint8_t *codes_t, cudaStream_t st) {
+  (void)rows;  // rows past the plan are never read
+  dim3 grid(static_cast<unsigned>((cols + kChunkCols - 1) / kChunkCols), static_cast<unsigned>(capacity));
+  chunk_codes_kernel<<<grid, kChunkThreads, 0, st>>>(codes, cols, offs, tpre, G, codes_t, capacity * kBlk);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------ rhs (K7)

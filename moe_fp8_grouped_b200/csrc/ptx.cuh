@@ -209,25 +209,7 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
 
 namespace gmm {
 
-// ------------------------------------------------ named barrier, registers
-
-// Barrier 1 over the 256 epilogue threads.
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-// Barrier 1 over the 256 epilogue threads that also ANDs a predicate across
-// them, so that every epilogue warp takes the same continue / stop decision.
-__device__ __forceinline__ bool epi_bar_and(bool p) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred ip, op;\n\t"
-      "setp.ne.u32 ip, %1, 0;\n\t"
-      "bar.red.and.pred op, 1, 256, ip;\n\t"
-      "selp.u32 %0, 1, 0, op;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(p))
-      : "memory");
-  return r != 0;
-}
+// ------------------------------------------------------------- registers
 
 template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {

@@ -141,6 +141,23 @@ def gmm_fwd(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | Non
     runs the bf16 family (rhs bf16, no scales).  A uint8 / float8 ``lhs`` is
     taken as already-quantized E4M3 codes: its scale is ``static_scale``
     (static) or ``lhs_scales`` [K/128, M] (dynamic, as gmm_quantize writes)."""
+    return _fwd(lhs, rhs, rhs_scales, group_sizes, rule, static_scale, transpose_rhs, out_dtype, out, ws,
+                lhs_scales, swiglu=False)
+
+
+def gmm_fwd_swiglu(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | None,
+                   group_sizes: torch.Tensor, rule="static", static_scale: torch.Tensor | None = None,
+                   transpose_rhs: bool = False, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                   ws: torch.Tensor | None = None, lhs_scales: torch.Tensor | None = None):
+    """Merged gate|up forward with SwiGLU fused: rhs is [W0 | W1] along N
+    (N = 2F); returns out[M, F] = silu(h[:, :F]) * h[:, F:] with h the merged
+    product, which is never written.  Arguments as for gmm_fwd."""
+    return _fwd(lhs, rhs, rhs_scales, group_sizes, rule, static_scale, transpose_rhs, out_dtype, out, ws,
+                lhs_scales, swiglu=True)
+
+
+def _fwd(lhs, rhs, rhs_scales, group_sizes, rule, static_scale, transpose_rhs, out_dtype, out, ws, lhs_scales,
+         swiglu):
     M, K = lhs.shape
     if transpose_rhs:
         G, N, K2 = rhs.shape
@@ -149,7 +166,7 @@ def gmm_fwd(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | Non
     assert K2 == K, "lhs / rhs contraction mismatch"
     r = _rule(rule)
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=lhs.device)
+        out = torch.empty((M, N // 2 if swiglu else N), dtype=out_dtype, device=lhs.device)
     if ws is None:
         ws = workspace(gmm_workspace_bytes(B.OP_FWD, M, K, N, G), lhs.device)
     if lhs.dtype in (torch.uint8, torch.float8_e4m3fn):
@@ -160,10 +177,11 @@ def gmm_fwd(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | Non
                      _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None, r)
     b = _operand(_dev(rhs, "rhs"), _TORCH_DT[rhs.dtype],
                  _dev(rhs_scales, "rhs_scales", torch.float32) if rhs_scales is not None else None, B.Q_NONE)
-    st = B.lib().gmm_fwd(a, b, int(transpose_rhs), _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,
-                         _dev(out, "out", (torch.bfloat16, torch.float32)), _TORCH_DT[out.dtype], ws.data_ptr(),
-                         ws.numel(), _stream(lhs))
-    _check(st, "gmm_fwd")
+    fn = B.lib().gmm_fwd_swiglu if swiglu else B.lib().gmm_fwd
+    st = fn(a, b, int(transpose_rhs), _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,
+            _dev(out, "out", (torch.bfloat16, torch.float32)), _TORCH_DT[out.dtype], ws.data_ptr(),
+            ws.numel(), _stream(lhs))
+    _check(st, "gmm_fwd_swiglu" if swiglu else "gmm_fwd")
     return out
 
 
@@ -197,7 +215,9 @@ def tgmm_drhs(lhs: torch.Tensor, dout: torch.Tensor, group_sizes: torch.Tensor, 
               static_scale: torch.Tensor | None = None, out_dtype=torch.float32, out: torch.Tensor | None = None,
               ws: torch.Tensor | None = None):
     """Weight gradient dW[g] = lhs[rows of g]^T @ dout[rows of g] ([G, K, N]),
-    both operands quantized per 128-row chunk of each group."""
+    both operands quantized per 128-row chunk of each group.  With rule
+    "static" a uint8 / float8 ``lhs`` is taken as the forward's E4M3 codes
+    (scale ``static_scale``) and only re-laid out."""
     M, K = lhs.shape
     M2, N = dout.shape
     assert M2 == M
@@ -207,8 +227,11 @@ def tgmm_drhs(lhs: torch.Tensor, dout: torch.Tensor, group_sizes: torch.Tensor, 
         out = torch.empty((G, K, N), dtype=out_dtype, device=lhs.device)
     if ws is None:
         ws = workspace(gmm_workspace_bytes(B.OP_DRHS, M, K, N, G), lhs.device)
-    a = _operand(_dev(lhs, "lhs", torch.bfloat16), B.DT_BF16,
-                 _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None, r)
+    sc = _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None
+    if lhs.dtype in (torch.uint8, torch.float8_e4m3fn):
+        a = _operand(_dev(lhs, "lhs"), B.DT_E4M3, sc, r)
+    else:
+        a = _operand(_dev(lhs, "lhs", torch.bfloat16), B.DT_BF16, sc, r)
     d = _operand(_dev(dout, "dout", torch.bfloat16), B.DT_BF16, None, B.Q_NONE if r == B.Q_NONE else B.Q_DYNAMIC)
     st = B.lib().tgmm_drhs(a, d, _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,
                            _dev(out, "out", (torch.bfloat16, torch.float32)), _TORCH_DT[out.dtype], ws.data_ptr(),

@@ -45,6 +45,7 @@ class Workload:
     routing: str
     tokens: int = 0
     topk: int = 0
+    merged: bool = False  # N holds the gate and up projections side by side (N = 2F)
 
     @property
     def flops_per_pass(self) -> int:
@@ -53,11 +54,12 @@ class Workload:
 
 
 WORKLOADS = {
-    "tiny": Workload("tiny", 8, 256, 512, 512, "static", "uniform_empty3"),
-    "mixtral": Workload("mixtral", 8, 16384, 4096, 28672, "static", "topk_uniform", tokens=8192, topk=2),
-    "dsv3_up": Workload("dsv3_up", 256, 32768, 7168, 4096, "dynamic", "zipf", tokens=4096, topk=8),
+    "tiny": Workload("tiny", 8, 256, 512, 512, "static", "uniform_empty3", merged=True),
+    "mixtral": Workload("mixtral", 8, 16384, 4096, 28672, "static", "topk_uniform", tokens=8192, topk=2,
+                        merged=True),
+    "dsv3_up": Workload("dsv3_up", 256, 32768, 7168, 4096, "dynamic", "zipf", tokens=4096, topk=8, merged=True),
     "dsv3_down": Workload("dsv3_down", 256, 32768, 2048, 7168, "dynamic", "zipf", tokens=4096, topk=8),
-    "ep_merged": Workload("ep_merged", 32, 8192, 7168, 512, "static", "uniform"),
+    "ep_merged": Workload("ep_merged", 32, 8192, 7168, 512, "static", "uniform", merged=True),
     "ep_separate": Workload("ep_separate", 32, 8192, 7168, 256, "static", "uniform"),
     "ragged": Workload("ragged", 256, 65536, 2048, 7168, "dynamic", "ragged_stress"),
     "ragged_bf16": Workload("ragged_bf16", 256, 65536, 2048, 7168, "none", "ragged_stress"),

@@ -257,6 +257,38 @@ def tgmm_drhs(x, rule: int, static_scale: float, dout, group_sizes, sel=None):
     return out, ab
 
 
+# ------------------------------------------------------------------ SwiGLU
+
+# max over the reals of |silu'(z)|, reached near z = 2.3994 (value 1.09984);
+# rounded up.  Bounds how an error in the gate moves silu(gate).
+SILU_LIPSCHITZ = 1.1
+
+
+def silu(z):
+    """silu(z) = z * sigmoid(z) = z / (1 + exp(-z)), fp64, elementwise: the
+    activation of the SwiGLU MLP whose gate and up projections the merged gmm
+    computes ("FP8 Megablox for batch split", maxtext PR #3770, Description
+    (2): W0 and W1 concatenated into one gmm).  exp(-z) overflows to inf for
+    z below about -709, which gives -0.0, the limit."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def gmm_fwd_swiglu(lhs, rule: int, static_scale: float, qr: np.ndarray, sr: np.ndarray, group_sizes,
+                   rows=None):
+    """SwiGLU of the merged forward.  qr / sr are the codes and scales of the
+    merged rhs [W0 | W1] ([G, K, 2F], [G, 2F]).  The forward h is this
+    module's gmm_fwd (fp64); the result is silu(h[:, :F]) * h[:, F:].
+
+    Returns (out [rows, F], (gate, up, absum_gate, absum_up)); the second item
+    feeds the propagated tolerance of a reduced-precision implementation."""
+    h, ab = gmm_fwd(lhs, rule, static_scale, qr, sr, group_sizes, rows)
+    F = h.shape[1] // 2
+    gate, up = h[:, :F], h[:, F:]
+    return silu(gate) * up, (gate, up, ab[:, :F], ab[:, F:])
+
+
 def gmm_fwd_bf16(lhs, w, group_sizes, rows=None):
     lb, wb = _bf16_bits(lhs), _bf16_bits(w)
     M, K = lb.shape

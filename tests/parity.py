@@ -67,3 +67,30 @@ def check_guards(raw: torch.Tensor, pad: int, n: int, fill=0x5A):
     r = raw.cpu()
     assert bool((r[:pad] == fill).all()), "write before the output buffer"
     assert bool((r[pad + n:] == fill).all()), "write past the output buffer"
+
+
+def swiglu_bound(gpu_dtype, terms, ref, eps: float = TOL):
+    """Elementwise bound for out = silu(g) * u when the gate g and the up value
+    u each carry the forward's error, |dg| <= eps * A_g and |du| <= eps * A_u:
+      |silu(g + dg)(u + du) - silu(g) u|
+        <= L eps A_g |u| + (|silu(g)| + L eps A_g) eps A_u,
+    with L = max |silu'| (oracle.SILU_LIPSCHITZ).  Added: the output's own
+    bf16 rounding (2^-8 |ref|) and 1e-5 |ref| for the fp32 evaluation of silu
+    and the product."""
+    gate, up, ag, au = terms
+    L = oracle.SILU_LIPSCHITZ
+    b = L * eps * ag * np.abs(up) + (np.abs(oracle.silu(gate)) + L * eps * ag) * eps * au
+    b = b + 1e-5 * np.abs(ref)
+    if gpu_dtype == torch.bfloat16:
+        b = b + 2.0 ** -8 * np.abs(ref)
+    return b
+
+
+def assert_within(gpu: torch.Tensor, ref: np.ndarray, bound: np.ndarray, what: str = ""):
+    g = to_np(gpu).reshape(ref.shape)
+    err = np.abs(g - ref)
+    bad = ~(err <= bound)  # NaN fails too
+    if bad.any():
+        worst = np.unravel_index(np.argmax(np.where(np.isnan(err), np.inf, err - bound)), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} elements outside the bound; worst at "
+                             f"{worst}: gpu={g[worst]!r} ref={ref[worst]!r} bound={bound[worst]!r}")

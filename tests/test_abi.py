@@ -81,6 +81,11 @@ def test_host_errors(L):
     assert f(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, None, big, None) == 9  # no workspace
     assert f(_op(FAKE, B.DT_E4M3, None, B.Q_DYNAMIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big,
              None) == 1  # pre-quantized lhs without its scales
+    sw = L.gmm_fwd_swiglu
+    assert sw(lhs, rhs, 0, gs, 8, 256, 512, 384, out, B.DT_BF16, ws, big, None) == 2  # N = 2F, F % 128
+    assert sw(lhs, rhs, 0, gs, 8, 256, 512, 0, out, B.DT_BF16, ws, big, None) == 2
+    assert sw(lhs, rhs, 0, None, 8, 256, 512, 512, out, B.DT_BF16, ws, big, None) == 1
+    assert sw(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, 1024, None) == 9
     d = L.gmm_dlhs
     assert d(_op(FAKE, B.DT_E4M3, FAKE, B.Q_DYNAMIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big,
              None) == 1  # dout must be bf16 (the rhs scale is folded in)

@@ -15,7 +15,7 @@ import torch
 import moe_fp8_grouped_b200 as gm
 import oracle
 from moe_fp8_grouped_b200 import synth
-from parity import assert_close
+from parity import assert_close, assert_within, swiglu_bound
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -48,6 +48,8 @@ def test_fullsize_sampled(name):
     out = gm.gmm_fwd(inp.lhs, codes, scales, gs, rule=rule, static_scale=sarg, ws=ws)
     dl = gm.gmm_dlhs(inp.dout, codes, scales, gs, ws=ws, rule="none" if bf16 else "dynamic")
     dw = gm.tgmm_drhs(inp.lhs, inp.dout, gs, rule=rule, static_scale=sarg, ws=ws)
+    # merged gate|up workloads: the forward with SwiGLU fused, too
+    sw = gm.gmm_fwd_swiglu(inp.lhs, codes, scales, gs, rule=rule, static_scale=sarg, ws=ws) if w.merged else None
     st, bits = gm.gmm_read_device_status(ws)
     assert st == 0, (st, bits)
 
@@ -74,6 +76,9 @@ def test_fullsize_sampled(name):
         else:
             ref, ab = oracle.gmm_fwd(lhs_r, qrule, inp.static_scale, qr, sr, one)
             assert_close(out[rows], ref, ab, f"{name} fwd g={g}")
+            if sw is not None:
+                ref, terms = oracle.gmm_fwd_swiglu(lhs_r, qrule, inp.static_scale, qr, sr, one)
+                assert_within(sw[rows], ref, swiglu_bound(sw.dtype, terms, ref), f"{name} swiglu g={g}")
             ref, ab = oracle.gmm_dlhs(dout_r, qr, sr, one)
             assert_close(dl[rows], ref, ab, f"{name} dlhs g={g}")
         # drhs rows (g, k): the whole group is the sub-problem
@@ -90,5 +95,6 @@ def test_fullsize_sampled(name):
     tail = int(offs[-1])
     if tail < M:
         assert not torch.any(out[tail:] != 0) and not torch.any(dl[tail:] != 0)
-    del inp, codes, scales, out, dl, dw, ws
+        assert sw is None or not torch.any(sw[tail:] != 0)
+    del inp, codes, scales, out, dl, dw, ws, sw
     torch.cuda.empty_cache()

@@ -15,7 +15,7 @@ import torch
 import moe_fp8_grouped_b200 as gm
 import oracle
 from moe_fp8_grouped_b200 import synth
-from parity import assert_close, check_guards, guarded, rule_code, untranspose_chunks
+from parity import assert_close, assert_within, check_guards, guarded, rule_code, swiglu_bound, untranspose_chunks
 
 pytestmark = pytest.mark.gpu
 
@@ -173,6 +173,24 @@ def test_fwd_prequantized_lhs(dev, rule, transpose):
     assert_close(outside, ref, ab, f"prequantized fwd {rule}")
 
 
+@pytest.mark.parametrize("name", ["ragged", "big_group"])
+def test_drhs_reuses_static_forward_codes(dev, name):
+    """Static rule: the forward's lhs codes (quantized once, as for an
+    expert-parallel all-gather in E4M3) feed the tgmm unchanged; the result
+    equals quantizing inside the tgmm bit for bit."""
+    inp = case_inputs(name)
+    lhs, _, dout, gs, s = to_dev(inp, dev)
+    ql, _ = gm.gmm_quantize(lhs, "static", axis=1, static_scale=s)
+    inside = gm.tgmm_drhs(lhs, dout, gs, rule="static", static_scale=s)
+    reused = gm.tgmm_drhs(ql, dout, gs, rule="static", static_scale=s)
+    assert gm.last_launch_count() == 4
+    assert torch.equal(inside, reused)
+    ref, ab = oracle.tgmm_drhs(inp.lhs, oracle.Q_STATIC, inp.static_scale, inp.dout, inp.group_sizes)
+    assert_close(reused, ref, ab, f"drhs with forward codes {name}")
+    with pytest.raises(gm.GmmError, match="invalid argument"):
+        gm.tgmm_drhs(ql, dout, gs, rule="dynamic", static_scale=s)
+
+
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
 def test_bf16_family(dev, name):
     inp = case_inputs(name)
@@ -186,6 +204,66 @@ def test_bf16_family(dev, name):
     r = gm.tgmm_drhs(lhs, dout, gs, rule="none", out_dtype=torch.float32)
     ref, ab = oracle.tgmm_drhs_bf16(inp.lhs, inp.dout, inp.group_sizes)
     assert_close(r, ref, ab, "bf16 drhs")
+
+
+# --------------------------------------------------------------- SwiGLU
+
+SWIGLU_CASES = {
+    "tiny": None,
+    "ragged": (5, 700, 384, 768, [1, 129, 0, 300, 200]),  # F = 384: a tile pair beyond 256
+    "g1": (1, 300, 256, 256, [300]),                        # F = 128: one column tile
+    "big_group": (2, 1100, 512, 512, [1000, 100]),
+}
+
+
+@pytest.mark.parametrize("name", list(SWIGLU_CASES))
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fwd_swiglu(dev, name, rule, transpose, out_dtype):
+    """Merged gate|up forward with silu(gate) * up fused into the epilogue,
+    against the oracle within the forward's tolerance carried through the
+    activation."""
+    c = SWIGLU_CASES[name]
+    inp = synth.make_inputs("tiny", seed=0) if c is None else synth.small_case(*c[:4], seed=9, sizes=c[4])
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    M, N = lhs.shape[0], w.shape[2]
+    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
+    raw, out, pad, n = guarded((M, N // 2), out_dtype)
+    gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule=rule, static_scale=s if rule == "static" else None,
+                      transpose_rhs=transpose, out=out)
+    assert gm.last_launch_count() == 3
+    torch.cuda.synchronize()
+    check_guards(raw, pad, n)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    ref, terms = oracle.gmm_fwd_swiglu(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+    assert_within(out, ref, swiglu_bound(out_dtype, terms, ref), f"swiglu {name} {rule} t={transpose}")
+
+
+def test_fwd_swiglu_bf16_family_and_prequantized(dev):
+    inp = synth.small_case(*SWIGLU_CASES["ragged"][:4], seed=10, sizes=SWIGLU_CASES["ragged"][4])
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    # bf16 family: the same fused epilogue on the kind::f16 path
+    out = gm.gmm_fwd_swiglu(lhs, w, None, gs, rule="none", out_dtype=torch.float32)
+    h, ab = oracle.gmm_fwd_bf16(inp.lhs, inp.w, inp.group_sizes)
+    F = h.shape[1] // 2
+    ref = oracle.silu(h[:, :F]) * h[:, F:]
+    assert_within(out, ref, swiglu_bound(torch.float32, (h[:, :F], h[:, F:], ab[:, :F], ab[:, F:]), ref),
+                  "swiglu bf16 family")
+    # pre-quantized lhs gives the same result as quantizing inside the call
+    codes, scales = gm.gmm_quantize_rhs(w)
+    ql, _ = gm.gmm_quantize(lhs, "static", axis=1, static_scale=s)
+    a = gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule="static", static_scale=s, out_dtype=torch.float32)
+    b = gm.gmm_fwd_swiglu(ql, codes, scales, gs, rule="static", static_scale=s, out_dtype=torch.float32)
+    assert torch.equal(a, b)
+
+
+def test_fwd_swiglu_rejects_n_not_two_tiles_of_128(dev):
+    inp = synth.small_case(*CASES["ragged"][:4], seed=7, sizes=CASES["ragged"][4])  # N = 640: F = 320
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    codes, scales = gm.gmm_quantize_rhs(w)
+    with pytest.raises(gm.GmmError, match="shape"):
+        gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule="static", static_scale=s)
 
 
 # ------------------------------------------------------------ identities
@@ -267,6 +345,12 @@ def test_unusable_static_scale_reports_and_outputs_zero(dev, bad):
     out = gm.gmm_fwd(lhs, c, sc, gs, rule="static", static_scale=torch.tensor([bad], device=dev), ws=ws)
     st, bits = gm.gmm_read_device_status(ws)
     assert st == 4 and bits & 2  # GMM_ERR_SCALE
+    assert not out.float().abs().sum().item()
+    # codes quantized before the call: the GEMM itself reports the scale
+    codes = torch.ones_like(lhs, dtype=torch.uint8)
+    out = gm.gmm_fwd(codes, c, sc, gs, rule="static", static_scale=torch.tensor([bad], device=dev), ws=ws)
+    st, bits = gm.gmm_read_device_status(ws)
+    assert st == 4 and bits & 2
     assert not out.float().abs().sum().item()
 
 
