@@ -426,6 +426,154 @@ void gmo_gmm_dlhs(const uint16_t *dout, const uint8_t *qr, const float *sr, cons
   free(offs);
 }
 
+/* ------------------------------------------------ block-wise rhs scales */
+
+/* Weights with one scale per 128-block along one axis of W[g] ("Support
+ * quantization for tokamax gmm v2", maxtext PR #4451, review thread on the
+ * rhs scale: a 2-D scale is per channel, a 3-D scale block-wise):
+ *   axis 0: blocks of 128 k for each column n, scales [G, K/128, N] -- block-
+ *           wise along the forward's contraction;
+ *   axis 1: blocks of 128 n for each row k, scales [G, N/128, K] -- block-
+ *           wise along the contraction of dlhs.
+ * codes keep W's layout [G, K, N].  Each block: s = fl32(amax / 448),
+ * inv = fl32(1 / s) (0 when s is 0 or the inverse overflows), code =
+ * e4m3(fl32(w * inv)).  K and N are multiples of 128. */
+void gmo_quantize_rhs_blocks(const uint16_t *w, int32_t G, int64_t K, int64_t N, int32_t axis, uint8_t *codes,
+                             float *scales) {
+  const int64_t kb_n = K / BLK, nb_n = N / BLK;
+#pragma omp parallel for schedule(static)
+  for (int32_t g = 0; g < G; ++g) {
+    const uint16_t *wg = w + (int64_t)g * K * N;
+    uint8_t *cg = codes + (int64_t)g * K * N;
+    if (axis == 0) {
+      for (int64_t kb = 0; kb < kb_n; ++kb)
+        for (int64_t n = 0; n < N; ++n) {
+          float amax = 0.0f;
+          for (int64_t k = kb * BLK; k < (kb + 1) * BLK; ++k) {
+            float v = fabsf(gmo_bf16_to_f32(wg[k * N + n]));
+            if (v > amax) amax = v;
+          }
+          float sc, inv;
+          dyn_scale(amax, &sc, &inv);
+          scales[((int64_t)g * kb_n + kb) * N + n] = sc;
+          for (int64_t k = kb * BLK; k < (kb + 1) * BLK; ++k)
+            cg[k * N + n] = gmo_e4m3_encode((double)(gmo_bf16_to_f32(wg[k * N + n]) * inv));
+        }
+    } else {
+      for (int64_t k = 0; k < K; ++k)
+        for (int64_t nb = 0; nb < nb_n; ++nb) {
+          float amax = 0.0f;
+          for (int64_t n = nb * BLK; n < (nb + 1) * BLK; ++n) {
+            float v = fabsf(gmo_bf16_to_f32(wg[k * N + n]));
+            if (v > amax) amax = v;
+          }
+          float sc, inv;
+          dyn_scale(amax, &sc, &inv);
+          scales[((int64_t)g * nb_n + nb) * K + k] = sc;
+          for (int64_t n = nb * BLK; n < (nb + 1) * BLK; ++n)
+            cg[k * N + n] = gmo_e4m3_encode((double)(gmo_bf16_to_f32(wg[k * N + n]) * inv));
+        }
+    }
+  }
+}
+
+/* Forward gmm with block-wise rhs scales s_r[g, b, n] ([G, K/128, N]) on
+ * selected rows:
+ *   out[m, n] = sum_b s_l[m, b] * s_r[g, b, n] * sum_{k in b} dec(q_l[m,k]) * dec(q_r[g,k,n])
+ * with s_l[m, b] = s for the static rule.  Rows outside every group are 0. */
+void gmo_gmm_fwd_blockwise(const uint16_t *lhs, int32_t rule, float s_static, const uint8_t *qr, const float *srb,
+                           const int32_t *sizes, int32_t G, int64_t M, int64_t K, int64_t N, const int64_t *rows,
+                           int64_t nrows, double *out, double *absum) {
+  int64_t *offs = (int64_t *)malloc(sizeof(int64_t) * (G + 1));
+  gmo_plan(sizes, G, M, offs, NULL);
+  double tab[256];
+  decode_table(tab);
+  int64_t nb = K / BLK;
+#pragma omp parallel
+  {
+    uint8_t *ql = (uint8_t *)malloc((size_t)K);
+    float *sl = (float *)malloc(sizeof(float) * nb);
+    double *blk = (double *)malloc(sizeof(double) * N);
+    double *bab = (double *)malloc(sizeof(double) * N);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+      int64_t m = rows[i];
+      double *o = out + i * N, *a = absum + i * N;
+      for (int64_t n = 0; n < N; ++n) o[n] = a[n] = 0.0;
+      int32_t g = group_of_row(offs, G, m);
+      if (g < 0) continue;
+      gmo_quantize_rows(lhs + m * K, 1, K, rule, s_static, ql, sl, NULL);
+      for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t n = 0; n < N; ++n) blk[n] = bab[n] = 0.0;
+        for (int64_t k = b * BLK; k < (b + 1) * BLK; ++k) {
+          double x = tab[ql[k]];
+          const uint8_t *wrow = qr + ((int64_t)g * K + k) * N;
+          for (int64_t n = 0; n < N; ++n) {
+            double p = x * tab[wrow[n]];
+            blk[n] += p;
+            bab[n] += fabs(p);
+          }
+        }
+        const float *sb = srb + ((int64_t)g * nb + b) * N;
+        for (int64_t n = 0; n < N; ++n) {
+          o[n] += (double)sl[b] * (double)sb[n] * blk[n];
+          a[n] += (double)sl[b] * (double)sb[n] * bab[n];
+        }
+      }
+    }
+    free(ql);
+    free(sl);
+    free(blk);
+    free(bab);
+  }
+  free(offs);
+}
+
+/* dlhs with block-wise rhs scales along n, s_r[g, b, k] ([G, N/128, K]), on
+ * selected rows.  dout is quantized on its own (dynamic 128-blocks along n;
+ * no rhs scale is folded in, since it now varies along k too):
+ *   dlhs[m, k] = sum_b s_d[m, b] * s_r[g, b, k] * sum_{n in b} dec(q_d[m,n]) * dec(q_r[g,k,n]) */
+void gmo_gmm_dlhs_blockwise(const uint16_t *dout, const uint8_t *qr, const float *srb, const int32_t *sizes,
+                            int32_t G, int64_t M, int64_t K, int64_t N, const int64_t *rows, int64_t nrows,
+                            double *out, double *absum) {
+  int64_t *offs = (int64_t *)malloc(sizeof(int64_t) * (G + 1));
+  gmo_plan(sizes, G, M, offs, NULL);
+  double tab[256];
+  decode_table(tab);
+  int64_t nb = N / BLK;
+#pragma omp parallel
+  {
+    uint8_t *qd = (uint8_t *)malloc((size_t)N);
+    float *sd = (float *)malloc(sizeof(float) * nb);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+      int64_t m = rows[i];
+      double *o = out + i * K, *a = absum + i * K;
+      for (int64_t k = 0; k < K; ++k) o[k] = a[k] = 0.0;
+      int32_t g = group_of_row(offs, G, m);
+      if (g < 0) continue;
+      gmo_quantize_rows(dout + m * N, 1, N, GMO_Q_DYNAMIC, 0.0f, qd, sd, NULL);
+      for (int64_t k = 0; k < K; ++k) {
+        const uint8_t *wrow = qr + ((int64_t)g * K + k) * N;
+        for (int64_t b = 0; b < nb; ++b) {
+          double sum = 0.0, sab = 0.0;
+          for (int64_t n = b * BLK; n < (b + 1) * BLK; ++n) {
+            double p = tab[qd[n]] * tab[wrow[n]];
+            sum += p;
+            sab += fabs(p);
+          }
+          double f = (double)sd[b] * (double)srb[((int64_t)g * nb + b) * K + k];
+          o[k] += f * sum;
+          a[k] += f * sab;
+        }
+      }
+    }
+    free(qd);
+    free(sd);
+  }
+  free(offs);
+}
+
 /* Transposed gmm (weight gradient) on selected (g, k) rows of dW:
  *   dW[g, k, n] = sum_c s_x[c, k] * s_d[c, n] * sum_{m in chunk c} dec(q_x[m,k]) * dec(q_d[m,n])
  * over the 128-row chunks c of group g; an empty group gives dW[g] = 0.

@@ -58,6 +58,11 @@ def lib():
         L.gmo_quantize_rows.argtypes = [_P(u16), i64, i64, i32, f32, _P(u8), _P(f32), _P(i32)]
         L.gmo_quantize_rows_scaled.argtypes = [_P(u16), i64, i64, _P(f32), _P(i32), i32, _P(u8), _P(f32)]
         L.gmo_quantize_rhs.argtypes = [_P(u16), i32, i64, i64, _P(u8), _P(f32)]
+        L.gmo_quantize_rhs_blocks.argtypes = [_P(u16), i32, i64, i64, i32, _P(u8), _P(f32)]
+        L.gmo_gmm_fwd_blockwise.argtypes = [_P(u16), i32, f32, _P(u8), _P(f32), _P(i32), i32, i64, i64, i64,
+                                            _P(i64), i64, _P(f64), _P(f64)]
+        L.gmo_gmm_dlhs_blockwise.argtypes = [_P(u16), _P(u8), _P(f32), _P(i32), i32, i64, i64, i64, _P(i64), i64,
+                                             _P(f64), _P(f64)]
         L.gmo_num_chunks.argtypes = [_P(i32), i32, i64]
         L.gmo_num_chunks.restype = i64
         L.gmo_quantize_chunks.argtypes = [_P(u16), i64, i64, i32, f32, _P(i32), i32, _P(u8), _P(f32)]
@@ -178,6 +183,18 @@ def quantize_rhs(w):
     return codes, scales
 
 
+def quantize_rhs_blocks(w, axis: int):
+    """W [G, K, N] bf16 -> codes [G, K, N] and block-wise scales: axis 0
+    [G, K/128, N] (blocks along K), axis 1 [G, N/128, K] (blocks along N)."""
+    wb = _bf16_bits(w)
+    G, K, N = wb.shape
+    codes = np.empty((G, K, N), dtype=np.uint8)
+    scales = np.empty((G, K // BLOCK, N) if axis == 0 else (G, N // BLOCK, K), dtype=np.float32)
+    lib().gmo_quantize_rhs_blocks(_ptr(wb, ctypes.c_uint16), G, K, N, axis, _ptr(codes, ctypes.c_uint8),
+                                  _ptr(scales, ctypes.c_float))
+    return codes, scales
+
+
 def num_chunks(group_sizes, M: int) -> int:
     gs = _sizes(group_sizes)
     return int(lib().gmo_num_chunks(_ptr(gs, ctypes.c_int32), gs.size, M))
@@ -254,6 +271,40 @@ def tgmm_drhs(x, rule: int, static_scale: float, dout, group_sizes, sel=None):
                         _ptr(out, ctypes.c_double), _ptr(ab, ctypes.c_double))
     if sel is None:
         return out.reshape(G, K, N), ab.reshape(G, K, N)
+    return out, ab
+
+
+def gmm_fwd_blockwise(lhs, rule: int, static_scale: float, qr: np.ndarray, srb: np.ndarray, group_sizes,
+                      rows=None):
+    """Forward gmm with block-wise rhs scales srb [G, K/128, N] -> (out, absum)."""
+    lb = _bf16_bits(lhs)
+    M, K = lb.shape
+    G, K2, N = qr.shape
+    assert K2 == K and srb.shape == (G, K // BLOCK, N)
+    gs, r = _sizes(group_sizes), _rows(rows, M)
+    qr = np.ascontiguousarray(qr, dtype=np.uint8)
+    srb = np.ascontiguousarray(srb, dtype=np.float32)
+    out = np.empty((r.size, N)); ab = np.empty((r.size, N))
+    lib().gmo_gmm_fwd_blockwise(_ptr(lb, ctypes.c_uint16), rule, static_scale, _ptr(qr, ctypes.c_uint8),
+                                _ptr(srb, ctypes.c_float), _ptr(gs, ctypes.c_int32), G, M, K, N,
+                                _ptr(r, ctypes.c_int64), r.size, _ptr(out, ctypes.c_double),
+                                _ptr(ab, ctypes.c_double))
+    return out, ab
+
+
+def gmm_dlhs_blockwise(dout, qr: np.ndarray, srb: np.ndarray, group_sizes, rows=None):
+    """dlhs with block-wise rhs scales along N, srb [G, N/128, K] -> (dlhs, absum)."""
+    db = _bf16_bits(dout)
+    M, N = db.shape
+    G, K, N2 = qr.shape
+    assert N2 == N and srb.shape == (G, N // BLOCK, K)
+    gs, r = _sizes(group_sizes), _rows(rows, M)
+    qr = np.ascontiguousarray(qr, dtype=np.uint8)
+    srb = np.ascontiguousarray(srb, dtype=np.float32)
+    out = np.empty((r.size, K)); ab = np.empty((r.size, K))
+    lib().gmo_gmm_dlhs_blockwise(_ptr(db, ctypes.c_uint16), _ptr(qr, ctypes.c_uint8), _ptr(srb, ctypes.c_float),
+                                 _ptr(gs, ctypes.c_int32), G, M, K, N, _ptr(r, ctypes.c_int64), r.size,
+                                 _ptr(out, ctypes.c_double), _ptr(ab, ctypes.c_double))
     return out, ab
 
 
