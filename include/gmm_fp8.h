@@ -115,6 +115,21 @@ gmm_status gmm_quantize_rhs(const void *w_bf16, int32_t G, int64_t K, int64_t N,
                             uint8_t *codes, float *scales, void *stream);
 
 /*
+ * Weight quantization with block-wise scales ("Support quantization for
+ * tokamax gmm v2", maxtext PR #4451, review thread on the rhs scale: a 2-D
+ * scale is per channel, a 3-D scale block-wise).  w_bf16: [G, K, N].  codes:
+ * [G, K, N] E4M3.  One scale per block of 128 weights along
+ *   axis 0: K (the forward's contraction): scales [G, K/128, N];
+ *   axis 1: N (the contraction of dlhs):    scales [G, N/128, K].
+ * Each block: s = fl32(amax / 448), code = e4m3_rn(fl32(w * fl32(1 / s)))
+ * (0 for an all-zero block).  Pass the codes to gmm_fwd (axis 0) or gmm_dlhs
+ * (axis 1) as an E4M3 rhs with rule GMM_Q_DYNAMIC.  Runs once per weight
+ * update, outside the passes.
+ */
+gmm_status gmm_quantize_rhs_blocks(const void *w_bf16, int32_t G, int64_t K, int64_t N, int axis, uint8_t *codes,
+                                   float *scales, void *stream);
+
+/*
  * Activation / gradient quantization, the step each pass runs first.  x_bf16
  * is [rows, cols] bf16.
  * axis == 1: blocks of 128 along each row (the forward lhs, the dlhs dout).
@@ -146,7 +161,11 @@ gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrul
  * re-applied after the matmul), with lhs.scale the static scale (rule STATIC,
  * one float) or the block scales [K/128, M] (rule DYNAMIC, the layout
  * gmm_quantize writes for axis 1); the quantize step is then skipped.  rhs: E4M3 codes with scales [G, N] (or bf16 for the bf16
- * family), [G, K, N] when transpose_rhs == 0, [G, N, K] when 1.
+ * family), [G, K, N] when transpose_rhs == 0, [G, N, K] when 1.  rhs.rule
+ * NONE: per-channel scales [G, N]; rhs.rule DYNAMIC: block-wise scales
+ * [G, K/128, N] from gmm_quantize_rhs_blocks axis 0 (transpose_rhs 0 only;
+ * else GMM_ERR_UNSUPPORTED), applied per 128-block of K:
+ *   out[m, n] = sum_b s_l[m, b] * s_r[g, b, n] * sum_{k in b} q_l[m, k] * q_r[g, k, n]
  * group_sizes: device int32 [G]; rows are sorted by group.
  * out: [M, N] of out_dtype (BF16 or F32):
  *   out[m, n] = s_r[g, n] * sum_b s_l[m, b] * sum_{k in b} q_l[m, k] * q_r[g, k, n]
@@ -204,6 +223,10 @@ gmm_status gmm_fwd_noalloc(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
  * for gmm_fwd with the same transpose_rhs.  dlhs: [M, K] of out_dtype:
  *   dlhs[m, k] = sum_b s_t[m, b] * sum_{n in b} q_t[m, n] * q_r[g, k, n],
  *   q_t, s_t = quantize(fl32(dout[m, n] * s_r[g, n]))
+ * With block-wise weights (rhs.rule DYNAMIC: codes [G, K, N] and scales
+ * [G, N/128, K] from gmm_quantize_rhs_blocks axis 1; transpose_rhs 0 only)
+ * dout is quantized on its own and
+ *   dlhs[m, k] = sum_b s_d[m, b] * s_r[g, b, k] * sum_{n in b} q_d[m, n] * q_r[g, k, n]
  */
 gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
                     int64_t M, int64_t K, int64_t N, void *dlhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,

@@ -193,7 +193,9 @@ static gmm_status classify(const gmm_operand &x, const gmm_operand &w, bool w_is
   }
   if (x.rule == GMM_Q_STATIC && !x.scale) return GMM_ERR_INVALID_ARG;  // a present rule must be applied
   if (w_is_rhs) {
+    // rule NONE: per-channel scales [G, N]; DYNAMIC: block-wise scales
     if (w.dtype != GMM_E4M3 || !w.scale) return GMM_ERR_INVALID_ARG;
+    if (w.rule != GMM_Q_NONE && w.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
   } else {
     if (w.dtype != GMM_BF16 || w.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;
   }
@@ -222,7 +224,7 @@ const char *gmm_status_string(gmm_status s) {
     case GMM_ERR_SHAPE: return "invalid shape (sizes must be positive, K and N multiples of 128)";
     case GMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case GMM_ERR_SCALE: return "static scale not finite or not above FLT_MIN";
-    case GMM_ERR_UNSUPPORTED: return "unsupported size";
+    case GMM_ERR_UNSUPPORTED: return "unsupported size or option combination";
     case GMM_ERR_CUDA: return "CUDA runtime error";
     case GMM_ERR_GROUP_SIZES: return "group_sizes negative or summing past M";
     case GMM_ERR_TIMEOUT: return "a device wait timed out";
@@ -247,6 +249,21 @@ gmm_status gmm_quantize_rhs(const void *w_bf16, int32_t G, int64_t K, int64_t N,
     return launch_quant_rhs(w_bf16, G, K, N, transpose_out != 0, codes, scales, st);
   }));
   if (s == GMM_OK) g_launches = 3;
+  return s;
+}
+
+gmm_status gmm_quantize_rhs_blocks(const void *w_bf16, int32_t G, int64_t K, int64_t N, int axis, uint8_t *codes,
+                                   float *scales, void *stream) {
+  g_launches = 0;
+  if (!w_bf16 || !codes || !scales || (axis != 0 && axis != 1)) return GMM_ERR_INVALID_ARG;
+  gmm_status s = check_sizes(1, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!al16(w_bf16) || !al16(codes) || !al16(scales)) return GMM_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = cuda_status(prof("quant_rhs_blocks", st, [&] {
+    return launch_quant_rhs_blocks(w_bf16, G, K, N, axis, codes, scales, st);
+  }));
+  if (s == GMM_OK) g_launches = 1;
   return s;
 }
 
@@ -319,6 +336,8 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   int n = 1;
   const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
   const bool preq = lhs.dtype == GMM_E4M3;  // codes and scales supplied by the caller
+  const bool blk = elem == 1 && rhs.rule == GMM_Q_DYNAMIC;  // block-wise rhs scales [G, K/128, N]
+  if (blk && transpose_rhs) return GMM_ERR_UNSUPPORTED;
   const void *A = lhs.data;
   if (elem == 1 && !preq) {
     s = cuda_status(prof("quant_rows", st, [&] {
@@ -349,14 +368,17 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   p.tpre = P.tpre;
   p.row_scale = (elem == 1 && dyn) ? (preq ? lhs.scale : P.scales_a) : nullptr;
   p.row_scale_ld = M;
-  p.col_scale = elem == 1 ? rhs.scale : nullptr;
+  p.col_scale = (elem == 1 && !blk) ? rhs.scale : nullptr;
+  p.colblk_scale = blk ? rhs.scale : nullptr;
+  p.colblk_ld = N;
   p.static_scale = (elem == 1 && !dyn) ? lhs.scale : nullptr;
   p.out = out;
   p.out_f32 = out_dtype == GMM_F32;
   p.ld_out = F ? F : N;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1 && dyn};
+  // per-block promotion for dynamic lhs scales or block-wise rhs scales
+  const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk)};
   const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   if ((s = cuda_status(prof(F ? "gemm_fwd_swiglu" : "gemm_fwd", st,
@@ -403,11 +425,15 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
   int n = 1;
   const void *A = dout.data;
+  // block-wise rhs scales along n ([G, N/128, K]): they vary along k as well,
+  // so dout is quantized on its own and both scales are applied per block
+  const bool blk = elem == 1 && rhs.rule == GMM_Q_DYNAMIC;
+  if (blk && transpose_rhs) return GMM_ERR_UNSUPPORTED;
   if (elem == 1) {
-    // t = fl32(dout * s_r[g(m), n]), dynamic 128-blocks along n
+    // per-channel rhs: t = fl32(dout * s_r[g(m), n]); dynamic 128-blocks along n
     s = cuda_status(prof("quant_rows", st, [&] {
-      return launch_quant_rows(dout.data, M, N, true, nullptr, rhs.scale, P.offs, G, P.codes_a, P.scales_a,
-                               P.status, st);
+      return launch_quant_rows(dout.data, M, N, true, nullptr, blk ? nullptr : rhs.scale, P.offs, G, P.codes_a,
+                               P.scales_a, P.status, st);
     }));
     if (s != GMM_OK) return s;
     ++n;
@@ -431,6 +457,8 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   p.row_scale = elem == 1 ? P.scales_a : nullptr;
   p.row_scale_ld = M;
   p.col_scale = nullptr;
+  p.colblk_scale = blk ? rhs.scale : nullptr;
+  p.colblk_ld = K;
   p.static_scale = nullptr;
   p.out = dlhs;
   p.out_f32 = out_dtype == GMM_F32;

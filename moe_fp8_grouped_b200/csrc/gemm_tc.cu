@@ -245,12 +245,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // Which scales each TMEM unit carries (the same decision in every role):
-  //   column scales: forward s_r[g, n] (every unit of a tile); tgmm with a
-  //                  dynamic lhs rule: s_x[chunk, k]
-  //   row scales:    promoted row-ragged passes (s_l / s_t per 128-block);
-  //                  tgmm: s_d[chunk, n]
-  const bool need_col = kTg ? (kPromote && p.colblk_scale != nullptr) : (p.col_scale != nullptr);
-  const bool need_row = kPromote;
+  //   column scales: forward s_r[g, n] (every unit of a tile, applied at the
+  //                  end); block-wise rhs scales s_r[g, b, n] (one set per
+  //                  unit, applied per unit); tgmm with a dynamic lhs rule:
+  //                  s_x[chunk, k] (per unit)
+  //   row scales:    promoted row-ragged passes with a dynamic row operand
+  //                  (s_l / s_t per 128-block); tgmm: s_d[chunk, n]
+  const bool need_col = kTg ? (kPromote && p.colblk_scale != nullptr)
+                            : (p.col_scale != nullptr || p.colblk_scale != nullptr);
+  const bool need_row = kPromote && p.row_scale != nullptr;
+  const bool unit_col = kPromote && p.colblk_scale != nullptr;  // column scales change per unit
   const bool use_ring = need_col || need_row;
 
   if (threadIdx.x == 0) {
@@ -415,8 +419,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // columns >= ncols are never read
             const int n = kTg ? t.ct * kBN + 8 * lane : tile_col_n(t.ct, 8 * lane, p.swiglu_f);
             if (n < p.ncols) {
-              const float *src = kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
-                                     : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n;
+              const float *src =
+                  kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
+                      : (p.colblk_scale ? p.colblk_scale + (static_cast<int64_t>(t.g) * p.kblocks + j) * p.colblk_ld + n
+                                        : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n);
               float *dst = s_scol + slot * kBN + 8 * lane;
               cp_async_16(dst, src);
               cp_async_16(dst + 4, src + 4);
@@ -543,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const float rs = s_srow[slot * kBM + row];
+          const float rs = need_row ? s_srow[slot * kBM + row] : 1.0f;
           const float2 rs2 = make_float2(rs, rs);
           const float *cs = s_scol + slot * kBN;
 #pragma unroll
@@ -557,15 +563,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int half = 0; half < 2; ++half) {
               const uint32_t *vv = half ? vb : va;
               const int c = 2 * cp + half;
-              if (!(kTg && need_col)) {
+              if (!unit_col) {
                 // one scale per accumulator row
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                   acc[c * 16 + i] = __ffma2_rn(make_float2(__uint_as_float(vv[2 * i]), __uint_as_float(vv[2 * i + 1])),
                                                rs2, acc[c * 16 + i]);
               } else {
-                // tgmm with a dynamic lhs rule: the lhs chunk scale varies
-                // along the columns k
+                // tgmm with a dynamic lhs rule (lhs chunk scale along the
+                // columns k) or block-wise rhs scales (along the columns n)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                   const float4 c4 = *reinterpret_cast<const float4 *>(cs + colt(c) + 4 * i);
@@ -589,9 +595,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (row_ok) {
-          // forward: the rhs column scale (in every unit's slot); static tgmm: s
-          const float fin = (kTg && p.static_scale) ? s_eff : 1.0f;
-          const bool colmul = !kTg && need_col;
+          // per-channel rhs column scale (in every unit's slot); static lhs: s
+          const float fin = p.static_scale ? s_eff : 1.0f;
+          const bool colmul = !kTg && p.col_scale != nullptr;
           const float *cf = s_scol + slot * kBN;
           if (sw) {
 #pragma unroll
@@ -601,8 +607,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float2 a = acc[c * 16 + i], b2 = acc[(c + 2) * 16 + i];
-                o[2 * i] = silu(a.x * fg[2 * i]) * (b2.x * fu[2 * i]);
-                o[2 * i + 1] = silu(a.y * fg[2 * i + 1]) * (b2.y * fu[2 * i + 1]);
+                const float g0 = (colmul ? a.x * fg[2 * i] : a.x) * fin;
+                const float g1 = (colmul ? a.y * fg[2 * i + 1] : a.y) * fin;
+                const float u0 = (colmul ? b2.x * fu[2 * i] : b2.x) * fin;
+                const float u1 = (colmul ? b2.y * fu[2 * i + 1] : b2.y) * fin;
+                o[2 * i] = silu(g0) * u0;
+                o[2 * i + 1] = silu(g1) * u1;
               }
               emit(t.ct * 128 + h * 64 + c * 32, o);
             }

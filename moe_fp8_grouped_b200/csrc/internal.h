@@ -60,6 +60,10 @@ cudaError_t launch_chunk_codes(const uint8_t *codes, int64_t rows, int64_t cols,
 cudaError_t launch_quant_rhs(const void *w, int G, int64_t K, int64_t N, bool transpose_out, uint8_t *codes,
                              float *scales, cudaStream_t st);
 
+// Block-wise weight quantizer: axis 0 scales [G, K/128, N], axis 1 [G, N/128, K].
+cudaError_t launch_quant_rhs_blocks(const void *w, int G, int64_t K, int64_t N, int axis, uint8_t *codes,
+                                    float *scales, cudaStream_t st);
+
 cudaError_t launch_timeout_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t st);
 
 enum GemmMode { MODE_ROWS = 0, MODE_TGMM = 1 };
@@ -81,7 +85,9 @@ struct GemmParams {
   const int *tpre;     // [G + 1]
   const float *row_scale;     // MODE_ROWS: [kblocks][M]; MODE_TGMM: dout chunk scales [chunk][N]
   int64_t row_scale_ld;
-  const float *colblk_scale;  // MODE_TGMM, dynamic x: lhs chunk scales [chunk][K]
+  const float *colblk_scale;  // per-unit column scales.  MODE_TGMM, dynamic x: lhs chunk
+                              // scales [chunk][K]; MODE_ROWS: block-wise rhs scales
+                              // [G][kblocks][ncols] (then col_scale is NULL)
   int64_t colblk_ld;
   const float *col_scale;     // MODE_ROWS: [G][ncols] final per-column scale, or NULL
   const float *static_scale;  // device scalar multiplied in at the end, or NULL

@@ -544,6 +544,70 @@ cudaError_t launch_quant_rhs(const void *w, int G, int64_t K, int64_t N, bool tr
   return cudaGetLastError();
 }
 
+// Block-wise weight scales: one scale per 128-block of W[g] along K (kAxis 0,
+// scales [G, K/128, N]) or along N (kAxis 1, scales [G, N/128, K]).  One CTA
+// per 128 x 128 tile (rows k, columns n); a tile holds exactly one block per
+// column (axis 0) or per row (axis 1).  Codes keep W's layout [G, K, N].
+template <int kAxis>
+__global__ void __launch_bounds__(256) rhs_blocks_kernel(const __nv_bfloat16 *__restrict__ w, int64_t K, int64_t N,
+                                                         uint8_t *__restrict__ codes, float *__restrict__ scales) {
+  __shared__ __align__(16) __nv_bfloat16 tile[kBlk][kBlk + 8];
+  __shared__ float s_inv[kBlk];
+  const int g = blockIdx.z;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBlk, k0 = static_cast<int64_t>(blockIdx.y) * kBlk;
+  for (int i = threadIdx.x; i < kBlk * 16; i += 256) {
+    const int rr = i >> 4, cc = (i & 15) * 8;
+    *reinterpret_cast<uint4 *>(&tile[rr][cc]) =
+        __ldg(reinterpret_cast<const uint4 *>(w + (g * K + k0 + rr) * N + n0 + cc));
+  }
+  __syncthreads();
+  if (threadIdx.x < kBlk) {
+    const int t = threadIdx.x;
+    float m = 0.0f;
+    if constexpr (kAxis == 0) {
+      for (int r = 0; r < kBlk; ++r) m = fmaxf(m, fabsf(__bfloat162float(tile[r][t])));  // column t
+    } else {
+      for (int c = 0; c < kBlk; ++c) m = fmaxf(m, fabsf(__bfloat162float(tile[t][c])));  // row t
+    }
+    float sc, inv;
+    dyn_scale(m, sc, inv);
+    s_inv[t] = inv;
+    if constexpr (kAxis == 0)
+      scales[(static_cast<int64_t>(g) * (K / kBlk) + blockIdx.y) * N + n0 + t] = sc;
+    else
+      scales[(static_cast<int64_t>(g) * (N / kBlk) + blockIdx.x) * K + k0 + t] = sc;
+  }
+  __syncthreads();
+  // thread (row t, half h): 64 columns of row k0 + t
+  const int t = threadIdx.x & 127, h = threadIdx.x >> 7;
+  uint8_t *dst = codes + (g * K + k0 + t) * N + n0 + 64 * h;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t wv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = 64 * h + q * 16 + e * 4;
+      float a[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        a[i] = __fmul_rn(__bfloat162float(tile[t][c + i]), kAxis == 0 ? s_inv[c + i] : s_inv[t]);
+      wv[e] = static_cast<uint32_t>(cvt_e4m3x2(a[0], a[1])) | (static_cast<uint32_t>(cvt_e4m3x2(a[2], a[3])) << 16);
+    }
+    *reinterpret_cast<uint4 *>(dst + q * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  }
+}
+
+cudaError_t launch_quant_rhs_blocks(const void *w, int G, int64_t K, int64_t N, int axis, uint8_t *codes,
+                                    float *scales, cudaStream_t st) {
+  const __nv_bfloat16 *wb = static_cast<const __nv_bfloat16 *>(w);
+  dim3 grid(static_cast<unsigned>(N / kBlk), static_cast<unsigned>(K / kBlk), G);
+  if (axis == 0)
+    rhs_blocks_kernel<0><<<grid, 256, 0, st>>>(wb, K, N, codes, scales);
+  else
+    rhs_blocks_kernel<1><<<grid, 256, 0, st>>>(wb, K, N, codes, scales);
+  return cudaGetLastError();
+}
+
 // -------------------------------------------------- bounded-wait self-test
 
 // Waits on a barrier that nothing arrives on; the bounded wait gives up after

@@ -132,6 +132,27 @@ def _operand(data, dtype_code, scale, rule):
     return B.Operand(data, dtype_code, scale, rule)
 
 
+def _rhs_operand(rhs, rhs_scales):
+    """rhs with its scales: 2-D scales [G, N] are per channel (rule NONE), 3-D
+    scales block-wise (rule DYNAMIC, from gmm_quantize_rhs_blocks)."""
+    blockwise = rhs_scales is not None and rhs_scales.dim() == 3
+    return _operand(_dev(rhs, "rhs"), _TORCH_DT[rhs.dtype],
+                    _dev(rhs_scales, "rhs_scales", torch.float32) if rhs_scales is not None else None,
+                    B.Q_DYNAMIC if blockwise else B.Q_NONE)
+
+
+def gmm_quantize_rhs_blocks(w: torch.Tensor, axis: int = 0):
+    """W [G, K, N] bf16 -> (codes uint8 [G, K, N], block-wise scales fp32):
+    axis 0 [G, K/128, N] for gmm_fwd, axis 1 [G, N/128, K] for gmm_dlhs."""
+    G, K, N = w.shape
+    codes = torch.empty((G, K, N), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((G, K // 128, N) if axis == 0 else (G, N // 128, K), dtype=torch.float32, device=w.device)
+    st = B.lib().gmm_quantize_rhs_blocks(_dev(w, "w", torch.bfloat16), G, K, N, int(axis), codes.data_ptr(),
+                                         scales.data_ptr(), _stream(w))
+    _check(st, "gmm_quantize_rhs_blocks")
+    return codes, scales
+
+
 def gmm_fwd(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | None, group_sizes: torch.Tensor,
             rule="static", static_scale: torch.Tensor | None = None, transpose_rhs: bool = False,
             out_dtype=torch.bfloat16, out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
@@ -175,8 +196,7 @@ def _fwd(lhs, rhs, rhs_scales, group_sizes, rule, static_scale, transpose_rhs, o
     else:
         a = _operand(_dev(lhs, "lhs", torch.bfloat16), B.DT_BF16,
                      _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None, r)
-    b = _operand(_dev(rhs, "rhs"), _TORCH_DT[rhs.dtype],
-                 _dev(rhs_scales, "rhs_scales", torch.float32) if rhs_scales is not None else None, B.Q_NONE)
+    b = _rhs_operand(rhs, rhs_scales)
     fn = B.lib().gmm_fwd_swiglu if swiglu else B.lib().gmm_fwd
     st = fn(a, b, int(transpose_rhs), _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,
             _dev(out, "out", (torch.bfloat16, torch.float32)), _TORCH_DT[out.dtype], ws.data_ptr(),
@@ -202,8 +222,7 @@ def gmm_dlhs(dout: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | N
     if ws is None:
         ws = workspace(gmm_workspace_bytes(B.OP_DLHS, M, K, N, G), dout.device)
     a = _operand(_dev(dout, "dout", torch.bfloat16), B.DT_BF16, None, r)
-    b = _operand(_dev(rhs, "rhs"), _TORCH_DT[rhs.dtype],
-                 _dev(rhs_scales, "rhs_scales", torch.float32) if rhs_scales is not None else None, B.Q_NONE)
+    b = _rhs_operand(rhs, rhs_scales)
     st = B.lib().gmm_dlhs(a, b, int(transpose_rhs), _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,
                           _dev(out, "out", (torch.bfloat16, torch.float32)), _TORCH_DT[out.dtype], ws.data_ptr(),
                           ws.numel(), _stream(dout))

@@ -98,3 +98,44 @@ def test_fullsize_sampled(name):
         assert sw is None or not torch.any(sw[tail:] != 0)
     del inp, codes, scales, out, dl, dw, ws, sw
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["dsv3_up", "mixtral"])
+def test_fullsize_blockwise_rhs_sampled(name):
+    """Block-wise weight scales at full size: gmm_fwd with [G, K/128, N]
+    scales and gmm_dlhs with [G, N/128, K] scales, checked on sampled rows
+    (each row depends only on itself and its group's weights)."""
+    dev = torch.device("cuda:0")
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w, seed=0, device="cuda")
+    gs_h = inp.group_sizes.numpy().astype(np.int64)
+    gs = inp.group_sizes.to(dev)
+    M, K, N, G = w.M, w.K, w.N, w.G
+    s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    sarg = s if w.rule == "static" else None
+    ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, N, G) for op in (0, 1)), dtype=torch.uint8, device=dev)
+    c0, s0 = gm.gmm_quantize_rhs_blocks(inp.w, 0)
+    out = gm.gmm_fwd(inp.lhs, c0, s0, gs, rule=w.rule, static_scale=sarg, ws=ws)
+    del c0
+    c1, s1 = gm.gmm_quantize_rhs_blocks(inp.w, 1)
+    dl = gm.gmm_dlhs(inp.dout, c1, s1, gs, ws=ws)
+    del c1
+    st, bits = gm.gmm_read_device_status(ws)
+    assert st == 0, (st, bits)
+    offs = np.concatenate([[0], np.cumsum(gs_h)])
+    rng = np.random.default_rng(1)
+    qrule = {"static": oracle.Q_STATIC, "dynamic": oracle.Q_DYNAMIC}[w.rule]
+    for g in pick_groups(gs_h, rng):
+        a, b = int(offs[g]), int(offs[g + 1])
+        wg = inp.w[g:g + 1].cpu()
+        qr0, sr0 = oracle.quantize_rhs_blocks(wg, 0)
+        qr1, sr1 = oracle.quantize_rhs_blocks(wg, 1)
+        assert np.array_equal(s0[g].cpu().numpy(), sr0[0]) and np.array_equal(s1[g].cpu().numpy(), sr1[0])
+        rows = sorted({a, b - 1, int(rng.integers(a, b))})
+        one = np.array([len(rows)], np.int32)
+        ref, ab = oracle.gmm_fwd_blockwise(inp.lhs[rows].cpu(), qrule, inp.static_scale, qr0, sr0, one)
+        assert_close(out[rows], ref, ab, f"{name} blockwise fwd g={g}")
+        ref, ab = oracle.gmm_dlhs_blockwise(inp.dout[rows].cpu(), qr1, sr1, one)
+        assert_close(dl[rows], ref, ab, f"{name} blockwise dlhs g={g}")
+    del inp, out, dl, ws, s0, s1
+    torch.cuda.empty_cache()

@@ -266,6 +266,79 @@ def test_fwd_swiglu_rejects_n_not_two_tiles_of_128(dev):
         gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule="static", static_scale=s)
 
 
+# ------------------------------------------------- block-wise rhs scales
+
+@pytest.mark.parametrize("axis", [0, 1])
+def test_quantize_rhs_blocks_bitexact(dev, axis):
+    inp = case_inputs("ragged")
+    w = inp.w.to(dev)
+    codes, scales = gm.gmm_quantize_rhs_blocks(w, axis)
+    qr, sr = oracle.quantize_rhs_blocks(inp.w, axis)
+    assert np.array_equal(codes.cpu().numpy(), qr)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), sr.view(np.uint32))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fwd_blockwise(dev, name, rule, out_dtype):
+    """Forward with one rhs scale per 128-block of K and column: every
+    contraction block is promoted with s_l[m, b] * s_r[g, b, n]."""
+    inp = case_inputs(name)
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    M, N = lhs.shape[0], w.shape[2]
+    codes, scales = gm.gmm_quantize_rhs_blocks(w, 0)
+    raw, out, pad, n = guarded((M, N), out_dtype)
+    gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=s if rule == "static" else None, out=out)
+    torch.cuda.synchronize()
+    check_guards(raw, pad, n)
+    qr, sr = oracle.quantize_rhs_blocks(inp.w, 0)
+    ref, ab = oracle.gmm_fwd_blockwise(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+    assert_close(out, ref, ab, f"blockwise fwd {name} {rule}")
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_dlhs_blockwise(dev, name, out_dtype):
+    inp = case_inputs(name)
+    _, w, dout, gs, _ = to_dev(inp, dev)
+    M, K = dout.shape[0], w.shape[1]
+    codes, scales = gm.gmm_quantize_rhs_blocks(w, 1)
+    raw, out, pad, n = guarded((M, K), out_dtype)
+    gm.gmm_dlhs(dout, codes, scales, gs, out=out)
+    torch.cuda.synchronize()
+    check_guards(raw, pad, n)
+    qr, sr = oracle.quantize_rhs_blocks(inp.w, 1)
+    ref, ab = oracle.gmm_dlhs_blockwise(inp.dout, qr, sr, inp.group_sizes)
+    assert_close(out, ref, ab, f"blockwise dlhs {name}")
+
+
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+def test_fwd_swiglu_blockwise(dev, rule):
+    c = SWIGLU_CASES["ragged"]
+    inp = synth.small_case(*c[:4], seed=12, sizes=c[4])
+    lhs, w, _, gs, s = to_dev(inp, dev)
+    codes, scales = gm.gmm_quantize_rhs_blocks(w, 0)
+    out = gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule=rule, static_scale=s if rule == "static" else None,
+                            out_dtype=torch.float32)
+    qr, sr = oracle.quantize_rhs_blocks(inp.w, 0)
+    h, ab = oracle.gmm_fwd_blockwise(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+    F = h.shape[1] // 2
+    ref = oracle.silu(h[:, :F]) * h[:, F:]
+    assert_within(out, ref, swiglu_bound(torch.float32, (h[:, :F], h[:, F:], ab[:, :F], ab[:, F:]), ref),
+                  f"blockwise swiglu {rule}")
+
+
+def test_blockwise_rejects_transposed_rhs(dev):
+    inp = case_inputs("g1")
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    codes, scales = gm.gmm_quantize_rhs_blocks(w, 0)
+    with pytest.raises(gm.GmmError, match="unsupported"):
+        gm.gmm_fwd(lhs, codes, scales, gs, rule="static", static_scale=s, transpose_rhs=True)
+    with pytest.raises(gm.GmmError, match="unsupported"):
+        gm.gmm_dlhs(dout, codes, scales, gs, transpose_rhs=True)
+
+
 # ------------------------------------------------------------ identities
 
 def test_merged_gate_up_identity_gpu(dev):
