@@ -253,6 +253,37 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
                      void *stream);
 
 /*
+ * Row movement for expert parallelism, the steps either side of the NCCL
+ * all-to-all that carries routed token rows to the rank holding their expert
+ * ("add static LHS scaling support for GMM v2 FWD", maxtext PR #4735, rebase
+ * commit text: activations quantized before the expert-parallel exchange and
+ * ragged sort, so E4M3 rows move instead of bf16; permute / unpermute).
+ *
+ * gmm_gather_rows: dst[i, :] = src[idx[i], :] for i < nrows, rows of
+ * row_bytes bytes (a multiple of 16; E4M3 codes or bf16).  src has src_rows
+ * rows; an index outside [0, src_rows) writes a row of zeros.  idx: device
+ * int32 [nrows].  src and dst 16-byte aligned, not overlapping.  Returns
+ * GMM_ERR_SHAPE for row_bytes % 16, GMM_ERR_ALIGNMENT, GMM_ERR_INVALID_ARG for
+ * negative sizes or NULL pointers (nrows == 0 is a no-op).
+ */
+gmm_status gmm_gather_rows(const void *src, const int32_t *idx, int64_t nrows, int64_t row_bytes, int64_t src_rows,
+                           void *dst, void *stream);
+
+/*
+ * gmm_combine_rows: the weighted sum that returns expert outputs to their
+ * tokens (the unpermute of the MoE combine):
+ *   y[t, :] = sum_{j < k} weight[t, j] * rows[slot[t, j], :]
+ * rows: bf16 [nrows, N] (gmm_fwd outputs in the order they came back from
+ * the exchange); slot: device int32 [T, k], the row of token t's j-th expert
+ * choice (outside [0, nrows): no contribution); weight: device float [T, k].
+ * Accumulated in fp32 in the order j = 0 .. k-1 (deterministic); y: [T, N]
+ * of y_dtype (BF16 or F32).  N must be a multiple of 8; rows and y 16-byte
+ * aligned.
+ */
+gmm_status gmm_combine_rows(const void *rows_bf16, int64_t nrows, const int32_t *slot, const float *weight, int64_t T,
+                            int32_t k, int64_t N, void *y, gmm_dtype y_dtype, void *stream);
+
+/*
  * Synchronizes `stream`, then reads the device status word that the last call
  * using `ws` left.  *bits_out (may be NULL) receives the raw GMM_DEV_* bits.
  * Returns GMM_OK, or the most severe device error: TIMEOUT, SCALE,

@@ -25,7 +25,8 @@ DEV_GROUP_SIZES, DEV_SCALE, DEV_TIMEOUT = 1, 2, 4
 EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm_quantize", "gmm_fwd",
            "gmm_dlhs", "tgmm_drhs", "gmm_read_device_status", "gmm_selftest_timeout", "gmm_set_wait_limit_ns",
            "gmm_status_string", "gmm_last_launch_count", "gmm_profile_enable", "gmm_profile_collect",
-           "gmm_fwd_noalloc", "gmm_fwd_swiglu", "gmm_quantize_rhs_blocks"]
+           "gmm_fwd_noalloc", "gmm_fwd_swiglu", "gmm_quantize_rhs_blocks", "gmm_gather_rows",
+           "gmm_combine_rows"]
 
 
 class Operand(ctypes.Structure):
@@ -63,6 +64,10 @@ def lib():
     L.gmm_fwd_swiglu.argtypes = L.gmm_fwd.argtypes
     L.gmm_quantize_rhs_blocks.argtypes = [vp, i32, i64, i64, ctypes.c_int, vp, vp, vp]
     L.gmm_quantize_rhs_blocks.restype = st
+    L.gmm_gather_rows.argtypes = [vp, vp, i64, i64, i64, vp, vp]
+    L.gmm_gather_rows.restype = st
+    L.gmm_combine_rows.argtypes = [vp, i64, vp, vp, i64, i32, i64, vp, ctypes.c_int, vp]
+    L.gmm_combine_rows.restype = st
     L.gmm_fwd_swiglu.restype = st
     L.gmm_fwd_noalloc.argtypes = [Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp]
     L.gmm_fwd_noalloc.restype = st

@@ -575,8 +575,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                   const float4 c4 = *reinterpret_cast<const float4 *>(cs + colt(c) + 4 * i);
-                  const float2 c01 = __fmul2_rn(make_float2(c4.x, c4.y), rs2);
-                  const float2 c23 = __fmul2_rn(make_float2(c4.z, c4.w), rs2);
+                  // without row scales (static lhs: s is applied at the end)
+                  // the column scale multiplies the unit directly
+                  const float2 c01 = need_row ? __fmul2_rn(make_float2(c4.x, c4.y), rs2) : make_float2(c4.x, c4.y);
+                  const float2 c23 = need_row ? __fmul2_rn(make_float2(c4.z, c4.w), rs2) : make_float2(c4.z, c4.w);
                   acc[c * 16 + 2 * i] = __ffma2_rn(
                       make_float2(__uint_as_float(vv[4 * i]), __uint_as_float(vv[4 * i + 1])), c01,
                       acc[c * 16 + 2 * i]);

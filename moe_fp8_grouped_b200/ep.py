@@ -1,0 +1,159 @@
+"""Expert parallelism around the grouped matmul.
+
+Each of P ranks holds E/P consecutive experts.  A token routed to k experts
+sends one row per choice to the rank that holds the expert; the rank runs
+gmm_fwd on the rows it received, grouped by its local experts (the
+group_offset view of a ragged dot: "FP8 Megablox for batch split", maxtext
+PR #3770, Description item 3), and the results travel back to be summed per
+token with the routing weights.  Rows are quantized before they move, so
+E4M3 codes (one byte per element) cross the links instead of bf16 ("add
+static LHS scaling support for GMM v2 FWD", maxtext PR #4735, rebase commit
+text: quantize before the expert-parallel exchange and ragged sort).  That
+needs a scale that does not depend on the row's position, i.e. the static
+rule.
+
+Split of the work:
+  - routing metadata (``route``, ``exchange_counts``, ``local_order``): small
+    integer tensors and their exchange, on any device (tested on CPU with
+    gloo ranks);
+  - the row exchange (``exchange_rows``): ``torch.distributed`` all-to-all,
+    NCCL on GPUs;
+  - row movement and arithmetic (``ep_moe_fwd``): the library's kernels
+    (gmm_gather_rows, gmm_fwd, gmm_combine_rows), CUDA only.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+import torch.distributed as dist
+
+from . import _binding as B
+from .ops import _check, _dev, _stream, gmm_fwd
+
+
+@dataclass
+class Route:
+    """Where each (token, choice) row goes.  Experts are owned in contiguous
+    blocks: rank r holds experts [r * E/P, (r + 1) * E/P)."""
+    E: int
+    P: int
+    k: int
+    order: torch.Tensor         # int64 [T*k]: flat positions t*k + j sorted by expert (stable)
+    counts: torch.Tensor        # int64 [E]: rows per expert from this rank
+    send_splits: list           # rows sent to each rank
+
+
+def route(expert_ids: torch.Tensor, E: int, P: int) -> Route:
+    """Sort this rank's routed rows by expert: the send order of the exchange."""
+    if E % P:
+        raise ValueError(f"{E} experts do not split over {P} ranks")
+    T, k = expert_ids.shape
+    flat = expert_ids.reshape(-1).to(torch.int64)
+    if flat.numel() and (int(flat.min()) < 0 or int(flat.max()) >= E):
+        raise ValueError("expert id out of range")
+    order = torch.argsort(flat, stable=True)
+    counts = torch.bincount(flat, minlength=E)
+    send = counts.view(P, E // P).sum(dim=1)
+    return Route(E, P, k, order, counts, [int(v) for v in send.tolist()])
+
+
+def exchange_counts(rt: Route, group=None) -> torch.Tensor:
+    """int64 [P, E/P]: rows each source rank sends to each of this rank's
+    experts.  One all-to-all of E integers."""
+    El = rt.E // rt.P
+    if rt.P == 1:
+        return rt.counts.view(1, El).clone()
+    recv = torch.empty_like(rt.counts)
+    dist.all_to_all_single(recv, rt.counts, group=group)  # E / P counts to each rank
+    return recv.view(rt.P, El)
+
+
+def local_order(recv_counts: torch.Tensor):
+    """Rows arrive grouped by source rank, then by expert.  Returns (perm,
+    group_sizes): perm[i] is the arrival index of the i-th row when the rows
+    are grouped by local expert (then by source rank), and group_sizes the
+    rows per local expert."""
+    P, El = recv_counts.shape
+    cnt = recv_counts.reshape(-1)
+    start = torch.cumsum(cnt, 0) - cnt  # arrival offset of block (p, e)
+    by_expert = torch.arange(P * El, device=cnt.device).view(P, El).t().reshape(-1)  # blocks (e, p)
+    c = cnt[by_expert]
+    total = int(c.sum())
+    first = torch.repeat_interleave(start[by_expert], c)
+    within = torch.arange(total, device=cnt.device) - torch.repeat_interleave(torch.cumsum(c, 0) - c, c)
+    return first + within, recv_counts.sum(dim=0)
+
+
+def exchange_rows(buf: torch.Tensor, in_splits, out_splits, group=None) -> torch.Tensor:
+    """All-to-all of rows: in_splits rows of buf go to each rank; out_splits
+    rows arrive from each rank, in rank order."""
+    out = torch.empty((sum(out_splits),) + tuple(buf.shape[1:]), dtype=buf.dtype, device=buf.device)
+    if len(in_splits) == 1:
+        out.copy_(buf)
+        return out
+    dist.all_to_all_single(out, buf, output_split_sizes=list(out_splits), input_split_sizes=list(in_splits),
+                           group=group)
+    return out
+
+
+def gather_rows(src: torch.Tensor, idx: torch.Tensor) -> torch.Tensor:
+    """dst[i] = src[idx[i]] with the library's row gather (CUDA)."""
+    idx32 = idx.to(device=src.device, dtype=torch.int32).contiguous()
+    dst = torch.empty((idx32.numel(),) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else dst[0].numel() * dst.element_size()
+    st = B.lib().gmm_gather_rows(_dev(src, "src"), idx32.data_ptr(), idx32.numel(), row_bytes, src.shape[0],
+                                 dst.data_ptr(), _stream(src))
+    _check(st, "gmm_gather_rows")
+    return dst
+
+
+def combine_rows(rows: torch.Tensor, slot: torch.Tensor, weight: torch.Tensor, out_dtype=torch.bfloat16):
+    """y[t] = sum_j weight[t, j] * rows[slot[t, j]] with the library's kernel."""
+    T, k = slot.shape
+    N = rows.shape[1]
+    y = torch.empty((T, N), dtype=out_dtype, device=rows.device)
+    s32 = slot.to(torch.int32).contiguous()
+    w32 = weight.to(torch.float32).contiguous()
+    st = B.lib().gmm_combine_rows(_dev(rows, "rows", torch.bfloat16), rows.shape[0], _dev(s32, "slot"),
+                                  _dev(w32, "weight"), T, k, N, y.data_ptr(),
+                                  B.DT_F32 if out_dtype == torch.float32 else B.DT_BF16, _stream(rows))
+    _check(st, "gmm_combine_rows")
+    return y
+
+
+def ep_moe_fwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: torch.Tensor,
+               weights: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, group=None,
+               out_dtype=torch.bfloat16) -> torch.Tensor:
+    """One expert-parallel expert projection for this rank's T tokens.
+
+    x_codes: E4M3 codes [T, K] of the tokens (static rule, ``static_scale``
+    one float on the device); expert_ids / weights: [T, k] routing; w_codes /
+    w_scales: this rank's experts [E/P, K, N] and [E/P, N].  Returns
+    y [T, N] = sum_j weights[t, j] * (x[t] @ W[expert_ids[t, j]]).
+    """
+    P = dist.get_world_size(group) if dist.is_initialized() else 1
+    El, K, N = w_codes.shape
+    T, k = expert_ids.shape
+    rt = route(expert_ids, El * P, P)
+    order = rt.order.to(x_codes.device)
+    # permute: this rank's routed rows in expert order, E4M3 codes
+    send = gather_rows(x_codes, order // k)
+    recv_counts = exchange_counts(rt, group)
+    arrive = [int(v) for v in recv_counts.sum(dim=1).tolist()]
+    recv = exchange_rows(send, rt.send_splits, arrive, group)
+    perm, gsz = local_order(recv_counts.to(x_codes.device))
+    lhs = gather_rows(recv, perm)
+    if lhs.shape[0]:
+        h = gmm_fwd(lhs, w_codes, w_scales, gsz.to(device=x_codes.device, dtype=torch.int32), rule="static",
+                    static_scale=static_scale, out_dtype=torch.bfloat16)
+    else:  # no rows for this rank's experts
+        h = torch.empty((0, N), dtype=torch.bfloat16, device=x_codes.device)
+    # back in arrival order, then to the source ranks
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(perm.numel(), device=perm.device)
+    back = exchange_rows(gather_rows(h, inv), arrive, rt.send_splits, group)
+    # back[i] is the result of flat position order[i]; slot of (t, j) = i
+    slot = torch.empty_like(order)
+    slot[order] = torch.arange(order.numel(), device=order.device)
+    return combine_rows(back, slot.view(T, k), weights, out_dtype)
