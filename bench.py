@@ -372,6 +372,39 @@ def run_ours(args):
                                             "product; timed apart from the step, L2 flushed per call"}
         del sw_out, flush
 
+    # expert-parallel forward (ep_moe_fwd: row gather by expert, exchange,
+    # gmm_fwd on the local experts, return and weighted combine) on the
+    # EP-shrunk workload: M rows = T tokens x top-2; one rank, so the
+    # exchange is the identity and the time is the data movement around the
+    # gmm plus the gmm itself
+    if w.name == "ep_merged" and rule == "static" and world == 1 and not blocks:
+        from moe_fp8_grouped_b200 import ep
+        T, kk = M // 2, 2
+        gen = torch.Generator(device=dev).manual_seed(1)
+        ids = torch.stack([torch.randperm(G, generator=gen, device=dev)[:kk] for _ in range(T)]).to(torch.int32)
+        wts = torch.softmax(torch.randn(T, kk, generator=gen, device=dev), dim=1)
+        xq, _ = gm.gmm_quantize(lhs[:T].contiguous(), "static", axis=1, static_scale=s_static)
+        for _ in range(3):
+            ep.ep_moe_fwd(xq, s_static, ids, wts, codes, rscales)
+        barrier()
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        evs = []
+        for _ in range(min(args.steps, 20)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            ep.ep_moe_fwd(xq, s_static, ids, wts, codes, rscales)
+            b.record()
+            evs.append((a, b))
+        barrier()
+        ep_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+        passes["ep_moe_fwd"] = {"ms": round(ep_ms, 4), "tflops": round(flops_pass / (ep_ms / 1e3) / 1e12, 1),
+                                "gemm_fwd_ms": passes.get("fwd", {}).get("gemm_ms"),
+                                "note": f"{T} tokens x top-{kk} over {G} experts, one rank: gather E4M3 rows "
+                                        "by expert, gmm_fwd, gather back, weighted combine (bf16 out); "
+                                        "host-side routing metadata included; L2 flushed per call"}
+        del flush
+
     # end to end: pinned host buffers, copies inside the timed region.  Steps
     # are pipelined over three streams (upload, compute, download) with two
     # device buffer sets, so step i's download overlaps step i+1's upload and

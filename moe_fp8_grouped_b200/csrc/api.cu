@@ -378,7 +378,7 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
   // per-block promotion for dynamic lhs scales or block-wise rhs scales
-  const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk)};
+  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk)};
   const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   if ((s = cuda_status(prof(F ? "gemm_fwd_swiglu" : "gemm_fwd", st,
@@ -465,7 +465,7 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   p.ld_out = K;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{MODE_ROWS, elem, bmn, elem == 1};
+  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1};
   const int64_t items = ((M + 127) / 128 + G) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   if ((s = cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)

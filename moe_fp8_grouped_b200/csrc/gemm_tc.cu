@@ -110,7 +110,7 @@ template <int kMode>
 __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const int *s_offs, const int *s_tpre,
                                             int tn) {
   Item t;
-  if constexpr (kMode == MODE_ROWS) {
+  if constexpr (kMode != MODE_TGMM) {
     // items of group g: (tpre[g+1] - tpre[g]) row tiles x tn column tiles,
     // row tiles fastest
     int lo = 0, hi = p.G + 1;  // first i with tpre[i] * tn > w
@@ -251,10 +251,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   //                  s_x[chunk, k] (per unit)
   //   row scales:    promoted row-ragged passes with a dynamic row operand
   //                  (s_l / s_t per 128-block); tgmm: s_d[chunk, n]
-  const bool need_col = kTg ? (kPromote && p.colblk_scale != nullptr)
-                            : (p.col_scale != nullptr || p.colblk_scale != nullptr);
-  const bool need_row = kPromote && p.row_scale != nullptr;
-  const bool unit_col = kPromote && p.colblk_scale != nullptr;  // column scales change per unit
+  constexpr bool kBlkScales = (kMode == MODE_ROWS_BLK);
+  const bool need_col = kTg ? (kPromote && p.colblk_scale != nullptr) : (kBlkScales || p.col_scale != nullptr);
+  // block-wise rhs with a static lhs has no row scales (s is applied at the end)
+  const bool need_row = kPromote && (!kBlkScales || p.row_scale != nullptr);
+  const bool unit_col = kBlkScales || (kTg && kPromote && p.colblk_scale != nullptr);  // column scales per unit
   const bool use_ring = need_col || need_row;
 
   if (threadIdx.x == 0) {
@@ -421,8 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n < p.ncols) {
               const float *src =
                   kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
-                      : (p.colblk_scale ? p.colblk_scale + (static_cast<int64_t>(t.g) * p.kblocks + j) * p.colblk_ld + n
-                                        : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n);
+                      : (kBlkScales ? p.colblk_scale + (static_cast<int64_t>(t.g) * p.kblocks + j) * p.colblk_ld + n
+                              : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n);
               float *dst = s_scol + slot * kBN + 8 * lane;
               cp_async_16(dst, src);
               cp_async_16(dst + 4, src + 4);
@@ -577,8 +578,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const float4 c4 = *reinterpret_cast<const float4 *>(cs + colt(c) + 4 * i);
                   // without row scales (static lhs: s is applied at the end)
                   // the column scale multiplies the unit directly
-                  const float2 c01 = need_row ? __fmul2_rn(make_float2(c4.x, c4.y), rs2) : make_float2(c4.x, c4.y);
-                  const float2 c23 = need_row ? __fmul2_rn(make_float2(c4.z, c4.w), rs2) : make_float2(c4.z, c4.w);
+                  const bool rowmul = kTg || need_row;  // tgmm always has dout chunk scales
+                  const float2 c01 = rowmul ? __fmul2_rn(make_float2(c4.x, c4.y), rs2) : make_float2(c4.x, c4.y);
+                  const float2 c23 = rowmul ? __fmul2_rn(make_float2(c4.z, c4.w), rs2) : make_float2(c4.z, c4.w);
                   acc[c * 16 + 2 * i] = __ffma2_rn(
                       make_float2(__uint_as_float(vv[4 * i]), __uint_as_float(vv[4 * i + 1])), c01,
                       acc[c * 16 + 2 * i]);
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (row_ok) {
           // per-channel rhs column scale (in every unit's slot); static lhs: s
-          const float fin = p.static_scale ? s_eff : 1.0f;
+          const float fin = ((kTg || kBlkScales) && p.static_scale) ? s_eff : 1.0f;
           const bool colmul = !kTg && p.col_scale != nullptr;
           const float *cf = s_scol + slot * kBN;
           if (sw) {
@@ -756,6 +758,11 @@ cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUt
     if (cfg.elem_bytes == 1 && cfg.promote) return launch_inst<1, false, true, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
     if (cfg.elem_bytes == 2 && !cfg.promote) return launch_inst<2, false, false, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
     return cudaErrorInvalidValue;
+  }
+  if (cfg.mode == MODE_ROWS_BLK) {  // block-wise rhs scales: promoted fp8 only
+    if (cfg.elem_bytes != 1 || !cfg.promote) return cudaErrorInvalidValue;
+    return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK>(tmA, tmB, tmOut, p, grid, st)
+                          : launch_inst<1, false, true, MODE_ROWS_BLK>(tmA, tmB, tmOut, p, grid, st);
   }
   if (cfg.elem_bytes == 1) {
     if (cfg.b_mn_major)

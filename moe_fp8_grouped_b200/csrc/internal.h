@@ -66,7 +66,10 @@ cudaError_t launch_quant_rhs_blocks(const void *w, int G, int64_t K, int64_t N, 
 
 cudaError_t launch_timeout_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t st);
 
-enum GemmMode { MODE_ROWS = 0, MODE_TGMM = 1 };
+// MODE_ROWS_BLK: MODE_ROWS whose rhs has block-wise scales (a column scale per
+// contraction block, applied per TMEM unit); a separate instantiation so that
+// the per-channel kernels carry none of its code.
+enum GemmMode { MODE_ROWS = 0, MODE_TGMM = 1, MODE_ROWS_BLK = 2 };
 
 // Tile space of one GEMM launch.  MODE_ROWS (forward, dlhs): tile rows are
 // 128-row slices of one group's rows, tile columns the output columns.

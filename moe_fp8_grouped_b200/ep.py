@@ -45,17 +45,22 @@ class Route:
 
 
 def route(expert_ids: torch.Tensor, E: int, P: int) -> Route:
-    """Sort this rank's routed rows by expert: the send order of the exchange."""
+    """Sort this rank's routed rows by expert: the send order of the exchange.
+    One host synchronization: the range check of the ids, together with the
+    send splits when there is more than one rank."""
     if E % P:
         raise ValueError(f"{E} experts do not split over {P} ranks")
     T, k = expert_ids.shape
     flat = expert_ids.reshape(-1).to(torch.int64)
-    if flat.numel() and (int(flat.min()) < 0 or int(flat.max()) >= E):
-        raise ValueError("expert id out of range")
+    bad = ((flat < 0) | (flat >= E)).sum().view(1)
     order = torch.argsort(flat, stable=True)
-    counts = torch.bincount(flat, minlength=E)
+    counts = torch.zeros(E, dtype=torch.int64, device=flat.device)
+    counts.index_add_(0, flat.clamp(0, E - 1), torch.ones_like(flat))
     send = counts.view(P, E // P).sum(dim=1)
-    return Route(E, P, k, order, counts, [int(v) for v in send.tolist()])
+    host = torch.cat([bad, send]).tolist() if P > 1 else bad.tolist()
+    if host[0]:
+        raise ValueError("expert id out of range")
+    return Route(E, P, k, order, counts, host[1:] if P > 1 else [T * k])
 
 
 def exchange_counts(rt: Route, group=None) -> torch.Tensor:
@@ -135,25 +140,28 @@ def ep_moe_fwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
     P = dist.get_world_size(group) if dist.is_initialized() else 1
     El, K, N = w_codes.shape
     T, k = expert_ids.shape
-    rt = route(expert_ids, El * P, P)
-    order = rt.order.to(x_codes.device)
+    rt = route(expert_ids.to(x_codes.device), El * P, P)
+    order = rt.order
     # permute: this rank's routed rows in expert order, E4M3 codes
     send = gather_rows(x_codes, order // k)
-    recv_counts = exchange_counts(rt, group)
-    arrive = [int(v) for v in recv_counts.sum(dim=1).tolist()]
-    recv = exchange_rows(send, rt.send_splits, arrive, group)
-    perm, gsz = local_order(recv_counts.to(x_codes.device))
-    lhs = gather_rows(recv, perm)
-    if lhs.shape[0]:
-        h = gmm_fwd(lhs, w_codes, w_scales, gsz.to(device=x_codes.device, dtype=torch.int32), rule="static",
-                    static_scale=static_scale, out_dtype=torch.bfloat16)
+    if P == 1:
+        # nothing to exchange: the sorted rows are already grouped by expert
+        back_rows, gsz = send, rt.counts
+    else:
+        recv_counts = exchange_counts(rt, group)
+        arrive = [int(v) for v in recv_counts.sum(dim=1).tolist()]
+        recv = exchange_rows(send, rt.send_splits, arrive, group)
+        perm, gsz = local_order(recv_counts)
+        back_rows = gather_rows(recv, perm)
+    if back_rows.shape[0]:
+        h = gmm_fwd(back_rows, w_codes, w_scales, gsz.to(torch.int32), rule="static", static_scale=static_scale,
+                    out_dtype=torch.bfloat16)
     else:  # no rows for this rank's experts
         h = torch.empty((0, N), dtype=torch.bfloat16, device=x_codes.device)
-    # back in arrival order, then to the source ranks
-    inv = torch.empty_like(perm)
-    inv[perm] = torch.arange(perm.numel(), device=perm.device)
-    back = exchange_rows(gather_rows(h, inv), arrive, rt.send_splits, group)
-    # back[i] is the result of flat position order[i]; slot of (t, j) = i
-    slot = torch.empty_like(order)
-    slot[order] = torch.arange(order.numel(), device=order.device)
-    return combine_rows(back, slot.view(T, k), weights, out_dtype)
+    if P > 1:
+        # back in arrival order, then to the source ranks
+        inv = torch.empty_like(perm).scatter_(0, perm, torch.arange(perm.numel(), device=perm.device))
+        h = exchange_rows(gather_rows(h, inv), arrive, rt.send_splits, group)
+    # h[i] is the result of flat position order[i]; slot of (t, j) = i
+    slot = torch.empty_like(order).scatter_(0, order, torch.arange(order.numel(), device=order.device))
+    return combine_rows(h, slot.view(T, k), weights, out_dtype)
