@@ -398,12 +398,35 @@ def run_ours(args):
             evs.append((a, b))
         barrier()
         ep_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+        # the same call captured as a CUDA graph (one rank: no host synchronization)
+        try:
+            graph = ep.EPForwardGraph(xq, s_static, ids, wts, codes, rscales)
+        except RuntimeError as exc:  # capture refused by the runtime: report the eager time only
+            graph, graph_err = None, str(exc).splitlines()[0]
+        ep_graph_ms = None
+        if graph is not None:
+            barrier()
+            evs = []
+            for _ in range(min(args.steps, 20)):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                graph.replay()
+                b.record()
+                evs.append((a, b))
+            barrier()
+            ep_graph_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
         passes["ep_moe_fwd"] = {"ms": round(ep_ms, 4), "tflops": round(flops_pass / (ep_ms / 1e3) / 1e12, 1),
+                                "graph_ms": round(ep_graph_ms, 4) if ep_graph_ms else None,
+                                "graph_tflops": (round(flops_pass / (ep_graph_ms / 1e3) / 1e12, 1)
+                                                 if ep_graph_ms else None),
+                                **({} if graph is not None else {"graph_error": graph_err}),
                                 "gemm_fwd_ms": passes.get("fwd", {}).get("gemm_ms"),
-                                "note": f"{T} tokens x top-{kk} over {G} experts, one rank: gather E4M3 rows "
-                                        "by expert, gmm_fwd, gather back, weighted combine (bf16 out); "
-                                        "host-side routing metadata included; L2 flushed per call"}
-        del flush
+                                "note": f"{T} tokens x top-{kk} over {G} experts, one rank: route (sort by "
+                                        "expert), gather E4M3 rows, gmm_fwd, weighted combine (bf16 out); ms: "
+                                        "eager calls (ids checked each call); graph_ms: the same kernels "
+                                        "replayed from a CUDA graph; L2 flushed per call"}
+        del flush, graph
 
     # end to end: pinned host buffers, copies inside the timed region.  Steps
     # are pipelined over three streams (upload, compute, download) with two

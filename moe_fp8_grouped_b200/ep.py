@@ -44,10 +44,13 @@ class Route:
     send_splits: list           # rows sent to each rank
 
 
-def route(expert_ids: torch.Tensor, E: int, P: int) -> Route:
+def route(expert_ids: torch.Tensor, E: int, P: int, validate: bool = True) -> Route:
     """Sort this rank's routed rows by expert: the send order of the exchange.
     One host synchronization: the range check of the ids, together with the
-    send splits when there is more than one rank."""
+    send splits when there is more than one rank.  validate=False (one rank
+    only) skips the check and the synchronization, for ids already checked
+    (for example in a captured CUDA graph); out-of-range ids are then counted
+    against the nearest valid expert."""
     if E % P:
         raise ValueError(f"{E} experts do not split over {P} ranks")
     T, k = expert_ids.shape
@@ -57,6 +60,8 @@ def route(expert_ids: torch.Tensor, E: int, P: int) -> Route:
     counts = torch.zeros(E, dtype=torch.int64, device=flat.device)
     counts.index_add_(0, flat.clamp(0, E - 1), torch.ones_like(flat))
     send = counts.view(P, E // P).sum(dim=1)
+    if P == 1 and not validate:
+        return Route(E, P, k, order, counts, [T * k])
     host = torch.cat([bad, send]).tolist() if P > 1 else bad.tolist()
     if host[0]:
         raise ValueError("expert id out of range")
@@ -129,18 +134,20 @@ def combine_rows(rows: torch.Tensor, slot: torch.Tensor, weight: torch.Tensor, o
 
 def ep_moe_fwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: torch.Tensor,
                weights: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, group=None,
-               out_dtype=torch.bfloat16) -> torch.Tensor:
+               out_dtype=torch.bfloat16, validate: bool = True) -> torch.Tensor:
     """One expert-parallel expert projection for this rank's T tokens.
 
     x_codes: E4M3 codes [T, K] of the tokens (static rule, ``static_scale``
     one float on the device); expert_ids / weights: [T, k] routing; w_codes /
     w_scales: this rank's experts [E/P, K, N] and [E/P, N].  Returns
     y [T, N] = sum_j weights[t, j] * (x[t] @ W[expert_ids[t, j]]).
+    On one rank with validate=False nothing synchronizes with the host, so
+    the call can be captured in a CUDA graph (see EPForwardGraph).
     """
     P = dist.get_world_size(group) if dist.is_initialized() else 1
     El, K, N = w_codes.shape
     T, k = expert_ids.shape
-    rt = route(expert_ids.to(x_codes.device), El * P, P)
+    rt = route(expert_ids.to(x_codes.device), El * P, P, validate=validate or P > 1)
     order = rt.order
     # permute: this rank's routed rows in expert order, E4M3 codes
     send = gather_rows(x_codes, order // k)
@@ -165,3 +172,31 @@ def ep_moe_fwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
     # h[i] is the result of flat position order[i]; slot of (t, j) = i
     slot = torch.empty_like(order).scatter_(0, order, torch.arange(order.numel(), device=order.device))
     return combine_rows(h, slot.view(T, k), weights, out_dtype)
+
+
+class EPForwardGraph:
+    """ep_moe_fwd on one rank captured once as a CUDA graph over fixed
+    buffers: every replay runs the same kernels without their per-call host
+    cost.  The routing ids are checked once, when the graph is made; to run
+    new inputs, copy them into ``x_codes`` / ``expert_ids`` / ``weights``
+    (check new ids first, with ``route(ids, E, 1)``) and call ``replay()``;
+    the result is ``out``."""
+
+    def __init__(self, x_codes, static_scale, expert_ids, weights, w_codes, w_scales, out_dtype=torch.bfloat16):
+        if dist.is_initialized() and dist.get_world_size() > 1:
+            raise ValueError("a captured EP forward covers one rank only (the exchange sizes are data-dependent)")
+        self.args = (x_codes, static_scale, expert_ids, weights, w_codes, w_scales)
+        ep_moe_fwd(*self.args, out_dtype=out_dtype)  # checks the ids, sets up the workspace
+        side = torch.cuda.Stream(device=x_codes.device)
+        side.wait_stream(torch.cuda.current_stream(x_codes.device))
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                ep_moe_fwd(*self.args, out_dtype=out_dtype, validate=False)
+        torch.cuda.current_stream(x_codes.device).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.out = ep_moe_fwd(*self.args, out_dtype=out_dtype, validate=False)
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.out

@@ -76,3 +76,21 @@ def test_ep_moe_fwd_single_rank(dev, T, E, k, K, N, out_dtype):
             mag[sel] += np.abs(wj * h[sel])
     bound += k * 2.0 ** -23 * mag + (2.0 ** -8 * np.abs(ref) if out_dtype == torch.bfloat16 else 0.0)
     assert_within(y, ref, bound, f"ep_moe_fwd T={T} E={E} k={k}")
+
+
+def test_ep_forward_graph_replays_the_eager_result(dev):
+    g = torch.Generator().manual_seed(5)
+    T, E, k, K, N = 64, 8, 2, 256, 256
+    x = torch.randn(T, K, generator=g).bfloat16().to(dev)
+    w = (torch.randn(E, K, N, generator=g) * 0.02).bfloat16().to(dev)
+    ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(dev)
+    wts = torch.softmax(torch.randn(T, k, generator=g), dim=1).to(dev)
+    s = torch.tensor([4.0 / 448.0], device=dev)
+    codes, scales = gm.gmm_quantize_rhs(w)
+    xq, _ = gm.gmm_quantize(x, "static", axis=1, static_scale=s)
+    eager = ep.ep_moe_fwd(xq, s, ids, wts, codes, scales)
+    graph = ep.EPForwardGraph(xq, s, ids, wts, codes, scales)
+    assert torch.equal(graph.replay(), eager)
+    # new routing weights copied into the captured buffer change the result
+    wts.copy_(wts.flip(1))
+    assert torch.equal(graph.replay(), ep.ep_moe_fwd(xq, s, ids, wts, codes, scales))
