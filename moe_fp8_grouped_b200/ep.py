@@ -56,7 +56,7 @@ def route(expert_ids: torch.Tensor, E: int, P: int, validate: bool = True) -> Ro
     T, k = expert_ids.shape
     flat = expert_ids.reshape(-1).to(torch.int64)
     bad = ((flat < 0) | (flat >= E)).sum().view(1)
-    order = torch.argsort(flat, stable=True)
+    order = torch.argsort(flat.to(torch.int32), stable=True)  # 32-bit keys: half the radix passes
     counts = torch.zeros(E, dtype=torch.int64, device=flat.device)
     counts.index_add_(0, flat.clamp(0, E - 1), torch.ones_like(flat))
     send = counts.view(P, E // P).sum(dim=1)
