@@ -139,10 +139,11 @@ gmm_status gmm_quantize_rhs_blocks(const void *w_bf16, int32_t G, int64_t K, int
  *   (this folds the rhs scale into dout for dlhs); group_sizes is then needed.
  * axis == 0: the tgmm operand.  Each group's rows are cut into 128-row chunks
  *   starting at the group's first row; chunk j (over all groups, in group
- *   order) gets one scale per column.  codes are stored transposed and
- *   padded: [cols, 128 * gmm_chunk_capacity(rows, G)], chunk j in columns
- *   [128 j, 128 j + 128), pad rows 0.  scales [gmm_chunk_capacity, cols]
- *   (written for STATIC too, all equal to the static scale).
+ *   order) gets one scale per column.  codes are stored transposed,
+ *   chunk-major and padded: [gmm_chunk_capacity(rows, G), cols, 128], the
+ *   128 codes of chunk j and column c contiguous (its rows in order, pad rows
+ *   0).  scales [gmm_chunk_capacity, cols] (written for STATIC too, all equal
+ *   to the static scale).
  * rule: STATIC (static_scale = device pointer to one float) or DYNAMIC.
  * ws: workspace of at least gmm_workspace_bytes(...) for the pass that
  * consumes this operand.

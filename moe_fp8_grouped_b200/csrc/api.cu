@@ -508,12 +508,15 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   }));
   if (s != GMM_OK) return s;
   const uint32_t bke = 128 / elem;
-  const uint64_t ldt = static_cast<uint64_t>(cap) * kBlk;  // elements per transposed row
   // tile rows = dout columns n (A = dout^T chunks), tile columns = lhs columns
-  // k (B = lhs^T chunks); the epilogue writes dW[g, k, n]
+  // k (B = lhs^T chunks); the epilogue writes dW[g, k, n].  The chunk-major
+  // operands [chunk][column][128] are 2-D tensors of 128-element lines: chunk
+  // j's line of column c is row j * C + c, so every box is one contiguous block.
   CUtensorMap tmA, tmB;
-  if (!make_map(&tmA, P.codes_b, elem, ldt, N, ldt * elem, bke, 128)) return GMM_ERR_CUDA;
-  if (!make_map(&tmB, P.codes_a, elem, ldt, K, ldt * elem, bke, 256)) return GMM_ERR_CUDA;
+  if (!make_map(&tmA, P.codes_b, elem, kBlk, static_cast<uint64_t>(cap) * N, kBlk * elem, bke, 128))
+    return GMM_ERR_CUDA;
+  if (!make_map(&tmB, P.codes_a, elem, kBlk, static_cast<uint64_t>(cap) * K, kBlk * elem, bke, 256))
+    return GMM_ERR_CUDA;
   CUtensorMap tmOut;  // dW as [G*K, N]: each epilogue warp stores 32 k-rows x 32 n
   if (!make_out_map(&tmOut, drhs, out_dtype == GMM_F32, N, static_cast<uint64_t>(G) * K, 32, 32))
     return GMM_ERR_CUDA;

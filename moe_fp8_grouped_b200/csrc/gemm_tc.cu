@@ -325,10 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               by = t.g * p.b_group_rows + t.ct * kBN;
             }
           } else {
-            ax = s_tpre[t.g] * kBlk + b * kBKe;  // the group's chunks in the transposed operands
-            ay = t.rt * kBM;                     // dout columns n
+            // chunk jj of the group (stages_per_chunk stages each) in the
+            // chunk-major operands: line rows jj * N + n and jj * K + k
+            const int jj = s_tpre[t.g] + b / p.stages_per_chunk;
+            ax = (b % p.stages_per_chunk) * kBKe;
+            ay = jj * (p.rtiles * kBM) + t.rt * kBM;  // dout columns n
             bx = ax;
-            by = t.ct * kBN;                     // lhs columns k
+            by = jj * p.ncols + t.ct * kBN;           // lhs columns k (rows past K belong to the
+                                                      // next chunk: their columns are never stored)
           }
           tma_load_2d(sA + s * kAStage, &tmA, ax, ay, &full[s]);
           if constexpr (kBMN) {

@@ -241,8 +241,8 @@ cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dy
 // One CTA of 128 threads per (256-column slice, chunk).  The chunk's rows (at
 // most 128, the rest zero) are staged in shared memory with cp.async; thread t
 // owns the adjacent columns 2t and 2t+1: it takes each column's absmax over the
-// chunk and writes each column's 128 codes as one 128-byte line of the
-// transposed code matrix.
+// chunk and writes each column's 128 codes as one line of the chunk-major
+// transposed layout [chunk][column][128], so a CTA writes one contiguous block.
 constexpr int kChunkCols = 256;
 constexpr int kChunkThreads = 128;
 constexpr int kChunkPitch = kChunkCols + 8;  // bf16 per staged row (16-byte aligned rows)
@@ -274,8 +274,8 @@ __device__ __forceinline__ bool find_chunk(int j, const int *offs, const int *tp
 template <bool kDynamic, bool kCopy>
 __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
     const __nv_bfloat16 *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ static_scale,
-    const int *__restrict__ offs, const int *__restrict__ tpre, int G, void *codes_t, int64_t ld_t,
-    float *__restrict__ scales, uint32_t *__restrict__ status) {
+    const int *__restrict__ offs, const int *__restrict__ tpre, int G, void *codes_t, float *__restrict__ scales,
+    uint32_t *__restrict__ status) {
   extern __shared__ __align__(16) uint8_t qsm[];
   __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(qsm);  // [128][kChunkPitch]
   __shared__ int s_info[3];
@@ -301,10 +301,11 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
   auto pair = [&](int r) -> float2 {
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t32[(r * kChunkPitch + col) >> 1]));
   };
+  const int64_t line = (static_cast<int64_t>(j) * cols + c0 + col) * kBlk;  // element offset of column col's line
   if constexpr (kCopy) {
     // bf16 family: transposed bf16 copy, no scale
-    uint16_t *dst0 = static_cast<uint16_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
-    uint16_t *dst1 = dst0 + ld_t;
+    uint16_t *dst0 = static_cast<uint16_t *>(codes_t) + line;
+    uint16_t *dst1 = dst0 + kBlk;
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
       uint32_t w0[4], w1[4];
@@ -339,8 +340,8 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
       s0 = s1 = s;
       inv0 = inv1 = inv;
     }
-    uint8_t *dst0 = static_cast<uint8_t *>(codes_t) + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
-    uint8_t *dst1 = dst0 + ld_t;
+    uint8_t *dst0 = static_cast<uint8_t *>(codes_t) + line;
+    uint8_t *dst1 = dst0 + kBlk;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       uint32_t w0[4], w1[4];
@@ -363,13 +364,12 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
 template <bool kDynamic, bool kCopy>
 static cudaError_t launch_chunks_inst(dim3 grid, cudaStream_t st, const __nv_bfloat16 *xb, int64_t rows,
                                       int64_t cols, const float *static_scale, const int *offs, const int *tpre,
-                                      int G, void *codes_t, int64_t ld_t, float *scales, uint32_t *status) {
+                                      int G, void *codes_t, float *scales, uint32_t *status) {
   auto kern = quant_chunks_kernel<kDynamic, kCopy>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kChunkSmem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kChunkThreads, kChunkSmem, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t, scales,
-                                                status);
+  kern<<<grid, kChunkThreads, kChunkSmem, st>>>(xb, rows, cols, static_scale, offs, tpre, G, codes_t, scales, status);
   return cudaGetLastError();
 }
 
@@ -378,15 +378,14 @@ cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool 
                                 float *scales, bool bf16_copy, uint32_t *status, cudaStream_t st) {
   dim3 grid(static_cast<unsigned>((cols + kChunkCols - 1) / kChunkCols), static_cast<unsigned>(capacity));
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-  const int64_t ld_t = capacity * kBlk;
   if (bf16_copy)
-    return launch_chunks_inst<false, true>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t,
-                                           scales, status);
+    return launch_chunks_inst<false, true>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, scales,
+                                           status);
   if (dynamic)
-    return launch_chunks_inst<true, false>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t,
-                                           scales, status);
-  return launch_chunks_inst<false, false>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, ld_t,
-                                          scales, status);
+    return launch_chunks_inst<true, false>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, scales,
+                                           status);
+  return launch_chunks_inst<false, false>(grid, st, xb, rows, cols, static_scale, offs, tpre, G, codes_t, scales,
+                                          status);
 }
 
 // Already-quantized E4M3 lhs (static rule): its codes laid out as the chunk
@@ -397,7 +396,7 @@ constexpr int kCodePitch = kChunkCols + 16;  // bytes per staged row (16-byte al
 __global__ void __launch_bounds__(kChunkThreads) chunk_codes_kernel(const uint8_t *__restrict__ x, int64_t cols,
                                                                     const int *__restrict__ offs,
                                                                     const int *__restrict__ tpre, int G,
-                                                                    uint8_t *__restrict__ codes_t, int64_t ld_t) {
+                                                                    uint8_t *__restrict__ codes_t) {
   __shared__ __align__(16) uint8_t tile[kBlk * kCodePitch];
   __shared__ int s_info[3];
   const int j = blockIdx.y;
@@ -416,8 +415,8 @@ __global__ void __launch_bounds__(kChunkThreads) chunk_codes_kernel(const uint8_
   __syncthreads();
   const int col = 2 * threadIdx.x;  // and col + 1
   if (c0 + col >= cols) return;     // cols is a multiple of 128: both columns are in or out
-  uint8_t *dst0 = codes_t + (c0 + col) * ld_t + static_cast<int64_t>(kBlk) * j;
-  uint8_t *dst1 = dst0 + ld_t;
+  uint8_t *dst0 = codes_t + (static_cast<int64_t>(j) * cols + c0 + col) * kBlk;
+  uint8_t *dst1 = dst0 + kBlk;
   auto pair = [&](int r) -> uint32_t { return *reinterpret_cast<const uint16_t *>(tile + r * kCodePitch + col); };
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -438,7 +437,7 @@ cudaError_t launch_chunk_codes(const uint8_t *codes, int64_t rows, int64_t cols,
                                int G, int64_t capacity, uint8_t *codes_t, cudaStream_t st) {
   (void)rows;  // rows past the plan are never read
   dim3 grid(static_cast<unsigned>((cols + kChunkCols - 1) / kChunkCols), static_cast<unsigned>(capacity));
-  chunk_codes_kernel<<<grid, kChunkThreads, 0, st>>>(codes, cols, offs, tpre, G, codes_t, capacity * kBlk);
+  chunk_codes_kernel<<<grid, kChunkThreads, 0, st>>>(codes, cols, offs, tpre, G, codes_t);
   return cudaGetLastError();
 }
 

@@ -113,7 +113,7 @@ def gmm_quantize(x: torch.Tensor, rule="dynamic", axis: int = 1, static_scale: t
         scales = torch.empty((cols // 128, rows), dtype=torch.float32, device=x.device)
     else:
         cap = gmm_chunk_capacity(rows, G)
-        codes = torch.empty((cols, 128 * cap), dtype=torch.uint8, device=x.device)
+        codes = torch.empty((cap, cols, 128), dtype=torch.uint8, device=x.device)
         scales = torch.empty((cap, cols), dtype=torch.float32, device=x.device)
     nbytes = gmm_workspace_bytes(B.OP_FWD, rows, cols, cols, G)
     if ws is None:

@@ -36,19 +36,19 @@ def rule_code(rule: str) -> int:
 
 
 def untranspose_chunks(codes_t: torch.Tensor, scales: torch.Tensor, offs: np.ndarray, M: int):
-    """GPU axis-0 layout (codes [C, 128*cap], scales [cap, C]) -> the oracle's
-    (codes [M, C] in row order, scales [num_chunks, C])."""
+    """GPU axis-0 layout (codes [cap, C, 128] chunk-major, scales [cap, C]) ->
+    the oracle's (codes [M, C] in row order, scales [num_chunks, C])."""
     ct = codes_t.cpu().numpy()
     sc = scales.cpu().numpy()
-    C = ct.shape[0]
+    C = ct.shape[1]
     out = np.zeros((M, C), dtype=np.uint8)
     j = 0
     for g in range(len(offs) - 1):
         for a in range(int(offs[g]), int(offs[g + 1]), 128):
             b = min(a + 128, int(offs[g + 1]))
-            out[a:b] = ct[:, 128 * j: 128 * j + (b - a)].T
+            out[a:b] = ct[j, :, :b - a].T
             # pad rows of the chunk must be zero codes
-            assert not ct[:, 128 * j + (b - a): 128 * (j + 1)].any(), "chunk padding not zero"
+            assert not ct[j, :, b - a:].any(), "chunk padding not zero"
             j += 1
     return out, sc[:j]
 
