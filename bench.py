@@ -377,7 +377,7 @@ def run_ours(args):
     # EP-shrunk workload: M rows = T tokens x top-2; one rank, so the
     # exchange is the identity and the time is the data movement around the
     # gmm plus the gmm itself
-    if w.name == "ep_merged" and rule == "static" and world == 1 and not blocks:
+    if w.name == "ep_merged" and parts == 1 and rule == "static" and world == 1 and not blocks:
         from moe_fp8_grouped_b200 import ep
         T, kk = M // 2, 2
         gen = torch.Generator(device=dev).manual_seed(1)
