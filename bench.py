@@ -50,6 +50,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate-backward", action="store_true",
+                    help="run dlhs and drhs as two calls (gmm_dlhs, tgmm_drhs) instead of gmm_backward, which "
+                         "quantizes dout once for both")
     ap.add_argument("--rhs-blocks", action="store_true",
                     help="block-wise weight scales: forward codes with [G, K/128, N] scales, dlhs codes with "
                          "[G, N/128, K] scales (two weight copies, made outside the timed step)")
@@ -231,8 +234,9 @@ def run_ours(args):
     out = torch.empty((M, Np), dtype=torch.bfloat16, device=dev)
     dl = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
     dw = torch.empty((G, K, Np), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, Np, G) for op in (0, 1, 2)), dtype=torch.uint8,
+    ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, Np, G) for op in (0, 1, 2, 3)), dtype=torch.uint8,
                      device=dev)
+    fused_bwd = not args.separate_backward
     sarg = s_static if rule == "static" else None
     grule = "none" if bf16_family else "dynamic"
     launches = [0]
@@ -245,10 +249,14 @@ def run_ours(args):
             launches[0] += gm.last_launch_count()
             if blocks:
                 c_, r_ = dl_codes, dl_scales
-            gm.gmm_dlhs(d_, c_, r_, gs_, out=dl, ws=ws, rule=grule)
-            launches[0] += gm.last_launch_count()
-            gm.tgmm_drhs(lhs_, d_, gs_, rule=rule, static_scale=sarg, out=dw, ws=ws)
-            launches[0] += gm.last_launch_count()
+            if fused_bwd:
+                gm.gmm_backward(lhs_, d_, c_, r_, gs_, rule=rule, static_scale=sarg, dlhs=dl, drhs=dw, ws=ws)
+                launches[0] += gm.last_launch_count()
+            else:
+                gm.gmm_dlhs(d_, c_, r_, gs_, out=dl, ws=ws, rule=grule)
+                launches[0] += gm.last_launch_count()
+                gm.tgmm_drhs(lhs_, d_, gs_, rule=rule, static_scale=sarg, out=dw, ws=ws)
+                launches[0] += gm.last_launch_count()
 
     def barrier():
         torch.cuda.synchronize()
@@ -472,10 +480,15 @@ def run_ours(args):
                     s_cmp.wait_event(down_done[b])  # download of step i-2 has read this output set
                 gm.gmm_fwd(a_lhs, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, out=o_out, ws=ws2[b])
                 launches[0] += gm.last_launch_count()
-                gm.gmm_dlhs(a_dout, a_codes, a_rs, a_gs, out=o_dl, ws=ws2[b], rule=grule)
-                launches[0] += gm.last_launch_count()
-                gm.tgmm_drhs(a_lhs, a_dout, a_gs, rule=rule, static_scale=sarg, out=o_dw, ws=ws2[b])
-                launches[0] += gm.last_launch_count()
+                if fused_bwd:
+                    gm.gmm_backward(a_lhs, a_dout, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, dlhs=o_dl,
+                                    drhs=o_dw, ws=ws2[b])
+                    launches[0] += gm.last_launch_count()
+                else:
+                    gm.gmm_dlhs(a_dout, a_codes, a_rs, a_gs, out=o_dl, ws=ws2[b], rule=grule)
+                    launches[0] += gm.last_launch_count()
+                    gm.tgmm_drhs(a_lhs, a_dout, a_gs, rule=rule, static_scale=sarg, out=o_dw, ws=ws2[b])
+                    launches[0] += gm.last_launch_count()
                 cmp_done[b].record(s_cmp)
             with torch.cuda.stream(s_down):
                 s_down.wait_event(cmp_done[b])
@@ -499,7 +512,7 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(ems / args.e2e_steps, 3),
                "path": "per step: pinned host -> device copies of lhs, dout, rhs codes + scales, group sizes; "
-                       "gmm_fwd + gmm_dlhs + tgmm_drhs; device -> pinned host copies of out, dlhs, dW. Steps "
+                       "gmm_fwd + gmm_backward (dlhs, drhs); device -> pinned host copies of out, dlhs, dW. Steps "
                        "pipelined over upload / compute / download streams with two device buffer sets."}
 
     cpu = None
@@ -517,6 +530,8 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if bf16_family else "e4m3", "data": "synthetic",
         "config": config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                                 "calls_per_pass": parts,
+                                "backward": ("gmm_backward (dout quantized once for dlhs and drhs)" if fused_bwd
+                                             else "gmm_dlhs + tgmm_drhs"),
                                 "rhs_scales": ("block-wise: fwd [G, K/128, N], dlhs [G, N/128, K]" if blocks
                                                else "per channel [G, N]"),
                                 **({"l2": "flushed before every step (256 MiB write outside the timed events; "

@@ -73,7 +73,7 @@ typedef enum {
 
 typedef enum { GMM_BF16 = 0, GMM_F32 = 1, GMM_E4M3 = 2 } gmm_dtype;
 
-typedef enum { GMM_OP_FWD = 0, GMM_OP_DLHS = 1, GMM_OP_DRHS = 2 } gmm_op;
+typedef enum { GMM_OP_FWD = 0, GMM_OP_DLHS = 1, GMM_OP_DRHS = 2, GMM_OP_BWD = 3 } gmm_op;
 
 /* Device status bits (gmm_read_device_status, `bits_out`). */
 #define GMM_DEV_GROUP_SIZES 1u
@@ -96,9 +96,9 @@ typedef struct {
   gmm_qrule rule;
 } gmm_operand;
 
-/* Bytes of workspace that gmm_fwd (op FWD), gmm_dlhs (DLHS) or tgmm_drhs
- * (DRHS) needs for these sizes; also enough for gmm_quantize with the same
- * operand.  Returns 0 for invalid sizes. */
+/* Bytes of workspace that gmm_fwd (op FWD), gmm_dlhs (DLHS), tgmm_drhs (DRHS)
+ * or gmm_backward (BWD) needs for these sizes; also enough for gmm_quantize
+ * with the same operand.  Returns 0 for invalid sizes. */
 size_t gmm_workspace_bytes(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G);
 
 /* Number of 128-row chunks a tgmm operand of `rows` rows and G groups can
@@ -252,6 +252,25 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
 gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_sizes, int32_t G, int64_t M,
                      int64_t K, int64_t N, void *drhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
                      void *stream);
+
+/*
+ * Both backward passes in one call: gmm_dlhs(dout, rhs) and tgmm_drhs(lhs,
+ * dout) with the arguments and results of those two calls, except that dout
+ * is read once: one kernel quantizes it into both operands (the dlhs row
+ * blocks, with the per-channel rhs scale folded in, and the tgmm chunk
+ * columns), which bit for bit equal what the two calls quantize.  The pages
+ * run dlhs and drhs as two kernels of the same backward ("Support
+ * quantization for tokamax gmm v2", maxtext PR #4451, Description); sharing
+ * the read of their common operand is a choice of this library.  lhs and
+ * dout are in the same family as for the separate calls (fp8: dout rule
+ * DYNAMIC; bf16 family: both NONE, rhs bf16).  Workspace:
+ * gmm_workspace_bytes(GMM_OP_BWD, M, K, N, G).  dlhs [M, K] of dlhs_dtype,
+ * drhs [G, K, N] of drhs_dtype.
+ */
+gmm_status gmm_backward(gmm_operand lhs, gmm_operand dout, gmm_operand rhs, int transpose_rhs,
+                        const int32_t *group_sizes, int32_t G, int64_t M, int64_t K, int64_t N, void *dlhs,
+                        gmm_dtype dlhs_dtype, void *drhs, gmm_dtype drhs_dtype, void *ws, size_t ws_bytes,
+                        void *stream);
 
 /*
  * Row movement for expert parallelism, the steps either side of the NCCL

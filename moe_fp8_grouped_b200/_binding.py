@@ -18,7 +18,7 @@ STATUS_NAMES = {0: "GMM_OK", 1: "GMM_ERR_INVALID_ARG", 2: "GMM_ERR_SHAPE", 3: "G
                 8: "GMM_ERR_TIMEOUT", 9: "GMM_ERR_WORKSPACE"}
 Q_NONE, Q_STATIC, Q_DYNAMIC = 0, 1, 2
 DT_BF16, DT_F32, DT_E4M3 = 0, 1, 2
-OP_FWD, OP_DLHS, OP_DRHS = 0, 1, 2
+OP_FWD, OP_DLHS, OP_DRHS, OP_BWD = 0, 1, 2, 3
 DEV_GROUP_SIZES, DEV_SCALE, DEV_TIMEOUT = 1, 2, 4
 
 # every symbol include/gmm_fp8.h declares
@@ -26,7 +26,7 @@ EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm
            "gmm_dlhs", "tgmm_drhs", "gmm_read_device_status", "gmm_selftest_timeout", "gmm_set_wait_limit_ns",
            "gmm_status_string", "gmm_last_launch_count", "gmm_profile_enable", "gmm_profile_collect",
            "gmm_fwd_noalloc", "gmm_fwd_swiglu", "gmm_quantize_rhs_blocks", "gmm_gather_rows",
-           "gmm_combine_rows"]
+           "gmm_combine_rows", "gmm_backward"]
 
 
 class Operand(ctypes.Structure):
@@ -64,6 +64,9 @@ def lib():
     L.gmm_fwd_swiglu.argtypes = L.gmm_fwd.argtypes
     L.gmm_quantize_rhs_blocks.argtypes = [vp, i32, i64, i64, ctypes.c_int, vp, vp, vp]
     L.gmm_quantize_rhs_blocks.restype = st
+    L.gmm_backward.argtypes = [Operand, Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int,
+                               vp, ctypes.c_int, vp, sz, vp]
+    L.gmm_backward.restype = st
     L.gmm_gather_rows.argtypes = [vp, vp, i64, i64, i64, vp, vp]
     L.gmm_gather_rows.restype = st
     L.gmm_combine_rows.argtypes = [vp, i64, vp, vp, i64, i32, i64, vp, ctypes.c_int, vp]

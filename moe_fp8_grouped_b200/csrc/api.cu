@@ -68,7 +68,9 @@ WsLayout ws_layout(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G) {
     L.scales_a = o;
     o += align256(sizeof(float) * static_cast<size_t>(M) * (C / kBlk));
     L.codes_b = L.scales_b = 0;
+    L.codes_r = L.scales_r = 0;
   } else {
+    L.codes_r = L.scales_r = 0;
     // transposed, chunk-padded operands; sized for 2-byte elements so that the
     // bf16 family fits as well
     const int64_t cap = chunk_capacity(M, G);
@@ -80,6 +82,12 @@ WsLayout ws_layout(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G) {
     o += align256(sizeof(float) * static_cast<size_t>(cap) * K);
     L.scales_b = o;
     o += align256(sizeof(float) * static_cast<size_t>(cap) * N);
+    if (op == GMM_OP_BWD) {  // + the dlhs row operand of dout
+      L.codes_r = o;
+      o += align256(static_cast<size_t>(M) * N);
+      L.scales_r = o;
+      o += align256(sizeof(float) * static_cast<size_t>(M) * (N / kBlk));
+    }
   }
   L.total = o;
   return L;
@@ -157,8 +165,8 @@ static gmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GMM_OK 
 struct WsPtrs {
   uint32_t *status;
   int *offs, *tpre;
-  uint8_t *codes_a, *codes_b;
-  float *scales_a, *scales_b;
+  uint8_t *codes_a, *codes_b, *codes_r;
+  float *scales_a, *scales_b, *scales_r;
 };
 
 static WsPtrs carve(void *ws, const WsLayout &L) {
@@ -171,6 +179,8 @@ static WsPtrs carve(void *ws, const WsLayout &L) {
   P.codes_b = L.codes_b ? w + L.codes_b : nullptr;
   P.scales_a = reinterpret_cast<float *>(w + L.scales_a);
   P.scales_b = L.scales_b ? reinterpret_cast<float *>(w + L.scales_b) : nullptr;
+  P.codes_r = L.codes_r ? w + L.codes_r : nullptr;
+  P.scales_r = L.scales_r ? reinterpret_cast<float *>(w + L.scales_r) : nullptr;
   return P;
 }
 
@@ -211,7 +221,7 @@ extern "C" {
 
 size_t gmm_workspace_bytes(gmm_op op, int64_t M, int64_t K, int64_t N, int32_t G) {
   if (check_sizes(M, K, N, G) != GMM_OK) return 0;
-  if (op != GMM_OP_FWD && op != GMM_OP_DLHS && op != GMM_OP_DRHS) return 0;
+  if (op != GMM_OP_FWD && op != GMM_OP_DLHS && op != GMM_OP_DRHS && op != GMM_OP_BWD) return 0;
   return ws_layout(op, M, K, N, G).total;
 }
 
@@ -404,41 +414,14 @@ gmm_status gmm_fwd_swiglu(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, c
   return fwd_impl(lhs, rhs, transpose_rhs, group_sizes, G, M, K, N, out, out_dtype, ws, ws_bytes, stream, N / 2);
 }
 
-gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
-                    int64_t M, int64_t K, int64_t N, void *dlhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
-                    void *stream) {
-  g_launches = 0;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  gmm_status s = check_sizes(M, K, N, G);
-  if (s != GMM_OK) return s;
-  if (!group_sizes || !dlhs) return GMM_ERR_INVALID_ARG;
-  if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
-  int elem = 0;
-  if ((s = classify(dout, rhs, true, &elem)) != GMM_OK) return s;
-  if (elem == 1 && dout.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;  // gradients: dynamic blocks
-  if (dout.dtype != GMM_BF16) return GMM_ERR_INVALID_ARG;                   // the rhs scale is folded in
-  if (!al16(dout.data) || !al16(rhs.data) || !al16(dlhs) || !al16(ws) || (rhs.scale && !al16(rhs.scale)))
-    return GMM_ERR_ALIGNMENT;
-  const WsLayout L = ws_layout(GMM_OP_DLHS, M, K, N, G);
-  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
-  WsPtrs P = carve(ws, L);
-  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
-  int n = 1;
-  const void *A = dout.data;
-  // block-wise rhs scales along n ([G, N/128, K]): they vary along k as well,
-  // so dout is quantized on its own and both scales are applied per block
-  const bool blk = elem == 1 && rhs.rule == GMM_Q_DYNAMIC;
-  if (blk && transpose_rhs) return GMM_ERR_UNSUPPORTED;
-  if (elem == 1) {
-    // per-channel rhs: t = fl32(dout * s_r[g(m), n]); dynamic 128-blocks along n
-    s = cuda_status(prof("quant_rows", st, [&] {
-      return launch_quant_rows(dout.data, M, N, true, nullptr, blk ? nullptr : rhs.scale, P.offs, G, P.codes_a,
-                               P.scales_a, P.status, st);
-    }));
-    if (s != GMM_OK) return s;
-    ++n;
-    A = P.codes_a;
-  }
+}  // extern "C"
+
+// dlhs GEMM on the row operand A [M, N]: E4M3 codes with block scales
+// A_scales [N/128, M] (elem 1) or bf16 dout (elem 2).  blk: block-wise rhs
+// scales [G, N/128, K] (A then carries no rhs scale).
+static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, const gmm_operand &rhs,
+                                int transpose_rhs, bool blk, const WsPtrs &P, int32_t G, int64_t M, int64_t K,
+                                int64_t N, void *dlhs, gmm_dtype out_dtype, cudaStream_t st) {
   const bool bmn = transpose_rhs != 0;  // [G, N, K]: K contiguous = MN-major B for dlhs
   const uint32_t bke = 128 / elem;
   CUtensorMap tmA, tmB;
@@ -454,7 +437,7 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   p.b_group_rows = static_cast<int>(bmn ? N : K);
   p.offs = P.offs;
   p.tpre = P.tpre;
-  p.row_scale = elem == 1 ? P.scales_a : nullptr;
+  p.row_scale = elem == 1 ? A_scales : nullptr;
   p.row_scale_ld = M;
   p.col_scale = nullptr;
   p.colblk_scale = blk ? rhs.scale : nullptr;
@@ -468,45 +451,14 @@ gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const 
   const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1};
   const int64_t items = ((M + 127) / 128 + G) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
-    return s;
-  g_launches = n + 1;
-  return GMM_OK;
+  return cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }));
 }
 
-gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_sizes, int32_t G, int64_t M,
-                     int64_t K, int64_t N, void *drhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
-                     void *stream) {
-  g_launches = 0;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  gmm_status s = check_sizes(M, K, N, G);
-  if (s != GMM_OK) return s;
-  if (!group_sizes || !drhs) return GMM_ERR_INVALID_ARG;
-  if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
-  int elem = 0;
-  if ((s = classify(lhs, dout, false, &elem)) != GMM_OK) return s;
-  if (!al16(lhs.data) || !al16(dout.data) || !al16(drhs) || !al16(ws)) return GMM_ERR_ALIGNMENT;
-  const WsLayout L = ws_layout(GMM_OP_DRHS, M, K, N, G);
-  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
-  WsPtrs P = carve(ws, L);
-  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
-  const int64_t cap = chunk_capacity(M, G);
-  const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
-  if (lhs.dtype == GMM_E4M3)  // static codes given: re-laid out only
-    s = cuda_status(prof("chunk_codes", st, [&] {
-      return launch_chunk_codes(static_cast<const uint8_t *>(lhs.data), M, K, P.offs, P.tpre, G, cap, P.codes_a, st);
-    }));
-  else
-    s = cuda_status(prof("quant_chunks", st, [&] {
-      return launch_quant_chunks(lhs.data, M, K, dyn, (elem == 1 && !dyn) ? lhs.scale : nullptr, P.offs, P.tpre, G,
-                                 cap, P.codes_a, P.scales_a, elem == 2, P.status, st);
-    }));
-  if (s != GMM_OK) return s;
-  s = cuda_status(prof("quant_chunks", st, [&] {
-    return launch_quant_chunks(dout.data, M, N, true, nullptr, P.offs, P.tpre, G, cap, P.codes_b, P.scales_b,
-                               elem == 2, P.status, st);
-  }));
-  if (s != GMM_OK) return s;
+// tgmm GEMM on the chunk-major operands in the workspace (codes_a: lhs,
+// codes_b: dout; scales_a / scales_b their chunk scales).
+static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, int64_t cap, const WsPtrs &P,
+                                int32_t G, int64_t M, int64_t K, int64_t N, void *drhs, gmm_dtype out_dtype,
+                                cudaStream_t st) {
   const uint32_t bke = 128 / elem;
   // tile rows = dout columns n (A = dout^T chunks), tile columns = lhs columns
   // k (B = lhs^T chunks); the epilogue writes dW[g, k, n].  The chunk-major
@@ -534,7 +486,7 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   p.row_scale_ld = N;
   p.colblk_scale = (elem == 1 && dyn) ? P.scales_a : nullptr;
   p.colblk_ld = K;
-  p.static_scale = (elem == 1 && !dyn) ? lhs.scale : nullptr;
+  p.static_scale = (elem == 1 && !dyn) ? static_scale : nullptr;
   p.out = drhs;
   p.out_f32 = out_dtype == GMM_F32;
   p.ld_out = N;
@@ -543,9 +495,152 @@ gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_siz
   const GemmConfig cfg{MODE_TGMM, elem, false, elem == 1};
   const int64_t items = static_cast<int64_t>(G) * (N / kBlk) * ((K + 255) / 256);
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  if ((s = cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, p, grid, st); }))) != GMM_OK)
+  return cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, p, grid, st); }));
+}
+
+// The tgmm lhs operand into the workspace: quantized per chunk, re-laid out
+// when the caller gives the forward's static codes, or copied (bf16 family).
+static gmm_status prepare_tgmm_lhs(const gmm_operand &lhs, int elem, int64_t cap, const WsPtrs &P, int32_t G,
+                                   int64_t M, int64_t K, cudaStream_t st) {
+  const bool dyn = lhs.rule == GMM_Q_DYNAMIC;
+  if (lhs.dtype == GMM_E4M3)  // static codes given: re-laid out only
+    return cuda_status(prof("chunk_codes", st, [&] {
+      return launch_chunk_codes(static_cast<const uint8_t *>(lhs.data), M, K, P.offs, P.tpre, G, cap, P.codes_a, st);
+    }));
+  return cuda_status(prof("quant_chunks", st, [&] {
+    return launch_quant_chunks(lhs.data, M, K, dyn, (elem == 1 && !dyn) ? lhs.scale : nullptr, P.offs, P.tpre, G, cap,
+                               P.codes_a, P.scales_a, elem == 2, P.status, st);
+  }));
+}
+
+// dlhs argument checks shared by gmm_dlhs and gmm_backward
+static gmm_status check_dlhs(const gmm_operand &dout, const gmm_operand &rhs, int transpose_rhs, int *elem) {
+  gmm_status s = classify(dout, rhs, true, elem);
+  if (s != GMM_OK) return s;
+  if (*elem == 1 && dout.rule != GMM_Q_DYNAMIC) return GMM_ERR_INVALID_ARG;  // gradients: dynamic blocks
+  if (dout.dtype != GMM_BF16) return GMM_ERR_INVALID_ARG;                    // the rhs scale is folded in
+  if (*elem == 1 && rhs.rule == GMM_Q_DYNAMIC && transpose_rhs) return GMM_ERR_UNSUPPORTED;
+  return GMM_OK;
+}
+
+extern "C" {
+
+gmm_status gmm_dlhs(gmm_operand dout, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
+                    int64_t M, int64_t K, int64_t N, void *dlhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                    void *stream) {
+  g_launches = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gmm_status s = check_sizes(M, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!group_sizes || !dlhs) return GMM_ERR_INVALID_ARG;
+  if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
+  int elem = 0;
+  if ((s = check_dlhs(dout, rhs, transpose_rhs, &elem)) != GMM_OK) return s;
+  if (!al16(dout.data) || !al16(rhs.data) || !al16(dlhs) || !al16(ws) || (rhs.scale && !al16(rhs.scale)))
+    return GMM_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(GMM_OP_DLHS, M, K, N, G);
+  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
+  WsPtrs P = carve(ws, L);
+  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
+  int n = 1;
+  const void *A = dout.data;
+  // block-wise rhs scales along n ([G, N/128, K]): they vary along k as well,
+  // so dout is quantized on its own and both scales are applied per block
+  const bool blk = elem == 1 && rhs.rule == GMM_Q_DYNAMIC;
+  if (elem == 1) {
+    // per-channel rhs: t = fl32(dout * s_r[g(m), n]); dynamic 128-blocks along n
+    s = cuda_status(prof("quant_rows", st, [&] {
+      return launch_quant_rows(dout.data, M, N, true, nullptr, blk ? nullptr : rhs.scale, P.offs, G, P.codes_a,
+                               P.scales_a, P.status, st);
+    }));
+    if (s != GMM_OK) return s;
+    ++n;
+    A = P.codes_a;
+  }
+  if ((s = run_dlhs_gemm(A, P.scales_a, elem, rhs, transpose_rhs, blk, P, G, M, K, N, dlhs, out_dtype, st)) != GMM_OK)
+    return s;
+  g_launches = n + 1;
+  return GMM_OK;
+}
+
+gmm_status tgmm_drhs(gmm_operand lhs, gmm_operand dout, const int32_t *group_sizes, int32_t G, int64_t M,
+                     int64_t K, int64_t N, void *drhs, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
+                     void *stream) {
+  g_launches = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gmm_status s = check_sizes(M, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!group_sizes || !drhs) return GMM_ERR_INVALID_ARG;
+  if (out_dtype != GMM_BF16 && out_dtype != GMM_F32) return GMM_ERR_INVALID_ARG;
+  int elem = 0;
+  if ((s = classify(lhs, dout, false, &elem)) != GMM_OK) return s;
+  if (!al16(lhs.data) || !al16(dout.data) || !al16(drhs) || !al16(ws)) return GMM_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(GMM_OP_DRHS, M, K, N, G);
+  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
+  WsPtrs P = carve(ws, L);
+  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
+  const int64_t cap = chunk_capacity(M, G);
+  if ((s = prepare_tgmm_lhs(lhs, elem, cap, P, G, M, K, st)) != GMM_OK) return s;
+  s = cuda_status(prof("quant_chunks", st, [&] {
+    return launch_quant_chunks(dout.data, M, N, true, nullptr, P.offs, P.tpre, G, cap, P.codes_b, P.scales_b,
+                               elem == 2, P.status, st);
+  }));
+  if (s != GMM_OK) return s;
+  if ((s = run_drhs_gemm(elem, lhs.rule == GMM_Q_DYNAMIC, lhs.scale, cap, P, G, M, K, N, drhs, out_dtype, st)) !=
+      GMM_OK)
     return s;
   g_launches = 4;
+  return GMM_OK;
+}
+
+gmm_status gmm_backward(gmm_operand lhs, gmm_operand dout, gmm_operand rhs, int transpose_rhs,
+                        const int32_t *group_sizes, int32_t G, int64_t M, int64_t K, int64_t N, void *dlhs,
+                        gmm_dtype dlhs_dtype, void *drhs, gmm_dtype drhs_dtype, void *ws, size_t ws_bytes,
+                        void *stream) {
+  g_launches = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gmm_status s = check_sizes(M, K, N, G);
+  if (s != GMM_OK) return s;
+  if (!group_sizes || !dlhs || !drhs) return GMM_ERR_INVALID_ARG;
+  if ((dlhs_dtype != GMM_BF16 && dlhs_dtype != GMM_F32) || (drhs_dtype != GMM_BF16 && drhs_dtype != GMM_F32))
+    return GMM_ERR_INVALID_ARG;
+  int elem = 0, elem_t = 0;
+  if ((s = check_dlhs(dout, rhs, transpose_rhs, &elem)) != GMM_OK) return s;
+  if ((s = classify(lhs, dout, false, &elem_t)) != GMM_OK) return s;
+  if (elem != elem_t) return GMM_ERR_INVALID_ARG;  // both passes in the same family
+  if (!al16(lhs.data) || !al16(dout.data) || !al16(rhs.data) || !al16(dlhs) || !al16(drhs) || !al16(ws) ||
+      (rhs.scale && !al16(rhs.scale)))
+    return GMM_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(GMM_OP_BWD, M, K, N, G);
+  if (!ws || ws_bytes < L.total) return GMM_ERR_WORKSPACE;
+  WsPtrs P = carve(ws, L);
+  if ((s = cuda_status(prof("plan", st, [&] { return launch_plan(group_sizes, G, M, P.offs, P.tpre, P.status, st); }))) != GMM_OK) return s;
+  const int64_t cap = chunk_capacity(M, G);
+  if ((s = prepare_tgmm_lhs(lhs, elem, cap, P, G, M, K, st)) != GMM_OK) return s;
+  const bool blk = elem == 1 && rhs.rule == GMM_Q_DYNAMIC;
+  const void *A = dout.data;
+  if (elem == 1) {
+    // one read of dout gives both operands: dlhs row blocks (per-channel rhs
+    // scale folded in) and the tgmm chunk columns
+    s = cuda_status(prof("quant_dout", st, [&] {
+      return launch_quant_dout_both(dout.data, M, N, blk ? nullptr : rhs.scale, P.offs, P.tpre, G, cap, P.codes_b,
+                                    P.scales_b, P.codes_r, P.scales_r, P.status, st);
+    }));
+    A = P.codes_r;
+  } else {
+    s = cuda_status(prof("quant_chunks", st, [&] {
+      return launch_quant_chunks(dout.data, M, N, true, nullptr, P.offs, P.tpre, G, cap, P.codes_b, P.scales_b, true,
+                                 P.status, st);
+    }));
+  }
+  if (s != GMM_OK) return s;
+  if ((s = run_dlhs_gemm(A, P.scales_r, elem, rhs, transpose_rhs, blk, P, G, M, K, N, dlhs, dlhs_dtype, st)) !=
+      GMM_OK)
+    return s;
+  if ((s = run_drhs_gemm(elem, lhs.rule == GMM_Q_DYNAMIC, lhs.scale, cap, P, G, M, K, N, drhs, drhs_dtype, st)) !=
+      GMM_OK)
+    return s;
+  g_launches = 5;
   return GMM_OK;
 }
 

@@ -30,6 +30,8 @@ struct WsLayout {
   size_t codes_b;      // operand B codes (tgmm only)
   size_t scales_a;     // fp32 scales of A
   size_t scales_b;     // fp32 scales of B (tgmm only)
+  size_t codes_r;      // dlhs row codes of dout (fused backward only)
+  size_t scales_r;     // their block scales [N/128, M]
   size_t total;
 };
 
@@ -51,6 +53,14 @@ cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dy
 cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool dynamic, const float *static_scale,
                                 const int *offs, const int *tpre, int G, int64_t capacity, void *codes_t,
                                 float *scales, bool bf16_copy, uint32_t *status, cudaStream_t st);
+
+// Backward dout, both quantized layouts from one read: the tgmm chunk operand
+// (as launch_quant_chunks, dynamic) and the dlhs row operand (as
+// launch_quant_rows, dynamic, col_scale folded in when not NULL).  Rows in no
+// group are left unwritten in the row operand (no GEMM tile keeps them).
+cudaError_t launch_quant_dout_both(const void *x, int64_t rows, int64_t cols, const float *col_scale, const int *offs,
+                                   const int *tpre, int G, int64_t capacity, void *codes_t, float *scales_t,
+                                   uint8_t *codes_r, float *scales_r, uint32_t *status, cudaStream_t st);
 
 // Already-quantized E4M3 rows [rows, cols] into the chunk layout of
 // launch_quant_chunks (codes only).

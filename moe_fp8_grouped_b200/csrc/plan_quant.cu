@@ -388,6 +388,144 @@ cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool 
                                           status);
 }
 
+// Backward dout from one read: the tgmm chunk operand and the dlhs row
+// operand.  One CTA per (chunk, 256-column slice) stages the chunk's rows as
+// quant_chunks_kernel does, then two warp roles work on the tile at once:
+// warps 0-3 the columns (thread t: columns 2t, 2t+1, absmax over the chunk's
+// rows, one code line per column), warps 4-11 the rows (warp w: rows w - 4,
+// w + 4, ...; half-warp h covers the 128-column block h of the slice, 8
+// columns per lane: t = fl32(dout * s_r[g, n]) when kFold, absmax over the
+// block by shuffles, codes and the block scale, exactly as quant_rows_kernel
+// computes them).
+constexpr int kDoutThreads = 384;
+constexpr int kDoutRowWarps = kDoutThreads / 32 - kChunkThreads / 32;
+
+template <bool kFold>
+__global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ col_scale,
+    const int *__restrict__ offs, const int *__restrict__ tpre, int G, uint8_t *__restrict__ codes_t,
+    float *__restrict__ scales_t, uint8_t *__restrict__ codes_r, float *__restrict__ scales_r) {
+  extern __shared__ __align__(16) uint8_t qsm[];
+  __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(qsm);  // [128][kChunkPitch]
+  __shared__ int s_info[4];
+  const int j = blockIdx.y;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kChunkCols;
+  if (threadIdx.x == 0) {
+    s_info[0] = find_chunk(j, offs, tpre, G, s_info[1], s_info[2]) ? 1 : 0;
+    if (s_info[0]) {  // the chunk's group
+      int lo = 0, hi = G + 1;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (tpre[mid] > j) hi = mid;
+        else lo = mid + 1;
+      }
+      s_info[3] = lo - 1;
+    }
+  }
+  __syncthreads();
+  if (!s_info[0]) return;
+  const int r0 = s_info[1], nr = s_info[2], g = s_info[3];
+  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 8); i += kDoutThreads) {
+    const int rr = i >> 5, cc = (i & 31) * 8;
+    const bool in = rr < nr && c0 + cc < cols;
+    const __nv_bfloat16 *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
+    cp_async_16_zfill(tile + rr * kChunkPitch + cc, src, in);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  // ---- rows: the dlhs operand
+  if (threadIdx.x >= kChunkThreads) {
+    const int lane = threadIdx.x & 31, warp = (threadIdx.x - kChunkThreads) >> 5;
+    const int half = lane >> 4, hl = lane & 15;
+    const int cl = half * 128 + hl * 8;  // the lane's 8 columns in the slice
+    const bool col_in = c0 + cl < cols;  // warp-half uniform (cols is a multiple of 128)
+    float cs[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cs[i] = 1.0f;
+    if (kFold && col_in) {
+      const float4 *c = reinterpret_cast<const float4 *>(col_scale + static_cast<int64_t>(g) * cols + c0 + cl);
+      const float4 a = __ldg(c), b = __ldg(c + 1);
+      cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
+      cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
+    }
+    for (int r = warp; r < nr; r += kDoutRowWarps) {
+      float v[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(tile + r * kChunkPitch + cl), v);
+      if constexpr (kFold) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], cs[i]);
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+      for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+      float sc, inv;
+      dyn_scale(amax, sc, inv);
+      if (col_in) {
+        uint2 out;
+        out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
+                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
+        out.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv))) |
+                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
+        const int64_t m = r0 + r;
+        *reinterpret_cast<uint2 *>(codes_r + m * cols + c0 + cl) = out;
+        if (hl == 0) scales_r[((c0 + cl) / kBlk) * rows + m] = sc;
+      }
+    }
+    return;
+  }
+  // ---- columns: the tgmm operand (quant_chunks_kernel, dynamic rule)
+  const int col = 2 * threadIdx.x;  // and col + 1
+  if (c0 + col >= cols) return;     // cols is a multiple of 128: both columns are in or out
+  const uint32_t *t32 = reinterpret_cast<const uint32_t *>(tile);
+  auto pair = [&](int r) -> float2 {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t32[(r * kChunkPitch + col) >> 1]));
+  };
+  float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll 8
+  for (int r = 0; r < kBlk; ++r) {
+    const float2 v = pair(r);
+    a0 = fmaxf(a0, fabsf(v.x));
+    a1 = fmaxf(a1, fabsf(v.y));
+  }
+  float s0, s1, inv0, inv1;
+  dyn_scale(a0, s0, inv0);
+  dyn_scale(a1, s1, inv1);
+  uint8_t *dst0 = codes_t + (static_cast<int64_t>(j) * cols + c0 + col) * kBlk;
+  uint8_t *dst1 = dst0 + kBlk;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint32_t w0[4], w1[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = q * 16 + e * 4;
+      const float2 v0 = pair(r), v1 = pair(r + 1), v2 = pair(r + 2), v3 = pair(r + 3);
+      w0[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.x, inv0), __fmul_rn(v1.x, inv0))) |
+              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.x, inv0), __fmul_rn(v3.x, inv0))) << 16);
+      w1[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.y, inv1), __fmul_rn(v1.y, inv1))) |
+              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.y, inv1), __fmul_rn(v3.y, inv1))) << 16);
+    }
+    *reinterpret_cast<uint4 *>(dst0 + q * 16) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    *reinterpret_cast<uint4 *>(dst1 + q * 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  }
+  *reinterpret_cast<float2 *>(scales_t + static_cast<int64_t>(j) * cols + c0 + col) = make_float2(s0, s1);
+}
+
+cudaError_t launch_quant_dout_both(const void *x, int64_t rows, int64_t cols, const float *col_scale, const int *offs,
+                                   const int *tpre, int G, int64_t capacity, void *codes_t, float *scales_t,
+                                   uint8_t *codes_r, float *scales_r, uint32_t *status, cudaStream_t st) {
+  (void)status;  // no static scale to check: gradients are dynamic
+  dim3 grid(static_cast<unsigned>((cols + kChunkCols - 1) / kChunkCols), static_cast<unsigned>(capacity));
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  auto kern = col_scale ? quant_dout_both_kernel<true> : quant_dout_both_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kChunkSmem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kDoutThreads, kChunkSmem, st>>>(xb, rows, cols, col_scale, offs, tpre, G,
+                                               static_cast<uint8_t *>(codes_t), scales_t, codes_r, scales_r);
+  return cudaGetLastError();
+}
+
 // Already-quantized E4M3 lhs (static rule): its codes laid out as the chunk
 // quantizer lays out the codes it makes (transposed, padded, zero pad rows),
 // bytes copied unchanged.  Same CTA shape as quant_chunks_kernel.

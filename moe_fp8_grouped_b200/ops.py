@@ -259,6 +259,39 @@ def tgmm_drhs(lhs: torch.Tensor, dout: torch.Tensor, group_sizes: torch.Tensor, 
     return out
 
 
+def gmm_backward(lhs: torch.Tensor, dout: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | None,
+                 group_sizes: torch.Tensor, rule="static", static_scale: torch.Tensor | None = None,
+                 transpose_rhs: bool = False, dlhs_dtype=torch.bfloat16, drhs_dtype=torch.float32,
+                 dlhs: torch.Tensor | None = None, drhs: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """Both backward passes in one call (dout read once): returns (dlhs [M, K],
+    dW [G, K, N]) equal bit for bit to gmm_dlhs and tgmm_drhs.  ``rule`` and
+    ``static_scale`` describe lhs as for tgmm_drhs ("none": bf16 family)."""
+    M, K = lhs.shape
+    M2, N = dout.shape
+    assert M2 == M
+    G = int(group_sizes.numel())
+    r = _rule(rule)
+    if dlhs is None:
+        dlhs = torch.empty((M, K), dtype=dlhs_dtype, device=lhs.device)
+    if drhs is None:
+        drhs = torch.empty((G, K, N), dtype=drhs_dtype, device=lhs.device)
+    if ws is None:
+        ws = workspace(gmm_workspace_bytes(B.OP_BWD, M, K, N, G), lhs.device)
+    sc = _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None
+    if lhs.dtype in (torch.uint8, torch.float8_e4m3fn):
+        a = _operand(_dev(lhs, "lhs"), B.DT_E4M3, sc, r)
+    else:
+        a = _operand(_dev(lhs, "lhs", torch.bfloat16), B.DT_BF16, sc, r)
+    d = _operand(_dev(dout, "dout", torch.bfloat16), B.DT_BF16, None, B.Q_NONE if r == B.Q_NONE else B.Q_DYNAMIC)
+    b = _rhs_operand(rhs, rhs_scales)
+    st = B.lib().gmm_backward(a, d, b, int(transpose_rhs), _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,
+                              _dev(dlhs, "dlhs", (torch.bfloat16, torch.float32)), _TORCH_DT[dlhs.dtype],
+                              _dev(drhs, "drhs", (torch.bfloat16, torch.float32)), _TORCH_DT[drhs.dtype],
+                              ws.data_ptr(), ws.numel(), _stream(lhs))
+    _check(st, "gmm_backward")
+    return dlhs, drhs
+
+
 def gmm_read_device_status(ws: torch.Tensor):
     """(status, bits) left in ``ws`` by the last call; synchronizes the stream."""
     bits = ctypes.c_uint32(0)

@@ -86,6 +86,13 @@ def test_host_errors(L):
     assert sw(lhs, rhs, 0, gs, 8, 256, 512, 0, out, B.DT_BF16, ws, big, None) == 2
     assert sw(lhs, rhs, 0, None, 8, 256, 512, 512, out, B.DT_BF16, ws, big, None) == 1
     assert sw(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, 1024, None) == 9
+    bw = L.gmm_backward
+    dop = _op(FAKE, B.DT_BF16, None, B.Q_DYNAMIC)
+    assert bw(lhs, dop, rhs, 0, gs, 8, 256, 500, 512, out, B.DT_BF16, out, B.DT_F32, ws, big, None) == 2  # K % 128
+    assert bw(lhs, dop, rhs, 0, gs, 8, 256, 512, 512, None, B.DT_BF16, out, B.DT_F32, ws, big, None) == 1
+    assert bw(lhs, dop, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, out, B.DT_F32, ws, 1024, None) == 9
+    assert bw(lhs, _op(FAKE, B.DT_BF16, None, B.Q_STATIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, out,
+              B.DT_F32, ws, big, None) == 1  # gradients are dynamic
     d = L.gmm_dlhs
     assert d(_op(FAKE, B.DT_E4M3, FAKE, B.Q_DYNAMIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big,
              None) == 1  # dout must be bf16 (the rhs scale is folded in)

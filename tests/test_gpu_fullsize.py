@@ -139,3 +139,28 @@ def test_fullsize_blockwise_rhs_sampled(name):
         assert_close(dl[rows], ref, ab, f"{name} blockwise dlhs g={g}")
     del inp, out, dl, ws, s0, s1
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["mixtral", "dsv3_up", "ragged"])
+def test_fullsize_backward_equals_the_two_calls(name):
+    """The fused backward at full size: dlhs and dW equal the separate calls
+    bit for bit (same codes from one read of dout)."""
+    dev = torch.device("cuda:0")
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w, seed=0, device="cuda")
+    gs = inp.group_sizes.to(dev)
+    M, K, N, G = w.M, w.K, w.N, w.G
+    s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    sarg = s if w.rule == "static" else None
+    codes, scales = gm.gmm_quantize_rhs(inp.w)
+    del inp.w
+    ws = torch.empty(gm.gmm_workspace_bytes(3, M, K, N, G), dtype=torch.uint8, device=dev)
+    dl, dw = gm.gmm_backward(inp.lhs, inp.dout, codes, scales, gs, rule=w.rule, static_scale=sarg, ws=ws)
+    st, bits = gm.gmm_read_device_status(ws)
+    assert st == 0, (st, bits)
+    assert torch.equal(dl, gm.gmm_dlhs(inp.dout, codes, scales, gs, ws=ws))
+    del dl
+    dw1 = gm.tgmm_drhs(inp.lhs, inp.dout, gs, rule=w.rule, static_scale=sarg, ws=ws)
+    assert torch.equal(dw, dw1)
+    del inp, dw, dw1, ws, codes, scales
+    torch.cuda.empty_cache()

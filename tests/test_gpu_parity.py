@@ -266,6 +266,60 @@ def test_fwd_swiglu_rejects_n_not_two_tiles_of_128(dev):
         gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule="static", static_scale=s)
 
 
+# ------------------------------------------------------ fused backward
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("transpose", [False, True])
+def test_backward_equals_the_two_calls(dev, name, rule, transpose):
+    """gmm_backward quantizes dout once for both passes; its codes are the
+    separate calls' codes, so dlhs and dW agree bit for bit, and with the
+    oracle within the tolerance."""
+    inp = case_inputs(name)
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    M, K, N, G = lhs.shape[0], lhs.shape[1], w.shape[2], w.shape[0]
+    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
+    sarg = s if rule == "static" else None
+    raw_d, dl, pad_d, n_d = guarded((M, K), torch.float32)
+    raw_w, dw, pad_w, n_w = guarded((G, K, N), torch.float32)
+    gm.gmm_backward(lhs, dout, codes, scales, gs, rule=rule, static_scale=sarg, transpose_rhs=transpose,
+                    dlhs=dl, drhs=dw)
+    assert gm.last_launch_count() == 5
+    torch.cuda.synchronize()
+    check_guards(raw_d, pad_d, n_d)
+    check_guards(raw_w, pad_w, n_w)
+    d1 = gm.gmm_dlhs(dout, codes, scales, gs, transpose_rhs=transpose, out_dtype=torch.float32)
+    w1 = gm.tgmm_drhs(lhs, dout, gs, rule=rule, static_scale=sarg)
+    assert torch.equal(dl, d1)
+    assert torch.equal(dw, w1)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    ref, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
+    assert_close(dl, ref, ab, f"backward dlhs {name}")
+    ref, ab = oracle.tgmm_drhs(inp.lhs, rule_code(rule), inp.static_scale, inp.dout, inp.group_sizes)
+    assert_close(dw, ref, ab, f"backward drhs {name}")
+
+
+def test_backward_bf16_family_blockwise_and_forward_codes(dev):
+    inp = case_inputs("ragged")
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    # bf16 family
+    dl, dw = gm.gmm_backward(lhs, dout, w, None, gs, rule="none", dlhs_dtype=torch.float32)
+    assert torch.equal(dl, gm.gmm_dlhs(dout, w, None, gs, rule="none", out_dtype=torch.float32))
+    assert torch.equal(dw, gm.tgmm_drhs(lhs, dout, gs, rule="none"))
+    # block-wise weights along N for dlhs (no fold)
+    c1, s1 = gm.gmm_quantize_rhs_blocks(w, 1)
+    dl, dw = gm.gmm_backward(lhs, dout, c1, s1, gs, rule="dynamic", dlhs_dtype=torch.float32)
+    assert torch.equal(dl, gm.gmm_dlhs(dout, c1, s1, gs, out_dtype=torch.float32))
+    assert torch.equal(dw, gm.tgmm_drhs(lhs, dout, gs, rule="dynamic"))
+    # the forward's static codes as the tgmm lhs
+    codes, scales = gm.gmm_quantize_rhs(w)
+    ql, _ = gm.gmm_quantize(lhs, "static", axis=1, static_scale=s)
+    dl, dw = gm.gmm_backward(ql, dout, codes, scales, gs, rule="static", static_scale=s)
+    assert torch.equal(dw, gm.tgmm_drhs(lhs, dout, gs, rule="static", static_scale=s))
+    with pytest.raises(gm.GmmError, match="invalid argument"):  # mixed families
+        gm.gmm_backward(lhs, dout, codes, scales, gs, rule="none")
+
+
 # ------------------------------------------------- block-wise rhs scales
 
 @pytest.mark.parametrize("axis", [0, 1])
