@@ -389,27 +389,30 @@ cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool 
 }
 
 // Backward dout from one read: the tgmm chunk operand and the dlhs row
-// operand.  One CTA per (chunk, 256-column slice) stages the chunk's rows as
-// quant_chunks_kernel does, then two warp roles work on the tile at once:
-// warps 0-3 the columns (thread t: columns 2t, 2t+1, absmax over the chunk's
-// rows, one code line per column), warps 4-11 the rows (warp w: rows w - 4,
-// w + 4, ...; half-warp h covers the 128-column block h of the slice, 8
-// columns per lane: t = fl32(dout * s_r[g, n]) when kFold, absmax over the
-// block by shuffles, codes and the block scale, exactly as quant_rows_kernel
-// computes them).
-constexpr int kDoutThreads = 384;
-constexpr int kDoutRowWarps = kDoutThreads / 32 - kChunkThreads / 32;
+// operand.  One CTA per (chunk, 128-column slice) stages the chunk's rows
+// (zero-filled past the chunk) by cp.async, then two warp roles work on the
+// tile at once: warps 0-1 the columns (thread t: columns 2t, 2t+1, absmax over
+// the chunk's rows, one code line per column), warps 2-5 the rows (a warp
+// takes two rows per step, one per half-warp, 8 columns per lane:
+// t = fl32(dout * s_r[g, n]) when kFold, absmax over the 128-column block by
+// shuffles, codes and the block scale, exactly as quant_rows_kernel computes
+// them).  The small tile (34 KB) keeps six CTAs per SM, so loads of some
+// overlap the arithmetic of others.
+constexpr int kDoutCols = 128;
+constexpr int kDoutPitch = kDoutCols + 8;                 // bf16 per staged row (16-byte aligned rows)
+constexpr int kDoutColThreads = kDoutCols / 2;            // two columns per thread
+constexpr int kDoutRowWarps = 4;
+constexpr int kDoutThreads = kDoutColThreads + 32 * kDoutRowWarps;
 
 template <bool kFold>
 __global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
     const __nv_bfloat16 *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ col_scale,
     const int *__restrict__ offs, const int *__restrict__ tpre, int G, uint8_t *__restrict__ codes_t,
     float *__restrict__ scales_t, uint8_t *__restrict__ codes_r, float *__restrict__ scales_r) {
-  extern __shared__ __align__(16) uint8_t qsm[];
-  __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(qsm);  // [128][kChunkPitch]
+  __shared__ __align__(16) __nv_bfloat16 tile[kBlk * kDoutPitch];
   __shared__ int s_info[4];
   const int j = blockIdx.y;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kChunkCols;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kDoutCols;  // cols is a multiple of 128
   if (threadIdx.x == 0) {
     s_info[0] = find_chunk(j, offs, tpre, G, s_info[1], s_info[2]) ? 1 : 0;
     if (s_info[0]) {  // the chunk's group
@@ -425,32 +428,32 @@ __global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
   __syncthreads();
   if (!s_info[0]) return;
   const int r0 = s_info[1], nr = s_info[2], g = s_info[3];
-  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 8); i += kDoutThreads) {
-    const int rr = i >> 5, cc = (i & 31) * 8;
-    const bool in = rr < nr && c0 + cc < cols;
+  for (int i = threadIdx.x; i < kBlk * (kDoutCols / 8); i += kDoutThreads) {
+    const int rr = i / (kDoutCols / 8), cc = (i % (kDoutCols / 8)) * 8;
+    const bool in = rr < nr;
     const __nv_bfloat16 *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
-    cp_async_16_zfill(tile + rr * kChunkPitch + cc, src, in);
+    cp_async_16_zfill(tile + rr * kDoutPitch + cc, src, in);
   }
   cp_async_wait_all();
   __syncthreads();
-  // ---- rows: the dlhs operand
-  if (threadIdx.x >= kChunkThreads) {
-    const int lane = threadIdx.x & 31, warp = (threadIdx.x - kChunkThreads) >> 5;
+  if (threadIdx.x >= kDoutColThreads) {
+    // ---- rows: the dlhs operand
+    const int lane = threadIdx.x & 31, warp = (threadIdx.x - kDoutColThreads) >> 5;
     const int half = lane >> 4, hl = lane & 15;
-    const int cl = half * 128 + hl * 8;  // the lane's 8 columns in the slice
-    const bool col_in = c0 + cl < cols;  // warp-half uniform (cols is a multiple of 128)
+    const int cl = hl * 8;  // the lane's 8 columns in the slice
     float cs[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) cs[i] = 1.0f;
-    if (kFold && col_in) {
+    if constexpr (kFold) {
       const float4 *c = reinterpret_cast<const float4 *>(col_scale + static_cast<int64_t>(g) * cols + c0 + cl);
       const float4 a = __ldg(c), b = __ldg(c + 1);
       cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
       cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
     }
-    for (int r = warp; r < nr; r += kDoutRowWarps) {
+    for (int rb = 2 * warp; rb < nr; rb += 2 * kDoutRowWarps) {
+      const int r = rb + half;  // rows past the chunk hold zeros and are not stored
       float v[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(tile + r * kChunkPitch + cl), v);
+      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(tile + r * kDoutPitch + cl), v);
       if constexpr (kFold) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], cs[i]);
@@ -462,7 +465,7 @@ __global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
       for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
       float sc, inv;
       dyn_scale(amax, sc, inv);
-      if (col_in) {
+      if (r < nr) {
         uint2 out;
         out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
                 (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
@@ -470,17 +473,16 @@ __global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
                 (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
         const int64_t m = r0 + r;
         *reinterpret_cast<uint2 *>(codes_r + m * cols + c0 + cl) = out;
-        if (hl == 0) scales_r[((c0 + cl) / kBlk) * rows + m] = sc;
+        if (hl == 0) scales_r[(c0 / kBlk) * rows + m] = sc;
       }
     }
     return;
   }
   // ---- columns: the tgmm operand (quant_chunks_kernel, dynamic rule)
   const int col = 2 * threadIdx.x;  // and col + 1
-  if (c0 + col >= cols) return;     // cols is a multiple of 128: both columns are in or out
   const uint32_t *t32 = reinterpret_cast<const uint32_t *>(tile);
   auto pair = [&](int r) -> float2 {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t32[(r * kChunkPitch + col) >> 1]));
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t32[(r * kDoutPitch + col) >> 1]));
   };
   float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll 8
@@ -516,13 +518,11 @@ cudaError_t launch_quant_dout_both(const void *x, int64_t rows, int64_t cols, co
                                    const int *tpre, int G, int64_t capacity, void *codes_t, float *scales_t,
                                    uint8_t *codes_r, float *scales_r, uint32_t *status, cudaStream_t st) {
   (void)status;  // no static scale to check: gradients are dynamic
-  dim3 grid(static_cast<unsigned>((cols + kChunkCols - 1) / kChunkCols), static_cast<unsigned>(capacity));
+  dim3 grid(static_cast<unsigned>(cols / kDoutCols), static_cast<unsigned>(capacity));
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
   auto kern = col_scale ? quant_dout_both_kernel<true> : quant_dout_both_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kChunkSmem));
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kDoutThreads, kChunkSmem, st>>>(xb, rows, cols, col_scale, offs, tpre, G,
-                                               static_cast<uint8_t *>(codes_t), scales_t, codes_r, scales_r);
+  kern<<<grid, kDoutThreads, 0, st>>>(xb, rows, cols, col_scale, offs, tpre, G, static_cast<uint8_t *>(codes_t),
+                                      scales_t, codes_r, scales_r);
   return cudaGetLastError();
 }
 
