@@ -238,13 +238,15 @@ cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dy
 
 // ---------------------------------------------------- chunks (axis 0)
 
-// One CTA of 128 threads per (256-column slice, chunk).  The chunk's rows (at
+// One CTA of 64 threads per (128-column slice, chunk).  The chunk's rows (at
 // most 128, the rest zero) are staged in shared memory with cp.async; thread t
 // owns the adjacent columns 2t and 2t+1: it takes each column's absmax over the
 // chunk and writes each column's 128 codes as one line of the chunk-major
 // transposed layout [chunk][column][128], so a CTA writes one contiguous block.
-constexpr int kChunkCols = 256;
-constexpr int kChunkThreads = 128;
+// The 34 KB tile keeps six CTAs per SM, so loads of some overlap the work of
+// others.
+constexpr int kChunkCols = 128;
+constexpr int kChunkThreads = kChunkCols / 2;
 constexpr int kChunkPitch = kChunkCols + 8;  // bf16 per staged row (16-byte aligned rows)
 constexpr size_t kChunkSmem = static_cast<size_t>(kBlk) * kChunkPitch * sizeof(__nv_bfloat16);
 
@@ -288,7 +290,7 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
   // 128 rows x 32 sixteen-byte pieces, all in flight; rows past the chunk and
   // columns past the matrix are zero-filled
   for (int i = threadIdx.x; i < kBlk * (kChunkCols / 8); i += kChunkThreads) {
-    const int rr = i >> 5, cc = (i & 31) * 8;
+    const int rr = i / (kChunkCols / 8), cc = (i % (kChunkCols / 8)) * 8;
     const bool in = rr < nr && c0 + cc < cols;
     const __nv_bfloat16 *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
     cp_async_16_zfill(tile + rr * kChunkPitch + cc, src, in);
@@ -544,7 +546,7 @@ __global__ void __launch_bounds__(kChunkThreads) chunk_codes_kernel(const uint8_
   if (!s_info[0]) return;
   const int r0 = s_info[1], nr = s_info[2];
   for (int i = threadIdx.x; i < kBlk * (kChunkCols / 16); i += kChunkThreads) {
-    const int rr = i >> 4, cc = (i & 15) * 16;
+    const int rr = i / (kChunkCols / 16), cc = (i % (kChunkCols / 16)) * 16;
     const bool in = rr < nr && c0 + cc < cols;
     const uint8_t *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
     cp_async_16_zfill(tile + rr * kCodePitch + cc, src, in);
