@@ -624,7 +624,7 @@ gmm_status gmm_backward(gmm_operand lhs, gmm_operand dout, gmm_operand rhs, int 
     // scale folded in) and the tgmm chunk columns
     s = cuda_status(prof("quant_dout", st, [&] {
       return launch_quant_dout_both(dout.data, M, N, blk ? nullptr : rhs.scale, P.offs, P.tpre, G, cap, P.codes_b,
-                                    P.scales_b, P.codes_r, P.scales_r, P.status, st);
+                                    P.scales_b, P.codes_r, P.scales_r, st);
     }));
     A = P.codes_r;
   } else {

@@ -60,7 +60,7 @@ cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool 
 // group are left unwritten in the row operand (no GEMM tile keeps them).
 cudaError_t launch_quant_dout_both(const void *x, int64_t rows, int64_t cols, const float *col_scale, const int *offs,
                                    const int *tpre, int G, int64_t capacity, void *codes_t, float *scales_t,
-                                   uint8_t *codes_r, float *scales_r, uint32_t *status, cudaStream_t st);
+                                   uint8_t *codes_r, float *scales_r, cudaStream_t st);
 
 // Already-quantized E4M3 rows [rows, cols] into the chunk layout of
 // launch_quant_chunks (codes only).

@@ -518,8 +518,7 @@ __global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
 
 cudaError_t launch_quant_dout_both(const void *x, int64_t rows, int64_t cols, const float *col_scale, const int *offs,
                                    const int *tpre, int G, int64_t capacity, void *codes_t, float *scales_t,
-                                   uint8_t *codes_r, float *scales_r, uint32_t *status, cudaStream_t st) {
-  (void)status;  // no static scale to check: gradients are dynamic
+                                   uint8_t *codes_r, float *scales_r, cudaStream_t st) {
   dim3 grid(static_cast<unsigned>(cols / kDoutCols), static_cast<unsigned>(capacity));
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
   auto kern = col_scale ? quant_dout_both_kernel<true> : quant_dout_both_kernel<false>;
