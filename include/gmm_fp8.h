@@ -290,6 +290,17 @@ gmm_status gmm_gather_rows(const void *src, const int32_t *idx, int64_t nrows, i
                            void *dst, void *stream);
 
 /*
+ * gmm_gather_scale_rows: the routed gradient rows of the expert-parallel
+ * backward, dst[i, :] = bf16(fl32(src[idx[i], :]) * scale[i]) (one
+ * round-to-nearest-even multiply per value, then the bf16 rounding); bf16
+ * rows of ncols values (a multiple of 8); idx device int32 [nrows], scale
+ * device float [nrows]; an index outside [0, src_rows) writes zeros.  Errors
+ * as for gmm_gather_rows.
+ */
+gmm_status gmm_gather_scale_rows(const void *src_bf16, const int32_t *idx, const float *scale, int64_t nrows,
+                                 int64_t ncols, int64_t src_rows, void *dst_bf16, void *stream);
+
+/*
  * gmm_combine_rows: the weighted sum that returns expert outputs to their
  * tokens (the unpermute of the MoE combine):
  *   y[t, :] = sum_{j < k} weight[t, j] * rows[slot[t, j], :]

@@ -26,7 +26,7 @@ EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm
            "gmm_dlhs", "tgmm_drhs", "gmm_read_device_status", "gmm_selftest_timeout", "gmm_set_wait_limit_ns",
            "gmm_status_string", "gmm_last_launch_count", "gmm_profile_enable", "gmm_profile_collect",
            "gmm_fwd_noalloc", "gmm_fwd_swiglu", "gmm_quantize_rhs_blocks", "gmm_gather_rows",
-           "gmm_combine_rows", "gmm_backward"]
+           "gmm_combine_rows", "gmm_backward", "gmm_gather_scale_rows"]
 
 
 class Operand(ctypes.Structure):
@@ -68,6 +68,8 @@ def lib():
                                vp, ctypes.c_int, vp, sz, vp]
     L.gmm_backward.restype = st
     L.gmm_gather_rows.argtypes = [vp, vp, i64, i64, i64, vp, vp]
+    L.gmm_gather_scale_rows.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
+    L.gmm_gather_scale_rows.restype = st
     L.gmm_gather_rows.restype = st
     L.gmm_combine_rows.argtypes = [vp, i64, vp, vp, i64, i32, i64, vp, ctypes.c_int, vp]
     L.gmm_combine_rows.restype = st

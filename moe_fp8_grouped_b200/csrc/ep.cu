@@ -29,6 +29,36 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
   }
 }
 
+// dst[i] = bf16(fl32(src[idx[i]]) * scale[i]) for bf16 rows of n8 * 8 values
+// (an index outside [0, src_rows) gives zeros).  One CTA per row, grid-stride.
+__global__ void __launch_bounds__(256) gather_scale_rows_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                                const int32_t *__restrict__ idx,
+                                                                const float *__restrict__ scale, int64_t nrows,
+                                                                int64_t n8, int64_t src_rows,
+                                                                __nv_bfloat16 *__restrict__ dst) {
+  for (int64_t i = blockIdx.x; i < nrows; i += gridDim.x) {
+    const int64_t r = idx[i];
+    const bool ok = r >= 0 && r < src_rows;
+    const float f = scale[i];
+    const uint4 *s = reinterpret_cast<const uint4 *>(src + (ok ? r : 0) * n8 * 8);
+    uint4 *d = reinterpret_cast<uint4 *>(dst + i * n8 * 8);
+    for (int64_t v = threadIdx.x; v < n8; v += blockDim.x) {
+      uint4 o = make_uint4(0, 0, 0, 0);
+      if (ok) {
+        const uint4 a = s[v];
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        __nv_bfloat162 *q = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = __bfloat1622float2(h[e]);
+          q[e] = __floats2bfloat162_rn(__fmul_rn(x.x, f), __fmul_rn(x.y, f));
+        }
+      }
+      d[v] = o;
+    }
+  }
+}
+
 // y[t, :] = sum_j weight[t, j] * rows[slot[t, j], :] (fp32, j in order; a
 // slot outside [0, nrows) contributes nothing).  One CTA per token, 8
 // columns per thread step.
@@ -88,6 +118,20 @@ gmm_status gmm_gather_rows(const void *src, const int32_t *idx, int64_t nrows, i
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   gather_rows_kernel<<<grid_for(nrows), 256, 0, st>>>(static_cast<const uint4 *>(src), idx, nrows, row_bytes / 16,
                                                       src_rows, static_cast<uint4 *>(dst));
+  return cudaGetLastError() == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
+}
+
+gmm_status gmm_gather_scale_rows(const void *src_bf16, const int32_t *idx, const float *scale, int64_t nrows,
+                                 int64_t ncols, int64_t src_rows, void *dst_bf16, void *stream) {
+  if (nrows < 0 || ncols <= 0 || src_rows < 0) return GMM_ERR_INVALID_ARG;
+  if (nrows == 0) return GMM_OK;
+  if (!src_bf16 || !idx || !scale || !dst_bf16) return GMM_ERR_INVALID_ARG;
+  if (ncols % 8) return GMM_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(src_bf16) | reinterpret_cast<uintptr_t>(dst_bf16)) & 15u) return GMM_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gather_scale_rows_kernel<<<grid_for(nrows), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(src_bf16), idx, scale,
+                                                            nrows, ncols / 8, src_rows,
+                                                            static_cast<__nv_bfloat16 *>(dst_bf16));
   return cudaGetLastError() == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
 }
 

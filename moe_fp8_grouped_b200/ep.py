@@ -18,8 +18,9 @@ Split of the work:
     gloo ranks);
   - the row exchange (``exchange_rows``): ``torch.distributed`` all-to-all,
     NCCL on GPUs;
-  - row movement and arithmetic (``ep_moe_fwd``): the library's kernels
-    (gmm_gather_rows, gmm_fwd, gmm_combine_rows), CUDA only.
+  - row movement and arithmetic (``ep_moe_fwd``, ``ep_moe_bwd``): the
+    library's kernels (gmm_gather_rows, gmm_gather_scale_rows, gmm_fwd,
+    gmm_backward, gmm_combine_rows), CUDA only.
 """
 from __future__ import annotations
 
@@ -29,7 +30,7 @@ import torch
 import torch.distributed as dist
 
 from . import _binding as B
-from .ops import _check, _dev, _stream, gmm_fwd
+from .ops import _check, _dev, _stream, gmm_backward, gmm_fwd
 
 
 @dataclass
@@ -118,6 +119,17 @@ def gather_rows(src: torch.Tensor, idx: torch.Tensor) -> torch.Tensor:
     return dst
 
 
+def gather_scale_rows(src: torch.Tensor, idx: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
+    """dst[i] = bf16(src[idx[i]] * scale[i]) for bf16 rows (library kernel)."""
+    idx32 = idx.to(device=src.device, dtype=torch.int32).contiguous()
+    f32 = scale.to(device=src.device, dtype=torch.float32).contiguous()
+    dst = torch.empty((idx32.numel(), src.shape[1]), dtype=torch.bfloat16, device=src.device)
+    st = B.lib().gmm_gather_scale_rows(_dev(src, "src", torch.bfloat16), idx32.data_ptr(), f32.data_ptr(),
+                                       idx32.numel(), src.shape[1], src.shape[0], dst.data_ptr(), _stream(src))
+    _check(st, "gmm_gather_scale_rows")
+    return dst
+
+
 def combine_rows(rows: torch.Tensor, slot: torch.Tensor, weight: torch.Tensor, out_dtype=torch.bfloat16):
     """y[t] = sum_j weight[t, j] * rows[slot[t, j]] with the library's kernel."""
     T, k = slot.shape
@@ -200,3 +212,46 @@ class EPForwardGraph:
     def replay(self) -> torch.Tensor:
         self.graph.replay()
         return self.out
+
+
+def ep_moe_bwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: torch.Tensor,
+               weights: torch.Tensor, dy: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, group=None,
+               dx_dtype=torch.bfloat16, dw_dtype=torch.float32):
+    """Backward of ep_moe_fwd for the gmm operands: given dy [T, N] (bf16)
+    returns dx [T, K] and this rank's expert weight gradient [E/P, K, N].
+
+    Each routed row carries dh = bf16(w[t, j] * dy[t]) to its expert's rank
+    together with the forward's E4M3 codes of x[t]; there gmm_backward (dout
+    quantized once) gives dlhs rows and dW; the dlhs rows return and are
+    summed per token: dx[t] = sum_j dlhs_{t, j}.  The routing weights'
+    gradient (dy . h) belongs to the router and is not computed here.
+    """
+    P = dist.get_world_size(group) if dist.is_initialized() else 1
+    El, K, N = w_codes.shape
+    T, k = expert_ids.shape
+    rt = route(expert_ids.to(x_codes.device), El * P, P)
+    order = rt.order
+    tok = order // k
+    send_x = gather_rows(x_codes, tok)
+    send_d = gather_scale_rows(dy, tok, weights.reshape(-1)[order])
+    if P == 1:
+        xr, dr, gsz, perm = send_x, send_d, rt.counts, None
+    else:
+        recv_counts = exchange_counts(rt, group)
+        arrive = [int(v) for v in recv_counts.sum(dim=1).tolist()]
+        perm, gsz = local_order(recv_counts)
+        xr = gather_rows(exchange_rows(send_x, rt.send_splits, arrive, group), perm)
+        dr = gather_rows(exchange_rows(send_d, rt.send_splits, arrive, group), perm)
+    dw = torch.empty((El, K, N), dtype=dw_dtype, device=x_codes.device)
+    if xr.shape[0]:
+        dl, dw = gmm_backward(xr, dr, w_codes, w_scales, gsz.to(torch.int32), rule="static",
+                              static_scale=static_scale, dlhs_dtype=torch.bfloat16, drhs=dw)
+    else:  # no rows for this rank's experts
+        dl = torch.empty((0, K), dtype=torch.bfloat16, device=x_codes.device)
+        dw.zero_()
+    if P > 1:
+        inv = torch.empty_like(perm).scatter_(0, perm, torch.arange(perm.numel(), device=perm.device))
+        dl = exchange_rows(gather_rows(dl, inv), arrive, rt.send_splits, group)
+    slot = torch.empty_like(order).scatter_(0, order, torch.arange(order.numel(), device=order.device))
+    ones = torch.ones((T, k), dtype=torch.float32, device=x_codes.device)
+    return combine_rows(dl, slot.view(T, k), ones, dx_dtype), dw

@@ -15,7 +15,7 @@ import torch
 import moe_fp8_grouped_b200 as gm
 import oracle
 from moe_fp8_grouped_b200 import ep
-from parity import assert_within
+from parity import assert_close, assert_within
 
 pytestmark = pytest.mark.gpu
 
@@ -94,3 +94,52 @@ def test_ep_forward_graph_replays_the_eager_result(dev):
     # new routing weights copied into the captured buffer change the result
     wts.copy_(wts.flip(1))
     assert torch.equal(graph.replay(), ep.ep_moe_fwd(xq, s, ids, wts, codes, scales))
+
+
+@pytest.mark.parametrize("T,E,k,K,N", [(96, 8, 2, 256, 384), (33, 4, 3, 384, 256)])
+def test_ep_moe_bwd_single_rank(dev, T, E, k, K, N):
+    """dx and the experts' dW of the one-rank expert-parallel backward against
+    the oracle: every routed row's gradient dh = bf16(w * dy) goes through the
+    oracle's dlhs and tgmm for its expert; dx sums a token's dlhs rows."""
+    g = torch.Generator().manual_seed(100 + T)
+    x = torch.randn(T, K, generator=g).bfloat16()
+    w = (torch.randn(E, K, N, generator=g) * 0.02).bfloat16()
+    dy = torch.randn(T, N, generator=g).bfloat16()
+    ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)])
+    wts = torch.softmax(torch.randn(T, k, generator=g), dim=1)
+    s_val = 4.0 / 448.0
+    s = torch.tensor([s_val], dtype=torch.float32, device=dev)
+    codes, scales = gm.gmm_quantize_rhs(w.to(dev))
+    xq, _ = gm.gmm_quantize(x.to(dev), "static", axis=1, static_scale=s)
+    dx, dw = ep.ep_moe_bwd(xq, s, ids.to(dev), wts.to(dev), dy.to(dev), codes, scales, dx_dtype=torch.float32)
+    torch.cuda.synchronize()
+    qr, sr = oracle.quantize_rhs(w)
+    ref_dx = np.zeros((T, K))
+    bound_dx = np.zeros((T, K))
+    mag = np.zeros((T, K))
+    for e in range(E):
+        rows = [(t, j) for t in range(T) for j in range(k) if int(ids[t, j]) == e]
+        if not rows:
+            assert not dw[e].any(), f"expert {e} without rows has nonzero dW"
+            continue
+        ts = [t for t, _ in rows]
+        dh = torch.stack([(dy[t].float() * wts[t, j]).bfloat16() for t, j in rows])
+        one = np.array([len(rows)], np.int32)
+        dl, ab = oracle.gmm_dlhs(dh, qr[e:e + 1], sr[e:e + 1], one)
+        for i, t in enumerate(ts):
+            ref_dx[t] += dl[i]
+            bound_dx[t] += 2e-3 * ab[i] + 2.0 ** -8 * np.abs(dl[i])
+            mag[t] += np.abs(dl[i])
+        ref_w, ab_w = oracle.tgmm_drhs(x[ts], oracle.Q_STATIC, s_val, dh, one)
+        assert_close(dw[e:e + 1], ref_w, ab_w, f"ep dW expert {e}")
+    assert_within(dx, ref_dx, bound_dx + k * 2.0 ** -23 * mag + 1e-30, f"ep dx T={T} E={E} k={k}")
+
+
+def test_gather_scale_rows(dev):
+    src = torch.randn(6, 40).bfloat16().to(dev)
+    idx = torch.tensor([5, -1, 0, 2], dtype=torch.int32, device=dev)
+    sc = torch.tensor([0.5, 3.0, -1.25, 0.1], device=dev)
+    out = ep.gather_scale_rows(src, idx, sc)
+    s = src.float()
+    want = torch.stack([(s[5] * 0.5), torch.zeros(40, device=dev), (s[0] * -1.25), (s[2] * sc[3])]).bfloat16()
+    assert torch.equal(out, want)
