@@ -164,16 +164,20 @@ class ClockSampler:
 
 # ----------------------------------------------------------- our arm
 
-def traffic_record(kernel: str):
-    """DRAM bytes per launch from a committed ncu capture, or None when the
-    kernel source changed since the capture."""
+def workload_key(w, blocks: bool) -> str:
+    return f"{w.name}/G{w.G}/M{w.M}/K{w.K}/N{w.N}/{w.rule}" + ("/blockwise" if blocks else "")
+
+
+def traffic_record(kernel: str, key: str):
+    """DRAM bytes per launch from a committed ncu capture of this kernel on this
+    workload, or None when there is none or the kernel source changed since."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
         src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()[:16]
-        r = rec.get(kernel)
-        if r and r.get("gemm_src_sha256_16") == src_hash:
-            return r.get("bytes_per_launch")
+        for r in rec.get(kernel, []):
+            if r.get("gemm_src_sha256_16") == src_hash and r.get("workload_key") == key:
+                return r.get("bytes_per_launch")
     except Exception:
         pass
     return None
@@ -346,7 +350,7 @@ def run_ours(args):
                     "unit": "GB/s", "frac": round(achieved / peak_bw, 4),
                     "peak_source": f"{peak_src} HBM copy bandwidth",
                     "algorithmic": f"{bytes_pass[dname]:.4g} bytes per launch (operands in, results out)"}
-    roofline["traffic"] = traffic_record(dom)
+    roofline["traffic"] = traffic_record(dom, workload_key(w, blocks))
 
     # merged gate|up workloads: the forward with SwiGLU fused into its
     # epilogue, timed on its own (not part of the step), with an L2 flush
