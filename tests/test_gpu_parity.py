@@ -393,6 +393,35 @@ def test_blockwise_rejects_transposed_rhs(dev):
         gm.gmm_dlhs(dout, codes, scales, gs, transpose_rhs=True)
 
 
+# ---------------------------------------------------------- limits
+
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+def test_maximum_group_count(dev, rule):
+    """G = 1024 (the largest supported), most groups empty, a few large,
+    rows left unrouted: all passes and the fused backward against the oracle."""
+    G, M, K, N = 1024, 3000, 256, 256
+    rng = np.random.default_rng(5)
+    sizes = np.zeros(G, np.int64)
+    hot = rng.choice(G, 40, replace=False)
+    sizes[hot] = rng.multinomial(2900, np.ones(40) / 40)  # 100 of the 3000 rows stay unrouted
+    inp = synth.small_case(G, M, K, N, seed=13, sizes=sizes.tolist())
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    sarg = s if rule == "static" else None
+    codes, scales = gm.gmm_quantize_rhs(w)
+    out = gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=sarg, out_dtype=torch.float32)
+    dl, dw = gm.gmm_backward(lhs, dout, codes, scales, gs, rule=rule, static_scale=sarg, dlhs_dtype=torch.float32)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    ref, ab = oracle.gmm_fwd(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+    assert_close(out, ref, ab, f"G=1024 fwd {rule}")
+    ref, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
+    assert_close(dl, ref, ab, f"G=1024 dlhs {rule}")
+    sel = np.concatenate([np.arange(0, G * K, K * 7), [hot[0] * K + 3, hot[1] * K + K - 1]])
+    ref, ab = oracle.tgmm_drhs(inp.lhs, rule_code(rule), inp.static_scale, inp.dout, inp.group_sizes, sel=sel)
+    assert_close(dw.view(G * K, N)[torch.as_tensor(sel, device=dev)], ref, ab, f"G=1024 drhs {rule}")
+    empty = np.flatnonzero(sizes == 0)
+    assert not dw[torch.as_tensor(empty, device=dev)].any()
+
+
 # ------------------------------------------------------------ identities
 
 def test_merged_gate_up_identity_gpu(dev):
