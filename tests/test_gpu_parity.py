@@ -422,6 +422,32 @@ def test_maximum_group_count(dev, rule):
     assert not dw[torch.as_tensor(empty, device=dev)].any()
 
 
+@pytest.mark.parametrize("G,M,K,N,sizes", [
+    (1, 1, 128, 128, [1]),            # one row, the smallest tile sizes
+    (3, 129, 128, 128, [0, 129, 0]),  # a 129-row group: one full and one 1-row tile / chunk
+    (4, 200, 256, 384, [0, 0, 0, 0]),  # every group empty: all outputs zero
+    (2, 300, 128, 256, [0, 17]),      # 283 unrouted rows
+])
+def test_degenerate_sizes(dev, G, M, K, N, sizes):
+    inp = synth.small_case(G, M, K, N, seed=31, sizes=sizes)
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    codes, scales = gm.gmm_quantize_rhs(w)
+    for rule in ("static", "dynamic"):
+        sarg = s if rule == "static" else None
+        out = gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=sarg, out_dtype=torch.float32)
+        dl, dw = gm.gmm_backward(lhs, dout, codes, scales, gs, rule=rule, static_scale=sarg,
+                                 dlhs_dtype=torch.float32)
+        qr, sr = oracle.quantize_rhs(inp.w)
+        ref, ab = oracle.gmm_fwd(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+        assert_close(out, ref, ab, f"degenerate fwd {sizes} {rule}")
+        ref, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
+        assert_close(dl, ref, ab, f"degenerate dlhs {sizes}")
+        ref, ab = oracle.tgmm_drhs(inp.lhs, rule_code(rule), inp.static_scale, inp.dout, inp.group_sizes)
+        assert_close(dw, ref, ab, f"degenerate drhs {sizes} {rule}")
+        if sum(sizes) == 0:
+            assert not out.any() and not dl.any() and not dw.any()
+
+
 # ------------------------------------------------------------ identities
 
 def test_merged_gate_up_identity_gpu(dev):
