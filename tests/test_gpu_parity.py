@@ -448,6 +448,46 @@ def test_degenerate_sizes(dev, G, M, K, N, sizes):
             assert not out.any() and not dl.any() and not dw.any()
 
 
+@pytest.mark.parametrize("seed", range(12))
+def test_random_shapes(dev, seed):
+    """Random sizes within the supported range (G up to 48, M up to 1600,
+    K and N multiples of 128 up to 768, some groups empty, some rows
+    unrouted), a random rule, rhs layout and output dtype: forward, fused
+    backward and, for even N, the SwiGLU forward against the oracle."""
+    rng = np.random.default_rng(1000 + seed)
+    G = int(rng.integers(1, 49))
+    M = int(rng.integers(1, 1601))
+    K = 128 * int(rng.integers(1, 7))
+    N = 128 * int(rng.integers(1, 7))
+    w = rng.random(G) * (rng.random(G) > 0.3)
+    routed = int(rng.integers(0, M + 1))
+    sizes = rng.multinomial(routed, w / w.sum()) if w.sum() > 0 else np.zeros(G, np.int64)
+    rule = ["static", "dynamic"][seed % 2]
+    transpose = bool(rng.integers(0, 2))
+    out_dtype = [torch.bfloat16, torch.float32][int(rng.integers(0, 2))]
+    inp = synth.small_case(G, M, K, N, seed=seed, sizes=sizes.tolist())
+    lhs, wt, dout, gs, s = to_dev(inp, dev)
+    sarg = s if rule == "static" else None
+    codes, scales = gm.gmm_quantize_rhs(wt, transpose_out=transpose)
+    out = gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=sarg, transpose_rhs=transpose,
+                     out_dtype=out_dtype)
+    dl, dw = gm.gmm_backward(lhs, dout, codes, scales, gs, rule=rule, static_scale=sarg, transpose_rhs=transpose,
+                             dlhs_dtype=out_dtype)
+    qr, sr = oracle.quantize_rhs(inp.w)
+    tag = f"seed {seed}: G={G} M={M} K={K} N={N} {rule} t={transpose} {out_dtype}"
+    ref, ab = oracle.gmm_fwd(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+    assert_close(out, ref, ab, "fwd " + tag)
+    ref, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
+    assert_close(dl, ref, ab, "dlhs " + tag)
+    ref, ab = oracle.tgmm_drhs(inp.lhs, rule_code(rule), inp.static_scale, inp.dout, inp.group_sizes)
+    assert_close(dw, ref, ab, "drhs " + tag)
+    if N % 256 == 0:
+        sw = gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule=rule, static_scale=sarg, transpose_rhs=transpose,
+                               out_dtype=out_dtype)
+        ref, terms = oracle.gmm_fwd_swiglu(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
+        assert_within(sw, ref, swiglu_bound(out_dtype, terms, ref), "swiglu " + tag)
+
+
 # ------------------------------------------------------------ identities
 
 def test_merged_gate_up_identity_gpu(dev):
