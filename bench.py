@@ -241,6 +241,9 @@ def run_ours(args):
     ws = torch.empty(max(gm.gmm_workspace_bytes(op, M, K, Np, G) for op in (0, 1, 2, 3)), dtype=torch.uint8,
                      device=dev)
     fused_bwd = not args.separate_backward
+    # static rule: the forward hands its lhs codes to the backward (tgmm lhs re-laid out, not quantized again)
+    keep_lhs = rule == "static" and not bf16_family
+    lhs_codes = torch.empty((M, K), dtype=torch.uint8, device=dev) if keep_lhs else None
     sarg = s_static if rule == "static" else None
     grule = "none" if bf16_family else "dynamic"
     launches = [0]
@@ -249,17 +252,22 @@ def run_ours(args):
         for i in range(parts):
             c_, r_ = (codes_, rscales_) if i == 0 else wparts[i]
             d_ = dout_ if i == 0 else douts[i]
-            gm.gmm_fwd(lhs_, c_, r_, gs_, rule=rule, static_scale=sarg, out=out, ws=ws)
+            if keep_lhs:
+                gm.gmm_fwd_keep_lhs(lhs_, c_, r_, gs_, rule=rule, static_scale=sarg, out=out, ws=ws,
+                                    lhs_codes=lhs_codes)
+            else:
+                gm.gmm_fwd(lhs_, c_, r_, gs_, rule=rule, static_scale=sarg, out=out, ws=ws)
             launches[0] += gm.last_launch_count()
+            x_ = lhs_codes if keep_lhs else lhs_  # the tgmm's lhs operand
             if blocks:
                 c_, r_ = dl_codes, dl_scales
             if fused_bwd:
-                gm.gmm_backward(lhs_, d_, c_, r_, gs_, rule=rule, static_scale=sarg, dlhs=dl, drhs=dw, ws=ws)
+                gm.gmm_backward(x_, d_, c_, r_, gs_, rule=rule, static_scale=sarg, dlhs=dl, drhs=dw, ws=ws)
                 launches[0] += gm.last_launch_count()
             else:
                 gm.gmm_dlhs(d_, c_, r_, gs_, out=dl, ws=ws, rule=grule)
                 launches[0] += gm.last_launch_count()
-                gm.tgmm_drhs(lhs_, d_, gs_, rule=rule, static_scale=sarg, out=dw, ws=ws)
+                gm.tgmm_drhs(x_, d_, gs_, rule=rule, static_scale=sarg, out=dw, ws=ws)
                 launches[0] += gm.last_launch_count()
 
     def barrier():
@@ -456,6 +464,7 @@ def run_ours(args):
         d_out = [(out if i == 0 else torch.empty_like(out), dl if i == 0 else torch.empty_like(dl),
                   dw if i == 0 else torch.empty_like(dw)) for i in range(2)]
         ws2 = [ws, torch.empty_like(ws)]
+        e2e_codes = [lhs_codes, torch.empty_like(lhs_codes)] if keep_lhs else None
         h2d = sum(t.numel() * t.element_size() for t in (h_lhs, h_dout, h_codes, h_rs, h_gs))
         d2h = sum(t.numel() * t.element_size() for t in (h_out[0], h_dl[0], h_dw[0]))
         s_up, s_cmp, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
@@ -482,16 +491,21 @@ def run_ours(args):
                 s_cmp.wait_event(up_done[b])
                 if used_out[b]:
                     s_cmp.wait_event(down_done[b])  # download of step i-2 has read this output set
-                gm.gmm_fwd(a_lhs, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, out=o_out, ws=ws2[b])
+                if keep_lhs:
+                    gm.gmm_fwd_keep_lhs(a_lhs, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, out=o_out,
+                                        ws=ws2[b], lhs_codes=e2e_codes[b])
+                else:
+                    gm.gmm_fwd(a_lhs, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, out=o_out, ws=ws2[b])
                 launches[0] += gm.last_launch_count()
+                a_x = e2e_codes[b] if keep_lhs else a_lhs
                 if fused_bwd:
-                    gm.gmm_backward(a_lhs, a_dout, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, dlhs=o_dl,
+                    gm.gmm_backward(a_x, a_dout, a_codes, a_rs, a_gs, rule=rule, static_scale=sarg, dlhs=o_dl,
                                     drhs=o_dw, ws=ws2[b])
                     launches[0] += gm.last_launch_count()
                 else:
                     gm.gmm_dlhs(a_dout, a_codes, a_rs, a_gs, out=o_dl, ws=ws2[b], rule=grule)
                     launches[0] += gm.last_launch_count()
-                    gm.tgmm_drhs(a_lhs, a_dout, a_gs, rule=rule, static_scale=sarg, out=o_dw, ws=ws2[b])
+                    gm.tgmm_drhs(a_x, a_dout, a_gs, rule=rule, static_scale=sarg, out=o_dw, ws=ws2[b])
                     launches[0] += gm.last_launch_count()
                 cmp_done[b].record(s_cmp)
             with torch.cuda.stream(s_down):
@@ -516,7 +530,7 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(ems / args.e2e_steps, 3),
                "path": "per step: pinned host -> device copies of lhs, dout, rhs codes + scales, group sizes; "
-                       "gmm_fwd + gmm_backward (dlhs, drhs); device -> pinned host copies of out, dlhs, dW. Steps "
+                       "gmm_fwd(_keep_lhs) + gmm_backward (dlhs, drhs); device -> pinned host copies of out, dlhs, dW. Steps "
                        "pipelined over upload / compute / download streams with two device buffer sets."}
 
     cpu = None
@@ -536,6 +550,8 @@ def run_ours(args):
                                 "calls_per_pass": parts,
                                 "backward": ("gmm_backward (dout quantized once for dlhs and drhs)" if fused_bwd
                                              else "gmm_dlhs + tgmm_drhs"),
+                                "lhs_codes": ("gmm_fwd_keep_lhs hands the forward's E4M3 lhs codes to the tgmm"
+                                              if keep_lhs else "the tgmm quantizes lhs itself"),
                                 "rhs_scales": ("block-wise: fwd [G, K/128, N], dlhs [G, N/128, K]" if blocks
                                                else "per channel [G, N]"),
                                 **({"l2": "flushed before every step (256 MiB write outside the timed events; "

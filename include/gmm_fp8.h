@@ -177,6 +177,24 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
                    void *stream);
 
 /*
+ * gmm_fwd that also hands its lhs quantization back to the caller
+ * ("add static LHS scaling support for GMM v2 FWD", maxtext PR #4735, rebase
+ * commit text: activations quantized once and the quantized array passed on).
+ * lhs must be bf16 with rule STATIC or DYNAMIC.  lhs_codes: device E4M3
+ * [M, K], written with the codes the forward multiplies (rows in no group
+ * included, as gmm_quantize axis 1 writes them); lhs_scales: device float
+ * [K/128, M] for DYNAMIC (unused and may be NULL for STATIC).  The codes are
+ * made in these buffers instead of the workspace, so the call costs the same
+ * as gmm_fwd.  With the static rule the codes are tgmm_drhs's / gmm_backward's
+ * lhs operand as they are (a pre-quantized lhs), which then skips its
+ * quantization of lhs.  Every other argument, result and error is gmm_fwd's;
+ * a NULL lhs_codes (or NULL lhs_scales with DYNAMIC) is GMM_ERR_INVALID_ARG.
+ */
+gmm_status gmm_fwd_keep_lhs(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes,
+                            int32_t G, int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws,
+                            size_t ws_bytes, uint8_t *lhs_codes, float *lhs_scales, void *stream);
+
+/*
  * Forward gmm of the merged gate|up weights with the SwiGLU activation fused
  * into its epilogue ("FP8 Megablox for batch split", maxtext PR #3770,
  * Description (2): W0 and W1 are concatenated so that one gmm call covers

@@ -26,7 +26,7 @@ EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm
            "gmm_dlhs", "tgmm_drhs", "gmm_read_device_status", "gmm_selftest_timeout", "gmm_set_wait_limit_ns",
            "gmm_status_string", "gmm_last_launch_count", "gmm_profile_enable", "gmm_profile_collect",
            "gmm_fwd_noalloc", "gmm_fwd_swiglu", "gmm_quantize_rhs_blocks", "gmm_gather_rows",
-           "gmm_combine_rows", "gmm_backward", "gmm_gather_scale_rows"]
+           "gmm_combine_rows", "gmm_backward", "gmm_gather_scale_rows", "gmm_fwd_keep_lhs"]
 
 
 class Operand(ctypes.Structure):
@@ -62,6 +62,9 @@ def lib():
     L.gmm_fwd.argtypes = [Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp, sz, vp]
     L.gmm_fwd.restype = st
     L.gmm_fwd_swiglu.argtypes = L.gmm_fwd.argtypes
+    L.gmm_fwd_keep_lhs.argtypes = [Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp, sz,
+                                   vp, vp, vp]
+    L.gmm_fwd_keep_lhs.restype = st
     L.gmm_quantize_rhs_blocks.argtypes = [vp, i32, i64, i64, ctypes.c_int, vp, vp, vp]
     L.gmm_quantize_rhs_blocks.restype = st
     L.gmm_backward.argtypes = [Operand, Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int,

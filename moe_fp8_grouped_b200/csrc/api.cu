@@ -324,10 +324,12 @@ gmm_status gmm_quantize(const void *x_bf16, int64_t rows, int64_t cols, gmm_qrul
 
 }  // extern "C"
 
-// Forward pass shared by gmm_fwd (F == 0) and gmm_fwd_swiglu (F = N / 2).
+// Forward pass shared by gmm_fwd (F == 0), gmm_fwd_swiglu (F = N / 2) and
+// gmm_fwd_keep_lhs (codes_out != NULL: the lhs codes and dynamic scales are
+// written to the caller's buffers instead of the workspace).
 static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes, int32_t G,
                            int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
-                           void *stream, int64_t F) {
+                           void *stream, int64_t F, uint8_t *codes_out = nullptr, float *scales_out = nullptr) {
   g_launches = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   gmm_status s = check_sizes(M, K, N, G);
@@ -349,14 +351,16 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   const bool blk = elem == 1 && rhs.rule == GMM_Q_DYNAMIC;  // block-wise rhs scales [G, K/128, N]
   if (blk && transpose_rhs) return GMM_ERR_UNSUPPORTED;
   const void *A = lhs.data;
+  uint8_t *codes = codes_out ? codes_out : P.codes_a;
+  float *qscales = (codes_out && dyn) ? scales_out : P.scales_a;
   if (elem == 1 && !preq) {
     s = cuda_status(prof("quant_rows", st, [&] {
-      return launch_quant_rows(lhs.data, M, K, dyn, dyn ? nullptr : lhs.scale, nullptr, P.offs, G, P.codes_a,
-                               P.scales_a, P.status, st);
+      return launch_quant_rows(lhs.data, M, K, dyn, dyn ? nullptr : lhs.scale, nullptr, P.offs, G, codes, qscales,
+                               P.status, st);
     }));
     if (s != GMM_OK) return s;
     ++n;
-    A = P.codes_a;
+    A = codes;
   }
   const bool bmn = transpose_rhs == 0;  // [G, K, N]: N contiguous = MN-major B
   const uint32_t bke = 128 / elem;
@@ -376,7 +380,7 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   p.b_group_rows = static_cast<int>(bmn ? K : N);
   p.offs = P.offs;
   p.tpre = P.tpre;
-  p.row_scale = (elem == 1 && dyn) ? (preq ? lhs.scale : P.scales_a) : nullptr;
+  p.row_scale = (elem == 1 && dyn) ? (preq ? lhs.scale : qscales) : nullptr;
   p.row_scale_ld = M;
   p.col_scale = (elem == 1 && !blk) ? rhs.scale : nullptr;
   p.colblk_scale = blk ? rhs.scale : nullptr;
@@ -404,6 +408,18 @@ gmm_status gmm_fwd(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const in
                    int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws, size_t ws_bytes,
                    void *stream) {
   return fwd_impl(lhs, rhs, transpose_rhs, group_sizes, G, M, K, N, out, out_dtype, ws, ws_bytes, stream, 0);
+}
+
+gmm_status gmm_fwd_keep_lhs(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes,
+                            int32_t G, int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype, void *ws,
+                            size_t ws_bytes, uint8_t *lhs_codes, float *lhs_scales, void *stream) {
+  g_launches = 0;
+  if (!lhs_codes || lhs.dtype != GMM_BF16 || (lhs.rule != GMM_Q_STATIC && lhs.rule != GMM_Q_DYNAMIC))
+    return GMM_ERR_INVALID_ARG;
+  if (lhs.rule == GMM_Q_DYNAMIC && !lhs_scales) return GMM_ERR_INVALID_ARG;
+  if (!al16(lhs_codes) || (lhs_scales && !al16(lhs_scales))) return GMM_ERR_ALIGNMENT;
+  return fwd_impl(lhs, rhs, transpose_rhs, group_sizes, G, M, K, N, out, out_dtype, ws, ws_bytes, stream, 0,
+                  lhs_codes, lhs_scales);
 }
 
 gmm_status gmm_fwd_swiglu(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes,

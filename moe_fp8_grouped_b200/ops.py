@@ -166,6 +166,41 @@ def gmm_fwd(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | Non
                 lhs_scales, swiglu=False)
 
 
+def gmm_fwd_keep_lhs(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | None,
+                     group_sizes: torch.Tensor, rule="static", static_scale: torch.Tensor | None = None,
+                     transpose_rhs: bool = False, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                     ws: torch.Tensor | None = None, lhs_codes: torch.Tensor | None = None,
+                     lhs_scales: torch.Tensor | None = None):
+    """gmm_fwd that also returns the E4M3 codes [M, K] (and, for the dynamic
+    rule, the block scales [K/128, M]) it made for lhs: (out, codes, scales),
+    written into ``lhs_codes`` / ``lhs_scales`` when given.
+    With the static rule the codes can be passed as the lhs of tgmm_drhs /
+    gmm_backward, which then skip their own quantization of lhs."""
+    M, K = lhs.shape
+    G, K2, N = (rhs.shape[0], rhs.shape[2], rhs.shape[1]) if transpose_rhs else rhs.shape
+    assert K2 == K, "lhs / rhs contraction mismatch"
+    r = _rule(rule)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=lhs.device)
+    if ws is None:
+        ws = workspace(gmm_workspace_bytes(B.OP_FWD, M, K, N, G), lhs.device)
+    codes = lhs_codes if lhs_codes is not None else torch.empty((M, K), dtype=torch.uint8, device=lhs.device)
+    scales = None
+    if r == B.Q_DYNAMIC:
+        scales = lhs_scales if lhs_scales is not None else torch.empty((K // 128, M), dtype=torch.float32,
+                                                                         device=lhs.device)
+    a = _operand(_dev(lhs, "lhs", torch.bfloat16), B.DT_BF16,
+                 _dev(static_scale, "static_scale", torch.float32) if static_scale is not None else None, r)
+    st = B.lib().gmm_fwd_keep_lhs(a, _rhs_operand(rhs, rhs_scales), int(transpose_rhs),
+                                  _dev(group_sizes, "group_sizes", torch.int32), G, M, K, N,
+                                  _dev(out, "out", (torch.bfloat16, torch.float32)), _TORCH_DT[out.dtype],
+                                  ws.data_ptr(), ws.numel(), _dev(codes, "lhs_codes", torch.uint8),
+                                  _dev(scales, "lhs_scales", torch.float32) if scales is not None else None,
+                                  _stream(lhs))
+    _check(st, "gmm_fwd_keep_lhs")
+    return out, codes, scales
+
+
 def gmm_fwd_swiglu(lhs: torch.Tensor, rhs: torch.Tensor, rhs_scales: torch.Tensor | None,
                    group_sizes: torch.Tensor, rule="static", static_scale: torch.Tensor | None = None,
                    transpose_rhs: bool = False, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,

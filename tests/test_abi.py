@@ -86,6 +86,11 @@ def test_host_errors(L):
     assert sw(lhs, rhs, 0, gs, 8, 256, 512, 0, out, B.DT_BF16, ws, big, None) == 2
     assert sw(lhs, rhs, 0, None, 8, 256, 512, 512, out, B.DT_BF16, ws, big, None) == 1
     assert sw(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, 1024, None) == 9
+    kl = L.gmm_fwd_keep_lhs
+    assert kl(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big, None, None, None) == 1  # no codes buffer
+    assert kl(_op(FAKE, B.DT_BF16, None, B.Q_DYNAMIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big, FAKE,
+              None, None) == 1  # dynamic rule without a scales buffer
+    assert kl(lhs, rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big, FAKE + 2, None, None) == 3
     bw = L.gmm_backward
     dop = _op(FAKE, B.DT_BF16, None, B.Q_DYNAMIC)
     assert bw(lhs, dop, rhs, 0, gs, 8, 256, 500, 512, out, B.DT_BF16, out, B.DT_F32, ws, big, None) == 2  # K % 128

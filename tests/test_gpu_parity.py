@@ -173,6 +173,33 @@ def test_fwd_prequantized_lhs(dev, rule, transpose):
     assert_close(outside, ref, ab, f"prequantized fwd {rule}")
 
 
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
+@pytest.mark.parametrize("transpose", [False, True])
+def test_fwd_keep_lhs_hands_back_its_codes(dev, rule, transpose):
+    """gmm_fwd_keep_lhs gives gmm_fwd's result bit for bit and the codes /
+    scales gmm_quantize makes; with the static rule those codes are the
+    backward's lhs operand, with the same dW."""
+    inp = case_inputs("ragged")
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    sarg = s if rule == "static" else None
+    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
+    out, qc, qs = gm.gmm_fwd_keep_lhs(lhs, codes, scales, gs, rule=rule, static_scale=sarg, transpose_rhs=transpose,
+                                      out_dtype=torch.float32)
+    assert gm.last_launch_count() == 3
+    ref = gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=sarg, transpose_rhs=transpose,
+                     out_dtype=torch.float32)
+    assert torch.equal(out, ref)
+    c2, s2 = gm.gmm_quantize(lhs, rule, axis=1, static_scale=sarg)
+    assert torch.equal(qc, c2)
+    if rule == "dynamic":
+        assert torch.equal(qs, s2)
+    else:
+        dl1, dw1 = gm.gmm_backward(qc, dout, codes, scales, gs, rule="static", static_scale=s, transpose_rhs=transpose)
+        dl2, dw2 = gm.gmm_backward(lhs, dout, codes, scales, gs, rule="static", static_scale=s,
+                                   transpose_rhs=transpose)
+        assert torch.equal(dl1, dl2) and torch.equal(dw1, dw2)
+
+
 @pytest.mark.parametrize("name", ["ragged", "big_group"])
 def test_drhs_reuses_static_forward_codes(dev, name):
     """Static rule: the forward's lhs codes (quantized once, as for an
