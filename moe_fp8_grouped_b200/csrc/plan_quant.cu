@@ -393,25 +393,51 @@ cudaError_t launch_quant_chunks(const void *x, int64_t rows, int64_t cols, bool 
 // Backward dout from one read: the tgmm chunk operand and the dlhs row
 // operand.  One CTA per (chunk, 128-column slice) stages the chunk's rows
 // (zero-filled past the chunk) by cp.async, then two warp roles work on the
-// tile at once: warps 0-1 the columns (thread t: columns 2t, 2t+1, absmax over
-// the chunk's rows, one code line per column), warps 2-5 the rows (a warp
-// takes two rows per step, one per half-warp, 8 columns per lane:
-// t = fl32(dout * s_r[g, n]) when kFold, absmax over the 128-column block by
-// shuffles, codes and the block scale, exactly as quant_rows_kernel computes
-// them).  The small tile (34 KB) keeps six CTAs per SM, so loads of some
-// overlap the arithmetic of others.
+// tile at once:
+//   warps 0-1, the columns: thread t holds columns 2t, 2t+1; the absmax over
+//     the chunk's rows is taken on packed bf16 pairs (exact: a max of bf16
+//     values), then each column's 128 codes form one code line;
+//   warps 2-5, the rows: a warp takes 8 rows per step, lane = row (lane & 7)
+//     and 32 columns (lane >> 3), so a quarter-warp reads 8 rows at one bank
+//     offset each (row pitch 68 words) and the block scale is computed once
+//     per 32 elements; t = fl32(dout * s_r[g, n]) when kFold, absmax over the
+//     128-column block by two shuffles, codes and the block scale exactly as
+//     quant_rows_kernel computes them.
+// Packed f32x2 multiplies and 32-byte stores keep the instruction count low
+// enough for the kernel to stream at memory speed.  The small tile (34 KB)
+// keeps six CTAs per SM, so loads of some overlap the arithmetic of others.
 constexpr int kDoutCols = 128;
 constexpr int kDoutPitch = kDoutCols + 8;                 // bf16 per staged row (16-byte aligned rows)
 constexpr int kDoutColThreads = kDoutCols / 2;            // two columns per thread
 constexpr int kDoutRowWarps = 4;
 constexpr int kDoutThreads = kDoutColThreads + 32 * kDoutRowWarps;
+constexpr int kDoutRowsPerStep = 8;                       // rows per row-warp step (lane & 7)
+constexpr int kDoutLaneCols = kDoutCols / 4;              // columns per row lane (lane >> 3)
+
+// 32 code bytes: one 256-bit store when dst is 32-byte aligned, else two
+// 128-bit stores (dst is always 16-byte aligned here).
+__device__ __forceinline__ void store_codes32(uint8_t *dst, const uint32_t (&w)[8], bool v8) {
+  if (v8) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+  } else {
+    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// column scale s_r[g, c0 + c] staged at c + 4 (c / 32): the four 32-column
+// groups start in different banks
+__device__ __forceinline__ int cs_slot(int c) { return c + ((c >> 5) << 2); }
 
 template <bool kFold>
-__global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
+__global__ void __launch_bounds__(kDoutThreads, 6) quant_dout_both_kernel(
     const __nv_bfloat16 *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ col_scale,
     const int *__restrict__ offs, const int *__restrict__ tpre, int G, uint8_t *__restrict__ codes_t,
     float *__restrict__ scales_t, uint8_t *__restrict__ codes_r, float *__restrict__ scales_r) {
   __shared__ __align__(16) __nv_bfloat16 tile[kBlk * kDoutPitch];
+  __shared__ __align__(16) float s_cs[kDoutCols + 16];
   __shared__ int s_info[4];
   const int j = blockIdx.y;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kDoutCols;  // cols is a multiple of 128
@@ -436,84 +462,91 @@ __global__ void __launch_bounds__(kDoutThreads) quant_dout_both_kernel(
     const __nv_bfloat16 *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
     cp_async_16_zfill(tile + rr * kDoutPitch + cc, src, in);
   }
+  if constexpr (kFold) {
+    for (int c = threadIdx.x; c < kDoutCols; c += kDoutThreads)
+      s_cs[cs_slot(c)] = __ldg(col_scale + static_cast<int64_t>(g) * cols + c0 + c);
+  }
   cp_async_wait_all();
   __syncthreads();
   if (threadIdx.x >= kDoutColThreads) {
     // ---- rows: the dlhs operand
     const int lane = threadIdx.x & 31, warp = (threadIdx.x - kDoutColThreads) >> 5;
-    const int half = lane >> 4, hl = lane & 15;
-    const int cl = hl * 8;  // the lane's 8 columns in the slice
-    float cs[8];
+    const int rl = lane & (kDoutRowsPerStep - 1), cl = (lane >> 3) * kDoutLaneCols;
+    const bool v8 = (reinterpret_cast<uintptr_t>(codes_r) & 31u) == 0;
+    for (int rb = kDoutRowsPerStep * warp; rb < nr; rb += kDoutRowsPerStep * kDoutRowWarps) {
+      const int r = rb + rl;  // < 128; rows past the chunk hold zeros and are not stored
+      float2 v[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) cs[i] = 1.0f;
-    if constexpr (kFold) {
-      const float4 *c = reinterpret_cast<const float4 *>(col_scale + static_cast<int64_t>(g) * cols + c0 + cl);
-      const float4 a = __ldg(c), b = __ldg(c + 1);
-      cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
-      cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
-    }
-    for (int rb = 2 * warp; rb < nr; rb += 2 * kDoutRowWarps) {
-      const int r = rb + half;  // rows past the chunk hold zeros and are not stored
-      float v[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(tile + r * kDoutPitch + cl), v);
+      for (int k = 0; k < 4; ++k) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(tile + r * kDoutPitch + cl + 8 * k);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[4 * k + e] = __bfloat1622float2(h[e]);
+      }
       if constexpr (kFold) {
+        const float4 *c4 = reinterpret_cast<const float4 *>(s_cs + cs_slot(cl));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], cs[i]);
+        for (int k = 0; k < 8; ++k) {
+          const float4 c = c4[k];
+          v[2 * k] = __fmul2_rn(v[2 * k], make_float2(c.x, c.y));
+          v[2 * k + 1] = __fmul2_rn(v[2 * k + 1], make_float2(c.z, c.w));
+        }
       }
       float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-      for (int d = 8; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 8));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
       float sc, inv;
       dyn_scale(amax, sc, inv);
       if (r < nr) {
-        uint2 out;
-        out.x = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
-                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
-        out.y = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv))) |
-                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv))) << 16);
+        const float2 inv2 = make_float2(inv, inv);
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 a = __fmul2_rn(v[2 * i], inv2), b = __fmul2_rn(v[2 * i + 1], inv2);
+          w[i] = static_cast<uint32_t>(cvt_e4m3x2(a.x, a.y)) | (static_cast<uint32_t>(cvt_e4m3x2(b.x, b.y)) << 16);
+        }
         const int64_t m = r0 + r;
-        *reinterpret_cast<uint2 *>(codes_r + m * cols + c0 + cl) = out;
-        if (hl == 0) scales_r[(c0 / kBlk) * rows + m] = sc;
+        store_codes32(codes_r + m * cols + c0 + cl, w, v8);
+        if (cl == 0) scales_r[(c0 / kBlk) * rows + m] = sc;
       }
     }
     return;
   }
   // ---- columns: the tgmm operand (quant_chunks_kernel, dynamic rule)
-  const int col = 2 * threadIdx.x;  // and col + 1
-  const uint32_t *t32 = reinterpret_cast<const uint32_t *>(tile);
-  auto pair = [&](int r) -> float2 {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t32[(r * kDoutPitch + col) >> 1]));
-  };
-  float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll 8
-  for (int r = 0; r < kBlk; ++r) {
-    const float2 v = pair(r);
-    a0 = fmaxf(a0, fabsf(v.x));
-    a1 = fmaxf(a1, fabsf(v.y));
-  }
+  const int t = threadIdx.x;  // columns 2t, 2t + 1
+  const __nv_bfloat162 *t2 = reinterpret_cast<const __nv_bfloat162 *>(tile);
+  constexpr int kPitch2 = kDoutPitch / 2;  // bf16 pairs per staged row
+  __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
+#pragma unroll 16
+  for (int r = 0; r < kBlk; ++r) m2 = __hmax2(m2, __habs2(t2[r * kPitch2 + t]));
+  const float2 am = __bfloat1622float2(m2);
   float s0, s1, inv0, inv1;
-  dyn_scale(a0, s0, inv0);
-  dyn_scale(a1, s1, inv1);
-  uint8_t *dst0 = codes_t + (static_cast<int64_t>(j) * cols + c0 + col) * kBlk;
+  dyn_scale(am.x, s0, inv0);
+  dyn_scale(am.y, s1, inv1);
+  const float2 inv = make_float2(inv0, inv1);
+  uint8_t *dst0 = codes_t + (static_cast<int64_t>(j) * cols + c0 + 2 * t) * kBlk;
   uint8_t *dst1 = dst0 + kBlk;
+  const bool v8 = (reinterpret_cast<uintptr_t>(codes_t) & 31u) == 0;
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    uint32_t w0[4], w1[4];
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w0[8], w1[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int r = q * 16 + e * 4;
-      const float2 v0 = pair(r), v1 = pair(r + 1), v2 = pair(r + 2), v3 = pair(r + 3);
-      w0[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.x, inv0), __fmul_rn(v1.x, inv0))) |
-              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.x, inv0), __fmul_rn(v3.x, inv0))) << 16);
-      w1[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.y, inv1), __fmul_rn(v1.y, inv1))) |
-              (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.y, inv1), __fmul_rn(v3.y, inv1))) << 16);
+    for (int e = 0; e < 8; ++e) {
+      const int r = q * 32 + e * 4;
+      float2 f[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f[i] = __fmul2_rn(__bfloat1622float2(t2[(r + i) * kPitch2 + t]), inv);
+      w0[e] = static_cast<uint32_t>(cvt_e4m3x2(f[0].x, f[1].x)) |
+              (static_cast<uint32_t>(cvt_e4m3x2(f[2].x, f[3].x)) << 16);
+      w1[e] = static_cast<uint32_t>(cvt_e4m3x2(f[0].y, f[1].y)) |
+              (static_cast<uint32_t>(cvt_e4m3x2(f[2].y, f[3].y)) << 16);
     }
-    *reinterpret_cast<uint4 *>(dst0 + q * 16) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-    *reinterpret_cast<uint4 *>(dst1 + q * 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    store_codes32(dst0 + q * 32, w0, v8);
+    store_codes32(dst1 + q * 32, w1, v8);
   }
-  *reinterpret_cast<float2 *>(scales_t + static_cast<int64_t>(j) * cols + c0 + col) = make_float2(s0, s1);
+  *reinterpret_cast<float2 *>(scales_t + static_cast<int64_t>(j) * cols + c0 + 2 * t) = make_float2(s0, s1);
 }
 
 cudaError_t launch_quant_dout_both(const void *x, int64_t rows, int64_t cols, const float *col_scale, const int *offs,
