@@ -238,15 +238,31 @@ cudaError_t launch_quant_rows(const void *x, int64_t rows, int64_t cols, bool dy
 
 // ---------------------------------------------------- chunks (axis 0)
 
-// One CTA of 64 threads per (128-column slice, chunk).  The chunk's rows (at
-// most 128, the rest zero) are staged in shared memory with cp.async; thread t
-// owns the adjacent columns 2t and 2t+1: it takes each column's absmax over the
-// chunk and writes each column's 128 codes as one line of the chunk-major
-// transposed layout [chunk][column][128], so a CTA writes one contiguous block.
-// The 34 KB tile keeps six CTAs per SM, so loads of some overlap the work of
-// others.
+// 32 code bytes: one 256-bit store when dst is 32-byte aligned, else two
+// 128-bit stores (dst is always 16-byte aligned here).
+__device__ __forceinline__ void store_codes32(uint8_t *dst, const uint32_t (&w)[8], bool v8) {
+  if (v8) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+  } else {
+    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+
+// One CTA of 128 threads per (128-column slice, chunk).  The chunk's rows (at
+// most 128, the rest zero) are staged in shared memory with cp.async; threads
+// t and t + 64 own the adjacent columns 2t and 2t+1, each for one half of the
+// rows: the halves' absmax (on packed bf16 pairs, exact) meet in shared
+// memory, and each thread writes its 64 rows of both columns' code lines in
+// the chunk-major transposed layout [chunk][column][128], so a CTA writes one
+// contiguous block.  The 34 KB tile keeps six CTAs per SM, so loads of some
+// overlap the work of others.
 constexpr int kChunkCols = 128;
-constexpr int kChunkThreads = kChunkCols / 2;
+constexpr int kChunkPairs = kChunkCols / 2;  // column pairs per slice
+constexpr int kChunkThreads = 2 * kChunkPairs;
 constexpr int kChunkPitch = kChunkCols + 8;  // bf16 per staged row (16-byte aligned rows)
 constexpr size_t kChunkSmem = static_cast<size_t>(kBlk) * kChunkPitch * sizeof(__nv_bfloat16);
 
@@ -281,13 +297,14 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
   extern __shared__ __align__(16) uint8_t qsm[];
   __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(qsm);  // [128][kChunkPitch]
   __shared__ int s_info[3];
+  __shared__ __nv_bfloat162 s_am[2][kChunkPairs];
   const int j = blockIdx.y;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kChunkCols;
   if (threadIdx.x == 0) s_info[0] = find_chunk(j, offs, tpre, G, s_info[1], s_info[2]) ? 1 : 0;
   __syncthreads();
   if (!s_info[0]) return;
   const int r0 = s_info[1], nr = s_info[2];
-  // 128 rows x 32 sixteen-byte pieces, all in flight; rows past the chunk and
+  // 128 rows x 16 sixteen-byte pieces, all in flight; rows past the chunk and
   // columns past the matrix are zero-filled
   for (int i = threadIdx.x; i < kBlk * (kChunkCols / 8); i += kChunkThreads) {
     const int rr = i / (kChunkCols / 8), cc = (i % (kChunkCols / 8)) * 8;
@@ -297,24 +314,26 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
   }
   cp_async_wait_all();
   __syncthreads();
-  const int col = 2 * threadIdx.x;  // and col + 1
-  if (c0 + col >= cols) return;     // cols is a multiple of 128: both columns are in or out
-  const uint32_t *t32 = reinterpret_cast<const uint32_t *>(tile);
-  auto pair = [&](int r) -> float2 {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t32[(r * kChunkPitch + col) >> 1]));
-  };
+  const int cp = threadIdx.x % kChunkPairs, rh = threadIdx.x / kChunkPairs;  // column pair, row half
+  const int col = 2 * cp;                                                     // and col + 1
+  const int rbeg = rh * (kBlk / 2);
+  const bool active = c0 + col < cols;  // both columns are in or out (cols is even)
+  const __nv_bfloat162 *t2 = reinterpret_cast<const __nv_bfloat162 *>(tile);
+  constexpr int kPitch2 = kChunkPitch / 2;  // bf16 pairs per staged row
   const int64_t line = (static_cast<int64_t>(j) * cols + c0 + col) * kBlk;  // element offset of column col's line
   if constexpr (kCopy) {
     // bf16 family: transposed bf16 copy, no scale
-    uint16_t *dst0 = static_cast<uint16_t *>(codes_t) + line;
+    if (!active) return;
+    const uint32_t *t32 = reinterpret_cast<const uint32_t *>(tile);
+    uint16_t *dst0 = static_cast<uint16_t *>(codes_t) + line + rbeg;
     uint16_t *dst1 = dst0 + kBlk;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
+    for (int q = 0; q < 8; ++q) {
       uint32_t w0[4], w1[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint32_t a = t32[((q * 8 + 2 * e) * kChunkPitch + col) >> 1];
-        const uint32_t b = t32[((q * 8 + 2 * e + 1) * kChunkPitch + col) >> 1];
+        const uint32_t a = t32[(rbeg + q * 8 + 2 * e) * kPitch2 + cp];
+        const uint32_t b = t32[(rbeg + q * 8 + 2 * e + 1) * kPitch2 + cp];
         w0[e] = (a & 0xFFFFu) | (b << 16);
         w1[e] = (a >> 16) | (b & 0xFFFF0000u);
       }
@@ -324,15 +343,14 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
   } else {
     float s0, s1, inv0, inv1;
     if constexpr (kDynamic) {
-      float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll 8
-      for (int r = 0; r < kBlk; ++r) {
-        const float2 v = pair(r);
-        a0 = fmaxf(a0, fabsf(v.x));
-        a1 = fmaxf(a1, fabsf(v.y));
-      }
-      dyn_scale(a0, s0, inv0);
-      dyn_scale(a1, s1, inv1);
+      __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
+#pragma unroll 16
+      for (int r = rbeg; r < rbeg + kBlk / 2; ++r) m2 = __hmax2(m2, __habs2(t2[r * kPitch2 + cp]));
+      s_am[rh][cp] = m2;
+      __syncthreads();
+      const float2 am = __bfloat1622float2(__hmax2(s_am[0][cp], s_am[1][cp]));
+      dyn_scale(am.x, s0, inv0);
+      dyn_scale(am.y, s1, inv1);
     } else {
       float s = *static_scale;
       const bool ok = static_scale_ok(s);
@@ -342,24 +360,30 @@ __global__ void __launch_bounds__(kChunkThreads) quant_chunks_kernel(
       s0 = s1 = s;
       inv0 = inv1 = inv;
     }
-    uint8_t *dst0 = static_cast<uint8_t *>(codes_t) + line;
+    if (!active) return;
+    const float2 inv = make_float2(inv0, inv1);
+    uint8_t *dst0 = static_cast<uint8_t *>(codes_t) + line + rbeg;
     uint8_t *dst1 = dst0 + kBlk;
+    const bool v8 = (reinterpret_cast<uintptr_t>(codes_t) & 31u) == 0;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t w0[4], w1[4];
+    for (int q = 0; q < 2; ++q) {
+      uint32_t w0[8], w1[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = q * 16 + e * 4;
-        const float2 v0 = pair(r), v1 = pair(r + 1), v2 = pair(r + 2), v3 = pair(r + 3);
-        w0[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.x, inv0), __fmul_rn(v1.x, inv0))) |
-                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.x, inv0), __fmul_rn(v3.x, inv0))) << 16);
-        w1[e] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v0.y, inv1), __fmul_rn(v1.y, inv1))) |
-                (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(v2.y, inv1), __fmul_rn(v3.y, inv1))) << 16);
+      for (int e = 0; e < 8; ++e) {
+        const int r = rbeg + q * 32 + e * 4;
+        float2 f[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = __fmul2_rn(__bfloat1622float2(t2[(r + i) * kPitch2 + cp]), inv);
+        w0[e] = static_cast<uint32_t>(cvt_e4m3x2(f[0].x, f[1].x)) |
+                (static_cast<uint32_t>(cvt_e4m3x2(f[2].x, f[3].x)) << 16);
+        w1[e] = static_cast<uint32_t>(cvt_e4m3x2(f[0].y, f[1].y)) |
+                (static_cast<uint32_t>(cvt_e4m3x2(f[2].y, f[3].y)) << 16);
       }
-      *reinterpret_cast<uint4 *>(dst0 + q * 16) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-      *reinterpret_cast<uint4 *>(dst1 + q * 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+      store_codes32(dst0 + q * 32, w0, v8);
+      store_codes32(dst1 + q * 32, w1, v8);
     }
-    *reinterpret_cast<float2 *>(scales + static_cast<int64_t>(j) * cols + c0 + col) = make_float2(s0, s1);
+    if (rh == 0)
+      *reinterpret_cast<float2 *>(scales + static_cast<int64_t>(j) * cols + c0 + col) = make_float2(s0, s1);
   }
 }
 
@@ -413,19 +437,6 @@ constexpr int kDoutRowWarps = 4;
 constexpr int kDoutThreads = kDoutColThreads + 32 * kDoutRowWarps;
 constexpr int kDoutRowsPerStep = 8;                       // rows per row-warp step (lane & 7)
 constexpr int kDoutLaneCols = kDoutCols / 4;              // columns per row lane (lane >> 3)
-
-// 32 code bytes: one 256-bit store when dst is 32-byte aligned, else two
-// 128-bit stores (dst is always 16-byte aligned here).
-__device__ __forceinline__ void store_codes32(uint8_t *dst, const uint32_t (&w)[8], bool v8) {
-  if (v8) {
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
-                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-                 : "memory");
-  } else {
-    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  }
-}
 
 // column scale s_r[g, c0 + c] staged at c + 4 (c / 32): the four 32-column
 // groups start in different banks
@@ -562,10 +573,12 @@ cudaError_t launch_quant_dout_both(const void *x, int64_t rows, int64_t cols, co
 
 // Already-quantized E4M3 lhs (static rule): its codes laid out as the chunk
 // quantizer lays out the codes it makes (transposed, padded, zero pad rows),
-// bytes copied unchanged.  Same CTA shape as quant_chunks_kernel.
+// bytes copied unchanged.  64 threads per (128-column slice, chunk), one
+// column pair each.
 constexpr int kCodePitch = kChunkCols + 16;  // bytes per staged row (16-byte aligned rows)
+constexpr int kCodeThreads = kChunkPairs;     // one column pair per thread
 
-__global__ void __launch_bounds__(kChunkThreads) chunk_codes_kernel(const uint8_t *__restrict__ x, int64_t cols,
+__global__ void __launch_bounds__(kCodeThreads) chunk_codes_kernel(const uint8_t *__restrict__ x, int64_t cols,
                                                                     const int *__restrict__ offs,
                                                                     const int *__restrict__ tpre, int G,
                                                                     uint8_t *__restrict__ codes_t) {
@@ -577,7 +590,7 @@ __global__ void __launch_bounds__(kChunkThreads) chunk_codes_kernel(const uint8_
   __syncthreads();
   if (!s_info[0]) return;
   const int r0 = s_info[1], nr = s_info[2];
-  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 16); i += kChunkThreads) {
+  for (int i = threadIdx.x; i < kBlk * (kChunkCols / 16); i += kCodeThreads) {
     const int rr = i / (kChunkCols / 16), cc = (i % (kChunkCols / 16)) * 16;
     const bool in = rr < nr && c0 + cc < cols;
     const uint8_t *src = in ? x + static_cast<int64_t>(r0 + rr) * cols + c0 + cc : x;
@@ -609,7 +622,7 @@ cudaError_t launch_chunk_codes(const uint8_t *codes, int64_t rows, int64_t cols,
                                int G, int64_t capacity, uint8_t *codes_t, cudaStream_t st) {
   (void)rows;  // rows past the plan are never read
   dim3 grid(static_cast<unsigned>((cols + kChunkCols - 1) / kChunkCols), static_cast<unsigned>(capacity));
-  chunk_codes_kernel<<<grid, kChunkThreads, 0, st>>>(codes, cols, offs, tpre, G, codes_t);
+  chunk_codes_kernel<<<grid, kCodeThreads, 0, st>>>(codes, cols, offs, tpre, G, codes_t);
   return cudaGetLastError();
 }
 
