@@ -657,3 +657,30 @@ def test_output_16_byte_aligned_only(dev, out_dtype):
         fn(out)
         ref, ab = ref_fn()
         assert_close(out, ref, ab, f"16B-aligned {shape}")
+
+
+def test_workspace_16_byte_aligned_only(dev):
+    """A workspace that is 16- but not 32-byte aligned puts the quantizers'
+    code buffers (forward rows, tgmm chunks, the fused backward's dout) on
+    their 16-byte store path: every pass equals its aligned-workspace result
+    bit for bit."""
+    inp = case_inputs("ragged")
+    lhs, w, dout, gs, s = to_dev(inp, dev)
+    M, K = lhs.shape
+    G, _, N = w.shape
+    c, sc = gm.gmm_quantize_rhs(w)
+    nbytes = max(gm.gmm_workspace_bytes(op, M, K, N, G) for op in (0, 1, 2, 3))
+    raw = torch.zeros(nbytes + 64, dtype=torch.uint8, device=dev)
+    off = (16 - raw.data_ptr() % 32) % 32 or 16  # 16 mod 32
+    ws16 = raw[off: off + nbytes]
+    assert ws16.data_ptr() % 32 == 16
+    for rule in ("static", "dynamic"):
+        sarg = s if rule == "static" else None
+        assert torch.equal(gm.gmm_fwd(lhs, c, sc, gs, rule=rule, static_scale=sarg),
+                           gm.gmm_fwd(lhs, c, sc, gs, rule=rule, static_scale=sarg, ws=ws16))
+        assert torch.equal(gm.tgmm_drhs(lhs, dout, gs, rule=rule, static_scale=sarg),
+                           gm.tgmm_drhs(lhs, dout, gs, rule=rule, static_scale=sarg, ws=ws16))
+        dl_a, dw_a = gm.gmm_backward(lhs, dout, c, sc, gs, rule=rule, static_scale=sarg)
+        dl_b, dw_b = gm.gmm_backward(lhs, dout, c, sc, gs, rule=rule, static_scale=sarg, ws=ws16)
+        assert torch.equal(dl_a, dl_b)
+        assert torch.equal(dw_a, dw_b)
