@@ -560,9 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cp = 0; cp < 2; ++cp) {
             // chunks 2 cp, 2 cp + 1 (compile-time accumulator indices)
+            // colt(2 cp + 1) = colt(2 cp) + 32: one 64-column load
             uint32_t va[32], vb[32];
-            tmem_ld32(tl + buf * kBN + colt(2 * cp), va);
-            tmem_ld32(tl + buf * kBN + colt(2 * cp + 1), vb);
+            tmem_ld64(tl + buf * kBN + colt(2 * cp), va, vb);
             tmem_wait_ld();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
