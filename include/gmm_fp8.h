@@ -40,7 +40,9 @@
  *    code = E4M3 round-to-nearest-even of fl32(x * inv) saturated to +-448.
  *    A dynamic scale is fl32(amax / 448) over a block of 128 values along the
  *    contraction axis; a scale whose inverse overflows counts as 0.
- *  - Shapes: K and N multiples of 128, all sizes positive, G <= 1024.
+ *  - Shapes: K and N multiples of 128, all sizes positive, G <= 1024;
+ *    M <= 2^24 with ceil(M / 128) + G <= 65535, K and N <= 2^20 (larger
+ *    requests return GMM_ERR_UNSUPPORTED).
  */
 #ifndef GMM_FP8_H
 #define GMM_FP8_H

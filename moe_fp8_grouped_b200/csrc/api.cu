@@ -157,6 +157,8 @@ static gmm_status check_sizes(int64_t M, int64_t K, int64_t N, int32_t G) {
   // 32-bit tile coordinates and row indices
   if (M > (1 << 24) || K > (1 << 20) || N > (1 << 20) || static_cast<int64_t>(G) * (K > N ? K : N) > INT_MAX)
     return GMM_ERR_UNSUPPORTED;
+  // the chunk quantizers index chunks by gridDim.y: ceil(M / 128) + G chunks at most
+  if ((M + kBlk - 1) / kBlk + G > 65535) return GMM_ERR_UNSUPPORTED;
   return GMM_OK;
 }
 

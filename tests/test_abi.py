@@ -67,6 +67,8 @@ def test_host_errors(L):
     assert f(lhs, rhs, 0, gs, 8, 256, 500, 512, out, B.DT_BF16, ws, big, None) == 2  # K % 128
     assert f(lhs, rhs, 0, gs, 8, 256, 512, 200, out, B.DT_BF16, ws, big, None) == 2  # N % 128
     assert f(lhs, rhs, 0, gs, 2000, 256, 512, 512, out, B.DT_BF16, ws, big, None) == 5  # G > 1024
+    assert f(lhs, rhs, 0, gs, 8, 65528 * 128 + 1, 512, 512, out, B.DT_BF16, ws, big, None) == 5  # chunks > 65535
+    assert f(lhs, rhs, 0, gs, 8, 65527 * 128, 512, 512, out, B.DT_BF16, ws, 1024, None) == 9  # at the limit
     assert f(lhs, rhs, 0, None, 8, 256, 512, 512, out, B.DT_BF16, ws, big, None) == 1  # no group_sizes
     assert f(_op(FAKE, B.DT_BF16, None, B.Q_STATIC), rhs, 0, gs, 8, 256, 512, 512, out, B.DT_BF16, ws, big,
              None) == 1  # static rule without its scale
