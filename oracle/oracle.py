@@ -28,13 +28,30 @@ BLOCK = 128
 _lib = None
 
 
+_CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
 def build(force: bool = False) -> str:
     """Compile oracle.c into liboracle.so next to it; returns the path."""
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-               "-o", _LIB_PATH, _SRC, "-lm"]
-        subprocess.run(cmd, check=True)
+        subprocess.run(["gcc", *_CFLAGS, "-o", _LIB_PATH, _SRC, "-lm"], check=True)
     return _LIB_PATH
+
+
+def source_text() -> str:
+    """The C source of this oracle."""
+    with open(_SRC) as f:
+        return f.read()
+
+
+def build_variant(src_text: str, directory: str, name: str) -> str:
+    """Compile a variant of the C source (same flags) into directory/name.so."""
+    c_path = os.path.join(directory, name + ".c")
+    so_path = os.path.join(directory, name + ".so")
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", *_CFLAGS, "-o", so_path, c_path, "-lm"], check=True)
+    return so_path
 
 
 def _P(t):
@@ -44,40 +61,51 @@ def _P(t):
 def lib():
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build())
-        i32, i64, f32, u8, u16, f64 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_uint8,
-                                       ctypes.c_uint16, ctypes.c_double)
-        L.gmo_num_threads.restype = ctypes.c_int
-        L.gmo_e4m3_decode.argtypes = [u8]
-        L.gmo_e4m3_decode.restype = f64
-        L.gmo_e4m3_encode.argtypes = [f64]
-        L.gmo_e4m3_encode.restype = u8
-        L.gmo_static_scale_ok.argtypes = [f32]
-        L.gmo_static_scale_ok.restype = ctypes.c_int
-        L.gmo_plan.argtypes = [_P(i32), i32, i64, _P(i64), _P(i32)]
-        L.gmo_quantize_rows.argtypes = [_P(u16), i64, i64, i32, f32, _P(u8), _P(f32), _P(i32)]
-        L.gmo_quantize_rows_scaled.argtypes = [_P(u16), i64, i64, _P(f32), _P(i32), i32, _P(u8), _P(f32)]
-        L.gmo_quantize_rhs.argtypes = [_P(u16), i32, i64, i64, _P(u8), _P(f32)]
-        L.gmo_quantize_rhs_blocks.argtypes = [_P(u16), i32, i64, i64, i32, _P(u8), _P(f32)]
-        L.gmo_gmm_fwd_blockwise.argtypes = [_P(u16), i32, f32, _P(u8), _P(f32), _P(i32), i32, i64, i64, i64,
-                                            _P(i64), i64, _P(f64), _P(f64)]
-        L.gmo_gmm_dlhs_blockwise.argtypes = [_P(u16), _P(u8), _P(f32), _P(i32), i32, i64, i64, i64, _P(i64), i64,
-                                             _P(f64), _P(f64)]
-        L.gmo_num_chunks.argtypes = [_P(i32), i32, i64]
-        L.gmo_num_chunks.restype = i64
-        L.gmo_quantize_chunks.argtypes = [_P(u16), i64, i64, i32, f32, _P(i32), i32, _P(u8), _P(f32)]
-        L.gmo_gmm_fwd.argtypes = [_P(u16), i32, f32, _P(u8), _P(f32), _P(i32), i32, i64, i64, i64,
-                                  _P(i64), i64, _P(f64), _P(f64)]
-        L.gmo_gmm_dlhs.argtypes = [_P(u16), _P(u8), _P(f32), _P(i32), i32, i64, i64, i64, _P(i64), i64,
-                                   _P(f64), _P(f64)]
-        L.gmo_tgmm_drhs.argtypes = [_P(u16), i32, f32, _P(u16), _P(i32), i32, i64, i64, i64, _P(i64), i64,
-                                    _P(f64), _P(f64)]
-        L.gmo_gmm_fwd_bf16.argtypes = [_P(u16), _P(u16), _P(i32), i32, i64, i64, i64, _P(i64), i64,
-                                       _P(f64), _P(f64)]
-        L.gmo_gmm_dlhs_bf16.argtypes = L.gmo_gmm_fwd_bf16.argtypes
-        L.gmo_tgmm_drhs_bf16.argtypes = L.gmo_gmm_fwd_bf16.argtypes
-        _lib = L
+        _lib = _bind(ctypes.CDLL(build()))
     return _lib
+
+
+def load_variant(so_path: str):
+    """A separately compiled build of this oracle's C source (for example a
+    copy with a deliberate mistake, made by a test to show that the pins
+    reject it), with the same signatures bound.  Pass it as ``_L`` to the
+    wrappers that take one."""
+    return _bind(ctypes.CDLL(so_path))
+
+
+def _bind(L):
+    i32, i64, f32, u8, u16, f64 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_uint8,
+                                   ctypes.c_uint16, ctypes.c_double)
+    L.gmo_num_threads.restype = ctypes.c_int
+    L.gmo_e4m3_decode.argtypes = [u8]
+    L.gmo_e4m3_decode.restype = f64
+    L.gmo_e4m3_encode.argtypes = [f64]
+    L.gmo_e4m3_encode.restype = u8
+    L.gmo_static_scale_ok.argtypes = [f32]
+    L.gmo_static_scale_ok.restype = ctypes.c_int
+    L.gmo_plan.argtypes = [_P(i32), i32, i64, _P(i64), _P(i32)]
+    L.gmo_quantize_rows.argtypes = [_P(u16), i64, i64, i32, f32, _P(u8), _P(f32), _P(i32)]
+    L.gmo_quantize_rows_scaled.argtypes = [_P(u16), i64, i64, _P(f32), _P(i32), i32, _P(u8), _P(f32)]
+    L.gmo_quantize_rhs.argtypes = [_P(u16), i32, i64, i64, _P(u8), _P(f32)]
+    L.gmo_quantize_rhs_blocks.argtypes = [_P(u16), i32, i64, i64, i32, _P(u8), _P(f32)]
+    L.gmo_gmm_fwd_blockwise.argtypes = [_P(u16), i32, f32, _P(u8), _P(f32), _P(i32), i32, i64, i64, i64,
+                                        _P(i64), i64, _P(f64), _P(f64)]
+    L.gmo_gmm_dlhs_blockwise.argtypes = [_P(u16), _P(u8), _P(f32), _P(i32), i32, i64, i64, i64, _P(i64), i64,
+                                         _P(f64), _P(f64)]
+    L.gmo_num_chunks.argtypes = [_P(i32), i32, i64]
+    L.gmo_num_chunks.restype = i64
+    L.gmo_quantize_chunks.argtypes = [_P(u16), i64, i64, i32, f32, _P(i32), i32, _P(u8), _P(f32)]
+    L.gmo_gmm_fwd.argtypes = [_P(u16), i32, f32, _P(u8), _P(f32), _P(i32), i32, i64, i64, i64,
+                              _P(i64), i64, _P(f64), _P(f64)]
+    L.gmo_gmm_dlhs.argtypes = [_P(u16), _P(u8), _P(f32), _P(i32), i32, i64, i64, i64, _P(i64), i64,
+                               _P(f64), _P(f64)]
+    L.gmo_tgmm_drhs.argtypes = [_P(u16), i32, f32, _P(u16), _P(i32), i32, i64, i64, i64, _P(i64), i64,
+                                _P(f64), _P(f64)]
+    L.gmo_gmm_fwd_bf16.argtypes = [_P(u16), _P(u16), _P(i32), i32, i64, i64, i64, _P(i64), i64,
+                                   _P(f64), _P(f64)]
+    L.gmo_gmm_dlhs_bf16.argtypes = L.gmo_gmm_fwd_bf16.argtypes
+    L.gmo_tgmm_drhs_bf16.argtypes = L.gmo_gmm_fwd_bf16.argtypes
+    return L
 
 
 # ----------------------------------------------------------------- helpers
@@ -340,31 +368,36 @@ def gmm_fwd_swiglu(lhs, rule: int, static_scale: float, qr: np.ndarray, sr: np.n
     return silu(gate) * up, (gate, up, ab[:, :F], ab[:, F:])
 
 
-def gmm_fwd_bf16(lhs, w, group_sizes, rows=None):
+def gmm_fwd_bf16(lhs, w, group_sizes, rows=None, _L=None):
+    """bf16-family forward: out[m, :] = lhs[m, :] @ W[g(m)] with the bf16
+    operands widened exactly, fp64 sums -> (out, absum)."""
     lb, wb = _bf16_bits(lhs), _bf16_bits(w)
     M, K = lb.shape
     G, _, N = wb.shape
     gs, r = _sizes(group_sizes), _rows(rows, M)
     out = np.empty((r.size, N)); ab = np.empty((r.size, N))
-    lib().gmo_gmm_fwd_bf16(_ptr(lb, ctypes.c_uint16), _ptr(wb, ctypes.c_uint16), _ptr(gs, ctypes.c_int32), G,
+    (_L or lib()).gmo_gmm_fwd_bf16(_ptr(lb, ctypes.c_uint16), _ptr(wb, ctypes.c_uint16), _ptr(gs, ctypes.c_int32), G,
                            M, K, N, _ptr(r, ctypes.c_int64), r.size, _ptr(out, ctypes.c_double),
                            _ptr(ab, ctypes.c_double))
     return out, ab
 
 
-def gmm_dlhs_bf16(dout, w, group_sizes, rows=None):
+def gmm_dlhs_bf16(dout, w, group_sizes, rows=None, _L=None):
+    """bf16-family dlhs: dlhs[m, :] = dout[m, :] @ W[g(m)]^T -> (dlhs, absum)."""
     db, wb = _bf16_bits(dout), _bf16_bits(w)
     M, N = db.shape
     G, K, _ = wb.shape
     gs, r = _sizes(group_sizes), _rows(rows, M)
     out = np.empty((r.size, K)); ab = np.empty((r.size, K))
-    lib().gmo_gmm_dlhs_bf16(_ptr(db, ctypes.c_uint16), _ptr(wb, ctypes.c_uint16), _ptr(gs, ctypes.c_int32), G,
+    (_L or lib()).gmo_gmm_dlhs_bf16(_ptr(db, ctypes.c_uint16), _ptr(wb, ctypes.c_uint16), _ptr(gs, ctypes.c_int32), G,
                             M, K, N, _ptr(r, ctypes.c_int64), r.size, _ptr(out, ctypes.c_double),
                             _ptr(ab, ctypes.c_double))
     return out, ab
 
 
-def tgmm_drhs_bf16(x, dout, group_sizes, sel=None):
+def tgmm_drhs_bf16(x, dout, group_sizes, sel=None, _L=None):
+    """bf16-family tgmm: dW[g] = x[rows of g]^T @ dout[rows of g] on the
+    selected (g, k) rows (index g*K + k; all by default) -> (dW, absum)."""
     xb, db = _bf16_bits(x), _bf16_bits(dout)
     M, K = xb.shape
     _, N = db.shape
@@ -372,7 +405,7 @@ def tgmm_drhs_bf16(x, dout, group_sizes, sel=None):
     G = gs.size
     s = np.arange(G * K, dtype=np.int64) if sel is None else np.ascontiguousarray(np.asarray(sel, np.int64))
     out = np.empty((s.size, N)); ab = np.empty((s.size, N))
-    lib().gmo_tgmm_drhs_bf16(_ptr(xb, ctypes.c_uint16), _ptr(db, ctypes.c_uint16), _ptr(gs, ctypes.c_int32), G,
+    (_L or lib()).gmo_tgmm_drhs_bf16(_ptr(xb, ctypes.c_uint16), _ptr(db, ctypes.c_uint16), _ptr(gs, ctypes.c_int32), G,
                              M, K, N, _ptr(s, ctypes.c_int64), s.size, _ptr(out, ctypes.c_double),
                              _ptr(ab, ctypes.c_double))
     if sel is None:
