@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--separate-backward", action="store_true",
                     help="run dlhs and drhs as two calls (gmm_dlhs, tgmm_drhs) instead of gmm_backward, which "
                          "quantizes dout once for both")
+    ap.add_argument("--no-forward-shapes", dest="forward_shapes", action="store_false",
+                    help="skip the forward measurement on the DeepSeek-V3 and EP-shrunk shapes that the default "
+                         "(Mixtral, one GPU) run adds to its line")
     ap.add_argument("--rhs-blocks", action="store_true",
                     help="block-wise weight scales: forward codes with [G, K/128, N] scales, dlhs codes with "
                          "[G, N/128, K] scales (two weight copies, made outside the timed step)")
@@ -70,6 +73,19 @@ def load_peaks():
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def tensor_peak(peaks, src, region_s: float, bf16_family: bool):
+    """The tensor peak a kernel timed inside a region of region_s seconds is
+    held to: the burst cuBLAS bf16 figure for regions under 2 s (the clock has
+    not settled under the power cap yet), the sustained one for longer regions;
+    x2 (the nominal dense fp8 / bf16 ratio, 4.5 / 2.25 PFLOP/s) for fp8."""
+    sustained = region_s >= 2.0
+    v = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * (1.0 if bf16_family else FP8_OVER_BF16)
+    desc = (f"{src} bf16 {'sustained' if sustained else 'burst'} cuBLAS"
+            + ("" if bf16_family else f" x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)")
+            + f"; timed region {region_s:.2f} s")
+    return v, desc
 
 
 def max_over_ranks(ms: float, world: int, device=None) -> float:
@@ -101,6 +117,39 @@ def algorithmic_bytes(M, K, N, G, G_ne, rule):
             "drhs": 2 * M * K + 2 * M * N + 4 * G * K * N,
             # merged gate|up forward with SwiGLU fused: the [M, N/2] bf16 result only
             "fwd_swiglu": 2 * M * K + lsc + wb * G_ne * K * N + wsc + M * N}
+
+
+def needs_l2_flush(w):
+    """True when one step's operands (lhs, dout, weights) could stay in L2
+    (126 MB) from one step to the next."""
+    op_bytes = w.M * w.K * 2 + w.M * w.N * 2 + w.G * w.K * w.N * (2 if w.rule == "none" else 1)
+    return op_bytes < 4 * L2_BYTES
+
+
+def step_config(w, args, world):
+    """The config of one bench step for workload w under these arguments (the
+    same dict on both arms)."""
+    separate = w.name == "ep_separate"
+    parts = 2 if separate else 1
+    Np = w.N // parts
+    bf16_family = w.rule == "none"
+    fused_bwd = not args.separate_backward
+    keep_lhs = w.rule == "static" and not bf16_family
+    blocks = bool(args.rhs_blocks)
+    flush_l2 = needs_l2_flush(w)
+    return config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                         "calls_per_pass": parts,
+                         "backward": ("gmm_backward (dout quantized once for dlhs and drhs)" if fused_bwd
+                                      else "gmm_dlhs + tgmm_drhs"),
+                         "lhs_codes": ("gmm_fwd_keep_lhs hands the forward's E4M3 lhs codes to the tgmm"
+                                       if keep_lhs else "the tgmm quantizes lhs itself"),
+                         "rhs_scales": ("block-wise: fwd [G, K/128, N], dlhs [G, N/128, K]" if blocks
+                                        else "per channel [G, N]"),
+                         **({"l2": "flushed before every step (256 MiB write outside the timed events; "
+                                   "the operands would fit in L2 across steps)"} if flush_l2 else {}),
+                         **({"workload": f"ep_separate: G={w.G} M={w.M} K={w.K}, two N={Np} calls per pass "
+                                         f"(W0, W1 apart), lhs rule {w.rule}, fwd+dlhs+drhs"}
+                            if separate else {})})
 
 
 def config_of(w, extra=None):
@@ -202,11 +251,12 @@ def run_ours(args):
     # ep_separate: the EP-shrunk workload as two separate N=256 calls per pass
     # (W0 and W1 apart) instead of one merged N=512 call
     separate = args.workload == "ep_separate"
+    w_named = synth.WORKLOADS[args.workload]
     w = synth.WORKLOADS["ep_merged" if separate else args.workload]
     if args.m_override:
-        w = synth.with_rows(w, args.m_override)
+        w = w_named = synth.with_rows(w, args.m_override)
     if args.n_override:
-        w = synth.with_cols(w, args.n_override)
+        w = w_named = synth.with_cols(w, args.n_override)
     inp = synth.make_inputs(w, seed=rank, device=str(dev))
     gs = inp.group_sizes.to(dev)
     rows_routed = int(inp.group_sizes.sum())
@@ -290,9 +340,7 @@ def run_ours(args):
     launches[0] = 0
     # operands that could stay in L2 (126 MB) from one step to the next: flush
     # L2 between steps with a 256 MiB write outside the timed events
-    op_bytes = lhs.numel() * 2 + sum(d.numel() * 2 for d in douts) + sum(
-        c.numel() * c.element_size() for c, _ in wparts)
-    flush_l2 = op_bytes < 4 * L2_BYTES
+    flush_l2 = needs_l2_flush(w)
     barrier()
     if flush_l2:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -324,7 +372,7 @@ def run_ours(args):
     value = job_tflops(flops_step, world, args.steps, ms)
 
     peaks, peak_src = load_peaks()
-    peak_tc = peaks["bf16_tflops_sustained"] * (1.0 if bf16_family else FP8_OVER_BF16)
+    peak_tc, peak_tc_src = tensor_peak(peaks, peak_src, ms / 1e3, bf16_family)
     peak_bw = peaks["hbm_gbs"]
     bytes_pass = algorithmic_bytes(M, K, Np, G, G_ne, rule)
     passes = {}
@@ -349,8 +397,7 @@ def run_ours(args):
         achieved = flops_pass / (dt / dn / 1e3) / 1e12
         roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tc, 1),
                     "unit": "TFLOP/s", "frac": round(achieved / peak_tc, 4),
-                    "peak_source": f"{peak_src} bf16 sustained cuBLAS" +
-                                   ("" if bf16_family else f" x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)"),
+                    "peak_source": peak_tc_src,
                     "algorithmic": f"2*sum(group_sizes)*K*N = {flops_pass:.4g} FLOP per launch"}
     else:
         achieved = bytes_pass[dname] / (dt / dn / 1e3) / 1e9
@@ -533,6 +580,15 @@ def run_ours(args):
                        "gmm_fwd(_keep_lhs) + gmm_backward (dlhs, drhs); device -> pinned host copies of out, dlhs, dW. Steps "
                        "pipelined over upload / compute / download streams with two device buffer sets."}
 
+    # the forward on the HBM-bound shapes (DeepSeek-V3 up / down, EP-shrunk
+    # merged), measured in the same process on one GPU: the shapes whose
+    # forward throughput and HBM GB/s the metric asks for next to the step
+    fwd_shapes = None
+    if world == 1 and args.workload == "mixtral" and not args.m_override and not args.n_override \
+            and args.forward_shapes:
+        fwd_shapes = measure_forward_shapes(dev, ("dsv3_up", "dsv3_down", "ep_merged"), min(args.steps, 20), peaks,
+                                            peak_src)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_sample(w, args.cpu_seconds)
@@ -546,26 +602,93 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if bf16_family else "e4m3", "data": "synthetic",
-        "config": config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                                "calls_per_pass": parts,
-                                "backward": ("gmm_backward (dout quantized once for dlhs and drhs)" if fused_bwd
-                                             else "gmm_dlhs + tgmm_drhs"),
-                                "lhs_codes": ("gmm_fwd_keep_lhs hands the forward's E4M3 lhs codes to the tgmm"
-                                              if keep_lhs else "the tgmm quantizes lhs itself"),
-                                "rhs_scales": ("block-wise: fwd [G, K/128, N], dlhs [G, N/128, K]" if blocks
-                                               else "per channel [G, N]"),
-                                **({"l2": "flushed before every step (256 MiB write outside the timed events; "
-                                          "the operands would fit in L2 across steps)"} if flush_l2 else {}),
-                                **({"workload": f"ep_separate: G={G} M={M} K={K}, two N={Np} calls per pass "
-                                                f"(W0, W1 apart), lhs rule {rule}, fwd+dlhs+drhs"}
-                                   if separate else {})}),
+        "config": step_config(w_named, args, world),
         "pct_peak": {"vs_nominal": round(value / world / (2250.0 if bf16_family else 4500.0) * 100, 2),
-                     "vs_measured_sustained": round(value / world / peak_tc * 100, 2),
-                     "peak": "dense bf16" if bf16_family else "dense fp8"},
+                     "vs_measured": round(value / world / peak_tc * 100, 2),
+                     "peak": "dense bf16" if bf16_family else "dense fp8", "measured_peak": peak_tc_src},
+        **({"forward_shapes": fwd_shapes} if fwd_shapes else {}),
         "passes": passes, "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": timed_launches, "clocks": clk,
     }
     print(json.dumps(line))
+
+
+def measure_forward_shapes(dev, names, calls, peaks, peak_src):
+    """gmm_fwd on each named workload (weights quantized outside the timed
+    calls, a 256 MiB L2 flush before every call, outside its events): the whole
+    call (group plan, lhs quantization, GEMM) and the GEMM kernel alone, as
+    TFLOP/s, % of the nominal dense FP8 peak, algorithmic HBM GB/s and the
+    fraction of the roofline max(FLOP / tensor peak, bytes / HBM peak)."""
+    import torch
+
+    import moe_fp8_grouped_b200 as gm
+    from moe_fp8_grouped_b200 import synth
+
+    res = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for name in names:
+        w = synth.WORKLOADS[name]
+        inp = synth.make_inputs(w, seed=0, device=str(dev))
+        inp.dout = None
+        gs = inp.group_sizes.to(dev)
+        codes, rs = gm.gmm_quantize_rhs(inp.w)
+        inp.w = None
+        s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev) if w.rule == "static" else None
+        out = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(gm.gmm_workspace_bytes(0, w.M, w.K, w.N, w.G), dtype=torch.uint8, device=dev)
+
+        def call():
+            gm.gmm_fwd(inp.lhs, codes, rs, gs, rule=w.rule, static_scale=s, out=out, ws=ws)
+
+        for _ in range(3):
+            call()
+        st, bits = gm.gmm_read_device_status(ws)
+        if st != 0:
+            raise RuntimeError(f"{name}: device status {st} bits {bits}")
+        clk = ClockSampler(dev.index if dev.index is not None else 0)
+        clk.start()
+        time.sleep(0.3)
+        gm.profile_enable(True)
+        evs = []
+        for _ in range(calls):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        gm.profile_enable(False)
+        prof = gm.profile_collect()
+        clocks = clk.stop()
+        call_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+        n, tot = prof.get("gemm_fwd", (0, 0.0))
+        gemm_ms = tot / n if n else None
+        rows = int(inp.group_sizes.sum())
+        G_ne = int((inp.group_sizes > 0).sum())
+        flops = 2.0 * rows * w.K * w.N
+        nbytes = algorithmic_bytes(w.M, w.K, w.N, w.G, G_ne, w.rule)["fwd"]
+        peak_tc, tc_src = tensor_peak(peaks, peak_src, sum(a.elapsed_time(b) for a, b in evs) / 1e3, False)
+        floor_ms = max(flops / (peak_tc * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+
+        def figures(t_ms):
+            return {"ms": round(t_ms, 4), "tflops": round(flops / (t_ms / 1e3) / 1e12, 1),
+                    "pct_nominal_fp8": round(flops / (t_ms / 1e3) / 1e12 / 4500.0 * 100, 2),
+                    "gb_per_s": round(nbytes / (t_ms / 1e3) / 1e9, 1),
+                    "frac_roofline": round(floor_ms / t_ms, 4)}
+
+        res[name] = {"workload": f"{name}: G={w.G} M={w.M} K={w.K} N={w.N}, lhs rule {w.rule}, forward only",
+                     "call": figures(call_ms), "gemm": figures(gemm_ms) if gemm_ms else None,
+                     "bound": "hbm" if nbytes / (peaks["hbm_gbs"] * 1e9) > flops / (peak_tc * 1e12) else "tensor",
+                     "roofline_ms": round(floor_ms, 4), "algorithmic_bytes": nbytes, "flop": flops,
+                     "peak_tflops": round(peak_tc, 1), "peak_source": f"{tc_src}; HBM {peak_src} copy",
+                     "clocks_sm_mhz": clocks.get("sm_mhz") if clocks else None,
+                     "calls": calls, "l2": "flushed before every call (256 MiB write outside the events)"}
+        del inp, gs, codes, rs, out, ws, s
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------ CPU (oracle) side
@@ -648,7 +771,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, {"parallelism": "CPU oracle on rank 0"}),
+        "config": step_config(w, args, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
                          "sample": f"per step: {r['sample']}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

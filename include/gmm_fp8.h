@@ -216,26 +216,42 @@ gmm_status gmm_fwd_swiglu(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, c
 
 /*
  * Forward gmm without a workspace argument, for callers that cannot allocate
- * device memory: code that runs where cudaMalloc is not allowed (a host
- * function enqueued on a stream), or that runs under a runtime which owns all
- * device memory and forbids allocations after start-up (cudaMalloc would also
- * synchronize the device).  The pages have no counterpart; it is a
- * convenience of this library.
+ * device memory: code under a runtime or framework that owns all device
+ * memory (a caching allocator or a fixed memory plan that reserved it at
+ * start-up and forbids allocations afterwards), where a cudaMalloc would fail
+ * or break the plan, and latency-bound callers that cannot afford the device
+ * synchronization cudaMalloc and cudaFree imply.  The pages have no
+ * counterpart; it is a convenience of this library.
  * Arguments and results are gmm_fwd's, minus ws and ws_bytes.  The scratch
- * lives in one 32 MiB array of device memory inside the library, which every
- * device holds, once the library is used on it, until the process exits.  A
- * call whose gmm_workspace_bytes(GMM_OP_FWD, M, K, N, G) exceeds 32 MiB
- * returns GMM_ERR_WORKSPACE before anything runs.  Nothing is allocated.
- * The first call on a device looks up the array's device address; make that
- * first call before any stream capture.  All calls share the array, which
+ * lives in one 32 MiB array of device memory inside the library, which each
+ * CUDA context holds until it is destroyed or the process exits.  With lazy
+ * module loading (the CUDA default) the array is committed on the first call
+ * in a context; with eager loading, when the library loads.  A call whose
+ * gmm_workspace_bytes(GMM_OP_FWD, M, K, N, G) exceeds 32 MiB returns
+ * GMM_ERR_WORKSPACE before anything runs.  No cudaMalloc, cudaFree or other
+ * allocating routine is called.  The first call in a context (of this entry
+ * point or of gmm_fwd_noalloc_status) looks up the array's device address:
+ * make it at start-up, before any stream capture, so that the 32 MiB are
+ * committed while memory is still free.  All calls share the array, which
  * keeps the last call's contents (each call rewrites all it reads): calls
  * whose kernels overlap on the GPU (concurrent streams) race, so serialize
- * them.  Device-detected errors still clamp or zero as in gmm_fwd, but their
- * status word is not readable through this entry point.
+ * them.  Device-detected errors clamp or zero as in gmm_fwd; read them with
+ * gmm_fwd_noalloc_status.
  */
 gmm_status gmm_fwd_noalloc(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, const int32_t *group_sizes,
                            int32_t G, int64_t M, int64_t K, int64_t N, void *out, gmm_dtype out_dtype,
                            void *stream);
+
+/*
+ * Device status of the last gmm_fwd_noalloc call in the current context (the
+ * GMM_DEV_* bits of its scratch array's status word), as
+ * gmm_read_device_status does for a workspace: synchronizes `stream`, writes
+ * the bits to *bits_out (if not NULL) and returns GMM_ERR_TIMEOUT,
+ * GMM_ERR_SCALE or GMM_ERR_GROUP_SIZES when the matching bit is set, else
+ * GMM_OK.  Read it after the call whose status it should report and before
+ * the next one.  The pages have no counterpart.  Allocates nothing.
+ */
+gmm_status gmm_fwd_noalloc_status(uint32_t *bits_out, void *stream);
 
 /*
  * Backward gmm wrt lhs.  dout: bf16 [M, N], always quantized with DYNAMIC

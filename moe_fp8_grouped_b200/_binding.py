@@ -26,7 +26,8 @@ EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm
            "gmm_dlhs", "tgmm_drhs", "gmm_read_device_status", "gmm_selftest_timeout", "gmm_set_wait_limit_ns",
            "gmm_status_string", "gmm_last_launch_count", "gmm_profile_enable", "gmm_profile_collect",
            "gmm_fwd_noalloc", "gmm_fwd_swiglu", "gmm_quantize_rhs_blocks", "gmm_gather_rows",
-           "gmm_combine_rows", "gmm_backward", "gmm_gather_scale_rows", "gmm_fwd_keep_lhs"]
+           "gmm_combine_rows", "gmm_backward", "gmm_gather_scale_rows", "gmm_fwd_keep_lhs",
+           "gmm_fwd_noalloc_status"]
 
 
 class Operand(ctypes.Structure):
@@ -79,6 +80,8 @@ def lib():
     L.gmm_fwd_swiglu.restype = st
     L.gmm_fwd_noalloc.argtypes = [Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp]
     L.gmm_fwd_noalloc.restype = st
+    L.gmm_fwd_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
+    L.gmm_fwd_noalloc_status.restype = st
     L.gmm_dlhs.argtypes = L.gmm_fwd.argtypes
     L.gmm_dlhs.restype = st
     L.tgmm_drhs.argtypes = [Operand, Operand, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp, sz, vp]

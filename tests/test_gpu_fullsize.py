@@ -164,3 +164,70 @@ def test_fullsize_backward_equals_the_two_calls(name):
     assert torch.equal(dw, dw1)
     del inp, dw, dw1, ws, codes, scales
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["mixtral", "dsv3_up", "ragged"])
+def test_fullsize_activation_codes_bit_exact(name):
+    """Activation codes and scales at full size, bit for bit against the oracle:
+    the lhs along K (the forward's operand, the workload's rule), dout along N
+    with the weight column scale folded in (the dlhs operand), and both per
+    128-row chunk of each group (the tgmm operands).  Quantization is local to
+    a row (axis 1) or to a group's rows (axis 0), so sampled rows and sampled
+    groups are exact sub-problems; every group's first and last row is among
+    the sampled rows."""
+    dev = torch.device("cuda:0")
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w, seed=0, device="cuda")
+    gs_h = inp.group_sizes.numpy().astype(np.int64)
+    gs = inp.group_sizes.to(dev)
+    M = w.M
+    static = w.rule == "static"
+    qrule = oracle.Q_STATIC if static else oracle.Q_DYNAMIC
+    s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    sarg = s if static else None
+    offs = np.concatenate([[0], np.cumsum(gs_h)])
+    rng = np.random.default_rng(2)
+    nz = np.flatnonzero(gs_h > 0)
+    rows = sorted(set(offs[nz].tolist()) | set((offs[nz + 1] - 1).tolist())
+                  | set(rng.integers(0, M, 256).tolist()))
+
+    # axis 1: lhs rows (the forward's operand)
+    codes, scales = gm.gmm_quantize(inp.lhs, w.rule, axis=1, static_scale=sarg)
+    qc, qs, _ = oracle.quantize_rows(inp.lhs[rows].cpu(), qrule, inp.static_scale)
+    assert np.array_equal(codes[rows].cpu().numpy(), qc), f"{name}: lhs row codes"
+    if not static:
+        assert np.array_equal(scales[:, rows].cpu().numpy().T, qs), f"{name}: lhs row scales"
+    del codes, scales
+
+    # axis 1 with the weight column scale folded in: dout rows (the dlhs operand)
+    _, wscales = gm.gmm_quantize_rhs(inp.w)
+    inp.w = None
+    codes, scales = gm.gmm_quantize(inp.dout, "dynamic", axis=1, group_sizes=gs, col_scale=wscales)
+    sr = wscales.cpu().numpy()
+    for g in pick_groups(gs_h, rng):
+        a, b = int(offs[g]), int(offs[g + 1])
+        rg = [r for r in rows if a <= r < b]
+        qc, qs = oracle.quantize_rows_scaled(inp.dout[rg].cpu(), sr[g:g + 1], np.array([len(rg)], np.int32))
+        assert np.array_equal(codes[rg].cpu().numpy(), qc), f"{name}: dout row codes, group {g}"
+        assert np.array_equal(scales[:, rg].cpu().numpy().T, qs), f"{name}: dout row scales, group {g}"
+    del codes, scales
+
+    # axis 0: 128-row chunks of each group (the tgmm operands)
+    first_chunk = np.concatenate([[0], np.cumsum((gs_h + 127) // 128)])
+    for x, rule_x, what in ((inp.lhs, w.rule, "lhs"), (inp.dout, "dynamic", "dout")):
+        ct, cs = gm.gmm_quantize(x, rule_x, axis=0, static_scale=sarg if rule_x == "static" else None,
+                                 group_sizes=gs)
+        for g in pick_groups(gs_h, rng):
+            a, b = int(offs[g]), int(offs[g + 1])
+            qc, qs = oracle.quantize_chunks(x[a:b].cpu(), oracle.Q_STATIC if rule_x == "static" else oracle.Q_DYNAMIC,
+                                            inp.static_scale, np.array([b - a], np.int32))
+            j0 = int(first_chunk[g])
+            for c in range((b - a + 127) // 128):
+                n = min(128, b - a - 128 * c)
+                got = ct[j0 + c, :, :n].cpu().numpy().T
+                assert np.array_equal(got, qc[128 * c:128 * c + n]), f"{name}: {what} chunk {c} of group {g}"
+                assert not ct[j0 + c, :, n:].any(), f"{name}: {what} chunk padding of group {g}"
+            assert np.array_equal(cs[j0:j0 + len(qs)].cpu().numpy(), qs), f"{name}: {what} chunk scales, group {g}"
+        del ct, cs
+    del inp
+    torch.cuda.empty_cache()

@@ -161,3 +161,38 @@ def test_plan_clamps_and_flags():
     assert list(offs) == [0, 8, 12, 12] and flags == oracle.FLAG_GROUP_SIZES
     offs, flags = oracle.plan([0, 0], 5)
     assert list(offs) == [0, 0, 0] and flags == 0
+
+
+def _codes_division_vs_reciprocal(s: np.float32):
+    """Over every finite bf16 value x: the number of inputs whose code differs
+    between e4m3(fl32(x / s)) (the LhsRef docstring's clip(lhs / scale)) and
+    e4m3(fl32(x * fl32(1 / s))) (the inner_kernel form this oracle follows),
+    and the number whose fp32 intermediates differ."""
+    bits = np.arange(65536, dtype=np.uint32)
+    x = (bits << 16).view(np.float32)
+    x = x[np.isfinite(x)]
+    inv = np.float32(1.0) / s
+    with np.errstate(over="ignore"):
+        q = (x / s).astype(np.float32)
+        p = (x * inv).astype(np.float32)
+    d = q != p
+    if not d.any():
+        return 0, 0
+    cq = oracle.e4m3_encode(q[d].astype(np.float64))
+    cp = oracle.e4m3_encode(p[d].astype(np.float64))
+    return int((cq != cp).sum()), int(d.sum())
+
+
+def test_static_rule_division_and_reciprocal_give_the_same_codes():
+    """Reading of the static rule ("add static LHS scaling support for GMM v2
+    FWD", maxtext PR #4735): the LhsRef docstring writes clip(lhs / scale), the
+    inner_kernel code multiplies by the inverse scale.  For the static scale of
+    every static workload (4/448), exhaustively over all bf16 inputs, the two
+    forms give the same E4M3 code although their fp32 intermediates differ on
+    about a third of the inputs; the same holds for 40 log-uniform scales in
+    [1e-4, 1].  So the choice changes no code on these inputs."""
+    diff, fp32_diff = _codes_division_vs_reciprocal(np.float32(4.0) / np.float32(448.0))
+    assert diff == 0 and fp32_diff > 20000
+    rng = np.random.default_rng(0)
+    for s in np.exp(rng.uniform(np.log(1e-4), 0.0, 40)).astype(np.float32):
+        assert _codes_division_vs_reciprocal(s)[0] == 0, s
