@@ -337,6 +337,24 @@ gmm_status gmm_gather_scale_rows(const void *src_bf16, const int32_t *idx, const
                                  int64_t ncols, int64_t src_rows, void *dst_bf16, void *stream);
 
 /*
+ * gmm_ep_local_order: regrouping of the rows an expert-parallel all-to-all
+ * delivers.  recv_counts: device int64 [P, El], the rows each source rank p
+ * sent for each local expert e; they arrive in source order, then expert
+ * order within a source ("FP8 Megablox for batch split", maxtext PR #3770,
+ * Description item 3: a rank's experts as a group_offset slice of the ragged
+ * dot).  Writes, on the device, perm [total] (perm[j] = arrival index of the
+ * j-th row once grouped by local expert, then by source rank), inv [total]
+ * (its inverse: the grouped position of each arrival row) and group_sizes
+ * [El] (rows per local expert).  total = sum of recv_counts, known on the
+ * host (it is the receive size the exchange needed).  No host
+ * synchronization.  P * El > 1024 or total > INT32_MAX returns
+ * GMM_ERR_UNSUPPORTED; counts that do not sum to total leave the rows they
+ * would misplace unwritten.
+ */
+gmm_status gmm_ep_local_order(const int64_t *recv_counts, int32_t P, int32_t El, int64_t total, int32_t *perm,
+                              int32_t *inv, int32_t *group_sizes, void *stream);
+
+/*
  * gmm_combine_rows: the weighted sum that returns expert outputs to their
  * tokens (the unpermute of the MoE combine):
  *   y[t, :] = sum_{j < k} weight[t, j] * rows[slot[t, j], :]
@@ -368,6 +386,23 @@ gmm_status gmm_selftest_timeout(void *ws, uint64_t limit_ns, void *stream);
 
 /* Time limit of every pipeline wait in the kernels (default 4e9 ns). */
 void gmm_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * GEMM tile choice for the calls that follow (process-wide; a tuning and
+ * testing knob, results are the same up to fp32 summation order, which does
+ * not change either: both tiles accumulate each output in the same order).
+ *   GMM_TILES_AUTO       (default) 256-row tiles over a pair of CTAs (a
+ *                        two-CTA cluster sharing each M = 256 tensor-core
+ *                        MMA) when the groups average at least 512 rows,
+ *                        else 128-row tiles on one CTA;
+ *   GMM_TILES_ONE_CTA    always 128-row tiles on one CTA;
+ *   GMM_TILES_CTA_PAIRS  always CTA pairs (the tgmm keeps one-CTA tiles when
+ *                        N is not a multiple of 256).
+ * Any other value returns GMM_ERR_INVALID_ARG.  Not part of the pages: how a
+ * tile maps onto the B200's SMs is this library's choice.
+ */
+enum { GMM_TILES_AUTO = 0, GMM_TILES_ONE_CTA = 1, GMM_TILES_CTA_PAIRS = 2 };
+gmm_status gmm_set_tiles(int32_t mode);
 
 /* Static text for a status code. */
 const char *gmm_status_string(gmm_status s);

@@ -9,6 +9,6 @@ there is no CPU fallback.
 from .ops import (  # noqa: F401
     DType, GmmError, QRule, gmm_backward, gmm_chunk_capacity, gmm_dlhs, gmm_fwd, gmm_fwd_keep_lhs, gmm_fwd_swiglu,
     gmm_plan, gmm_quantize, gmm_quantize_rhs, gmm_quantize_rhs_blocks, gmm_read_device_status, gmm_selftest_timeout,
-    gmm_set_wait_limit_ns, gmm_status_string, gmm_workspace_bytes, last_launch_count, profile_collect,
+    gmm_set_tiles, gmm_set_wait_limit_ns, gmm_status_string, gmm_workspace_bytes, last_launch_count, profile_collect,
     profile_enable, tgmm_drhs, workspace,
 )

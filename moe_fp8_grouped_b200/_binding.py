@@ -20,6 +20,7 @@ Q_NONE, Q_STATIC, Q_DYNAMIC = 0, 1, 2
 DT_BF16, DT_F32, DT_E4M3 = 0, 1, 2
 OP_FWD, OP_DLHS, OP_DRHS, OP_BWD = 0, 1, 2, 3
 DEV_GROUP_SIZES, DEV_SCALE, DEV_TIMEOUT = 1, 2, 4
+TILES_AUTO, TILES_ONE_CTA, TILES_CTA_PAIRS = 0, 1, 2
 
 # every symbol include/gmm_fp8.h declares
 EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm_quantize", "gmm_fwd",
@@ -27,7 +28,7 @@ EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm
            "gmm_status_string", "gmm_last_launch_count", "gmm_profile_enable", "gmm_profile_collect",
            "gmm_fwd_noalloc", "gmm_fwd_swiglu", "gmm_quantize_rhs_blocks", "gmm_gather_rows",
            "gmm_combine_rows", "gmm_backward", "gmm_gather_scale_rows", "gmm_fwd_keep_lhs",
-           "gmm_fwd_noalloc_status"]
+           "gmm_fwd_noalloc_status", "gmm_set_tiles", "gmm_ep_local_order"]
 
 
 class Operand(ctypes.Structure):
@@ -77,6 +78,8 @@ def lib():
     L.gmm_gather_rows.restype = st
     L.gmm_combine_rows.argtypes = [vp, i64, vp, vp, i64, i32, i64, vp, ctypes.c_int, vp]
     L.gmm_combine_rows.restype = st
+    L.gmm_ep_local_order.argtypes = [vp, i32, i32, i64, vp, vp, vp, vp]
+    L.gmm_ep_local_order.restype = st
     L.gmm_fwd_swiglu.restype = st
     L.gmm_fwd_noalloc.argtypes = [Operand, Operand, ctypes.c_int, vp, i32, i64, i64, i64, vp, ctypes.c_int, vp]
     L.gmm_fwd_noalloc.restype = st
@@ -92,6 +95,8 @@ def lib():
     L.gmm_selftest_timeout.restype = st
     L.gmm_set_wait_limit_ns.argtypes = [u64]
     L.gmm_set_wait_limit_ns.restype = None
+    L.gmm_set_tiles.argtypes = [i32]
+    L.gmm_set_tiles.restype = st
     L.gmm_status_string.argtypes = [ctypes.c_int]
     L.gmm_status_string.restype = ctypes.c_char_p
     L.gmm_last_launch_count.argtypes = []

@@ -13,6 +13,19 @@
 namespace gmm {
 
 static uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+static int g_cta_pairs = GMM_TILES_AUTO;
+static constexpr bool kAutoPairs = false;  // the automatic choice takes one-CTA tiles
+
+// 256-row tiles over a CTA pair for the row passes when the groups average at
+// least two such tiles (a group's last pair tile is half empty when its
+// 128-row tile count is odd); for the tgmm when its rows do too and its dout
+// columns split into 256-wide pair tiles.
+static bool use_pairs(bool tgmm, int64_t M, int64_t N, int32_t G) {
+  if (g_cta_pairs == GMM_TILES_ONE_CTA) return false;
+  if (tgmm && N % 256) return false;
+  if (g_cta_pairs == GMM_TILES_CTA_PAIRS) return true;
+  return kAutoPairs && M >= 512 * static_cast<int64_t>(G);
+}
 static thread_local int32_t g_launches = 0;
 
 // ------------------------------------------------------------ profiling
@@ -164,6 +177,15 @@ static gmm_status check_sizes(int64_t M, int64_t K, int64_t N, int32_t G) {
 
 static gmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA; }
 
+// Launch size of a row pass (forward, dlhs) over `cols` output columns: one CTA
+// per SM at most; for pairs the number of pair items (the launch caps it)
+static int row_pass_grid(bool pairs, int64_t M, int64_t cols, int32_t G) {
+  const int64_t rows = pairs ? 256 : 128;
+  const int64_t items = ((M + rows - 1) / rows + G) * ((cols + 255) / 256);
+  if (pairs) return static_cast<int>(items < INT_MAX ? items : INT_MAX);
+  return static_cast<int>(items < num_sms() ? items : num_sms());
+}
+
 struct WsPtrs {
   uint32_t *status;
   int *offs, *tpre;
@@ -248,6 +270,12 @@ const char *gmm_status_string(gmm_status s) {
 int32_t gmm_last_launch_count(void) { return g_launches; }
 
 void gmm_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns = limit_ns ? limit_ns : kDefaultWaitLimitNs; }
+
+gmm_status gmm_set_tiles(int32_t mode) {
+  if (mode != GMM_TILES_AUTO && mode != GMM_TILES_ONE_CTA && mode != GMM_TILES_CTA_PAIRS) return GMM_ERR_INVALID_ARG;
+  g_cta_pairs = mode;
+  return GMM_OK;
+}
 
 gmm_status gmm_quantize_rhs(const void *w_bf16, int32_t G, int64_t K, int64_t N, int transpose_out,
                             uint8_t *codes, float *scales, void *stream) {
@@ -370,8 +398,10 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   if (!make_map(&tmA, A, elem, K, M, K * elem, bke, 128)) return GMM_ERR_CUDA;
   // SwiGLU tiles take the gate rows and the up rows of a K-major rhs as two
   // 128-row boxes
+  const bool pairs = use_pairs(false, M, N, G);
   const bool okB = bmn ? make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, bke)
-                       : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, F ? 128 : 256);
+                       : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke,
+                                  (F || pairs) ? 128 : 256);
   if (!okB) return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
@@ -394,9 +424,8 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
   // per-block promotion for dynamic lhs scales or block-wise rhs scales
-  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk)};
-  const int64_t items = ((M + 127) / 128 + G) * ((N + 255) / 256);
-  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk), pairs};
+  const int grid = row_pass_grid(pairs, M, N, G);
   if ((s = cuda_status(prof(F ? "gemm_fwd_swiglu" : "gemm_fwd", st,
                             [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
     return s;
@@ -442,10 +471,12 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
                                 int64_t N, void *dlhs, gmm_dtype out_dtype, cudaStream_t st) {
   const bool bmn = transpose_rhs != 0;  // [G, N, K]: K contiguous = MN-major B for dlhs
   const uint32_t bke = 128 / elem;
+  const bool pairs = use_pairs(false, M, K, G);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, A, elem, N, M, N * elem, bke, 128)) return GMM_ERR_CUDA;
   const bool okB = bmn ? make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, bke)
-                       : make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, 256);
+                       : make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke,
+                                  pairs ? 128 : 256);
   if (!okB) return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
@@ -466,9 +497,8 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
   p.ld_out = K;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1};
-  const int64_t items = ((M + 127) / 128 + G) * ((K + 255) / 256);
-  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1, pairs};
+  const int grid = row_pass_grid(pairs, M, K, G);
   return cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }));
 }
 
@@ -482,10 +512,11 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   // k (B = lhs^T chunks); the epilogue writes dW[g, k, n].  The chunk-major
   // operands [chunk][column][128] are 2-D tensors of 128-element lines: chunk
   // j's line of column c is row j * C + c, so every box is one contiguous block.
+  const bool pairs = use_pairs(true, M, N, G);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, P.codes_b, elem, kBlk, static_cast<uint64_t>(cap) * N, kBlk * elem, bke, 128))
     return GMM_ERR_CUDA;
-  if (!make_map(&tmB, P.codes_a, elem, kBlk, static_cast<uint64_t>(cap) * K, kBlk * elem, bke, 256))
+  if (!make_map(&tmB, P.codes_a, elem, kBlk, static_cast<uint64_t>(cap) * K, kBlk * elem, bke, pairs ? 128 : 256))
     return GMM_ERR_CUDA;
   CUtensorMap tmOut;  // dW as [G*K, N]: each epilogue warp stores 32 k-rows x 32 n
   if (!make_out_map(&tmOut, drhs, out_dtype == GMM_F32, N, static_cast<uint64_t>(G) * K, 32, 32))
@@ -510,9 +541,10 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   p.ld_out = N;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{MODE_TGMM, elem, false, elem == 1};
-  const int64_t items = static_cast<int64_t>(G) * (N / kBlk) * ((K + 255) / 256);
-  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  const GemmConfig cfg{MODE_TGMM, elem, false, elem == 1, pairs};
+  const int64_t items = static_cast<int64_t>(G) * (N / (pairs ? 2 * kBlk : kBlk)) * ((K + 255) / 256);
+  const int grid = pairs ? static_cast<int>(items < INT_MAX ? items : INT_MAX)
+                         : static_cast<int>(items < num_sms() ? items : num_sms());
   return cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, p, grid, st); }));
 }
 

@@ -11,6 +11,8 @@
 // issued by the caller between these kernels.
 #include <cuda_bf16.h>
 
+#include <climits>
+
 #include "internal.h"
 
 namespace gmm {
@@ -97,6 +99,74 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(const __nv_bfloat16 *
   }
 }
 
+// Regrouping of the rows that arrive from an all-to-all: they come in source
+// rank order, then expert order within each source (block (p, e) holds
+// cnt[p * El + e] rows); the gmm wants them grouped by local expert, then by
+// source rank.  For arrival row i of block (p, e):
+//   pos = D[e, p] + (i - A[p, e]),  perm[pos] = i,  inv[i] = pos,
+// A the arrival offsets (prefix over (p, e) order), D the grouped offsets
+// (prefix over (e, p) order).  Every CTA builds A and D in shared memory
+// (warp 0 scans A, warp 1 scans D), then its threads take one arrival row
+// each.  CTA 0 also writes gsz[e] = sum_p cnt[p * El + e].  A row whose pos
+// falls outside [0, total) (counts that do not sum to total) is skipped.
+constexpr int kMaxEpBlocks = 1024;  // P * El
+
+__device__ __forceinline__ void warp_scan_blocks(const int64_t *cnt, int n, int P, int El, bool by_expert, int *out,
+                                                 int lane) {
+  // entry j of the scan order: (p, e) = (j / El, j % El) for arrival order,
+  // (j % P, j / P) for grouped order; out[p * El + e] = exclusive prefix
+  const int per = (n + 31) / 32;
+  const int j0 = min(lane * per, n), j1 = min(j0 + per, n);
+  auto cnt_at = [&](int j) -> int {
+    const int p = by_expert ? j % P : j / El, e = by_expert ? j / P : j % El;
+    return static_cast<int>(cnt[p * El + e]);
+  };
+  int sum = 0;
+  for (int j = j0; j < j1; ++j) sum += cnt_at(j);
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  int run = incl - sum;
+  for (int j = j0; j < j1; ++j) {
+    const int p = by_expert ? j % P : j / El, e = by_expert ? j / P : j % El;
+    out[p * El + e] = run;
+    run += cnt_at(j);
+  }
+}
+
+__global__ void __launch_bounds__(256) ep_local_order_kernel(const int64_t *__restrict__ cnt, int P, int El,
+                                                             int total, int32_t *__restrict__ perm,
+                                                             int32_t *__restrict__ inv, int32_t *__restrict__ gsz) {
+  __shared__ int sA[kMaxEpBlocks], sD[kMaxEpBlocks];
+  const int n = P * El;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) warp_scan_blocks(cnt, n, P, El, false, sA, lane);
+  if (warp == 1) warp_scan_blocks(cnt, n, P, El, true, sD, lane);
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e < El; e += blockDim.x) {
+      int64_t t = 0;
+      for (int p = 0; p < P; ++p) t += cnt[p * El + e];
+      gsz[e] = static_cast<int32_t>(t);
+    }
+  __syncthreads();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    // the last block b with A[b] <= i (A is non-decreasing; that block is non-empty)
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sA[mid] <= i) lo = mid;
+      else hi = mid - 1;
+    }
+    const int pos = sD[lo] + (i - sA[lo]);
+    if (pos < 0 || pos >= total) continue;
+    perm[pos] = i;
+    inv[i] = pos;
+  }
+}
+
 static unsigned grid_for(int64_t n) {
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   return static_cast<unsigned>(n < cap ? (n > 0 ? n : 1) : cap);
@@ -132,6 +202,18 @@ gmm_status gmm_gather_scale_rows(const void *src_bf16, const int32_t *idx, const
   gather_scale_rows_kernel<<<grid_for(nrows), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(src_bf16), idx, scale,
                                                             nrows, ncols / 8, src_rows,
                                                             static_cast<__nv_bfloat16 *>(dst_bf16));
+  return cudaGetLastError() == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
+}
+
+gmm_status gmm_ep_local_order(const int64_t *recv_counts, int32_t P, int32_t El, int64_t total, int32_t *perm,
+                              int32_t *inv, int32_t *group_sizes, void *stream) {
+  if (P <= 0 || El <= 0 || total < 0) return GMM_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(P) * El > kMaxEpBlocks || total > INT32_MAX) return GMM_ERR_UNSUPPORTED;
+  if (!recv_counts || !group_sizes || (total > 0 && (!perm || !inv))) return GMM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t blocks = (total + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(blocks < 1 ? 1 : (blocks < num_sms() * 4 ? blocks : num_sms() * 4));
+  ep_local_order_kernel<<<grid, 256, 0, st>>>(recv_counts, P, El, static_cast<int>(total), perm, inv, group_sizes);
   return cudaGetLastError() == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
 }
 

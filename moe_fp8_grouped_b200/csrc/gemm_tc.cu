@@ -57,7 +57,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 256;
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 8;    // ring of per-unit scale slots (scale loader -> epilogue)
-constexpr int kNumBars = 32;      // mbarriers reserved in shared memory
+constexpr int kNumBars = 40;      // mbarriers reserved in shared memory
 // Register split (setmaxnreg): the control warpgroup gives registers to the
 // two epilogue warpgroups.  Sum must not exceed the launch allocation
 // (registers per thread at launch x 384); launch_inst checks it.
@@ -68,26 +68,34 @@ constexpr int regs_ctl() { return kPromote ? 40 : 72; }
 template <bool kPromote>
 constexpr int regs_epi() { return kPromote ? 232 : 216; }
 
-// tgmm keeps 3 pipeline stages and uses the freed shared memory to stage its
-// output for TMA stores (one 4 KB block per epilogue warp)
-template <int kMode>
-constexpr int stages_of() { return kMode == MODE_TGMM ? 3 : kStages; }
+// Pipeline stages.  One CTA: A 16 KB + B 32 KB per stage, 4 stages (tgmm: 3,
+// the freed shared memory stages its output for TMA stores, one 4 KB block
+// per epilogue warp).  A CTA pair (kCta = 2): each CTA holds its 128 rows of A
+// and half of B (16 KB + 16 KB), 6 stages (tgmm: 4).
+template <int kCta, int kMode>
+constexpr int stages_of() {
+  return kCta == 2 ? (kMode == MODE_TGMM ? 4 : 6) : (kMode == MODE_TGMM ? 3 : kStages);
+}
 constexpr int kStageOut = 4096;  // bytes of one output staging buffer (tgmm); two per epilogue warp
 
 // scale ring slots: tgmm keeps 4 to make room for its output staging
 template <int kMode>
 constexpr int ring_of() { return kMode == MODE_TGMM ? 4 : kScaleSlots; }
 
-template <int kMode>
+template <int kCta, int kMode>
 constexpr size_t gemm_smem_bytes() {
   return 1024                                    // alignment slack
-         + static_cast<size_t>(stages_of<kMode>()) * (kAStage + kBStage)
+         + static_cast<size_t>(stages_of<kCta, kMode>()) * (kAStage + kBStage / kCta)
          + kNumBars * 8                          // mbarriers
          + 16                                    // tmem slot, abort flags
          + ring_of<kMode>() * (kBN + kBM) * sizeof(float)  // scale ring
-         + 2 * (kMaxGroups + 1) * sizeof(int)    // plan copy
+         + (kCta == 2 ? 3 : 2) * (kMaxGroups + 1) * sizeof(int)  // plan copy (+ pair-tile prefix)
          + (kMode == MODE_TGMM ? 128 + kEpiWarps * 2 * kStageOut : 0);  // + alignment slack
 }
+static_assert(gemm_smem_bytes<2, MODE_ROWS>() <= 232448, "pair-tile shared memory");
+static_assert(gemm_smem_bytes<2, MODE_TGMM>() <= 232448, "pair-tile tgmm shared memory");
+static_assert(gemm_smem_bytes<1, MODE_ROWS>() <= 232448, "shared memory");
+static_assert(gemm_smem_bytes<1, MODE_TGMM>() <= 232448, "tgmm shared memory");
 
 // One work item: tile row index rt (MODE_ROWS: rows r0 .. rend of group g;
 // MODE_TGMM: dout columns 128 rt ..), tile column index ct, and the number of
@@ -106,35 +114,39 @@ __device__ __forceinline__ int tile_col_n(int ct, int c, int F) {
 // x * sigmoid(x); -0 for large negative x, where exp(-x) overflows
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 
-template <int kMode>
+// A CTA pair (kCta = 2) takes one item of twice the rows: rank r of the pair
+// holds tile rows 128 r .. 128 r + 127 of it.
+template <int kMode, int kCta>
 __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const int *s_offs, const int *s_tpre,
-                                            int tn) {
+                                            const int *s_ppre, int tn, int rank) {
   Item t;
   if constexpr (kMode != MODE_TGMM) {
-    // items of group g: (tpre[g+1] - tpre[g]) row tiles x tn column tiles,
-    // row tiles fastest
-    int lo = 0, hi = p.G + 1;  // first i with tpre[i] * tn > w
+    // items of group g: (pre[g+1] - pre[g]) row tiles (128 rows, or 256 for a
+    // pair) x tn column tiles, row tiles fastest
+    const int *pre = kCta == 2 ? s_ppre : s_tpre;
+    int lo = 0, hi = p.G + 1;  // first i with pre[i] * tn > w
     while (lo < hi) {
       int mid = (lo + hi) >> 1;
-      if (s_tpre[mid] * tn > w) hi = mid;
+      if (pre[mid] * tn > w) hi = mid;
       else lo = mid + 1;
     }
     const int g = lo - 1;
-    const int mt_g = s_tpre[g + 1] - s_tpre[g];
-    const int local = w - s_tpre[g] * tn;
+    const int mt_g = pre[g + 1] - pre[g];
+    const int local = w - pre[g] * tn;
     t.g = g;
     t.rt = local % mt_g;
     t.ct = local / mt_g;
-    t.r0 = s_offs[g] + kBM * t.rt;
-    t.rend = min(s_offs[g + 1], t.r0 + kBM);
+    t.r0 = s_offs[g] + kCta * kBM * t.rt + kBM * rank;
+    t.rend = min(s_offs[g + 1], t.r0 + kBM);  // at or before r0: the pair's second half is past the group
     t.nblocks = p.kblocks;
   } else {
-    // items of group g: rtiles row tiles x tn column tiles, column tiles
-    // fastest (the group's lhs chunks stay in L2 across the row tiles)
-    const int per_g = p.rtiles * tn;
+    // items of group g: rtiles / kCta row tiles x tn column tiles, column
+    // tiles fastest (the group's lhs chunks stay in L2 across the row tiles);
+    // pairs need an even rtiles
+    const int per_g = (p.rtiles / kCta) * tn;
     const int g = w / per_g, local = w % per_g;
     t.g = g;
-    t.rt = local / tn;
+    t.rt = (local / tn) * kCta + rank;
     t.ct = local % tn;
     t.r0 = 0;
     t.rend = 0;
@@ -205,25 +217,34 @@ __device__ __forceinline__ void store_col32(void *out, int64_t off_elems, int64_
   }
 }
 
-template <int kElem, bool kBMN, bool kPromote, int kMode>
+// kCta = 2: the kernel runs as clusters of two CTAs (a pair) that share each
+// M = 256 MMA (tcgen05 cta_group::2): rank r holds rows 128 r .. of every
+// item's A tile and columns 128 r .. 128 r + 127 of its B tile, and receives
+// its 128 rows of the accumulator.  Rank 0 issues the MMAs.  Halving B per SM
+// halves the shared-memory traffic per MMA (TMA writes plus tensor-core
+// reads), which bounds the one-CTA tile.
+template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta>
 __global__ void __launch_bounds__(kThreads, 1)
     gmm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   constexpr bool kF16 = (kElem == 2);
   constexpr bool kTg = (kMode == MODE_TGMM);
+  constexpr bool kPair = (kCta == 2);
   constexpr int kBKe = 128 / kElem;                 // contraction elements per stage
   constexpr int kMmaK = 32 / kElem;                 // contraction elements per MMA
-  constexpr int kBBoxes = kBMN ? 2 * kElem : 1;     // TMA boxes per B stage
-  constexpr int kBBoxBytes = kBStage / kBBoxes;
-  constexpr uint32_t kIdesc = instr_desc(kF16, kBMN);
-  constexpr int kSt = stages_of<kMode>();
+  constexpr int kBS = kBStage / kCta;               // bytes of B per CTA per stage
+  constexpr int kBBoxes = kBMN ? (2 / kCta) * kElem : 1;  // TMA boxes per B stage (128-byte wide if MN-major)
+  constexpr int kBBoxBytes = kBS / kBBoxes;
+  constexpr uint32_t kIdesc = instr_desc(kF16, kBMN, kPair ? 256u : 128u);
+  constexpr int kSt = stages_of<kCta, kMode>();
   constexpr int kRing = ring_of<kMode>();
+  constexpr uint32_t kStageTx = kCta * (kAStage + kBS);  // bytes completing one stage (both CTAs)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + kSt * kAStage;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kSt * kBStage);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kSt * kBS);
   uint64_t *full = bars;                    // [kSt] TMA -> MMA
   uint64_t *empty = bars + kSt;         // [kSt] MMA -> TMA
   uint64_t *tfull = bars + 2 * kSt;     // [2] MMA -> epilogue
@@ -238,11 +259,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *s_srow = s_scol + kRing * kBN;                // [kRing][128] row scales per unit
   int *s_offs = reinterpret_cast<int *>(s_srow + kRing * kBM);
   int *s_tpre = s_offs + (kMaxGroups + 1);
+  int *s_ppre = s_tpre + (kMaxGroups + 1);  // prefix of 256-row pair tiles per group (kPair, row passes)
   // tgmm output staging, 128-byte aligned (TMA store sources must be aligned)
   uint8_t *s_stage_out =
-      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(s_tpre + (kMaxGroups + 1)) + 127) & ~uintptr_t(127));
+      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(s_tpre + kCta * (kMaxGroups + 1)) + 127) &
+                                  ~uintptr_t(127));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = kPair ? static_cast<int>(cluster_ctarank()) : 0;
+  const bool leader = rank == 0;
+  // items: one per CTA, or one per pair (consecutive blockIdx.x form a cluster)
+  const int w0 = kPair ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int wstep = kPair ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
 
   // Which scales each TMEM unit carries (the same decision in every role):
   //   column scales: forward s_r[g, n] (every unit of a tile, applied at the
@@ -265,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], kEpiWarps);
+      mbar_init(&tempty[i], kCta * kEpiWarps);  // a pair: the epilogue warps of both CTAs arrive on rank 0's
     }
     mbar_init(drain, 1);
     for (int i = 0; i < kRing; ++i) {
@@ -280,13 +308,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
+  if constexpr (kPair) {
+    // the other CTA's barriers are used (remote arrivals, byte counts,
+    // multicast commits) only after both CTAs initialized theirs
+    cluster_sync();
+  }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   for (int i = threadIdx.x; i <= p.G; i += kThreads) {
     s_offs[i] = p.offs[i];
     s_tpre[i] = p.tpre[i];
+  }
+  if constexpr (kPair && !kTg) {
+    __syncthreads();
+    if (warp == 2) {
+      // pair tiles per group: ceil(row tiles / 2); lane l scans groups
+      // [l * per, (l + 1) * per), then the lane totals are scanned across the warp
+      const int per = (p.G + 31) / 32;
+      const int g0 = min(lane * per, p.G), g1 = min(g0 + per, p.G);
+      int sum = 0;
+      for (int g = g0; g < g1; ++g) sum += (s_tpre[g + 1] - s_tpre[g] + 1) >> 1;
+      int incl = sum;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      int run = incl - sum;
+      for (int g = g0; g < g1; ++g) {
+        s_ppre[g] = run;
+        run += (s_tpre[g + 1] - s_tpre[g] + 1) >> 1;
+      }
+      if (lane == 31) s_ppre[p.G] = incl;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -294,7 +355,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_slot;
 
   const int tn = (p.ncols + kBN - 1) / kBN;
-  const int total = kTg ? p.G * p.rtiles * tn : s_tpre[p.G] * tn;
+  const int total = kTg ? p.G * (p.rtiles / kCta) * tn : (kPair ? s_ppre[p.G] : s_tpre[p.G]) * tn;
+  // rank 0's barriers as shared::cluster addresses (a pair's shared barriers)
+  const uint32_t full0_cl = kPair ? mapa_shared(smem_u32(full), 0) : 0;
+  const uint32_t tempty0_cl = kPair ? mapa_shared(smem_u32(tempty), 0) : 0;
   const WaitCtl ctl{p.wait_limit_ns, abort_flag, p.status};
   const WaitCtl ctl_drain{p.wait_limit_ns, no_abort, p.status};
 
@@ -304,15 +368,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------- TMA producer
       int it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-        const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+      // a pair's loads complete on rank 0's full barrier, which rank 0 arms
+      // with both CTAs' bytes
+      auto load = [&](void *dst, const CUtensorMap *map, int x, int y, int s) {
+        if constexpr (kPair) tma_load_2d_pair(dst, map, x, y, full0_cl + 8u * s);
+        else tma_load_2d(dst, map, x, y, &full[s]);
+      };
+      for (int w = w0; ok && w < total; w += wstep) {
+        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
         for (int b = 0; b < t.nblocks; ++b, ++it) {
           const int s = it % kSt;
           if (!mbar_wait(&empty[s], ((it / kSt) & 1) ^ 1, ctl)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], kAStage + kBStage);
+          if (leader) mbar_arrive_expect_tx(&full[s], kStageTx);
           int ax, ay, bx, by;
           if constexpr (!kTg) {
             ax = b * kBKe;
@@ -322,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               by = t.g * p.b_group_rows + b * kBKe;
             } else {
               bx = b * kBKe;
-              by = t.g * p.b_group_rows + t.ct * kBN;
+              by = t.g * p.b_group_rows + t.ct * kBN + (kBN / kCta) * rank;
             }
           } else {
             // chunk jj of the group (stages_per_chunk stages each) in the
@@ -331,37 +401,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             ax = (b % p.stages_per_chunk) * kBKe;
             ay = jj * (p.rtiles * kBM) + t.rt * kBM;  // dout columns n
             bx = ax;
-            by = jj * p.ncols + t.ct * kBN;           // lhs columns k (rows past K belong to the
-                                                      // next chunk: their columns are never stored)
+            by = jj * p.ncols + t.ct * kBN + (kBN / kCta) * rank;  // lhs columns k (rows past K belong
+                                                      // to the next chunk: their columns are never stored)
           }
-          tma_load_2d(sA + s * kAStage, &tmA, ax, ay, &full[s]);
+          load(sA + s * kAStage, &tmA, ax, ay, s);
           if constexpr (kBMN) {
-            // boxes of 128 bytes along n (columns of W[g] in [K, N])
+            // boxes of 128 bytes along n (columns of W[g] in [K, N]); a pair
+            // CTA takes tile columns 128 rank ..
 #pragma unroll
             for (int h = 0; h < kBBoxes; ++h)
-              tma_load_2d(sB + s * kBStage + h * kBBoxBytes, &tmB, tile_col_n(t.ct, h * kBKe, p.swiglu_f), by,
-                          &full[s]);
+              load(sB + s * kBS + h * kBBoxBytes, &tmB, tile_col_n(t.ct, (kBN / kCta) * rank + h * kBKe, p.swiglu_f),
+                   by, s);
           } else if (!kTg && p.swiglu_f) {
-            // two boxes of 128 rows (n) of W[g] in [N, K]: gate rows, up rows
+            // boxes of 128 rows (n) of W[g] in [N, K]: gate rows, up rows (a
+            // pair CTA loads one of them)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tma_load_2d(sB + s * kBStage + h * (kBStage / 2), &tmB, bx,
-                          t.g * p.b_group_rows + tile_col_n(t.ct, h * 128, p.swiglu_f), &full[s]);
+            for (int h = 0; h < 2 / kCta; ++h)
+              load(sB + s * kBS + h * (kBStage / 2), &tmB, bx,
+                   t.g * p.b_group_rows + tile_col_n(t.ct, (h + rank) * 128, p.swiglu_f), s);
           } else {
-            tma_load_2d(sB + s * kBStage, &tmB, bx, by, &full[s]);
+            load(sB + s * kBS, &tmB, bx, by, s);
           }
         }
       }
-      // let every issued copy land before the CTA can exit
-      for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
-        mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
+      // let every issued copy land before the CTA can exit.  A pair's copies
+      // complete on rank 0's barriers, so rank 0 waits for both CTAs' copies;
+      // rank 1 leaves only after the closing cluster barrier, which rank 0
+      // reaches after this wait.
+      if (leader)
+        for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
+          mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
     } else if (warp == 1) {
       // ----------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      if (lane == 0 && leader) {
         int it = 0, u = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-          const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+        for (int w = w0; ok && w < total; w += wstep) {
+          const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
@@ -379,23 +455,30 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBStage);
+            const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBS);
             const uint32_t d = tbase + buf * kBN;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
               const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
                                           : smem_desc_sw128(b0 + kk * 32, 16, 1024);
-              tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
+              // a pair's descriptors name rank 0's shared memory; the tensor
+              // core reads the same offsets in rank 1 for its half
+              if constexpr (kPair) tc_mma_pair<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
+              else tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
             }
-            tc_commit(&empty[s]);
+            // stage s free again / TMEM unit ready: in both CTAs of a pair
+            if constexpr (kPair) tc_commit_pair_both(&empty[s], 0x3);
+            else tc_commit(&empty[s]);
             if (kPromote || b == t.nblocks - 1) {
-              tc_commit(&tfull[buf]);
+              if constexpr (kPair) tc_commit_pair_both(&tfull[buf], 0x3);
+              else tc_commit(&tfull[buf]);
               ++u;
             }
           }
         }
-        tc_commit(drain);
+        if constexpr (kPair) tc_commit_pair_local(drain);
+        else tc_commit(drain);
         mbar_wait(drain, 0, ctl_drain);
       }
       __syncwarp();
@@ -405,8 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // them, so that no global-memory latency sits on the epilogue's path.
       int v = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-        const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+      for (int w = w0; ok && w < total; w += wstep) {
+        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
         const int units = kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0);
         const int64_t ch0 = kTg ? s_tpre[t.g] : 0;
         for (int j = 0; j < units; ++j, ++v) {
@@ -491,8 +574,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++v;
       }
     };
-    for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
-      const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+    // TMEM unit consumed: a pair's epilogue warps arrive on rank 0's barrier
+    auto release_unit = [&](uint32_t buf) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (kPair) mbar_arrive_cluster(tempty0_cl + 8u * buf);
+        else mbar_arrive(&tempty[buf]);
+      }
+    };
+    for (int w = w0; ok && w < total; w += wstep) {
+      const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
       const int col0 = t.ct * kBN + h * 128;
       int64_t orow;
       bool row_ok;
@@ -595,9 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
+          release_unit(buf);
           ++u;
           if (b + 1 < t.nblocks) release_slot(slot);  // the last slot is read again below
         }
@@ -690,9 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             emit(col, o);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[buf]);
+        release_unit(buf);
         ++u;
         release_slot(slot);
       }
@@ -719,9 +807,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair: neither CTA frees its tensor memory or leaves while the other may
+  // still read its shared memory (MMAs) or count bytes on its barriers (loads)
+  if constexpr (kPair) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, kTmemCols);
+    if constexpr (kPair) tmem_dealloc_pair(tbase, kTmemCols);
+    else tmem_dealloc(tbase, kTmemCols);
   }
 }
 
@@ -737,11 +829,11 @@ int num_sms() {
   return g_num_sms;
 }
 
-template <int kElem, bool kBMN, bool kPromote, int kMode>
+template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta>
 static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
                                const GemmParams &p, int grid, cudaStream_t st) {
-  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode>;
-  const size_t smem = gemm_smem_bytes<kMode>();
+  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode, kCta>;
+  const size_t smem = gemm_smem_bytes<kCta, kMode>();
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -751,33 +843,71 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
     return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(tmA, tmB, tmOut, p);
-  return cudaGetLastError();
+  if constexpr (kCta == 1) {
+    kern<<<grid, kThreads, smem, st>>>(tmA, tmB, tmOut, p);
+    return cudaGetLastError();
+  } else {
+    // clusters of two CTAs; as many pairs as can be resident at once (a
+    // persistent grid), never more than there are items
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    static int max_pairs = 0;  // per instantiation
+    if (max_pairs == 0) {
+      cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = num_sms() / 2;
+      max_pairs = n;
+    }
+    const int pairs = grid < max_pairs ? grid : max_pairs;  // grid counts items here
+    if (pairs <= 0) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmOut, p);
+  }
 }
 
-cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st) {
+template <int kCta>
+static cudaError_t launch_cta(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                              const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st) {
   if (cfg.mode == MODE_TGMM) {
     if (cfg.b_mn_major) return cudaErrorInvalidValue;
-    if (cfg.elem_bytes == 1 && cfg.promote) return launch_inst<1, false, true, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
-    if (cfg.elem_bytes == 2 && !cfg.promote) return launch_inst<2, false, false, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
+    if (cfg.elem_bytes == 1 && cfg.promote)
+      return launch_inst<1, false, true, MODE_TGMM, kCta>(tmA, tmB, tmOut, p, grid, st);
+    if (cfg.elem_bytes == 2 && !cfg.promote)
+      return launch_inst<2, false, false, MODE_TGMM, kCta>(tmA, tmB, tmOut, p, grid, st);
     return cudaErrorInvalidValue;
   }
   if (cfg.mode == MODE_ROWS_BLK) {  // block-wise rhs scales: promoted fp8 only
     if (cfg.elem_bytes != 1 || !cfg.promote) return cudaErrorInvalidValue;
-    return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK>(tmA, tmB, tmOut, p, grid, st)
-                          : launch_inst<1, false, true, MODE_ROWS_BLK>(tmA, tmB, tmOut, p, grid, st);
+    return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, p, grid, st)
+                          : launch_inst<1, false, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, p, grid, st);
   }
   if (cfg.elem_bytes == 1) {
     if (cfg.b_mn_major)
-      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
-                         : launch_inst<1, true, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
-    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
-                       : launch_inst<1, false, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
+      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st)
+                         : launch_inst<1, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st);
+    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st)
+                       : launch_inst<1, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st);
   }
   if (cfg.promote) return cudaErrorInvalidValue;
-  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
-                        : launch_inst<2, false, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
+  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st)
+                        : launch_inst<2, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st);
+}
+
+// grid: CTAs for one-CTA tiles; for pairs (cfg.cta_pairs) the number of pair
+// items, capped at the resident pairs
+cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st) {
+  return cfg.cta_pairs ? launch_cta<2>(cfg, tmA, tmB, tmOut, p, grid, st)
+                       : launch_cta<1>(cfg, tmA, tmB, tmOut, p, grid, st);
 }
 
 }  // namespace gmm

@@ -119,12 +119,15 @@ struct GemmConfig {
   int elem_bytes;   // 1: E4M3 (kind::f8f6f4), 2: BF16 (kind::f16)
   bool b_mn_major;  // B operand MN-major in shared memory
   bool promote;     // one TMEM unit per contraction block, promoted in registers
+  bool cta_pairs;   // 256-row tiles over a cluster of two CTAs (M = 256 MMAs);
+                    // the B tensor map's K-major box is then 128 rows
 };
 
 int num_sms();
 
 // tmOut: the output as a TMA tensor (MODE_TGMM: dW [G*K, N], box 32 x 32);
-// unused by MODE_ROWS.
+// unused by MODE_ROWS.  grid: CTAs (one-CTA tiles) or items (pairs; the
+// launch caps it at the pairs that fit on the GPU at once).
 cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
                         const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st);
 

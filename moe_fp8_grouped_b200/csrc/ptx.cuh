@@ -204,15 +204,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor: fp32 accumulator, M = 128, N = 256, A K-major,
-// B K-major or MN-major; E4M3 x E4M3 (kind::f8f6f4) or BF16 x BF16 (kind::f16).
-__host__ __device__ constexpr uint32_t instr_desc(bool f16, bool b_mn_major) {
+// Instruction descriptor: fp32 accumulator, M = 128 (one CTA) or 256 (a CTA
+// pair), N = 256, A K-major, B K-major or MN-major; E4M3 x E4M3
+// (kind::f8f6f4) or BF16 x BF16 (kind::f16).
+__host__ __device__ constexpr uint32_t instr_desc(bool f16, bool b_mn_major, uint32_t m = 128) {
   return (1u << 4)                              // D format F32
          | ((f16 ? 1u : 0u) << 7)               // A format: E4M3 = 0, BF16 = 1
          | ((f16 ? 1u : 0u) << 10)              // B format
          | ((b_mn_major ? 1u : 0u) << 16)       // B major
          | ((256u >> 3) << 17)                  // N
-         | ((128u >> 4) << 24);                 // M
+         | ((m >> 4) << 24);                    // M
 }
 
 // Two floats -> two E4M3 bytes (lo -> low byte), round to nearest even,
@@ -300,5 +301,106 @@ __device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap *map, int32_
 // Waits until at most one of this thread's committed bulk stores still reads
 // shared memory.
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+}  // namespace gmm
+
+namespace gmm {
+
+// ------------------------------------------------- CTA pairs (cta_group::2)
+//
+// Two CTAs of a cluster share one M = 256 MMA: each holds 128 rows of A and
+// half of B in its own shared memory, and each receives its 128 rows of the
+// accumulator in its own tensor memory.  The even CTA (rank 0) issues the
+// MMAs; barriers that both CTAs feed live in rank 0.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the object at shared-memory address `addr` of
+// this CTA, in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// every thread of both CTAs arrives and waits (release / acquire at cluster
+// scope)
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// arrive on an mbarrier given by its shared::cluster address (either CTA)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// 2-D tile load into this CTA's shared memory whose byte count completes on
+// an mbarrier of either CTA of the pair (shared::cluster address).  No
+// multicast: each CTA loads only its own part.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
+// tensor memory of the pair: issued by the same warp in both CTAs
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem of both CTAs] * B[smem of both CTAs]^T,
+// M = 256.  Issued by one thread of the even CTA.
+template <bool kF16>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  if constexpr (kF16) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// Arrive once on the mbarrier at this shared-memory offset in each CTA of
+// `cta_mask` when every pair MMA this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t *bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// The same for this CTA's own mbarrier only.
+__device__ __forceinline__ void tc_commit_pair_local(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
 
 }  // namespace gmm

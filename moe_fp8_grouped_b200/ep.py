@@ -42,16 +42,20 @@ class Route:
     k: int
     order: torch.Tensor         # int64 [T*k]: flat positions t*k + j sorted by expert (stable)
     counts: torch.Tensor        # int64 [E]: rows per expert from this rank
-    send_splits: list           # rows sent to each rank
+    send_splits: list | None    # rows sent to each rank (host ints; None until synchronized)
+    bad: torch.Tensor | None = None   # int64 [1] on the device: expert ids out of range
 
 
-def route(expert_ids: torch.Tensor, E: int, P: int, validate: bool = True) -> Route:
+def route(expert_ids: torch.Tensor, E: int, P: int, validate: bool = True, sync: bool = True) -> Route:
     """Sort this rank's routed rows by expert: the send order of the exchange.
-    One host synchronization: the range check of the ids, together with the
-    send splits when there is more than one rank.  validate=False (one rank
-    only) skips the check and the synchronization, for ids already checked
-    (for example in a captured CUDA graph); out-of-range ids are then counted
-    against the nearest valid expert."""
+
+    sync=True (the default): one host synchronization reads the range check of
+    the ids and, with more than one rank, the send splits.  sync=False: nothing
+    is read on the host; ``bad`` stays on the device and ``send_splits`` is
+    None (``exchange_counts`` then reads both with the arrival counts, in the
+    exchange's one synchronization).  validate=False (one rank only) skips the
+    check, for ids already checked (for example in a captured CUDA graph);
+    out-of-range ids are then counted against the nearest valid expert."""
     if E % P:
         raise ValueError(f"{E} experts do not split over {P} ranks")
     T, k = expert_ids.shape
@@ -63,37 +67,82 @@ def route(expert_ids: torch.Tensor, E: int, P: int, validate: bool = True) -> Ro
     send = counts.view(P, E // P).sum(dim=1)
     if P == 1 and not validate:
         return Route(E, P, k, order, counts, [T * k])
+    if not sync:
+        return Route(E, P, k, order, counts, None, bad)
     host = torch.cat([bad, send]).tolist() if P > 1 else bad.tolist()
     if host[0]:
         raise ValueError("expert id out of range")
     return Route(E, P, k, order, counts, host[1:] if P > 1 else [T * k])
 
 
-def exchange_counts(rt: Route, group=None) -> torch.Tensor:
-    """int64 [P, E/P]: rows each source rank sends to each of this rank's
-    experts.  One all-to-all of E integers."""
+def exchange_counts(rt: Route, group=None):
+    """One all-to-all of E + P integers: this rank's per-expert counts go to
+    the experts' ranks, each with this rank's count of out-of-range ids.
+    Returns (recv_counts int64 [P, E/P] on the device: rows each source rank
+    sends to each local expert; arrive: host list of rows arriving from each
+    rank).  When ``rt`` was routed without synchronizing, this is the
+    exchange's one host synchronization: it reads the send splits, the arrival
+    counts and every rank's bad-id count at once, and every rank raises when
+    any rank routed an id out of range (so that no rank enters the row
+    exchange alone)."""
     El = rt.E // rt.P
     if rt.P == 1:
-        return rt.counts.view(1, El).clone()
-    recv = torch.empty_like(rt.counts)
-    dist.all_to_all_single(recv, rt.counts, group=group)  # E / P counts to each rank
-    return recv.view(rt.P, El)
+        recv = rt.counts.view(1, El).clone()
+        if rt.send_splits is None:
+            if int(rt.bad.item()):
+                raise ValueError("expert id out of range")
+            rt.send_splits = [int(rt.counts.sum().item())]
+        return recv, list(rt.send_splits)
+    bad = rt.bad if rt.bad is not None else torch.zeros(1, dtype=torch.int64, device=rt.counts.device)
+    payload = torch.cat([rt.counts.view(rt.P, El), bad.expand(rt.P).view(rt.P, 1)], dim=1).contiguous()
+    recv = torch.empty_like(payload)
+    dist.all_to_all_single(recv, payload, group=group)  # E / P counts + 1 flag to each rank
+    recv_counts = recv[:, :El].contiguous()
+    if rt.send_splits is None:
+        send = rt.counts.view(rt.P, El).sum(dim=1)
+        host = torch.cat([send, recv_counts.sum(dim=1), recv[:, El]]).tolist()
+        P = rt.P
+        if any(host[2 * P:]):
+            raise ValueError("expert id out of range (on some rank)")
+        rt.send_splits = host[:P]
+        return recv_counts, host[P:2 * P]
+    return recv_counts, [int(v) for v in recv_counts.sum(dim=1).tolist()]
 
 
-def local_order(recv_counts: torch.Tensor):
-    """Rows arrive grouped by source rank, then by expert.  Returns (perm,
+def local_order(recv_counts: torch.Tensor, total: int | None = None):
+    """Rows arrive grouped by source rank, then by expert.  Returns (perm, inv,
     group_sizes): perm[i] is the arrival index of the i-th row when the rows
-    are grouped by local expert (then by source rank), and group_sizes the
-    rows per local expert."""
+    are grouped by local expert (then by source rank), inv its inverse (the
+    grouped position of each arrival row) and group_sizes the rows per local
+    expert.  On a CUDA device the library's kernel builds them
+    (gmm_ep_local_order, no host synchronization; ``total`` = the arrival
+    count, which the caller knows from the exchange); on the CPU (gloo ranks)
+    the same indices come from torch."""
     P, El = recv_counts.shape
+    if recv_counts.is_cuda:
+        if total is None:
+            raise ValueError("local_order on the device needs the arrival total")
+        cnt = recv_counts.to(torch.int64).contiguous()
+        perm = torch.empty(total, dtype=torch.int32, device=cnt.device)
+        inv = torch.empty(total, dtype=torch.int32, device=cnt.device)
+        gsz = torch.empty(El, dtype=torch.int32, device=cnt.device)
+        st = B.lib().gmm_ep_local_order(cnt.data_ptr(), P, El, total, perm.data_ptr() if total else None,
+                                        inv.data_ptr() if total else None, gsz.data_ptr(), _stream(cnt))
+        _check(st, "gmm_ep_local_order")
+        return perm, inv, gsz
     cnt = recv_counts.reshape(-1)
     start = torch.cumsum(cnt, 0) - cnt  # arrival offset of block (p, e)
     by_expert = torch.arange(P * El, device=cnt.device).view(P, El).t().reshape(-1)  # blocks (e, p)
     c = cnt[by_expert]
-    total = int(c.sum())
-    first = torch.repeat_interleave(start[by_expert], c)
-    within = torch.arange(total, device=cnt.device) - torch.repeat_interleave(torch.cumsum(c, 0) - c, c)
-    return first + within, recv_counts.sum(dim=0)
+    if total is None:
+        total = int(c.sum())
+    first = torch.repeat_interleave(start[by_expert], c, output_size=total)
+    within = torch.arange(total, device=cnt.device) - torch.repeat_interleave(torch.cumsum(c, 0) - c, c,
+                                                                              output_size=total)
+    perm = first + within
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(total, device=cnt.device)
+    return perm, inv, recv_counts.sum(dim=0)
 
 
 def exchange_rows(buf: torch.Tensor, in_splits, out_splits, group=None) -> torch.Tensor:
@@ -159,7 +208,9 @@ def ep_moe_fwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
     P = dist.get_world_size(group) if dist.is_initialized() else 1
     El, K, N = w_codes.shape
     T, k = expert_ids.shape
-    rt = route(expert_ids.to(x_codes.device), El * P, P, validate=validate or P > 1)
+    # P > 1: one host synchronization per call, in exchange_counts (the
+    # splits NCCL needs and the id check of every rank)
+    rt = route(expert_ids.to(x_codes.device), El * P, P, validate=validate or P > 1, sync=P == 1)
     order = rt.order
     # permute: this rank's routed rows in expert order, E4M3 codes
     send = gather_rows(x_codes, order // k)
@@ -167,10 +218,9 @@ def ep_moe_fwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
         # nothing to exchange: the sorted rows are already grouped by expert
         back_rows, gsz = send, rt.counts
     else:
-        recv_counts = exchange_counts(rt, group)
-        arrive = [int(v) for v in recv_counts.sum(dim=1).tolist()]
+        recv_counts, arrive = exchange_counts(rt, group)
         recv = exchange_rows(send, rt.send_splits, arrive, group)
-        perm, gsz = local_order(recv_counts)
+        perm, inv, gsz = local_order(recv_counts, sum(arrive))
         back_rows = gather_rows(recv, perm)
     if back_rows.shape[0]:
         h = gmm_fwd(back_rows, w_codes, w_scales, gsz.to(torch.int32), rule="static", static_scale=static_scale,
@@ -179,7 +229,6 @@ def ep_moe_fwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
         h = torch.empty((0, N), dtype=torch.bfloat16, device=x_codes.device)
     if P > 1:
         # back in arrival order, then to the source ranks
-        inv = torch.empty_like(perm).scatter_(0, perm, torch.arange(perm.numel(), device=perm.device))
         h = exchange_rows(gather_rows(h, inv), arrive, rt.send_splits, group)
     # h[i] is the result of flat position order[i]; slot of (t, j) = i
     slot = torch.empty_like(order).scatter_(0, order, torch.arange(order.numel(), device=order.device))
@@ -229,7 +278,7 @@ def ep_moe_bwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
     P = dist.get_world_size(group) if dist.is_initialized() else 1
     El, K, N = w_codes.shape
     T, k = expert_ids.shape
-    rt = route(expert_ids.to(x_codes.device), El * P, P)
+    rt = route(expert_ids.to(x_codes.device), El * P, P, sync=P == 1)
     order = rt.order
     tok = order // k
     send_x = gather_rows(x_codes, tok)
@@ -237,9 +286,8 @@ def ep_moe_bwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
     if P == 1:
         xr, dr, gsz, perm = send_x, send_d, rt.counts, None
     else:
-        recv_counts = exchange_counts(rt, group)
-        arrive = [int(v) for v in recv_counts.sum(dim=1).tolist()]
-        perm, gsz = local_order(recv_counts)
+        recv_counts, arrive = exchange_counts(rt, group)  # the one host synchronization
+        perm, inv, gsz = local_order(recv_counts, sum(arrive))
         xr = gather_rows(exchange_rows(send_x, rt.send_splits, arrive, group), perm)
         dr = gather_rows(exchange_rows(send_d, rt.send_splits, arrive, group), perm)
     dw = torch.empty((El, K, N), dtype=dw_dtype, device=x_codes.device)
@@ -250,7 +298,6 @@ def ep_moe_bwd(x_codes: torch.Tensor, static_scale: torch.Tensor, expert_ids: to
         dl = torch.empty((0, K), dtype=torch.bfloat16, device=x_codes.device)
         dw.zero_()
     if P > 1:
-        inv = torch.empty_like(perm).scatter_(0, perm, torch.arange(perm.numel(), device=perm.device))
         dl = exchange_rows(gather_rows(dl, inv), arrive, rt.send_splits, group)
     slot = torch.empty_like(order).scatter_(0, order, torch.arange(order.numel(), device=order.device))
     ones = torch.ones((T, k), dtype=torch.float32, device=x_codes.device)

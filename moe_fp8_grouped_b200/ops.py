@@ -342,6 +342,15 @@ def gmm_set_wait_limit_ns(limit_ns: int):
     B.lib().gmm_set_wait_limit_ns(limit_ns)
 
 
+TILES = {"auto": B.TILES_AUTO, "one_cta": B.TILES_ONE_CTA, "cta_pairs": B.TILES_CTA_PAIRS}
+
+
+def gmm_set_tiles(mode="auto"):
+    """GEMM tile choice for the calls that follow: "auto", "one_cta" (128-row
+    tiles) or "cta_pairs" (256-row tiles over a two-CTA cluster)."""
+    _check(B.lib().gmm_set_tiles(TILES[mode] if isinstance(mode, str) else int(mode)), "gmm_set_tiles")
+
+
 def gmm_plan(group_sizes: torch.Tensor, M: int):
     """Host-side helper (no kernel): clamped row offsets of the groups, as
     int64 CPU tensor [G + 1] (same rule as the device plan)."""
