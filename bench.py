@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--separate-backward", action="store_true",
                     help="run dlhs and drhs as two calls (gmm_dlhs, tgmm_drhs) instead of gmm_backward, which "
                          "quantizes dout once for both")
+    ap.add_argument("--tiles", default="auto", choices=["auto", "one_cta", "cta_pairs", "small_groups"],
+                    help="GEMM tile choice (gmm_set_tiles): automatic, 128-row tiles on one CTA, or 256-row tiles "
+                         "over CTA pairs")
     ap.add_argument("--no-forward-shapes", dest="forward_shapes", action="store_false",
                     help="skip the forward measurement on the DeepSeek-V3 and EP-shrunk shapes that the default "
                          "(Mixtral, one GPU) run adds to its line")
@@ -145,6 +148,7 @@ def step_config(w, args, world):
                                        if keep_lhs else "the tgmm quantizes lhs itself"),
                          "rhs_scales": ("block-wise: fwd [G, K/128, N], dlhs [G, N/128, K]" if blocks
                                         else "per channel [G, N]"),
+                         "tiles": args.tiles,
                          **({"l2": "flushed before every step (256 MiB write outside the timed events; "
                                    "the operands would fit in L2 across steps)"} if flush_l2 else {}),
                          **({"workload": f"ep_separate: G={w.G} M={w.M} K={w.K}, two N={Np} calls per pass "
@@ -250,6 +254,7 @@ def run_ours(args):
 
     # ep_separate: the EP-shrunk workload as two separate N=256 calls per pass
     # (W0 and W1 apart) instead of one merged N=512 call
+    gm.gmm_set_tiles(args.tiles)
     separate = args.workload == "ep_separate"
     w_named = synth.WORKLOADS[args.workload]
     w = synth.WORKLOADS["ep_merged" if separate else args.workload]

@@ -177,11 +177,23 @@ static gmm_status check_sizes(int64_t M, int64_t K, int64_t N, int32_t G) {
 
 static gmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA; }
 
+// Groups of at most this many rows take transposed small-group tiles (the
+// weights as the 128-row MMA operand, the group's rows as 64 MMA columns) in
+// the promoted E4M3 row passes on one-CTA tiles.
+constexpr int kSmallGroupRows = 64;
+
+static constexpr bool kAutoSmall = false;  // the automatic choice takes plain 128-row tiles for small groups
+
+static bool use_small(bool pairs, bool promote_fp8) {
+  if (!promote_fp8 || pairs) return false;
+  return g_cta_pairs == GMM_TILES_SMALL_GROUPS || (kAutoSmall && g_cta_pairs == GMM_TILES_AUTO);
+}
+
 // Launch size of a row pass (forward, dlhs) over `cols` output columns: one CTA
 // per SM at most; for pairs the number of pair items (the launch caps it)
 static int row_pass_grid(bool pairs, int64_t M, int64_t cols, int32_t G) {
   const int64_t rows = pairs ? 256 : 128;
-  const int64_t items = ((M + rows - 1) / rows + G) * ((cols + 255) / 256);
+  const int64_t items = ((M + rows - 1) / rows + G) * ((cols + 255) / 256) + static_cast<int64_t>(G) * (cols / 128);
   if (pairs) return static_cast<int>(items < INT_MAX ? items : INT_MAX);
   return static_cast<int>(items < num_sms() ? items : num_sms());
 }
@@ -272,7 +284,9 @@ int32_t gmm_last_launch_count(void) { return g_launches; }
 void gmm_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns = limit_ns ? limit_ns : kDefaultWaitLimitNs; }
 
 gmm_status gmm_set_tiles(int32_t mode) {
-  if (mode != GMM_TILES_AUTO && mode != GMM_TILES_ONE_CTA && mode != GMM_TILES_CTA_PAIRS) return GMM_ERR_INVALID_ARG;
+  if (mode != GMM_TILES_AUTO && mode != GMM_TILES_ONE_CTA && mode != GMM_TILES_CTA_PAIRS &&
+      mode != GMM_TILES_SMALL_GROUPS)
+    return GMM_ERR_INVALID_ARG;
   g_cta_pairs = mode;
   return GMM_OK;
 }
@@ -403,11 +417,18 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
                        : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke,
                                   (F || pairs) ? 128 : 256);
   if (!okB) return GMM_ERR_CUDA;
+  // small-group tiles: the weights as the 128-row operand (tmB itself when
+  // MN-major; a 128-row box of the K-major [G, N, K] weights otherwise)
+  const bool small = F == 0 && use_small(pairs, elem == 1 && dyn && !blk);
+  CUtensorMap tmW = tmB;
+  if (small && !bmn && !make_map(&tmW, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, 128))
+    return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
   p.M = static_cast<int>(M);
   p.ncols = static_cast<int>(N);
   p.swiglu_f = static_cast<int>(F);
+  p.small_rows = small ? kSmallGroupRows : 0;
   p.kblocks = static_cast<int>(K / bke);
   p.b_group_rows = static_cast<int>(bmn ? K : N);
   p.offs = P.offs;
@@ -427,7 +448,7 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk), pairs};
   const int grid = row_pass_grid(pairs, M, N, G);
   if ((s = cuda_status(prof(F ? "gemm_fwd_swiglu" : "gemm_fwd", st,
-                            [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
+                            [&] { return launch_gemm(cfg, tmA, tmB, tmA, tmW, p, grid, st); }))) != GMM_OK)
     return s;
   g_launches = n + 1;
   return GMM_OK;
@@ -478,10 +499,15 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
                        : make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke,
                                   pairs ? 128 : 256);
   if (!okB) return GMM_ERR_CUDA;
+  const bool small = use_small(pairs, elem == 1 && !blk);
+  CUtensorMap tmW = tmB;  // MN-major [G, N, K]: the 128 x 128 box of tmB
+  if (small && !bmn && !make_map(&tmW, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, 128))
+    return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
   p.M = static_cast<int>(M);
   p.ncols = static_cast<int>(K);
+  p.small_rows = small ? kSmallGroupRows : 0;
   p.kblocks = static_cast<int>(N / bke);
   p.b_group_rows = static_cast<int>(bmn ? N : K);
   p.offs = P.offs;
@@ -499,7 +525,7 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
   p.wait_limit_ns = g_wait_limit_ns;
   const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1, pairs};
   const int grid = row_pass_grid(pairs, M, K, G);
-  return cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }));
+  return cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, tmW, p, grid, st); }));
 }
 
 // tgmm GEMM on the chunk-major operands in the workspace (codes_a: lhs,
@@ -545,7 +571,7 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   const int64_t items = static_cast<int64_t>(G) * (N / (pairs ? 2 * kBlk : kBlk)) * ((K + 255) / 256);
   const int grid = pairs ? static_cast<int>(items < INT_MAX ? items : INT_MAX)
                          : static_cast<int>(items < num_sms() ? items : num_sms());
-  return cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, p, grid, st); }));
+  return cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, tmB, p, grid, st); }));
 }
 
 // The tgmm lhs operand into the workspace: quantized per chunk, re-laid out

@@ -82,6 +82,12 @@ constexpr int kStageOut = 4096;  // bytes of one output staging buffer (tgmm); t
 template <int kMode>
 constexpr int ring_of() { return kMode == MODE_TGMM ? 4 : kScaleSlots; }
 
+// int arrays [kMaxGroups + 1] in shared memory: group offsets, 128-row tile
+// prefix, and (CTA pairs or row passes) the item prefix of pair tiles or of
+// small-group tiles
+template <int kCta, int kMode>
+constexpr int plan_arrays() { return (kCta == 2 || kMode != MODE_TGMM) ? 3 : 2; }
+
 template <int kCta, int kMode>
 constexpr size_t gemm_smem_bytes() {
   return 1024                                    // alignment slack
@@ -89,20 +95,28 @@ constexpr size_t gemm_smem_bytes() {
          + kNumBars * 8                          // mbarriers
          + 16                                    // tmem slot, abort flags
          + ring_of<kMode>() * (kBN + kBM) * sizeof(float)  // scale ring
-         + (kCta == 2 ? 3 : 2) * (kMaxGroups + 1) * sizeof(int)  // plan copy (+ pair-tile prefix)
+         + plan_arrays<kCta, kMode>() * (kMaxGroups + 1) * sizeof(int)  // plan copy, item prefix
          + (kMode == MODE_TGMM ? 128 + kEpiWarps * 2 * kStageOut : 0);  // + alignment slack
 }
 static_assert(gemm_smem_bytes<2, MODE_ROWS>() <= 232448, "pair-tile shared memory");
 static_assert(gemm_smem_bytes<2, MODE_TGMM>() <= 232448, "pair-tile tgmm shared memory");
 static_assert(gemm_smem_bytes<1, MODE_ROWS>() <= 232448, "shared memory");
 static_assert(gemm_smem_bytes<1, MODE_TGMM>() <= 232448, "tgmm shared memory");
+static_assert(gemm_smem_bytes<1, MODE_ROWS>() == gemm_smem_bytes<1, MODE_ROWS_BLK>(), "row-pass shared memory");
 
 // One work item: tile row index rt (MODE_ROWS: rows r0 .. rend of group g;
 // MODE_TGMM: dout columns 128 rt ..), tile column index ct, and the number of
 // contraction stages.
 struct Item {
   int g, rt, ct, nblocks, r0, rend;
+  bool small;  // transposed small-group tile: output columns 128 ct .. as TMEM lanes,
+               // the group's rows r0 .. rend (at most 64) as TMEM columns
 };
+
+// Small-group tiles: M = 128 output columns (TMEM lanes), N = 64 rows of the
+// group (TMEM columns), 128-long contraction blocks.
+constexpr int kSmallN = 64;
+constexpr int kSmallCols = 128;
 
 // Column of the (2-D view of the) rhs held by tile column c (0 .. 255) of
 // column tile ct: plain tiles are 256 consecutive columns; SwiGLU tiles are
@@ -116,11 +130,42 @@ __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 
 // A CTA pair (kCta = 2) takes one item of twice the rows: rank r of the pair
 // holds tile rows 128 r .. 128 r + 127 of it.
+// small == true (one-CTA row passes with p.small_rows > 0): s_ppre holds the
+// prefix of items per group, tn column tiles per 128-row tile for ordinary
+// groups, ncols / 128 transposed tiles for groups of 1 .. p.small_rows rows.
 template <int kMode, int kCta>
 __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const int *s_offs, const int *s_tpre,
-                                            const int *s_ppre, int tn, int rank) {
+                                            const int *s_ppre, int tn, int rank, bool small) {
   Item t;
+  t.small = false;
   if constexpr (kMode != MODE_TGMM) {
+    if (kCta == 1 && small) {
+      int lo = 0, hi = p.G + 1;  // first i with s_ppre[i] > w
+      while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (s_ppre[mid] > w) hi = mid;
+        else lo = mid + 1;
+      }
+      const int g = lo - 1;
+      const int local = w - s_ppre[g];
+      const int size = s_offs[g + 1] - s_offs[g];
+      t.g = g;
+      t.nblocks = p.kblocks;
+      if (size > 0 && size <= p.small_rows) {
+        t.small = true;
+        t.rt = 0;
+        t.ct = local;  // 128-column tile
+        t.r0 = s_offs[g];
+        t.rend = s_offs[g + 1];
+      } else {
+        const int mt_g = s_tpre[g + 1] - s_tpre[g];
+        t.rt = local % mt_g;
+        t.ct = local / mt_g;
+        t.r0 = s_offs[g] + kBM * t.rt;
+        t.rend = min(s_offs[g + 1], t.r0 + kBM);
+      }
+      return t;
+    }
     // items of group g: (pre[g+1] - pre[g]) row tiles (128 rows, or 256 for a
     // pair) x tn column tiles, row tiles fastest
     const int *pre = kCta == 2 ? s_ppre : s_tpre;
@@ -226,7 +271,8 @@ __device__ __forceinline__ void store_col32(void *out, int64_t off_elems, int64_
 template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta>
 __global__ void __launch_bounds__(kThreads, 1)
     gmm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+                  const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmW,
+                  const GemmParams p) {
   constexpr bool kF16 = (kElem == 2);
   constexpr bool kTg = (kMode == MODE_TGMM);
   constexpr bool kPair = (kCta == 2);
@@ -259,11 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *s_srow = s_scol + kRing * kBN;                // [kRing][128] row scales per unit
   int *s_offs = reinterpret_cast<int *>(s_srow + kRing * kBM);
   int *s_tpre = s_offs + (kMaxGroups + 1);
-  int *s_ppre = s_tpre + (kMaxGroups + 1);  // prefix of 256-row pair tiles per group (kPair, row passes)
+  // item prefix per group: 256-row pair tiles (kPair, row passes) or
+  // ordinary and small-group items (one CTA, small tiles on)
+  int *s_ppre = s_tpre + (kMaxGroups + 1);
   // tgmm output staging, 128-byte aligned (TMA store sources must be aligned)
-  uint8_t *s_stage_out =
-      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(s_tpre + kCta * (kMaxGroups + 1)) + 127) &
-                                  ~uintptr_t(127));
+  uint8_t *s_stage_out = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(s_offs + plan_arrays<kCta, kMode>() * (kMaxGroups + 1)) + 127) & ~uintptr_t(127));
+  // transposed tiles for small groups: one-CTA promoted E4M3 row passes
+  constexpr bool kSmallOk = (kCta == 1 && kMode == MODE_ROWS && kElem == 1 && kPromote);
+  const bool small_on = kSmallOk && p.small_rows > 0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = kPair ? static_cast<int>(cluster_ctarank()) : 0;
@@ -307,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (small_on) tma_prefetch_desc(&tmW);
   }
   if constexpr (kPair) {
     // the other CTA's barriers are used (remote arrivals, byte counts,
@@ -326,15 +377,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_offs[i] = p.offs[i];
     s_tpre[i] = p.tpre[i];
   }
-  if constexpr (kPair && !kTg) {
+  const int tn = (p.ncols + kBN - 1) / kBN;
+  if ((kPair && !kTg) || small_on) {
     __syncthreads();
     if (warp == 2) {
-      // pair tiles per group: ceil(row tiles / 2); lane l scans groups
+      // items per group: pair tiles, ceil(row tiles / 2) x tn; or tn per row
+      // tile, ncols / 128 for a small group.  Lane l scans groups
       // [l * per, (l + 1) * per), then the lane totals are scanned across the warp
+      auto items_of = [&](int g) -> int {
+        const int mt = s_tpre[g + 1] - s_tpre[g];
+        if (kPair) return (mt + 1) >> 1;  // multiplied by tn where decoded
+        const int size = s_offs[g + 1] - s_offs[g];
+        return (size > 0 && size <= p.small_rows) ? p.ncols / kSmallCols : mt * tn;
+      };
       const int per = (p.G + 31) / 32;
       const int g0 = min(lane * per, p.G), g1 = min(g0 + per, p.G);
       int sum = 0;
-      for (int g = g0; g < g1; ++g) sum += (s_tpre[g + 1] - s_tpre[g] + 1) >> 1;
+      for (int g = g0; g < g1; ++g) sum += items_of(g);
       int incl = sum;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -344,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int run = incl - sum;
       for (int g = g0; g < g1; ++g) {
         s_ppre[g] = run;
-        run += (s_tpre[g + 1] - s_tpre[g] + 1) >> 1;
+        run += items_of(g);
       }
       if (lane == 31) s_ppre[p.G] = incl;
     }
@@ -354,8 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  const int tn = (p.ncols + kBN - 1) / kBN;
-  const int total = kTg ? p.G * (p.rtiles / kCta) * tn : (kPair ? s_ppre[p.G] : s_tpre[p.G]) * tn;
+  const int total = kTg ? p.G * (p.rtiles / kCta) * tn
+                        : (small_on ? s_ppre[p.G] : (kPair ? s_ppre[p.G] : s_tpre[p.G]) * tn);
   // rank 0's barriers as shared::cluster addresses (a pair's shared barriers)
   const uint32_t full0_cl = kPair ? mapa_shared(smem_u32(full), 0) : 0;
   const uint32_t tempty0_cl = kPair ? mapa_shared(smem_u32(tempty), 0) : 0;
@@ -375,12 +434,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         else tma_load_2d(dst, map, x, y, &full[s]);
       };
       for (int w = w0; ok && w < total; w += wstep) {
-        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
+        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
         for (int b = 0; b < t.nblocks; ++b, ++it) {
           const int s = it % kSt;
           if (!mbar_wait(&empty[s], ((it / kSt) & 1) ^ 1, ctl)) {
             ok = false;
             break;
+          }
+          if (kSmallOk && t.small) {
+            // weights (the 128 output columns as rows) into the A slot, the
+            // group's rows (a 128-row box, the first kSmallN used) into the B slot
+            mbar_arrive_expect_tx(&full[s], 2 * kAStage);
+            const int wo = t.g * p.b_group_rows;
+            if constexpr (kBMN) load(sA + s * kAStage, &tmW, t.ct * kSmallCols, wo + b * kBKe, s);
+            else load(sA + s * kAStage, &tmW, b * kBKe, wo + t.ct * kSmallCols, s);
+            load(sB + s * kBS, &tmA, b * kBKe, t.r0, s);
+            continue;
           }
           if (leader) mbar_arrive_expect_tx(&full[s], kStageTx);
           int ax, ay, bx, by;
@@ -437,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0, u = 0;
         bool ok = true;
         for (int w = w0; ok && w < total; w += wstep) {
-          const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
+          const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
@@ -457,6 +526,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBS);
             const uint32_t d = tbase + buf * kBN;
+            if (kSmallOk && t.small) {
+              // A: the weight tile, 128 output columns x 128 contraction (the
+              // major-ness of the weights in memory); B: kSmallN rows, K-major
+              constexpr uint32_t kIdescSmall = instr_desc_mn(kF16, kBMN, false, kSmallN, 128u);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t adesc = kBMN ? smem_desc_sw128(a0 + kk * kMmaK * 128, kAStage, 1024)
+                                            : smem_desc_sw128(a0 + kk * 32, 16, 1024);
+                const uint64_t bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+                tc_mma<kF16>(d, adesc, bdesc, kIdescSmall, (unit_start && kk == 0) ? 0u : 1u);
+              }
+              tc_commit(&empty[s]);
+              tc_commit(&tfull[buf]);
+              ++u;
+              continue;
+            }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
@@ -489,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int v = 0;
       bool ok = true;
       for (int w = w0; ok && w < total; w += wstep) {
-        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
+        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
         const int units = kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0);
         const int64_t ch0 = kTg ? s_tpre[t.g] : 0;
         for (int j = 0; j < units; ++j, ++v) {
@@ -502,6 +587,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // cp.async straight into the slot: the loader never waits for the
           // data, the slot's barrier completes when all 32 lanes' copies land
+          if (kSmallOk && t.small) {
+            // the group's row scales of block j (TMEM columns: 2 per lane) and
+            // the per-channel weight scales of the 128 output columns (TMEM
+            // lanes, applied at the end)
+            const float *src = p.row_scale + static_cast<int64_t>(j) * p.row_scale_ld;
+            const int64_t last = p.M - 1;
+            float *dc = s_scol + slot * kBN + 2 * lane;
+            cp_async_4(dc, src + min(static_cast<int64_t>(t.r0) + 2 * lane, last));
+            cp_async_4(dc + 1, src + min(static_cast<int64_t>(t.r0) + 2 * lane + 1, last));
+            if (p.col_scale)
+              cp_async_16(s_srow + slot * kBM + 4 * lane,
+                          p.col_scale + static_cast<int64_t>(t.g) * p.ncols + t.ct * kSmallCols + 4 * lane);
+            cp_async_mbar_arrive(&sfull[slot]);
+            continue;
+          }
           if (need_col) {
             // 8 columns per lane (never straddling a gate / up boundary);
             // columns >= ncols are never read
@@ -584,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     for (int w = w0; ok && w < total; w += wstep) {
-      const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
+      const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
       const int col0 = t.ct * kBN + h * 128;
       int64_t orow;
       bool row_ok;
@@ -624,6 +724,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
+      if (kSmallOk && t.small) {
+        // transposed small-group tile: TMEM lane = output column n (the
+        // thread's), TMEM columns = the group's rows; warp half h holds rows
+        // 32 h .. 32 h + 31.  acc += unit * s_row[block] per column.
+        float2 acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        int slot = 0;
+        for (int b = 0; b < t.nblocks; ++b) {
+          const uint32_t buf = u & 1;
+          slot = v % kRing;
+          if (!wait_unit(buf, slot)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t va[32];
+          tmem_ld32(tl + buf * kBN + 32 * h, va);
+          tmem_wait_ld();
+          const float2 *cs2 = reinterpret_cast<const float2 *>(s_scol + slot * kBN + 32 * h);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            acc[i] = __ffma2_rn(make_float2(__uint_as_float(va[2 * i]), __uint_as_float(va[2 * i + 1])), cs2[i],
+                                acc[i]);
+          release_unit(buf);
+          ++u;
+          if (b + 1 < t.nblocks) release_slot(slot);
+        }
+        if (!ok) break;
+        const float fin = p.col_scale ? s_srow[slot * kBM + row] : 1.0f;
+        const int64_t n = static_cast<int64_t>(t.ct) * kSmallCols + row;
+        const int m0 = t.r0 + 32 * h;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int m = m0 + 2 * i + e;
+            if (m >= t.rend) continue;
+            const float o = (e ? acc[i].y : acc[i].x) * fin;
+            if (p.out_f32) static_cast<float *>(p.out)[m * p.ld_out + n] = o;
+            else static_cast<__nv_bfloat16 *>(p.out)[m * p.ld_out + n] = __float2bfloat16_rn(o);
+          }
+        }
+        release_slot(slot);
+        continue;
+      }
       if (t.nblocks == 0) {  // empty group in tgmm: dW tile = 0
         float z[32];
 #pragma unroll
@@ -831,7 +977,7 @@ int num_sms() {
 
 template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta>
 static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                               const GemmParams &p, int grid, cudaStream_t st) {
+                               const CUtensorMap &tmW, const GemmParams &p, int grid, cudaStream_t st) {
   auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode, kCta>;
   const size_t smem = gemm_smem_bytes<kCta, kMode>();
   cudaFuncAttributes attr;
@@ -844,7 +990,7 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if constexpr (kCta == 1) {
-    kern<<<grid, kThreads, smem, st>>>(tmA, tmB, tmOut, p);
+    kern<<<grid, kThreads, smem, st>>>(tmA, tmB, tmOut, tmW, p);
     return cudaGetLastError();
   } else {
     // clusters of two CTAs; as many pairs as can be resident at once (a
@@ -870,44 +1016,49 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
     const int pairs = grid < max_pairs ? grid : max_pairs;  // grid counts items here
     if (pairs <= 0) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3(2 * pairs, 1, 1);
-    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmOut, p);
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmOut, tmW, p);
   }
 }
 
 template <int kCta>
 static cudaError_t launch_cta(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                              const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st) {
+                              const CUtensorMap &tmOut, const CUtensorMap &tmW, const GemmParams &p, int grid,
+                              cudaStream_t st) {
   if (cfg.mode == MODE_TGMM) {
     if (cfg.b_mn_major) return cudaErrorInvalidValue;
     if (cfg.elem_bytes == 1 && cfg.promote)
-      return launch_inst<1, false, true, MODE_TGMM, kCta>(tmA, tmB, tmOut, p, grid, st);
+      return launch_inst<1, false, true, MODE_TGMM, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
     if (cfg.elem_bytes == 2 && !cfg.promote)
-      return launch_inst<2, false, false, MODE_TGMM, kCta>(tmA, tmB, tmOut, p, grid, st);
+      return launch_inst<2, false, false, MODE_TGMM, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
     return cudaErrorInvalidValue;
   }
   if (cfg.mode == MODE_ROWS_BLK) {  // block-wise rhs scales: promoted fp8 only
     if (cfg.elem_bytes != 1 || !cfg.promote) return cudaErrorInvalidValue;
-    return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, p, grid, st)
-                          : launch_inst<1, false, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, p, grid, st);
+    return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
+                          : launch_inst<1, false, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
   }
   if (cfg.elem_bytes == 1) {
     if (cfg.b_mn_major)
-      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st)
-                         : launch_inst<1, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st);
-    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st)
-                       : launch_inst<1, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st);
+      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
+                         : launch_inst<1, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
+    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
+                       : launch_inst<1, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
   }
   if (cfg.promote) return cudaErrorInvalidValue;
-  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st)
-                        : launch_inst<2, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, p, grid, st);
+  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
+                        : launch_inst<2, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
 }
 
 // grid: CTAs for one-CTA tiles; for pairs (cfg.cta_pairs) the number of pair
 // items, capped at the resident pairs
 cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st) {
-  return cfg.cta_pairs ? launch_cta<2>(cfg, tmA, tmB, tmOut, p, grid, st)
-                       : launch_cta<1>(cfg, tmA, tmB, tmOut, p, grid, st);
+                        const CUtensorMap &tmOut, const CUtensorMap &tmW, const GemmParams &p, int grid,
+                        cudaStream_t st) {
+  if (p.small_rows > 0 && (cfg.cta_pairs || cfg.mode != MODE_ROWS || cfg.elem_bytes != 1 || !cfg.promote ||
+                           p.small_rows > kSmallN || p.ncols % kSmallCols || p.swiglu_f))
+    return cudaErrorInvalidValue;
+  return cfg.cta_pairs ? launch_cta<2>(cfg, tmA, tmB, tmOut, tmW, p, grid, st)
+                       : launch_cta<1>(cfg, tmA, tmB, tmOut, tmW, p, grid, st);
 }
 
 }  // namespace gmm

@@ -216,6 +216,14 @@ __host__ __device__ constexpr uint32_t instr_desc(bool f16, bool b_mn_major, uin
          | ((m >> 4) << 24);                    // M
 }
 
+// Instruction descriptor with both operand major-nesses and any legal M / N
+// (fp32 accumulator; N a multiple of 16 up to 256 for M = 128).
+__host__ __device__ constexpr uint32_t instr_desc_mn(bool f16, bool a_mn_major, bool b_mn_major, uint32_t n,
+                                                     uint32_t m) {
+  return (1u << 4) | ((f16 ? 1u : 0u) << 7) | ((f16 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
 // Two floats -> two E4M3 bytes (lo -> low byte), round to nearest even,
 // saturating to +-448.
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {

@@ -342,12 +342,14 @@ def gmm_set_wait_limit_ns(limit_ns: int):
     B.lib().gmm_set_wait_limit_ns(limit_ns)
 
 
-TILES = {"auto": B.TILES_AUTO, "one_cta": B.TILES_ONE_CTA, "cta_pairs": B.TILES_CTA_PAIRS}
+TILES = {"auto": B.TILES_AUTO, "one_cta": B.TILES_ONE_CTA, "cta_pairs": B.TILES_CTA_PAIRS,
+         "small_groups": B.TILES_SMALL_GROUPS}
 
 
 def gmm_set_tiles(mode="auto"):
     """GEMM tile choice for the calls that follow: "auto", "one_cta" (128-row
-    tiles) or "cta_pairs" (256-row tiles over a two-CTA cluster)."""
+    tiles), "cta_pairs" (256-row tiles over a two-CTA cluster) or
+    "small_groups" (transposed tiles for groups of at most 64 rows)."""
     _check(B.lib().gmm_set_tiles(TILES[mode] if isinstance(mode, str) else int(mode)), "gmm_set_tiles")
 
 
