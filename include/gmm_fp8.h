@@ -402,11 +402,23 @@ void gmm_set_wait_limit_ns(uint64_t limit_ns);
  *                           and dlhs (dynamic row scales, per-channel weight
  *                           scales, no SwiGLU) groups of at most 64 rows on
  *                           transposed tiles: the weights as the 128-row MMA
- *                           operand, the group's rows as 64 MMA columns.
+ *                           operand, the group's rows as 64 MMA columns;
+ *   GMM_TILES_CTA_PAIRS_NARROW  CTA pairs, and the promoted E4M3 passes whose
+ *                           weights or tgmm operand are K-major (dlhs with
+ *                           transpose_rhs 0, the dynamic forward with
+ *                           transpose_rhs 1, the tgmm) on 256 x 128 tiles:
+ *                           four 128-column tensor-memory accumulators per
+ *                           SM instead of two of 256.
  * Any other value returns GMM_ERR_INVALID_ARG.  Not part of the pages: how a
  * tile maps onto the B200's SMs is this library's choice.
  */
-enum { GMM_TILES_AUTO = 0, GMM_TILES_ONE_CTA = 1, GMM_TILES_CTA_PAIRS = 2, GMM_TILES_SMALL_GROUPS = 3 };
+enum {
+  GMM_TILES_AUTO = 0,
+  GMM_TILES_ONE_CTA = 1,
+  GMM_TILES_CTA_PAIRS = 2,
+  GMM_TILES_SMALL_GROUPS = 3,
+  GMM_TILES_CTA_PAIRS_NARROW = 4
+};
 gmm_status gmm_set_tiles(int32_t mode);
 
 /* Static text for a status code. */

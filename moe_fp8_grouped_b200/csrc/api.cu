@@ -21,10 +21,19 @@ static constexpr bool kAutoPairs = false;  // the automatic choice takes one-CTA
 // 128-row tile count is odd); for the tgmm when its rows do too and its dout
 // columns split into 256-wide pair tiles.
 static bool use_pairs(bool tgmm, int64_t M, int64_t N, int32_t G) {
-  if (g_cta_pairs == GMM_TILES_ONE_CTA) return false;
+  if (g_cta_pairs == GMM_TILES_ONE_CTA || g_cta_pairs == GMM_TILES_SMALL_GROUPS) return false;
   if (tgmm && N % 256) return false;
-  if (g_cta_pairs == GMM_TILES_CTA_PAIRS) return true;
+  if (g_cta_pairs == GMM_TILES_CTA_PAIRS || g_cta_pairs == GMM_TILES_CTA_PAIRS_NARROW) return true;
   return kAutoPairs && M >= 512 * static_cast<int64_t>(G);
+}
+
+// 128-column pair tiles (four TMEM accumulator buffers) for the promoted E4M3
+// passes whose B operand is K-major
+static constexpr bool kAutoNarrow = false;
+
+static int tile_cols(bool pairs, bool promote_fp8, bool b_k_major, bool swiglu) {
+  if (!pairs || !promote_fp8 || !b_k_major || swiglu) return 256;
+  return (g_cta_pairs == GMM_TILES_CTA_PAIRS_NARROW || (kAutoNarrow && g_cta_pairs == GMM_TILES_AUTO)) ? 128 : 256;
 }
 static thread_local int32_t g_launches = 0;
 
@@ -191,9 +200,9 @@ static bool use_small(bool pairs, bool promote_fp8) {
 
 // Launch size of a row pass (forward, dlhs) over `cols` output columns: one CTA
 // per SM at most; for pairs the number of pair items (the launch caps it)
-static int row_pass_grid(bool pairs, int64_t M, int64_t cols, int32_t G) {
+static int row_pass_grid(bool pairs, int64_t M, int64_t cols, int32_t G, int tn = 256) {
   const int64_t rows = pairs ? 256 : 128;
-  const int64_t items = ((M + rows - 1) / rows + G) * ((cols + 255) / 256) + static_cast<int64_t>(G) * (cols / 128);
+  const int64_t items = ((M + rows - 1) / rows + G) * ((cols + tn - 1) / tn) + static_cast<int64_t>(G) * (cols / 128);
   if (pairs) return static_cast<int>(items < INT_MAX ? items : INT_MAX);
   return static_cast<int>(items < num_sms() ? items : num_sms());
 }
@@ -285,7 +294,7 @@ void gmm_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns = limit_ns ? lim
 
 gmm_status gmm_set_tiles(int32_t mode) {
   if (mode != GMM_TILES_AUTO && mode != GMM_TILES_ONE_CTA && mode != GMM_TILES_CTA_PAIRS &&
-      mode != GMM_TILES_SMALL_GROUPS)
+      mode != GMM_TILES_SMALL_GROUPS && mode != GMM_TILES_CTA_PAIRS_NARROW)
     return GMM_ERR_INVALID_ARG;
   g_cta_pairs = mode;
   return GMM_OK;
@@ -413,9 +422,10 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   // SwiGLU tiles take the gate rows and the up rows of a K-major rhs as two
   // 128-row boxes
   const bool pairs = use_pairs(false, M, N, G);
+  const int tn = tile_cols(pairs, elem == 1 && (dyn || blk), !bmn, F != 0);
   const bool okB = bmn ? make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, bke)
                        : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke,
-                                  (F || pairs) ? 128 : 256);
+                                  pairs ? tn / 2 : (F ? 128 : 256));
   if (!okB) return GMM_ERR_CUDA;
   // small-group tiles: the weights as the 128-row operand (tmB itself when
   // MN-major; a 128-row box of the K-major [G, N, K] weights otherwise)
@@ -445,8 +455,9 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
   // per-block promotion for dynamic lhs scales or block-wise rhs scales
-  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk), pairs};
-  const int grid = row_pass_grid(pairs, M, N, G);
+  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1 && (dyn || blk), pairs,
+                       blk ? 256 : tn};
+  const int grid = row_pass_grid(pairs, M, N, G, cfg.tile_n);
   if ((s = cuda_status(prof(F ? "gemm_fwd_swiglu" : "gemm_fwd", st,
                             [&] { return launch_gemm(cfg, tmA, tmB, tmA, tmW, p, grid, st); }))) != GMM_OK)
     return s;
@@ -493,11 +504,12 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
   const bool bmn = transpose_rhs != 0;  // [G, N, K]: K contiguous = MN-major B for dlhs
   const uint32_t bke = 128 / elem;
   const bool pairs = use_pairs(false, M, K, G);
+  const int tn = blk ? 256 : tile_cols(pairs, elem == 1, !bmn, false);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, A, elem, N, M, N * elem, bke, 128)) return GMM_ERR_CUDA;
   const bool okB = bmn ? make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, bke)
                        : make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke,
-                                  pairs ? 128 : 256);
+                                  pairs ? tn / 2 : 256);
   if (!okB) return GMM_ERR_CUDA;
   const bool small = use_small(pairs, elem == 1 && !blk);
   CUtensorMap tmW = tmB;  // MN-major [G, N, K]: the 128 x 128 box of tmB
@@ -523,8 +535,8 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
   p.ld_out = K;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1, pairs};
-  const int grid = row_pass_grid(pairs, M, K, G);
+  const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1, pairs, tn};
+  const int grid = row_pass_grid(pairs, M, K, G, tn);
   return cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, tmW, p, grid, st); }));
 }
 
@@ -539,10 +551,11 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   // operands [chunk][column][128] are 2-D tensors of 128-element lines: chunk
   // j's line of column c is row j * C + c, so every box is one contiguous block.
   const bool pairs = use_pairs(true, M, N, G);
+  const int tn = tile_cols(pairs, elem == 1, true, false);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, P.codes_b, elem, kBlk, static_cast<uint64_t>(cap) * N, kBlk * elem, bke, 128))
     return GMM_ERR_CUDA;
-  if (!make_map(&tmB, P.codes_a, elem, kBlk, static_cast<uint64_t>(cap) * K, kBlk * elem, bke, pairs ? 128 : 256))
+  if (!make_map(&tmB, P.codes_a, elem, kBlk, static_cast<uint64_t>(cap) * K, kBlk * elem, bke, pairs ? tn / 2 : 256))
     return GMM_ERR_CUDA;
   CUtensorMap tmOut;  // dW as [G*K, N]: each epilogue warp stores 32 k-rows x 32 n
   if (!make_out_map(&tmOut, drhs, out_dtype == GMM_F32, N, static_cast<uint64_t>(G) * K, 32, 32))
@@ -567,8 +580,8 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   p.ld_out = N;
   p.status = P.status;
   p.wait_limit_ns = g_wait_limit_ns;
-  const GemmConfig cfg{MODE_TGMM, elem, false, elem == 1, pairs};
-  const int64_t items = static_cast<int64_t>(G) * (N / (pairs ? 2 * kBlk : kBlk)) * ((K + 255) / 256);
+  const GemmConfig cfg{MODE_TGMM, elem, false, elem == 1, pairs, tn};
+  const int64_t items = static_cast<int64_t>(G) * (N / (pairs ? 2 * kBlk : kBlk)) * ((K + tn - 1) / tn);
   const int grid = pairs ? static_cast<int>(items < INT_MAX ? items : INT_MAX)
                          : static_cast<int>(items < num_sms() ? items : num_sms());
   return cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, tmB, p, grid, st); }));

@@ -57,7 +57,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 256;
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 8;    // ring of per-unit scale slots (scale loader -> epilogue)
-constexpr int kNumBars = 40;      // mbarriers reserved in shared memory
+constexpr int kNumBars = 48;      // mbarriers reserved in shared memory
 // Register split (setmaxnreg): the control warpgroup gives registers to the
 // two epilogue warpgroups.  Sum must not exceed the launch allocation
 // (registers per thread at launch x 384); launch_inst checks it.
@@ -71,10 +71,12 @@ constexpr int regs_epi() { return kPromote ? 232 : 216; }
 // Pipeline stages.  One CTA: A 16 KB + B 32 KB per stage, 4 stages (tgmm: 3,
 // the freed shared memory stages its output for TMA stores, one 4 KB block
 // per epilogue warp).  A CTA pair (kCta = 2): each CTA holds its 128 rows of A
-// and half of B (16 KB + 16 KB), 6 stages (tgmm: 4).
-template <int kCta, int kMode>
+// and half of B: 16 KB + 16 KB with 256-column tiles, 6 stages (tgmm: 4);
+// 16 KB + 8 KB with 128-column tiles (kTN = 128), 8 stages (tgmm: 5).
+template <int kCta, int kMode, int kTN = 256>
 constexpr int stages_of() {
-  return kCta == 2 ? (kMode == MODE_TGMM ? 4 : 6) : (kMode == MODE_TGMM ? 3 : kStages);
+  return kCta == 2 ? (kTN == 128 ? (kMode == MODE_TGMM ? 5 : 8) : (kMode == MODE_TGMM ? 4 : 6))
+                   : (kMode == MODE_TGMM ? 3 : kStages);
 }
 constexpr int kStageOut = 4096;  // bytes of one output staging buffer (tgmm); two per epilogue warp
 
@@ -88,10 +90,10 @@ constexpr int ring_of() { return kMode == MODE_TGMM ? 4 : kScaleSlots; }
 template <int kCta, int kMode>
 constexpr int plan_arrays() { return (kCta == 2 || kMode != MODE_TGMM) ? 3 : 2; }
 
-template <int kCta, int kMode>
+template <int kCta, int kMode, int kTN = 256>
 constexpr size_t gemm_smem_bytes() {
   return 1024                                    // alignment slack
-         + static_cast<size_t>(stages_of<kCta, kMode>()) * (kAStage + kBStage / kCta)
+         + static_cast<size_t>(stages_of<kCta, kMode, kTN>()) * (kAStage + (kTN * 128) / kCta)
          + kNumBars * 8                          // mbarriers
          + 16                                    // tmem slot, abort flags
          + ring_of<kMode>() * (kBN + kBM) * sizeof(float)  // scale ring
@@ -103,6 +105,8 @@ static_assert(gemm_smem_bytes<2, MODE_TGMM>() <= 232448, "pair-tile tgmm shared 
 static_assert(gemm_smem_bytes<1, MODE_ROWS>() <= 232448, "shared memory");
 static_assert(gemm_smem_bytes<1, MODE_TGMM>() <= 232448, "tgmm shared memory");
 static_assert(gemm_smem_bytes<1, MODE_ROWS>() == gemm_smem_bytes<1, MODE_ROWS_BLK>(), "row-pass shared memory");
+static_assert(gemm_smem_bytes<2, MODE_ROWS, 128>() <= 232448, "narrow pair-tile shared memory");
+static_assert(gemm_smem_bytes<2, MODE_TGMM, 128>() <= 232448, "narrow pair-tile tgmm shared memory");
 
 // One work item: tile row index rt (MODE_ROWS: rows r0 .. rend of group g;
 // MODE_TGMM: dout columns 128 rt ..), tile column index ct, and the number of
@@ -114,15 +118,20 @@ struct Item {
 };
 
 // Small-group tiles: M = 128 output columns (TMEM lanes), N = 64 rows of the
-// group (TMEM columns), 128-long contraction blocks.
+// group (TMEM columns), 128-long contraction blocks.  kSmallStack consecutive
+// blocks share one 256-column TMEM unit, one 64-column slice each, so that a
+// unit carries as much MMA and promotion work as a 128 x 256 unit (and four
+// times the weight bytes of one block).
 constexpr int kSmallN = 64;
 constexpr int kSmallCols = 128;
+constexpr int kSmallStack = 256 / kSmallN;
 
-// Column of the (2-D view of the) rhs held by tile column c (0 .. 255) of
-// column tile ct: plain tiles are 256 consecutive columns; SwiGLU tiles are
-// gate columns 128 ct .. 128 ct + 127, then up columns F + 128 ct ..
-__device__ __forceinline__ int tile_col_n(int ct, int c, int F) {
-  return F ? (c < 128 ? 128 * ct + c : F + 128 * ct + (c - 128)) : kBN * ct + c;
+// Column of the (2-D view of the) rhs held by tile column c (0 .. tn - 1) of
+// column tile ct: plain tiles are tn (256 or 128) consecutive columns; SwiGLU
+// tiles (256 wide) are gate columns 128 ct .. 128 ct + 127, then up columns
+// F + 128 ct ..
+__device__ __forceinline__ int tile_col_n(int ct, int c, int F, int tn = kBN) {
+  return F ? (c < 128 ? 128 * ct + c : F + 128 * ct + (c - 128)) : tn * ct + c;
 }
 
 // x * sigmoid(x); -0 for large negative x, where exp(-x) overflows
@@ -268,7 +277,10 @@ __device__ __forceinline__ void store_col32(void *out, int64_t off_elems, int64_
 // its 128 rows of the accumulator.  Rank 0 issues the MMAs.  Halving B per SM
 // halves the shared-memory traffic per MMA (TMA writes plus tensor-core
 // reads), which bounds the one-CTA tile.
-template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta>
+// kTN: tile columns, 256, or 128 for CTA pairs in the promoted passes with a
+// K-major B (four 128-column TMEM buffers instead of two of 256: the MMA can
+// run three units ahead of the epilogue).
+template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta, bool kSmall, int kTN>
 __global__ void __launch_bounds__(kThreads, 1)
     gmm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmW,
@@ -278,11 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kPair = (kCta == 2);
   constexpr int kBKe = 128 / kElem;                 // contraction elements per stage
   constexpr int kMmaK = 32 / kElem;                 // contraction elements per MMA
-  constexpr int kBS = kBStage / kCta;               // bytes of B per CTA per stage
+  static_assert(kTN == 256 || (kTN == 128 && kPair && kPromote && !kBMN), "128-column tiles: pairs, promoted, K-major B");
+  constexpr int kBS = (kTN * 128) / kCta;           // bytes of B per CTA per stage
   constexpr int kBBoxes = kBMN ? (2 / kCta) * kElem : 1;  // TMA boxes per B stage (128-byte wide if MN-major)
   constexpr int kBBoxBytes = kBS / kBBoxes;
-  constexpr uint32_t kIdesc = instr_desc(kF16, kBMN, kPair ? 256u : 128u);
-  constexpr int kSt = stages_of<kCta, kMode>();
+  constexpr uint32_t kIdesc = instr_desc_mn(kF16, false, kBMN, kTN, kPair ? 256u : 128u);
+  constexpr int kSt = stages_of<kCta, kMode, kTN>();
+  constexpr int kNB = kTmemCols / kTN;              // TMEM accumulator buffers
+  constexpr int kCh = kTN / 64;                     // 32-column chunks per epilogue thread
   constexpr int kRing = ring_of<kMode>();
   constexpr uint32_t kStageTx = kCta * (kAStage + kBS);  // bytes completing one stage (both CTAs)
 
@@ -293,9 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kSt * kBS);
   uint64_t *full = bars;                    // [kSt] TMA -> MMA
   uint64_t *empty = bars + kSt;         // [kSt] MMA -> TMA
-  uint64_t *tfull = bars + 2 * kSt;     // [2] MMA -> epilogue
-  uint64_t *tempty = tfull + 2;             // [2] epilogue -> MMA
-  uint64_t *drain = tempty + 2;             // MMA completion at exit
+  uint64_t *tfull = bars + 2 * kSt;     // [kNB] MMA -> epilogue
+  uint64_t *tempty = tfull + kNB;           // [kNB] epilogue -> MMA
+  uint64_t *drain = tempty + kNB;           // MMA completion at exit
   uint64_t *sfull = drain + 1;              // [kRing] scale loader -> epilogue
   uint64_t *sempty = sfull + kRing;   // [kRing] epilogue -> scale loader
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
@@ -311,8 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // tgmm output staging, 128-byte aligned (TMA store sources must be aligned)
   uint8_t *s_stage_out = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(s_offs + plan_arrays<kCta, kMode>() * (kMaxGroups + 1)) + 127) & ~uintptr_t(127));
-  // transposed tiles for small groups: one-CTA promoted E4M3 row passes
-  constexpr bool kSmallOk = (kCta == 1 && kMode == MODE_ROWS && kElem == 1 && kPromote);
+  // transposed tiles for small groups: one-CTA promoted E4M3 row passes, in
+  // their own instantiation (kSmall) so that the other kernels carry none of
+  // their code or registers
+  constexpr bool kSmallOk = kSmall;
+  static_assert(!kSmall || (kCta == 1 && kMode == MODE_ROWS && kElem == 1 && kPromote), "small-group tiles");
   const bool small_on = kSmallOk && p.small_rows > 0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -341,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNB; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kCta * kEpiWarps);  // a pair: the epilogue warps of both CTAs arrive on rank 0's
     }
@@ -377,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_offs[i] = p.offs[i];
     s_tpre[i] = p.tpre[i];
   }
-  const int tn = (p.ncols + kBN - 1) / kBN;
+  const int tn = (p.ncols + kTN - 1) / kTN;
   if ((kPair && !kTg) || small_on) {
     __syncthreads();
     if (warp == 2) {
@@ -457,11 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ax = b * kBKe;
             ay = t.r0;
             if (kBMN) {
-              bx = t.ct * kBN;
+              bx = t.ct * kTN;
               by = t.g * p.b_group_rows + b * kBKe;
             } else {
               bx = b * kBKe;
-              by = t.g * p.b_group_rows + t.ct * kBN + (kBN / kCta) * rank;
+              by = t.g * p.b_group_rows + t.ct * kTN + (kTN / kCta) * rank;
             }
           } else {
             // chunk jj of the group (stages_per_chunk stages each) in the
@@ -470,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ax = (b % p.stages_per_chunk) * kBKe;
             ay = jj * (p.rtiles * kBM) + t.rt * kBM;  // dout columns n
             bx = ax;
-            by = jj * p.ncols + t.ct * kBN + (kBN / kCta) * rank;  // lhs columns k (rows past K belong
+            by = jj * p.ncols + t.ct * kTN + (kTN / kCta) * rank;  // lhs columns k (rows past K belong
                                                       // to the next chunk: their columns are never stored)
           }
           load(sA + s * kAStage, &tmA, ax, ay, s);
@@ -479,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // CTA takes tile columns 128 rank ..
 #pragma unroll
             for (int h = 0; h < kBBoxes; ++h)
-              load(sB + s * kBS + h * kBBoxBytes, &tmB, tile_col_n(t.ct, (kBN / kCta) * rank + h * kBKe, p.swiglu_f),
-                   by, s);
+              load(sB + s * kBS + h * kBBoxBytes, &tmB,
+                   tile_col_n(t.ct, (kTN / kCta) * rank + h * kBKe, p.swiglu_f, kTN), by, s);
           } else if (!kTg && p.swiglu_f) {
             // boxes of 128 rows (n) of W[g] in [N, K]: gate rows, up rows (a
             // pair CTA loads one of them)
@@ -509,10 +527,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
-            const bool unit_start = kPromote || b == 0;
+            const bool unit_start = (kSmallOk && t.small) ? (b % kSmallStack == 0) : (kPromote || b == 0);
             if (unit_start) {
-              buf = u & 1;
-              if (!mbar_wait(&tempty[buf], ((u >> 1) & 1) ^ 1, ctl)) {
+              buf = u % kNB;
+              if (!mbar_wait(&tempty[buf], ((u / kNB) & 1) ^ 1, ctl)) {
                 ok = false;
                 break;
               }
@@ -525,21 +543,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBS);
-            const uint32_t d = tbase + buf * kBN;
+            const uint32_t d = tbase + buf * kTN;
             if (kSmallOk && t.small) {
               // A: the weight tile, 128 output columns x 128 contraction (the
-              // major-ness of the weights in memory); B: kSmallN rows, K-major
+              // major-ness of the weights in memory); B: kSmallN rows, K-major.
+              // Block b fills slice b % kSmallStack of the unit.
               constexpr uint32_t kIdescSmall = instr_desc_mn(kF16, kBMN, false, kSmallN, 128u);
+              const uint32_t ds = d + (b % kSmallStack) * kSmallN;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t adesc = kBMN ? smem_desc_sw128(a0 + kk * kMmaK * 128, kAStage, 1024)
                                             : smem_desc_sw128(a0 + kk * 32, 16, 1024);
                 const uint64_t bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-                tc_mma<kF16>(d, adesc, bdesc, kIdescSmall, (unit_start && kk == 0) ? 0u : 1u);
+                tc_mma<kF16>(ds, adesc, bdesc, kIdescSmall, kk == 0 ? 0u : 1u);
               }
               tc_commit(&empty[s]);
-              tc_commit(&tfull[buf]);
-              ++u;
+              if (b % kSmallStack == kSmallStack - 1 || b == t.nblocks - 1) {
+                tc_commit(&tfull[buf]);
+                ++u;
+              }
               continue;
             }
 #pragma unroll
@@ -575,7 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int w = w0; ok && w < total; w += wstep) {
         const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
-        const int units = kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0);
+        const int units = (kSmallOk && t.small) ? (t.nblocks + kSmallStack - 1) / kSmallStack
+                                                : (kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0));
         const int64_t ch0 = kTg ? s_tpre[t.g] : 0;
         for (int j = 0; j < units; ++j, ++v) {
           const int slot = v % kRing;
@@ -588,14 +611,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           // cp.async straight into the slot: the loader never waits for the
           // data, the slot's barrier completes when all 32 lanes' copies land
           if (kSmallOk && t.small) {
-            // the group's row scales of block j (TMEM columns: 2 per lane) and
-            // the per-channel weight scales of the 128 output columns (TMEM
-            // lanes, applied at the end)
-            const float *src = p.row_scale + static_cast<int64_t>(j) * p.row_scale_ld;
+            // the group's row scales of the unit's blocks (slice s: 64 TMEM
+            // columns, 2 per lane) and the per-channel weight scales of the
+            // 128 output columns (TMEM lanes, applied at the end)
             const int64_t last = p.M - 1;
-            float *dc = s_scol + slot * kBN + 2 * lane;
-            cp_async_4(dc, src + min(static_cast<int64_t>(t.r0) + 2 * lane, last));
-            cp_async_4(dc + 1, src + min(static_cast<int64_t>(t.r0) + 2 * lane + 1, last));
+            const int64_t r = static_cast<int64_t>(t.r0) + 2 * lane;
+#pragma unroll
+            for (int sl = 0; sl < kSmallStack; ++sl) {
+              const int b = j * kSmallStack + sl;
+              if (b >= t.nblocks) break;
+              const float *src = p.row_scale + static_cast<int64_t>(b) * p.row_scale_ld;
+              float *dc = s_scol + slot * kBN + sl * kSmallN + 2 * lane;
+              cp_async_4(dc, src + min(r, last));
+              cp_async_4(dc + 1, src + min(r + 1, last));
+            }
             if (p.col_scale)
               cp_async_16(s_srow + slot * kBM + 4 * lane,
                           p.col_scale + static_cast<int64_t>(t.g) * p.ncols + t.ct * kSmallCols + 4 * lane);
@@ -603,17 +632,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           if (need_col) {
-            // 8 columns per lane (never straddling a gate / up boundary);
-            // columns >= ncols are never read
-            const int n = kTg ? t.ct * kBN + 8 * lane : tile_col_n(t.ct, 8 * lane, p.swiglu_f);
+            // kTN / 32 columns per lane (never straddling a gate / up
+            // boundary); columns >= ncols are never read
+            constexpr int kCpl = kTN / 32;
+            const int n = kTg ? t.ct * kTN + kCpl * lane : tile_col_n(t.ct, kCpl * lane, p.swiglu_f, kTN);
             if (n < p.ncols) {
               const float *src =
                   kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
                       : (kBlkScales ? p.colblk_scale + (static_cast<int64_t>(t.g) * p.kblocks + j) * p.colblk_ld + n
                               : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n);
-              float *dst = s_scol + slot * kBN + 8 * lane;
-              cp_async_16(dst, src);
-              cp_async_16(dst + 4, src + 4);
+              float *dst = s_scol + slot * kBN + kCpl * lane;
+#pragma unroll
+              for (int e = 0; e < kCpl; e += 4) cp_async_16(dst + e, src + e);
             }
           }
           if (need_row) {
@@ -644,7 +674,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile column of the thread's 32-column chunk c (0 .. 3): the column half h
     // of the tile, or for SwiGLU gate columns 64 h .. (c = 0, 1) and the
     // matching up columns 128 + 64 h .. (c = 2, 3)
-    auto colt = [&](int c) -> int { return sw ? ((c & 2) ? 128 : 0) + h * 64 + (c & 1) * 32 : h * 128 + c * 32; };
+    auto colt = [&](int c) -> int {
+      return sw ? ((c & 2) ? 128 : 0) + h * 64 + (c & 1) * 32 : h * (kTN / 2) + c * 32;
+    };
     float s_eff = 1.0f;
     if (p.static_scale) {
       const float v = *p.static_scale;
@@ -663,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // abort flag, which ends every other warp's next wait, and no barrier
     // among the epilogue warps is ever entered after that point.
     auto wait_unit = [&](uint32_t buf, int slot) -> bool {
-      bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
+      bool got = mbar_wait(&tfull[buf], (u / kNB) & 1, ctl);
       if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kRing) & 1, ctl);
       return __all_sync(0xffffffffu, got);
     };
@@ -685,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int w = w0; ok && w < total; w += wstep) {
       const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
-      const int col0 = t.ct * kBN + h * 128;
+      const int col0 = t.ct * kTN + h * (kTN / 2);
       int64_t orow;
       bool row_ok;
       if constexpr (!kTg) {
@@ -732,25 +764,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.0f, 0.0f);
         int slot = 0;
-        for (int b = 0; b < t.nblocks; ++b) {
-          const uint32_t buf = u & 1;
+        const int nunits = (t.nblocks + kSmallStack - 1) / kSmallStack;
+        for (int j = 0; j < nunits; ++j) {
+          const uint32_t buf = u % kNB;
           slot = v % kRing;
           if (!wait_unit(buf, slot)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          uint32_t va[32];
-          tmem_ld32(tl + buf * kBN + 32 * h, va);
-          tmem_wait_ld();
-          const float2 *cs2 = reinterpret_cast<const float2 *>(s_scol + slot * kBN + 32 * h);
+          const int nb = min(kSmallStack, t.nblocks - j * kSmallStack);  // blocks in this unit (warp-uniform)
+          // slices two at a time, blocks in contraction order: the same
+          // sequence of fused multiply-adds as a 128-row tile
+          for (int sp = 0; sp < nb; sp += 2) {
+            uint32_t va[32], vb[32];
+            tmem_ld32(tl + buf * kBN + sp * kSmallN + 32 * h, va);
+            if (sp + 1 < nb) tmem_ld32(tl + buf * kBN + (sp + 1) * kSmallN + 32 * h, vb);
+            tmem_wait_ld();
+            const float2 *ca = reinterpret_cast<const float2 *>(s_scol + slot * kBN + sp * kSmallN + 32 * h);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            acc[i] = __ffma2_rn(make_float2(__uint_as_float(va[2 * i]), __uint_as_float(va[2 * i + 1])), cs2[i],
-                                acc[i]);
+            for (int i = 0; i < 16; ++i)
+              acc[i] = __ffma2_rn(make_float2(__uint_as_float(va[2 * i]), __uint_as_float(va[2 * i + 1])), ca[i],
+                                  acc[i]);
+            if (sp + 1 < nb) {
+              const float2 *cb = ca + kSmallN / 2;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[i] = __ffma2_rn(make_float2(__uint_as_float(vb[2 * i]), __uint_as_float(vb[2 * i + 1])), cb[i],
+                                    acc[i]);
+            }
+          }
           release_unit(buf);
           ++u;
-          if (b + 1 < t.nblocks) release_slot(slot);
+          if (j + 1 < nunits) release_slot(slot);
         }
         if (!ok) break;
         const float fin = p.col_scale ? s_srow[slot * kBM + row] : 1.0f;
@@ -775,17 +821,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < kCh; ++c)
           if (col0 + c * 32 < p.ncols) emit(col0 + c * 32, z);
         continue;
       }
       if constexpr (kPromote) {
-        float2 acc[64];
+        float2 acc[kCh * 16];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int i = 0; i < kCh * 16; ++i) acc[i] = make_float2(0.0f, 0.0f);
         int slot = 0;
         for (int b = 0; b < t.nblocks; ++b) {
-          const uint32_t buf = u & 1;
+          const uint32_t buf = u % kNB;
           slot = v % kRing;
           if (!wait_unit(buf, slot)) {
             ok = false;
@@ -796,11 +842,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 rs2 = make_float2(rs, rs);
           const float *cs = s_scol + slot * kBN;
 #pragma unroll
-          for (int cp = 0; cp < 2; ++cp) {
+          for (int cp = 0; cp < kCh / 2; ++cp) {
             // chunks 2 cp, 2 cp + 1 (compile-time accumulator indices)
             // colt(2 cp + 1) = colt(2 cp) + 32: one 64-column load
             uint32_t va[32], vb[32];
-            tmem_ld64(tl + buf * kBN + colt(2 * cp), va, vb);
+            tmem_ld64(tl + buf * kTN + colt(2 * cp), va, vb);
             tmem_wait_ld();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -843,14 +889,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float fin = ((kTg || kBlkScales) && p.static_scale) ? s_eff : 1.0f;
           const bool colmul = !kTg && p.col_scale != nullptr;
           const float *cf = s_scol + slot * kBN;
-          if (sw) {
+          if (kTN == 256 && sw) {  // SwiGLU tiles are 256 wide (128 gate + 128 up columns)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               const float *fg = cf + colt(c), *fu = cf + colt(c + 2);
               float o[32];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float2 a = acc[c * 16 + i], b2 = acc[(c + 2) * 16 + i];
+                const float2 a = acc[c * 16 + i], b2 = acc[((c + 2) % kCh) * 16 + i];
                 const float g0 = (colmul ? a.x * fg[2 * i] : a.x) * fin;
                 const float g1 = (colmul ? a.y * fg[2 * i + 1] : a.y) * fin;
                 const float u0 = (colmul ? b2.x * fu[2 * i] : b2.x) * fin;
@@ -862,8 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int col = t.ct * kBN + colt(c);
+            for (int c = 0; c < kCh; ++c) {
+              const int col = t.ct * kTN + colt(c);
               if (col >= p.ncols) continue;
               float o[32];
 #pragma unroll
@@ -882,7 +928,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         release_slot(slot);
       } else {
-        const uint32_t buf = u & 1;
+        static_assert(kPromote || kTN == 256, "one unit per tile: 256-column tiles");
+        const uint32_t buf = u % kNB;
         const int slot = v % kRing;
         if (!wait_unit(buf, slot)) {
           ok = false;
@@ -895,8 +942,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cp = 0; cp < 2; ++cp) {
           const int ca = sw ? cp : 2 * cp, cb = sw ? cp + 2 : 2 * cp + 1;
           uint32_t va[32], vb[32];
-          tmem_ld32(tl + buf * kBN + colt(ca), va);
-          tmem_ld32(tl + buf * kBN + colt(cb), vb);
+          tmem_ld32(tl + buf * kTN + colt(ca), va);
+          tmem_ld32(tl + buf * kTN + colt(cb), vb);
           tmem_wait_ld();
           if (sw) {
             if (row_ok) {
@@ -915,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < 2; ++half) {
             const uint32_t *vv = half ? vb : va;
             const int c = half ? cb : ca;
-            const int col = t.ct * kBN + colt(c);
+            const int col = t.ct * kTN + colt(c);
             if (!row_ok || col >= p.ncols) continue;
             float o[32];
 #pragma unroll
@@ -975,11 +1022,11 @@ int num_sms() {
   return g_num_sms;
 }
 
-template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta>
+template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta, bool kSmall = false, int kTN = 256>
 static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
                                const CUtensorMap &tmW, const GemmParams &p, int grid, cudaStream_t st) {
-  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode, kCta>;
-  const size_t smem = gemm_smem_bytes<kCta, kMode>();
+  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode, kCta, kSmall, kTN>;
+  const size_t smem = gemm_smem_bytes<kCta, kMode, kTN>();
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -1037,6 +1084,22 @@ static cudaError_t launch_cta(const GemmConfig &cfg, const CUtensorMap &tmA, con
     return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
                           : launch_inst<1, false, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
   }
+  if constexpr (kCta == 2) {
+    if (cfg.tile_n == 128) {  // four 128-column TMEM buffers: promoted E4M3, K-major B
+      if (cfg.elem_bytes != 1 || !cfg.promote || cfg.b_mn_major) return cudaErrorInvalidValue;
+      if (cfg.mode == MODE_ROWS)
+        return launch_inst<1, false, true, MODE_ROWS, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
+      if (cfg.mode == MODE_TGMM)
+        return launch_inst<1, false, true, MODE_TGMM, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
+      return cudaErrorInvalidValue;
+    }
+  }
+  if (cfg.tile_n != 256) return cudaErrorInvalidValue;
+  if constexpr (kCta == 1) {
+    if (p.small_rows > 0)  // promoted E4M3 row pass with small-group tiles (checked by launch_gemm)
+      return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS, 1, true>(tmA, tmB, tmOut, tmW, p, grid, st)
+                            : launch_inst<1, false, true, MODE_ROWS, 1, true>(tmA, tmB, tmOut, tmW, p, grid, st);
+  }
   if (cfg.elem_bytes == 1) {
     if (cfg.b_mn_major)
       return cfg.promote ? launch_inst<1, true, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
@@ -1057,6 +1120,7 @@ cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUt
   if (p.small_rows > 0 && (cfg.cta_pairs || cfg.mode != MODE_ROWS || cfg.elem_bytes != 1 || !cfg.promote ||
                            p.small_rows > kSmallN || p.ncols % kSmallCols || p.swiglu_f))
     return cudaErrorInvalidValue;
+  if (cfg.tile_n == 128 && (!cfg.cta_pairs || p.swiglu_f)) return cudaErrorInvalidValue;
   return cfg.cta_pairs ? launch_cta<2>(cfg, tmA, tmB, tmOut, tmW, p, grid, st)
                        : launch_cta<1>(cfg, tmA, tmB, tmOut, tmW, p, grid, st);
 }

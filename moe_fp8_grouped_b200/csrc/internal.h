@@ -124,7 +124,9 @@ struct GemmConfig {
   bool b_mn_major;  // B operand MN-major in shared memory
   bool promote;     // one TMEM unit per contraction block, promoted in registers
   bool cta_pairs;   // 256-row tiles over a cluster of two CTAs (M = 256 MMAs);
-                    // the B tensor map's K-major box is then 128 rows
+                    // the B tensor map's K-major box is then tile_n / 2 rows
+  int tile_n;       // tile columns: 256, or 128 (CTA pairs, promoted E4M3,
+                    // K-major B: four TMEM accumulator buffers)
 };
 
 int num_sms();

@@ -341,9 +341,14 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// arrive on an mbarrier given by its shared::cluster address (either CTA)
+// arrive on an mbarrier given by its shared::cluster address (either CTA),
+// with the default release semantics at CTA scope: what the arrival orders
+// for the other CTA (the tensor-memory reads of a consumed accumulator) is
+// ordered by tcgen05.fence::before_thread_sync, not by the memory model's
+// scope; a cluster-scope release would also wait for this thread's global
+// stores
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // 2-D tile load into this CTA's shared memory whose byte count completes on

@@ -45,12 +45,17 @@ def dev():
     return torch.device("cuda:0")
 
 
-def both_tiles(fn):
-    """fn() on one-CTA tiles, then on CTA pairs (the auto choice restored)."""
+PAIR_MODES = ["cta_pairs", "cta_pairs_narrow"]
+
+
+def both_tiles(fn, mode="cta_pairs"):
+    """fn() on one-CTA tiles, then on CTA pairs (256-column tiles, or with
+    mode "cta_pairs_narrow" 128-column tiles in the promoted passes whose B
+    operand is K-major); the auto choice is restored."""
     try:
         gm.gmm_set_tiles("one_cta")
         one = fn()
-        gm.gmm_set_tiles("cta_pairs")
+        gm.gmm_set_tiles(mode)
         pair = fn()
     finally:
         gm.gmm_set_tiles("auto")
@@ -66,13 +71,14 @@ def to_dev(inp, dev):
 @pytest.mark.parametrize("name", list(CASES))
 @pytest.mark.parametrize("rule", ["static", "dynamic"])
 @pytest.mark.parametrize("transpose", [False, True])
-def test_fwd_pairs(dev, name, rule, transpose):
+@pytest.mark.parametrize("mode", PAIR_MODES)
+def test_fwd_pairs(dev, mode, name, rule, transpose):
     inp = case_inputs(name)
     lhs, w, _, gs, s = to_dev(inp, dev)
     codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
     sarg = s if rule == "static" else None
     one, pair = both_tiles(lambda: gm.gmm_fwd(lhs, codes, scales, gs, rule=rule, static_scale=sarg,
-                                              transpose_rhs=transpose, out_dtype=torch.float32))
+                                              transpose_rhs=transpose, out_dtype=torch.float32), mode)
     qr, sr = oracle.quantize_rhs(inp.w)
     ref, ab = oracle.gmm_fwd(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
     assert_close(pair, ref, ab, f"pair fwd {name} {rule} t={transpose}")
@@ -81,12 +87,13 @@ def test_fwd_pairs(dev, name, rule, transpose):
 
 @pytest.mark.parametrize("name", list(CASES))
 @pytest.mark.parametrize("transpose", [False, True])
-def test_dlhs_pairs(dev, name, transpose):
+@pytest.mark.parametrize("mode", PAIR_MODES)
+def test_dlhs_pairs(dev, mode, name, transpose):
     inp = case_inputs(name)
     _, w, dout, gs, _ = to_dev(inp, dev)
     codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
     one, pair = both_tiles(lambda: gm.gmm_dlhs(dout, codes, scales, gs, transpose_rhs=transpose,
-                                               out_dtype=torch.bfloat16))
+                                               out_dtype=torch.bfloat16), mode)
     qr, sr = oracle.quantize_rhs(inp.w)
     ref, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
     assert_close(pair, ref, ab, f"pair dlhs {name} t={transpose}")
@@ -95,29 +102,31 @@ def test_dlhs_pairs(dev, name, transpose):
 
 @pytest.mark.parametrize("name", list(CASES))
 @pytest.mark.parametrize("rule", ["static", "dynamic"])
-def test_drhs_and_backward_pairs(dev, name, rule):
+@pytest.mark.parametrize("mode", PAIR_MODES)
+def test_drhs_and_backward_pairs(dev, mode, name, rule):
     inp = case_inputs(name)
     lhs, w, dout, gs, s = to_dev(inp, dev)
     sarg = s if rule == "static" else None
-    one, pair = both_tiles(lambda: gm.tgmm_drhs(lhs, dout, gs, rule=rule, static_scale=sarg))
+    one, pair = both_tiles(lambda: gm.tgmm_drhs(lhs, dout, gs, rule=rule, static_scale=sarg), mode)
     ref, ab = oracle.tgmm_drhs(inp.lhs, rule_code(rule), inp.static_scale, inp.dout, inp.group_sizes)
     assert_close(pair, ref, ab, f"pair drhs {name} {rule}")
     assert torch.equal(pair, one)
     codes, scales = gm.gmm_quantize_rhs(w)
     (d1, w1), (d2, w2) = both_tiles(lambda: gm.gmm_backward(lhs, dout, codes, scales, gs, rule=rule,
-                                                            static_scale=sarg))
+                                                            static_scale=sarg), mode)
     assert torch.equal(d1, d2) and torch.equal(w1, w2)
     assert torch.equal(w2, pair)
 
 
 @pytest.mark.parametrize("name", ["tiny", "odd_tiles", "unrouted"])
 @pytest.mark.parametrize("transpose", [False, True])
-def test_swiglu_pairs(dev, name, transpose):
+@pytest.mark.parametrize("mode", PAIR_MODES)
+def test_swiglu_pairs(dev, mode, name, transpose):
     inp = case_inputs(name)
     lhs, w, _, gs, s = to_dev(inp, dev)
     codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
     one, pair = both_tiles(lambda: gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule="dynamic",
-                                                     transpose_rhs=transpose, out_dtype=torch.float32))
+                                                     transpose_rhs=transpose, out_dtype=torch.float32), mode)
     qr, sr = oracle.quantize_rhs(inp.w)
     ref, terms = oracle.gmm_fwd_swiglu(inp.lhs, oracle.Q_DYNAMIC, inp.static_scale, qr, sr, inp.group_sizes)
     assert_within(pair, ref, swiglu_bound(torch.float32, terms, ref), f"pair swiglu {name}")
@@ -125,47 +134,50 @@ def test_swiglu_pairs(dev, name, transpose):
 
 
 @pytest.mark.parametrize("name", ["tiny", "odd_tiles"])
-def test_bf16_family_pairs(dev, name):
+@pytest.mark.parametrize("mode", PAIR_MODES)
+def test_bf16_family_pairs(dev, mode, name):
     inp = case_inputs(name)
     lhs, w, dout, gs, _ = to_dev(inp, dev)
     for tr in (False, True):
         wt = w.transpose(1, 2).contiguous() if tr else w
         one, pair = both_tiles(lambda: gm.gmm_fwd(lhs, wt, None, gs, rule="none", transpose_rhs=tr,
-                                                  out_dtype=torch.float32))
+                                                  out_dtype=torch.float32), mode)
         ref, ab = oracle.gmm_fwd_bf16(inp.lhs, inp.w, inp.group_sizes)
         assert_close(pair, ref, ab, f"pair bf16 fwd t={tr}")
         assert torch.equal(pair, one)
-    one, pair = both_tiles(lambda: gm.gmm_dlhs(dout, w, None, gs, rule="none", out_dtype=torch.float32))
+    one, pair = both_tiles(lambda: gm.gmm_dlhs(dout, w, None, gs, rule="none", out_dtype=torch.float32), mode)
     ref, ab = oracle.gmm_dlhs_bf16(inp.dout, inp.w, inp.group_sizes)
     assert_close(pair, ref, ab, "pair bf16 dlhs")
     assert torch.equal(pair, one)
-    one, pair = both_tiles(lambda: gm.tgmm_drhs(lhs, dout, gs, rule="none", out_dtype=torch.float32))
+    one, pair = both_tiles(lambda: gm.tgmm_drhs(lhs, dout, gs, rule="none", out_dtype=torch.float32), mode)
     ref, ab = oracle.tgmm_drhs_bf16(inp.lhs, inp.dout, inp.group_sizes)
     assert_close(pair, ref, ab, "pair bf16 drhs")
     assert torch.equal(pair, one)
 
 
 @pytest.mark.parametrize("rule", ["static", "dynamic"])
-def test_blockwise_pairs(dev, rule):
+@pytest.mark.parametrize("mode", PAIR_MODES)
+def test_blockwise_pairs(dev, mode, rule):
     inp = case_inputs("odd_tiles")
     lhs, w, dout, gs, s = to_dev(inp, dev)
     sarg = s if rule == "static" else None
     c0, s0 = gm.gmm_quantize_rhs_blocks(w, 0)
     c1, s1 = gm.gmm_quantize_rhs_blocks(w, 1)
     one, pair = both_tiles(lambda: gm.gmm_fwd(lhs, c0, s0, gs, rule=rule, static_scale=sarg,
-                                              out_dtype=torch.float32))
+                                              out_dtype=torch.float32), mode)
     qr0, sr0 = oracle.quantize_rhs_blocks(inp.w, 0)
     ref, ab = oracle.gmm_fwd_blockwise(inp.lhs, rule_code(rule), inp.static_scale, qr0, sr0, inp.group_sizes)
     assert_close(pair, ref, ab, f"pair blockwise fwd {rule}")
     assert torch.equal(pair, one)
-    one, pair = both_tiles(lambda: gm.gmm_dlhs(dout, c1, s1, gs, out_dtype=torch.float32))
+    one, pair = both_tiles(lambda: gm.gmm_dlhs(dout, c1, s1, gs, out_dtype=torch.float32), mode)
     qr1, sr1 = oracle.quantize_rhs_blocks(inp.w, 1)
     ref, ab = oracle.gmm_dlhs_blockwise(inp.dout, qr1, sr1, inp.group_sizes)
     assert_close(pair, ref, ab, "pair blockwise dlhs")
     assert torch.equal(pair, one)
 
 
-def test_pairs_status_clean_and_max_groups(dev):
+@pytest.mark.parametrize("mode", PAIR_MODES)
+def test_pairs_status_clean_and_max_groups(dev, mode):
     """Many groups, most empty, a few large: pair items span the group
     boundaries the pair prefix is built from (1024 groups, the maximum)."""
     G, M, K, N = 1024, 2000, 256, 256
@@ -176,7 +188,7 @@ def test_pairs_status_clean_and_max_groups(dev):
     codes, scales = gm.gmm_quantize_rhs(w)
     ws = torch.empty(gm.gmm_workspace_bytes(0, M, K, N, G), dtype=torch.uint8, device=dev)
     one, pair = both_tiles(lambda: gm.gmm_fwd(lhs, codes, scales, gs, rule="static", static_scale=s, ws=ws,
-                                              out_dtype=torch.float32))
+                                              out_dtype=torch.float32), mode)
     st, bits = gm.gmm_read_device_status(ws)
     assert st == 0, (st, bits)
     rows = [0, 3, 699, 700, 1212, 1213, 1812, 1813, 1999]
