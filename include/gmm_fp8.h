@@ -405,8 +405,9 @@ void gmm_set_wait_limit_ns(uint64_t limit_ns);
  *                           operand, the group's rows as 64 MMA columns;
  *   GMM_TILES_CTA_PAIRS_NARROW  CTA pairs, and the promoted E4M3 passes whose
  *                           weights or tgmm operand are K-major (dlhs with
- *                           transpose_rhs 0, the dynamic forward with
- *                           transpose_rhs 1, the tgmm) on 256 x 128 tiles:
+ *                           transpose_rhs 0, per channel or block-wise, the
+ *                           dynamic forward with transpose_rhs 1, the tgmm)
+ *                           on 256 x 128 tiles:
  *                           four 128-column tensor-memory accumulators per
  *                           SM instead of two of 256.
  * Any other value returns GMM_ERR_INVALID_ARG.  Not part of the pages: how a

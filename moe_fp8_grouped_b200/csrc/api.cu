@@ -504,7 +504,7 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
   const bool bmn = transpose_rhs != 0;  // [G, N, K]: K contiguous = MN-major B for dlhs
   const uint32_t bke = 128 / elem;
   const bool pairs = use_pairs(false, M, K, G);
-  const int tn = blk ? 256 : tile_cols(pairs, elem == 1, !bmn, false);
+  const int tn = tile_cols(pairs, elem == 1, !bmn, false);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, A, elem, N, M, N * elem, bke, 128)) return GMM_ERR_CUDA;
   const bool okB = bmn ? make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, bke)
@@ -575,6 +575,8 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   p.colblk_scale = (elem == 1 && dyn) ? P.scales_a : nullptr;
   p.colblk_ld = K;
   p.static_scale = (elem == 1 && !dyn) ? static_scale : nullptr;
+  // groups averaging under 512 rows: row tiles fastest (see GemmParams)
+  p.tg_rows_fastest = M < 512 * static_cast<int64_t>(G) ? 1 : 0;
   p.out = drhs;
   p.out_f32 = out_dtype == GMM_F32;
   p.ld_out = N;

@@ -194,14 +194,18 @@ __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const in
     t.rend = min(s_offs[g + 1], t.r0 + kBM);  // at or before r0: the pair's second half is past the group
     t.nblocks = p.kblocks;
   } else {
-    // items of group g: rtiles / kCta row tiles x tn column tiles, column
-    // tiles fastest (the group's lhs chunks stay in L2 across the row tiles);
-    // pairs need an even rtiles
-    const int per_g = (p.rtiles / kCta) * tn;
+    // items of group g: rtiles / kCta row tiles x tn column tiles; column
+    // tiles fastest (the group's dout chunk columns are reused by consecutive
+    // items), or row tiles fastest (its lhs chunk columns are: for small
+    // groups, whose many items would otherwise space the reuses of a lhs
+    // tile further apart than the dW stream lets it stay in L2); pairs need
+    // an even rtiles
+    const int rtp = p.rtiles / kCta;
+    const int per_g = rtp * tn;
     const int g = w / per_g, local = w % per_g;
     t.g = g;
-    t.rt = (local / tn) * kCta + rank;
-    t.ct = local % tn;
+    t.rt = (p.tg_rows_fastest ? local % rtp : local / tn) * kCta + rank;
+    t.ct = p.tg_rows_fastest ? local / rtp : local % tn;
     t.r0 = 0;
     t.rend = 0;
     t.nblocks = (s_tpre[g + 1] - s_tpre[g]) * p.stages_per_chunk;
@@ -848,6 +852,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t va[32], vb[32];
             tmem_ld64(tl + buf * kTN + colt(2 * cp), va, vb);
             tmem_wait_ld();
+            // 128-column tiles: the unit is in registers now; hand its TMEM
+            // buffer back before the promotion math
+            if constexpr (kCh == 2) release_unit(buf);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
               const uint32_t *vv = half ? vb : va;
@@ -879,7 +886,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          release_unit(buf);
+          if constexpr (kCh != 2) release_unit(buf);
           ++u;
           if (b + 1 < t.nblocks) release_slot(slot);  // the last slot is read again below
         }
@@ -1091,6 +1098,8 @@ static cudaError_t launch_cta(const GemmConfig &cfg, const CUtensorMap &tmA, con
         return launch_inst<1, false, true, MODE_ROWS, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
       if (cfg.mode == MODE_TGMM)
         return launch_inst<1, false, true, MODE_TGMM, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
+      if (cfg.mode == MODE_ROWS_BLK)
+        return launch_inst<1, false, true, MODE_ROWS_BLK, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
       return cudaErrorInvalidValue;
     }
   }

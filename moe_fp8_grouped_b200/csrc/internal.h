@@ -110,6 +110,9 @@ struct GemmParams {
   int swiglu_f;               // MODE_ROWS forward: F > 0 fuses SwiGLU over the merged
                               // columns [0, F) gate | [F, 2F) up and writes [M, F];
                               // 0 writes the plain product
+  int tg_rows_fastest;        // MODE_TGMM item order within a group: 1 = row tiles (dout
+                              // columns) fastest, each lhs column tile reused by
+                              // consecutive items; 0 = column tiles fastest
   int small_rows;             // MODE_ROWS, promoted E4M3, one-CTA tiles: groups of 1 ..
                               // small_rows (<= 64) rows take transposed tiles (the
                               // weights as the 128-row operand, the group's rows as
