@@ -53,7 +53,7 @@ def parse_args():
     ap.add_argument("--separate-backward", action="store_true",
                     help="run dlhs and drhs as two calls (gmm_dlhs, tgmm_drhs) instead of gmm_backward, which "
                          "quantizes dout once for both")
-    ap.add_argument("--tiles", default="auto", choices=["auto", "one_cta", "cta_pairs", "small_groups", "cta_pairs_narrow"],
+    ap.add_argument("--tiles", default="auto", choices=["auto", "one_cta", "cta_pairs", "cta_pairs_narrow"],
                     help="GEMM tile choice (gmm_set_tiles): automatic, 128-row tiles on one CTA, or 256-row tiles "
                          "over CTA pairs")
     ap.add_argument("--no-forward-shapes", dest="forward_shapes", action="store_false",

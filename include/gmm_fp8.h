@@ -392,34 +392,23 @@ void gmm_set_wait_limit_ns(uint64_t limit_ns);
  * testing knob: every tile gives the same results bit for bit, each output
  * being accumulated over the same contraction steps in the same order).
  *   GMM_TILES_AUTO          (default) the tile this library measured fastest
- *                           for the call's shape: 128-row tiles on one CTA;
- *   GMM_TILES_ONE_CTA       always 128-row tiles on one CTA;
- *   GMM_TILES_CTA_PAIRS     256-row tiles over a pair of CTAs (a two-CTA
+ *                           for the call's shape and pass;
+ *   GMM_TILES_ONE_CTA       128 x 256 tiles on one CTA;
+ *   GMM_TILES_CTA_PAIRS     256 x 256 tiles over a pair of CTAs (a two-CTA
  *                           cluster sharing each M = 256 tensor-core MMA;
  *                           the tgmm keeps one-CTA tiles when N is not a
  *                           multiple of 256);
- *   GMM_TILES_SMALL_GROUPS  one-CTA tiles, and in the promoted E4M3 forward
- *                           and dlhs (dynamic row scales, per-channel weight
- *                           scales, no SwiGLU) groups of at most 64 rows on
- *                           transposed tiles: the weights as the 128-row MMA
- *                           operand, the group's rows as 64 MMA columns;
  *   GMM_TILES_CTA_PAIRS_NARROW  CTA pairs, and the promoted E4M3 passes whose
  *                           weights or tgmm operand are K-major (dlhs with
  *                           transpose_rhs 0, per channel or block-wise, the
  *                           dynamic forward with transpose_rhs 1, the tgmm)
- *                           on 256 x 128 tiles:
- *                           four 128-column tensor-memory accumulators per
- *                           SM instead of two of 256.
+ *                           on 256 x 128 tiles: four 128-column
+ *                           tensor-memory accumulators per SM instead of two
+ *                           of 256.
  * Any other value returns GMM_ERR_INVALID_ARG.  Not part of the pages: how a
  * tile maps onto the B200's SMs is this library's choice.
  */
-enum {
-  GMM_TILES_AUTO = 0,
-  GMM_TILES_ONE_CTA = 1,
-  GMM_TILES_CTA_PAIRS = 2,
-  GMM_TILES_SMALL_GROUPS = 3,
-  GMM_TILES_CTA_PAIRS_NARROW = 4
-};
+enum { GMM_TILES_AUTO = 0, GMM_TILES_ONE_CTA = 1, GMM_TILES_CTA_PAIRS = 2, GMM_TILES_CTA_PAIRS_NARROW = 3 };
 gmm_status gmm_set_tiles(int32_t mode);
 
 /* Static text for a status code. */

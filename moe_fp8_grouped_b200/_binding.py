@@ -20,7 +20,7 @@ Q_NONE, Q_STATIC, Q_DYNAMIC = 0, 1, 2
 DT_BF16, DT_F32, DT_E4M3 = 0, 1, 2
 OP_FWD, OP_DLHS, OP_DRHS, OP_BWD = 0, 1, 2, 3
 DEV_GROUP_SIZES, DEV_SCALE, DEV_TIMEOUT = 1, 2, 4
-TILES_AUTO, TILES_ONE_CTA, TILES_CTA_PAIRS, TILES_SMALL_GROUPS, TILES_CTA_PAIRS_NARROW = 0, 1, 2, 3, 4
+TILES_AUTO, TILES_ONE_CTA, TILES_CTA_PAIRS, TILES_CTA_PAIRS_NARROW = 0, 1, 2, 3
 
 # every symbol include/gmm_fp8.h declares
 EXPORTS = ["gmm_workspace_bytes", "gmm_chunk_capacity", "gmm_quantize_rhs", "gmm_quantize", "gmm_fwd",

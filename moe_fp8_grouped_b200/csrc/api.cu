@@ -21,7 +21,7 @@ static constexpr bool kAutoPairs = false;  // the automatic choice takes one-CTA
 // 128-row tile count is odd); for the tgmm when its rows do too and its dout
 // columns split into 256-wide pair tiles.
 static bool use_pairs(bool tgmm, int64_t M, int64_t N, int32_t G) {
-  if (g_cta_pairs == GMM_TILES_ONE_CTA || g_cta_pairs == GMM_TILES_SMALL_GROUPS) return false;
+  if (g_cta_pairs == GMM_TILES_ONE_CTA) return false;
   if (tgmm && N % 256) return false;
   if (g_cta_pairs == GMM_TILES_CTA_PAIRS || g_cta_pairs == GMM_TILES_CTA_PAIRS_NARROW) return true;
   return kAutoPairs && M >= 512 * static_cast<int64_t>(G);
@@ -186,23 +186,11 @@ static gmm_status check_sizes(int64_t M, int64_t K, int64_t N, int32_t G) {
 
 static gmm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA; }
 
-// Groups of at most this many rows take transposed small-group tiles (the
-// weights as the 128-row MMA operand, the group's rows as 64 MMA columns) in
-// the promoted E4M3 row passes on one-CTA tiles.
-constexpr int kSmallGroupRows = 64;
-
-static constexpr bool kAutoSmall = false;  // the automatic choice takes plain 128-row tiles for small groups
-
-static bool use_small(bool pairs, bool promote_fp8) {
-  if (!promote_fp8 || pairs) return false;
-  return g_cta_pairs == GMM_TILES_SMALL_GROUPS || (kAutoSmall && g_cta_pairs == GMM_TILES_AUTO);
-}
-
 // Launch size of a row pass (forward, dlhs) over `cols` output columns: one CTA
 // per SM at most; for pairs the number of pair items (the launch caps it)
 static int row_pass_grid(bool pairs, int64_t M, int64_t cols, int32_t G, int tn = 256) {
   const int64_t rows = pairs ? 256 : 128;
-  const int64_t items = ((M + rows - 1) / rows + G) * ((cols + tn - 1) / tn) + static_cast<int64_t>(G) * (cols / 128);
+  const int64_t items = ((M + rows - 1) / rows + G) * ((cols + tn - 1) / tn);
   if (pairs) return static_cast<int>(items < INT_MAX ? items : INT_MAX);
   return static_cast<int>(items < num_sms() ? items : num_sms());
 }
@@ -294,7 +282,7 @@ void gmm_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns = limit_ns ? lim
 
 gmm_status gmm_set_tiles(int32_t mode) {
   if (mode != GMM_TILES_AUTO && mode != GMM_TILES_ONE_CTA && mode != GMM_TILES_CTA_PAIRS &&
-      mode != GMM_TILES_SMALL_GROUPS && mode != GMM_TILES_CTA_PAIRS_NARROW)
+      mode != GMM_TILES_CTA_PAIRS_NARROW)
     return GMM_ERR_INVALID_ARG;
   g_cta_pairs = mode;
   return GMM_OK;
@@ -427,18 +415,11 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
                        : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke,
                                   pairs ? tn / 2 : (F ? 128 : 256));
   if (!okB) return GMM_ERR_CUDA;
-  // small-group tiles: the weights as the 128-row operand (tmB itself when
-  // MN-major; a 128-row box of the K-major [G, N, K] weights otherwise)
-  const bool small = F == 0 && use_small(pairs, elem == 1 && dyn && !blk);
-  CUtensorMap tmW = tmB;
-  if (small && !bmn && !make_map(&tmW, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke, 128))
-    return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
   p.M = static_cast<int>(M);
   p.ncols = static_cast<int>(N);
   p.swiglu_f = static_cast<int>(F);
-  p.small_rows = small ? kSmallGroupRows : 0;
   p.kblocks = static_cast<int>(K / bke);
   p.b_group_rows = static_cast<int>(bmn ? K : N);
   p.offs = P.offs;
@@ -459,7 +440,7 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
                        blk ? 256 : tn};
   const int grid = row_pass_grid(pairs, M, N, G, cfg.tile_n);
   if ((s = cuda_status(prof(F ? "gemm_fwd_swiglu" : "gemm_fwd", st,
-                            [&] { return launch_gemm(cfg, tmA, tmB, tmA, tmW, p, grid, st); }))) != GMM_OK)
+                            [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }))) != GMM_OK)
     return s;
   g_launches = n + 1;
   return GMM_OK;
@@ -511,15 +492,10 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
                        : make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke,
                                   pairs ? tn / 2 : 256);
   if (!okB) return GMM_ERR_CUDA;
-  const bool small = use_small(pairs, elem == 1 && !blk);
-  CUtensorMap tmW = tmB;  // MN-major [G, N, K]: the 128 x 128 box of tmB
-  if (small && !bmn && !make_map(&tmW, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, 128))
-    return GMM_ERR_CUDA;
   GemmParams p{};
   p.G = G;
   p.M = static_cast<int>(M);
   p.ncols = static_cast<int>(K);
-  p.small_rows = small ? kSmallGroupRows : 0;
   p.kblocks = static_cast<int>(N / bke);
   p.b_group_rows = static_cast<int>(bmn ? N : K);
   p.offs = P.offs;
@@ -537,7 +513,7 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
   p.wait_limit_ns = g_wait_limit_ns;
   const GemmConfig cfg{blk ? MODE_ROWS_BLK : MODE_ROWS, elem, bmn, elem == 1, pairs, tn};
   const int grid = row_pass_grid(pairs, M, K, G, tn);
-  return cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, tmW, p, grid, st); }));
+  return cuda_status(prof("gemm_dlhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmA, p, grid, st); }));
 }
 
 // tgmm GEMM on the chunk-major operands in the workspace (codes_a: lhs,
@@ -586,7 +562,7 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   const int64_t items = static_cast<int64_t>(G) * (N / (pairs ? 2 * kBlk : kBlk)) * ((K + tn - 1) / tn);
   const int grid = pairs ? static_cast<int>(items < INT_MAX ? items : INT_MAX)
                          : static_cast<int>(items < num_sms() ? items : num_sms());
-  return cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, tmB, p, grid, st); }));
+  return cuda_status(prof("gemm_drhs", st, [&] { return launch_gemm(cfg, tmA, tmB, tmOut, p, grid, st); }));
 }
 
 // The tgmm lhs operand into the workspace: quantized per chunk, re-laid out

@@ -34,6 +34,9 @@
 //                     epilogue accumulates acc += unit * row_scale (* the
 //                     block's column scale for dynamic-lhs tgmm) in registers.
 //
+// The same GEMM on tiles shared by a pair of CTAs (tcgen05 cta_group::2) is
+// gemm_pair.cu; launch_gemm dispatches to it for GemmConfig::cta_pairs.
+//
 // SwiGLU (forward only, p.swiglu_f = F > 0): the rhs holds the gate and up
 // weights side by side, W = [W0 | W1] along N = 2F ("FP8 Megablox for batch
 // split", maxtext PR #3770, Description (2): the merged gating gmm).  A tile
@@ -57,7 +60,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 256;
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 8;    // ring of per-unit scale slots (scale loader -> epilogue)
-constexpr int kNumBars = 48;      // mbarriers reserved in shared memory
+constexpr int kNumBars = 32;      // mbarriers reserved in shared memory
 // Register split (setmaxnreg): the control warpgroup gives registers to the
 // two epilogue warpgroups.  Sum must not exceed the launch allocation
 // (registers per thread at launch x 384); launch_inst checks it.
@@ -68,144 +71,77 @@ constexpr int regs_ctl() { return kPromote ? 40 : 72; }
 template <bool kPromote>
 constexpr int regs_epi() { return kPromote ? 232 : 216; }
 
-// Pipeline stages.  One CTA: A 16 KB + B 32 KB per stage, 4 stages (tgmm: 3,
-// the freed shared memory stages its output for TMA stores, one 4 KB block
-// per epilogue warp).  A CTA pair (kCta = 2): each CTA holds its 128 rows of A
-// and half of B: 16 KB + 16 KB with 256-column tiles, 6 stages (tgmm: 4);
-// 16 KB + 8 KB with 128-column tiles (kTN = 128), 8 stages (tgmm: 5).
-template <int kCta, int kMode, int kTN = 256>
-constexpr int stages_of() {
-  return kCta == 2 ? (kTN == 128 ? (kMode == MODE_TGMM ? 5 : 8) : (kMode == MODE_TGMM ? 4 : 6))
-                   : (kMode == MODE_TGMM ? 3 : kStages);
-}
+// tgmm keeps 3 pipeline stages and uses the freed shared memory to stage its
+// output for TMA stores (one 4 KB block per epilogue warp)
+template <int kMode>
+constexpr int stages_of() { return kMode == MODE_TGMM ? 3 : kStages; }
 constexpr int kStageOut = 4096;  // bytes of one output staging buffer (tgmm); two per epilogue warp
 
 // scale ring slots: tgmm keeps 4 to make room for its output staging
 template <int kMode>
 constexpr int ring_of() { return kMode == MODE_TGMM ? 4 : kScaleSlots; }
 
-// int arrays [kMaxGroups + 1] in shared memory: group offsets, 128-row tile
-// prefix, and (CTA pairs or row passes) the item prefix of pair tiles or of
-// small-group tiles
-template <int kCta, int kMode>
-constexpr int plan_arrays() { return (kCta == 2 || kMode != MODE_TGMM) ? 3 : 2; }
-
-template <int kCta, int kMode, int kTN = 256>
+template <int kMode>
 constexpr size_t gemm_smem_bytes() {
   return 1024                                    // alignment slack
-         + static_cast<size_t>(stages_of<kCta, kMode, kTN>()) * (kAStage + (kTN * 128) / kCta)
+         + static_cast<size_t>(stages_of<kMode>()) * (kAStage + kBStage)
          + kNumBars * 8                          // mbarriers
          + 16                                    // tmem slot, abort flags
          + ring_of<kMode>() * (kBN + kBM) * sizeof(float)  // scale ring
-         + plan_arrays<kCta, kMode>() * (kMaxGroups + 1) * sizeof(int)  // plan copy, item prefix
+         + 2 * (kMaxGroups + 1) * sizeof(int)    // plan copy
          + (kMode == MODE_TGMM ? 128 + kEpiWarps * 2 * kStageOut : 0);  // + alignment slack
 }
-static_assert(gemm_smem_bytes<2, MODE_ROWS>() <= 232448, "pair-tile shared memory");
-static_assert(gemm_smem_bytes<2, MODE_TGMM>() <= 232448, "pair-tile tgmm shared memory");
-static_assert(gemm_smem_bytes<1, MODE_ROWS>() <= 232448, "shared memory");
-static_assert(gemm_smem_bytes<1, MODE_TGMM>() <= 232448, "tgmm shared memory");
-static_assert(gemm_smem_bytes<1, MODE_ROWS>() == gemm_smem_bytes<1, MODE_ROWS_BLK>(), "row-pass shared memory");
-static_assert(gemm_smem_bytes<2, MODE_ROWS, 128>() <= 232448, "narrow pair-tile shared memory");
-static_assert(gemm_smem_bytes<2, MODE_TGMM, 128>() <= 232448, "narrow pair-tile tgmm shared memory");
 
 // One work item: tile row index rt (MODE_ROWS: rows r0 .. rend of group g;
 // MODE_TGMM: dout columns 128 rt ..), tile column index ct, and the number of
 // contraction stages.
 struct Item {
   int g, rt, ct, nblocks, r0, rend;
-  bool small;  // transposed small-group tile: output columns 128 ct .. as TMEM lanes,
-               // the group's rows r0 .. rend (at most 64) as TMEM columns
 };
 
-// Small-group tiles: M = 128 output columns (TMEM lanes), N = 64 rows of the
-// group (TMEM columns), 128-long contraction blocks.  kSmallStack consecutive
-// blocks share one 256-column TMEM unit, one 64-column slice each, so that a
-// unit carries as much MMA and promotion work as a 128 x 256 unit (and four
-// times the weight bytes of one block).
-constexpr int kSmallN = 64;
-constexpr int kSmallCols = 128;
-constexpr int kSmallStack = 256 / kSmallN;
-
-// Column of the (2-D view of the) rhs held by tile column c (0 .. tn - 1) of
-// column tile ct: plain tiles are tn (256 or 128) consecutive columns; SwiGLU
-// tiles (256 wide) are gate columns 128 ct .. 128 ct + 127, then up columns
-// F + 128 ct ..
-__device__ __forceinline__ int tile_col_n(int ct, int c, int F, int tn = kBN) {
-  return F ? (c < 128 ? 128 * ct + c : F + 128 * ct + (c - 128)) : tn * ct + c;
+// Column of the (2-D view of the) rhs held by tile column c (0 .. 255) of
+// column tile ct: plain tiles are 256 consecutive columns; SwiGLU tiles are
+// gate columns 128 ct .. 128 ct + 127, then up columns F + 128 ct ..
+__device__ __forceinline__ int tile_col_n(int ct, int c, int F) {
+  return F ? (c < 128 ? 128 * ct + c : F + 128 * ct + (c - 128)) : kBN * ct + c;
 }
 
 // x * sigmoid(x); -0 for large negative x, where exp(-x) overflows
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 
-// A CTA pair (kCta = 2) takes one item of twice the rows: rank r of the pair
-// holds tile rows 128 r .. 128 r + 127 of it.
-// small == true (one-CTA row passes with p.small_rows > 0): s_ppre holds the
-// prefix of items per group, tn column tiles per 128-row tile for ordinary
-// groups, ncols / 128 transposed tiles for groups of 1 .. p.small_rows rows.
-template <int kMode, int kCta>
+template <int kMode>
 __device__ __forceinline__ Item decode_item(int w, const GemmParams &p, const int *s_offs, const int *s_tpre,
-                                            const int *s_ppre, int tn, int rank, bool small) {
+                                            int tn) {
   Item t;
-  t.small = false;
   if constexpr (kMode != MODE_TGMM) {
-    if (kCta == 1 && small) {
-      int lo = 0, hi = p.G + 1;  // first i with s_ppre[i] > w
-      while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if (s_ppre[mid] > w) hi = mid;
-        else lo = mid + 1;
-      }
-      const int g = lo - 1;
-      const int local = w - s_ppre[g];
-      const int size = s_offs[g + 1] - s_offs[g];
-      t.g = g;
-      t.nblocks = p.kblocks;
-      if (size > 0 && size <= p.small_rows) {
-        t.small = true;
-        t.rt = 0;
-        t.ct = local;  // 128-column tile
-        t.r0 = s_offs[g];
-        t.rend = s_offs[g + 1];
-      } else {
-        const int mt_g = s_tpre[g + 1] - s_tpre[g];
-        t.rt = local % mt_g;
-        t.ct = local / mt_g;
-        t.r0 = s_offs[g] + kBM * t.rt;
-        t.rend = min(s_offs[g + 1], t.r0 + kBM);
-      }
-      return t;
-    }
-    // items of group g: (pre[g+1] - pre[g]) row tiles (128 rows, or 256 for a
-    // pair) x tn column tiles, row tiles fastest
-    const int *pre = kCta == 2 ? s_ppre : s_tpre;
-    int lo = 0, hi = p.G + 1;  // first i with pre[i] * tn > w
+    // items of group g: (tpre[g+1] - tpre[g]) row tiles x tn column tiles,
+    // row tiles fastest
+    int lo = 0, hi = p.G + 1;  // first i with tpre[i] * tn > w
     while (lo < hi) {
       int mid = (lo + hi) >> 1;
-      if (pre[mid] * tn > w) hi = mid;
+      if (s_tpre[mid] * tn > w) hi = mid;
       else lo = mid + 1;
     }
     const int g = lo - 1;
-    const int mt_g = pre[g + 1] - pre[g];
-    const int local = w - pre[g] * tn;
+    const int mt_g = s_tpre[g + 1] - s_tpre[g];
+    const int local = w - s_tpre[g] * tn;
     t.g = g;
     t.rt = local % mt_g;
     t.ct = local / mt_g;
-    t.r0 = s_offs[g] + kCta * kBM * t.rt + kBM * rank;
-    t.rend = min(s_offs[g + 1], t.r0 + kBM);  // at or before r0: the pair's second half is past the group
+    t.r0 = s_offs[g] + kBM * t.rt;
+    t.rend = min(s_offs[g + 1], t.r0 + kBM);
     t.nblocks = p.kblocks;
   } else {
-    // items of group g: rtiles / kCta row tiles x tn column tiles; column
-    // tiles fastest (the group's dout chunk columns are reused by consecutive
+    // items of group g: rtiles row tiles x tn column tiles; column tiles
+    // fastest (the group's dout chunk columns are reused by consecutive
     // items), or row tiles fastest (its lhs chunk columns are: for small
     // groups, whose many items would otherwise space the reuses of a lhs
-    // tile further apart than the dW stream lets it stay in L2); pairs need
-    // an even rtiles
-    const int rtp = p.rtiles / kCta;
-    const int per_g = rtp * tn;
+    // tile further apart than the dW stream lets it stay in L2)
+    const int per_g = p.rtiles * tn;
     const int g = w / per_g, local = w % per_g;
     t.g = g;
-    t.rt = (p.tg_rows_fastest ? local % rtp : local / tn) * kCta + rank;
-    t.ct = p.tg_rows_fastest ? local / rtp : local % tn;
+    t.rt = p.tg_rows_fastest ? local % p.rtiles : local / tn;
+    t.ct = p.tg_rows_fastest ? local / p.rtiles : local % tn;
     t.r0 = 0;
     t.rend = 0;
     t.nblocks = (s_tpre[g + 1] - s_tpre[g]) * p.stages_per_chunk;
@@ -275,46 +211,30 @@ __device__ __forceinline__ void store_col32(void *out, int64_t off_elems, int64_
   }
 }
 
-// kCta = 2: the kernel runs as clusters of two CTAs (a pair) that share each
-// M = 256 MMA (tcgen05 cta_group::2): rank r holds rows 128 r .. of every
-// item's A tile and columns 128 r .. 128 r + 127 of its B tile, and receives
-// its 128 rows of the accumulator.  Rank 0 issues the MMAs.  Halving B per SM
-// halves the shared-memory traffic per MMA (TMA writes plus tensor-core
-// reads), which bounds the one-CTA tile.
-// kTN: tile columns, 256, or 128 for CTA pairs in the promoted passes with a
-// K-major B (four 128-column TMEM buffers instead of two of 256: the MMA can
-// run three units ahead of the epilogue).
-template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta, bool kSmall, int kTN>
+template <int kElem, bool kBMN, bool kPromote, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     gmm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmW,
-                  const GemmParams p) {
+                  const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   constexpr bool kF16 = (kElem == 2);
   constexpr bool kTg = (kMode == MODE_TGMM);
-  constexpr bool kPair = (kCta == 2);
   constexpr int kBKe = 128 / kElem;                 // contraction elements per stage
   constexpr int kMmaK = 32 / kElem;                 // contraction elements per MMA
-  static_assert(kTN == 256 || (kTN == 128 && kPair && kPromote && !kBMN), "128-column tiles: pairs, promoted, K-major B");
-  constexpr int kBS = (kTN * 128) / kCta;           // bytes of B per CTA per stage
-  constexpr int kBBoxes = kBMN ? (2 / kCta) * kElem : 1;  // TMA boxes per B stage (128-byte wide if MN-major)
-  constexpr int kBBoxBytes = kBS / kBBoxes;
-  constexpr uint32_t kIdesc = instr_desc_mn(kF16, false, kBMN, kTN, kPair ? 256u : 128u);
-  constexpr int kSt = stages_of<kCta, kMode, kTN>();
-  constexpr int kNB = kTmemCols / kTN;              // TMEM accumulator buffers
-  constexpr int kCh = kTN / 64;                     // 32-column chunks per epilogue thread
+  constexpr int kBBoxes = kBMN ? 2 * kElem : 1;     // TMA boxes per B stage
+  constexpr int kBBoxBytes = kBStage / kBBoxes;
+  constexpr uint32_t kIdesc = instr_desc(kF16, kBMN);
+  constexpr int kSt = stages_of<kMode>();
   constexpr int kRing = ring_of<kMode>();
-  constexpr uint32_t kStageTx = kCta * (kAStage + kBS);  // bytes completing one stage (both CTAs)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + kSt * kAStage;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kSt * kBS);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kSt * kBStage);
   uint64_t *full = bars;                    // [kSt] TMA -> MMA
   uint64_t *empty = bars + kSt;         // [kSt] MMA -> TMA
-  uint64_t *tfull = bars + 2 * kSt;     // [kNB] MMA -> epilogue
-  uint64_t *tempty = tfull + kNB;           // [kNB] epilogue -> MMA
-  uint64_t *drain = tempty + kNB;           // MMA completion at exit
+  uint64_t *tfull = bars + 2 * kSt;     // [2] MMA -> epilogue
+  uint64_t *tempty = tfull + 2;             // [2] epilogue -> MMA
+  uint64_t *drain = tempty + 2;             // MMA completion at exit
   uint64_t *sfull = drain + 1;              // [kRing] scale loader -> epilogue
   uint64_t *sempty = sfull + kRing;   // [kRing] epilogue -> scale loader
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
@@ -324,25 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *s_srow = s_scol + kRing * kBN;                // [kRing][128] row scales per unit
   int *s_offs = reinterpret_cast<int *>(s_srow + kRing * kBM);
   int *s_tpre = s_offs + (kMaxGroups + 1);
-  // item prefix per group: 256-row pair tiles (kPair, row passes) or
-  // ordinary and small-group items (one CTA, small tiles on)
-  int *s_ppre = s_tpre + (kMaxGroups + 1);
   // tgmm output staging, 128-byte aligned (TMA store sources must be aligned)
-  uint8_t *s_stage_out = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(s_offs + plan_arrays<kCta, kMode>() * (kMaxGroups + 1)) + 127) & ~uintptr_t(127));
-  // transposed tiles for small groups: one-CTA promoted E4M3 row passes, in
-  // their own instantiation (kSmall) so that the other kernels carry none of
-  // their code or registers
-  constexpr bool kSmallOk = kSmall;
-  static_assert(!kSmall || (kCta == 1 && kMode == MODE_ROWS && kElem == 1 && kPromote), "small-group tiles");
-  const bool small_on = kSmallOk && p.small_rows > 0;
+  uint8_t *s_stage_out =
+      reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(s_tpre + (kMaxGroups + 1)) + 127) & ~uintptr_t(127));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rank = kPair ? static_cast<int>(cluster_ctarank()) : 0;
-  const bool leader = rank == 0;
-  // items: one per CTA, or one per pair (consecutive blockIdx.x form a cluster)
-  const int w0 = kPair ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
-  const int wstep = kPair ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
 
   // Which scales each TMEM unit carries (the same decision in every role):
   //   column scales: forward s_r[g, n] (every unit of a tile, applied at the
@@ -363,9 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < kNB; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], kCta * kEpiWarps);  // a pair: the epilogue warps of both CTAs arrive on rank 0's
+      mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
     for (int i = 0; i < kRing; ++i) {
@@ -379,67 +285,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (small_on) tma_prefetch_desc(&tmW);
-  }
-  if constexpr (kPair) {
-    // the other CTA's barriers are used (remote arrivals, byte counts,
-    // multicast commits) only after both CTAs initialized theirs
-    cluster_sync();
   }
   if (warp == 1) {
-    if constexpr (kPair) {
-      tmem_alloc_pair(tmem_slot, kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
   }
   for (int i = threadIdx.x; i <= p.G; i += kThreads) {
     s_offs[i] = p.offs[i];
     s_tpre[i] = p.tpre[i];
-  }
-  const int tn = (p.ncols + kTN - 1) / kTN;
-  if ((kPair && !kTg) || small_on) {
-    __syncthreads();
-    if (warp == 2) {
-      // items per group: pair tiles, ceil(row tiles / 2) x tn; or tn per row
-      // tile, ncols / 128 for a small group.  Lane l scans groups
-      // [l * per, (l + 1) * per), then the lane totals are scanned across the warp
-      auto items_of = [&](int g) -> int {
-        const int mt = s_tpre[g + 1] - s_tpre[g];
-        if (kPair) return (mt + 1) >> 1;  // multiplied by tn where decoded
-        const int size = s_offs[g + 1] - s_offs[g];
-        return (size > 0 && size <= p.small_rows) ? p.ncols / kSmallCols : mt * tn;
-      };
-      const int per = (p.G + 31) / 32;
-      const int g0 = min(lane * per, p.G), g1 = min(g0 + per, p.G);
-      int sum = 0;
-      for (int g = g0; g < g1; ++g) sum += items_of(g);
-      int incl = sum;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
-      }
-      int run = incl - sum;
-      for (int g = g0; g < g1; ++g) {
-        s_ppre[g] = run;
-        run += items_of(g);
-      }
-      if (lane == 31) s_ppre[p.G] = incl;
-    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  const int total = kTg ? p.G * (p.rtiles / kCta) * tn
-                        : (small_on ? s_ppre[p.G] : (kPair ? s_ppre[p.G] : s_tpre[p.G]) * tn);
-  // rank 0's barriers as shared::cluster addresses (a pair's shared barriers)
-  const uint32_t full0_cl = kPair ? mapa_shared(smem_u32(full), 0) : 0;
-  const uint32_t tempty0_cl = kPair ? mapa_shared(smem_u32(tempty), 0) : 0;
+  const int tn = (p.ncols + kBN - 1) / kBN;
+  const int total = kTg ? p.G * p.rtiles * tn : s_tpre[p.G] * tn;
   const WaitCtl ctl{p.wait_limit_ns, abort_flag, p.status};
   const WaitCtl ctl_drain{p.wait_limit_ns, no_abort, p.status};
 
@@ -449,41 +310,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------- TMA producer
       int it = 0;
       bool ok = true;
-      // a pair's loads complete on rank 0's full barrier, which rank 0 arms
-      // with both CTAs' bytes
-      auto load = [&](void *dst, const CUtensorMap *map, int x, int y, int s) {
-        if constexpr (kPair) tma_load_2d_pair(dst, map, x, y, full0_cl + 8u * s);
-        else tma_load_2d(dst, map, x, y, &full[s]);
-      };
-      for (int w = w0; ok && w < total; w += wstep) {
-        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
+      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+        const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
         for (int b = 0; b < t.nblocks; ++b, ++it) {
           const int s = it % kSt;
           if (!mbar_wait(&empty[s], ((it / kSt) & 1) ^ 1, ctl)) {
             ok = false;
             break;
           }
-          if (kSmallOk && t.small) {
-            // weights (the 128 output columns as rows) into the A slot, the
-            // group's rows (a 128-row box, the first kSmallN used) into the B slot
-            mbar_arrive_expect_tx(&full[s], 2 * kAStage);
-            const int wo = t.g * p.b_group_rows;
-            if constexpr (kBMN) load(sA + s * kAStage, &tmW, t.ct * kSmallCols, wo + b * kBKe, s);
-            else load(sA + s * kAStage, &tmW, b * kBKe, wo + t.ct * kSmallCols, s);
-            load(sB + s * kBS, &tmA, b * kBKe, t.r0, s);
-            continue;
-          }
-          if (leader) mbar_arrive_expect_tx(&full[s], kStageTx);
+          mbar_arrive_expect_tx(&full[s], kAStage + kBStage);
           int ax, ay, bx, by;
           if constexpr (!kTg) {
             ax = b * kBKe;
             ay = t.r0;
             if (kBMN) {
-              bx = t.ct * kTN;
+              bx = t.ct * kBN;
               by = t.g * p.b_group_rows + b * kBKe;
             } else {
               bx = b * kBKe;
-              by = t.g * p.b_group_rows + t.ct * kTN + (kTN / kCta) * rank;
+              by = t.g * p.b_group_rows + t.ct * kBN;
             }
           } else {
             // chunk jj of the group (stages_per_chunk stages each) in the
@@ -492,49 +337,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             ax = (b % p.stages_per_chunk) * kBKe;
             ay = jj * (p.rtiles * kBM) + t.rt * kBM;  // dout columns n
             bx = ax;
-            by = jj * p.ncols + t.ct * kTN + (kTN / kCta) * rank;  // lhs columns k (rows past K belong
-                                                      // to the next chunk: their columns are never stored)
+            by = jj * p.ncols + t.ct * kBN;           // lhs columns k (rows past K belong to the
+                                                      // next chunk: their columns are never stored)
           }
-          load(sA + s * kAStage, &tmA, ax, ay, s);
+          tma_load_2d(sA + s * kAStage, &tmA, ax, ay, &full[s]);
           if constexpr (kBMN) {
-            // boxes of 128 bytes along n (columns of W[g] in [K, N]); a pair
-            // CTA takes tile columns 128 rank ..
+            // boxes of 128 bytes along n (columns of W[g] in [K, N])
 #pragma unroll
             for (int h = 0; h < kBBoxes; ++h)
-              load(sB + s * kBS + h * kBBoxBytes, &tmB,
-                   tile_col_n(t.ct, (kTN / kCta) * rank + h * kBKe, p.swiglu_f, kTN), by, s);
+              tma_load_2d(sB + s * kBStage + h * kBBoxBytes, &tmB, tile_col_n(t.ct, h * kBKe, p.swiglu_f), by,
+                          &full[s]);
           } else if (!kTg && p.swiglu_f) {
-            // boxes of 128 rows (n) of W[g] in [N, K]: gate rows, up rows (a
-            // pair CTA loads one of them)
+            // two boxes of 128 rows (n) of W[g] in [N, K]: gate rows, up rows
 #pragma unroll
-            for (int h = 0; h < 2 / kCta; ++h)
-              load(sB + s * kBS + h * (kBStage / 2), &tmB, bx,
-                   t.g * p.b_group_rows + tile_col_n(t.ct, (h + rank) * 128, p.swiglu_f), s);
+            for (int h = 0; h < 2; ++h)
+              tma_load_2d(sB + s * kBStage + h * (kBStage / 2), &tmB, bx,
+                          t.g * p.b_group_rows + tile_col_n(t.ct, h * 128, p.swiglu_f), &full[s]);
           } else {
-            load(sB + s * kBS, &tmB, bx, by, s);
+            tma_load_2d(sB + s * kBStage, &tmB, bx, by, &full[s]);
           }
         }
       }
-      // let every issued copy land before the CTA can exit.  A pair's copies
-      // complete on rank 0's barriers, so rank 0 waits for both CTAs' copies;
-      // rank 1 leaves only after the closing cluster barrier, which rank 0
-      // reaches after this wait.
-      if (leader)
-        for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
-          mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
+      // let every issued copy land before the CTA can exit
+      for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
+        mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
     } else if (warp == 1) {
       // ----------------------------------------------------- MMA issuer
-      if (lane == 0 && leader) {
+      if (lane == 0) {
         int it = 0, u = 0;
         bool ok = true;
-        for (int w = w0; ok && w < total; w += wstep) {
-          const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
+        for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+          const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
-            const bool unit_start = (kSmallOk && t.small) ? (b % kSmallStack == 0) : (kPromote || b == 0);
+            const bool unit_start = kPromote || b == 0;
             if (unit_start) {
-              buf = u % kNB;
-              if (!mbar_wait(&tempty[buf], ((u / kNB) & 1) ^ 1, ctl)) {
+              buf = u & 1;
+              if (!mbar_wait(&tempty[buf], ((u >> 1) & 1) ^ 1, ctl)) {
                 ok = false;
                 break;
               }
@@ -546,50 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBS);
-            const uint32_t d = tbase + buf * kTN;
-            if (kSmallOk && t.small) {
-              // A: the weight tile, 128 output columns x 128 contraction (the
-              // major-ness of the weights in memory); B: kSmallN rows, K-major.
-              // Block b fills slice b % kSmallStack of the unit.
-              constexpr uint32_t kIdescSmall = instr_desc_mn(kF16, kBMN, false, kSmallN, 128u);
-              const uint32_t ds = d + (b % kSmallStack) * kSmallN;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t adesc = kBMN ? smem_desc_sw128(a0 + kk * kMmaK * 128, kAStage, 1024)
-                                            : smem_desc_sw128(a0 + kk * 32, 16, 1024);
-                const uint64_t bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-                tc_mma<kF16>(ds, adesc, bdesc, kIdescSmall, kk == 0 ? 0u : 1u);
-              }
-              tc_commit(&empty[s]);
-              if (b % kSmallStack == kSmallStack - 1 || b == t.nblocks - 1) {
-                tc_commit(&tfull[buf]);
-                ++u;
-              }
-              continue;
-            }
+            const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBStage);
+            const uint32_t d = tbase + buf * kBN;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
               const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
                                           : smem_desc_sw128(b0 + kk * 32, 16, 1024);
-              // a pair's descriptors name rank 0's shared memory; the tensor
-              // core reads the same offsets in rank 1 for its half
-              if constexpr (kPair) tc_mma_pair<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
-              else tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
+              tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
             }
-            // stage s free again / TMEM unit ready: in both CTAs of a pair
-            if constexpr (kPair) tc_commit_pair_both(&empty[s], 0x3);
-            else tc_commit(&empty[s]);
+            tc_commit(&empty[s]);
             if (kPromote || b == t.nblocks - 1) {
-              if constexpr (kPair) tc_commit_pair_both(&tfull[buf], 0x3);
-              else tc_commit(&tfull[buf]);
+              tc_commit(&tfull[buf]);
               ++u;
             }
           }
         }
-        if constexpr (kPair) tc_commit_pair_local(drain);
-        else tc_commit(drain);
+        tc_commit(drain);
         mbar_wait(drain, 0, ctl_drain);
       }
       __syncwarp();
@@ -599,10 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // them, so that no global-memory latency sits on the epilogue's path.
       int v = 0;
       bool ok = true;
-      for (int w = w0; ok && w < total; w += wstep) {
-        const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
-        const int units = (kSmallOk && t.small) ? (t.nblocks + kSmallStack - 1) / kSmallStack
-                                                : (kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0));
+      for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+        const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+        const int units = kPromote ? t.nblocks : (t.nblocks > 0 ? 1 : 0);
         const int64_t ch0 = kTg ? s_tpre[t.g] : 0;
         for (int j = 0; j < units; ++j, ++v) {
           const int slot = v % kRing;
@@ -614,40 +425,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // cp.async straight into the slot: the loader never waits for the
           // data, the slot's barrier completes when all 32 lanes' copies land
-          if (kSmallOk && t.small) {
-            // the group's row scales of the unit's blocks (slice s: 64 TMEM
-            // columns, 2 per lane) and the per-channel weight scales of the
-            // 128 output columns (TMEM lanes, applied at the end)
-            const int64_t last = p.M - 1;
-            const int64_t r = static_cast<int64_t>(t.r0) + 2 * lane;
-#pragma unroll
-            for (int sl = 0; sl < kSmallStack; ++sl) {
-              const int b = j * kSmallStack + sl;
-              if (b >= t.nblocks) break;
-              const float *src = p.row_scale + static_cast<int64_t>(b) * p.row_scale_ld;
-              float *dc = s_scol + slot * kBN + sl * kSmallN + 2 * lane;
-              cp_async_4(dc, src + min(r, last));
-              cp_async_4(dc + 1, src + min(r + 1, last));
-            }
-            if (p.col_scale)
-              cp_async_16(s_srow + slot * kBM + 4 * lane,
-                          p.col_scale + static_cast<int64_t>(t.g) * p.ncols + t.ct * kSmallCols + 4 * lane);
-            cp_async_mbar_arrive(&sfull[slot]);
-            continue;
-          }
           if (need_col) {
-            // kTN / 32 columns per lane (never straddling a gate / up
-            // boundary); columns >= ncols are never read
-            constexpr int kCpl = kTN / 32;
-            const int n = kTg ? t.ct * kTN + kCpl * lane : tile_col_n(t.ct, kCpl * lane, p.swiglu_f, kTN);
+            // 8 columns per lane (never straddling a gate / up boundary);
+            // columns >= ncols are never read
+            const int n = kTg ? t.ct * kBN + 8 * lane : tile_col_n(t.ct, 8 * lane, p.swiglu_f);
             if (n < p.ncols) {
               const float *src =
                   kTg ? p.colblk_scale + (ch0 + j) * p.colblk_ld + n
                       : (kBlkScales ? p.colblk_scale + (static_cast<int64_t>(t.g) * p.kblocks + j) * p.colblk_ld + n
                               : p.col_scale + static_cast<int64_t>(t.g) * p.ncols + n);
-              float *dst = s_scol + slot * kBN + kCpl * lane;
-#pragma unroll
-              for (int e = 0; e < kCpl; e += 4) cp_async_16(dst + e, src + e);
+              float *dst = s_scol + slot * kBN + 8 * lane;
+              cp_async_16(dst, src);
+              cp_async_16(dst + 4, src + 4);
             }
           }
           if (need_row) {
@@ -678,9 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile column of the thread's 32-column chunk c (0 .. 3): the column half h
     // of the tile, or for SwiGLU gate columns 64 h .. (c = 0, 1) and the
     // matching up columns 128 + 64 h .. (c = 2, 3)
-    auto colt = [&](int c) -> int {
-      return sw ? ((c & 2) ? 128 : 0) + h * 64 + (c & 1) * 32 : h * (kTN / 2) + c * 32;
-    };
+    auto colt = [&](int c) -> int { return sw ? ((c & 2) ? 128 : 0) + h * 64 + (c & 1) * 32 : h * 128 + c * 32; };
     float s_eff = 1.0f;
     if (p.static_scale) {
       const float v = *p.static_scale;
@@ -699,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // abort flag, which ends every other warp's next wait, and no barrier
     // among the epilogue warps is ever entered after that point.
     auto wait_unit = [&](uint32_t buf, int slot) -> bool {
-      bool got = mbar_wait(&tfull[buf], (u / kNB) & 1, ctl);
+      bool got = mbar_wait(&tfull[buf], (u >> 1) & 1, ctl);
       if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kRing) & 1, ctl);
       return __all_sync(0xffffffffu, got);
     };
@@ -710,18 +497,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++v;
       }
     };
-    // TMEM unit consumed: a pair's epilogue warps arrive on rank 0's barrier
-    auto release_unit = [&](uint32_t buf) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (kPair) mbar_arrive_cluster(tempty0_cl + 8u * buf);
-        else mbar_arrive(&tempty[buf]);
-      }
-    };
-    for (int w = w0; ok && w < total; w += wstep) {
-      const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank, small_on);
-      const int col0 = t.ct * kTN + h * (kTN / 2);
+    for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
+      const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+      const int col0 = t.ct * kBN + h * 128;
       int64_t orow;
       bool row_ok;
       if constexpr (!kTg) {
@@ -760,82 +538,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-      if (kSmallOk && t.small) {
-        // transposed small-group tile: TMEM lane = output column n (the
-        // thread's), TMEM columns = the group's rows; warp half h holds rows
-        // 32 h .. 32 h + 31.  acc += unit * s_row[block] per column.
-        float2 acc[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.0f, 0.0f);
-        int slot = 0;
-        const int nunits = (t.nblocks + kSmallStack - 1) / kSmallStack;
-        for (int j = 0; j < nunits; ++j) {
-          const uint32_t buf = u % kNB;
-          slot = v % kRing;
-          if (!wait_unit(buf, slot)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int nb = min(kSmallStack, t.nblocks - j * kSmallStack);  // blocks in this unit (warp-uniform)
-          // slices two at a time, blocks in contraction order: the same
-          // sequence of fused multiply-adds as a 128-row tile
-          for (int sp = 0; sp < nb; sp += 2) {
-            uint32_t va[32], vb[32];
-            tmem_ld32(tl + buf * kBN + sp * kSmallN + 32 * h, va);
-            if (sp + 1 < nb) tmem_ld32(tl + buf * kBN + (sp + 1) * kSmallN + 32 * h, vb);
-            tmem_wait_ld();
-            const float2 *ca = reinterpret_cast<const float2 *>(s_scol + slot * kBN + sp * kSmallN + 32 * h);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              acc[i] = __ffma2_rn(make_float2(__uint_as_float(va[2 * i]), __uint_as_float(va[2 * i + 1])), ca[i],
-                                  acc[i]);
-            if (sp + 1 < nb) {
-              const float2 *cb = ca + kSmallN / 2;
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                acc[i] = __ffma2_rn(make_float2(__uint_as_float(vb[2 * i]), __uint_as_float(vb[2 * i + 1])), cb[i],
-                                    acc[i]);
-            }
-          }
-          release_unit(buf);
-          ++u;
-          if (j + 1 < nunits) release_slot(slot);
-        }
-        if (!ok) break;
-        const float fin = p.col_scale ? s_srow[slot * kBM + row] : 1.0f;
-        const int64_t n = static_cast<int64_t>(t.ct) * kSmallCols + row;
-        const int m0 = t.r0 + 32 * h;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int m = m0 + 2 * i + e;
-            if (m >= t.rend) continue;
-            const float o = (e ? acc[i].y : acc[i].x) * fin;
-            if (p.out_f32) static_cast<float *>(p.out)[m * p.ld_out + n] = o;
-            else static_cast<__nv_bfloat16 *>(p.out)[m * p.ld_out + n] = __float2bfloat16_rn(o);
-          }
-        }
-        release_slot(slot);
-        continue;
-      }
       if (t.nblocks == 0) {  // empty group in tgmm: dW tile = 0
         float z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.0f;
 #pragma unroll
-        for (int c = 0; c < kCh; ++c)
+        for (int c = 0; c < 4; ++c)
           if (col0 + c * 32 < p.ncols) emit(col0 + c * 32, z);
         continue;
       }
       if constexpr (kPromote) {
-        float2 acc[kCh * 16];
+        float2 acc[64];
 #pragma unroll
-        for (int i = 0; i < kCh * 16; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
         int slot = 0;
         for (int b = 0; b < t.nblocks; ++b) {
-          const uint32_t buf = u % kNB;
+          const uint32_t buf = u & 1;
           slot = v % kRing;
           if (!wait_unit(buf, slot)) {
             ok = false;
@@ -846,15 +564,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 rs2 = make_float2(rs, rs);
           const float *cs = s_scol + slot * kBN;
 #pragma unroll
-          for (int cp = 0; cp < kCh / 2; ++cp) {
+          for (int cp = 0; cp < 2; ++cp) {
             // chunks 2 cp, 2 cp + 1 (compile-time accumulator indices)
             // colt(2 cp + 1) = colt(2 cp) + 32: one 64-column load
             uint32_t va[32], vb[32];
-            tmem_ld64(tl + buf * kTN + colt(2 * cp), va, vb);
+            tmem_ld64(tl + buf * kBN + colt(2 * cp), va, vb);
             tmem_wait_ld();
-            // 128-column tiles: the unit is in registers now; hand its TMEM
-            // buffer back before the promotion math
-            if constexpr (kCh == 2) release_unit(buf);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
               const uint32_t *vv = half ? vb : va;
@@ -886,7 +601,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          if constexpr (kCh != 2) release_unit(buf);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
           ++u;
           if (b + 1 < t.nblocks) release_slot(slot);  // the last slot is read again below
         }
@@ -896,14 +613,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float fin = ((kTg || kBlkScales) && p.static_scale) ? s_eff : 1.0f;
           const bool colmul = !kTg && p.col_scale != nullptr;
           const float *cf = s_scol + slot * kBN;
-          if (kTN == 256 && sw) {  // SwiGLU tiles are 256 wide (128 gate + 128 up columns)
+          if (sw) {
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               const float *fg = cf + colt(c), *fu = cf + colt(c + 2);
               float o[32];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float2 a = acc[c * 16 + i], b2 = acc[((c + 2) % kCh) * 16 + i];
+                const float2 a = acc[c * 16 + i], b2 = acc[(c + 2) * 16 + i];
                 const float g0 = (colmul ? a.x * fg[2 * i] : a.x) * fin;
                 const float g1 = (colmul ? a.y * fg[2 * i + 1] : a.y) * fin;
                 const float u0 = (colmul ? b2.x * fu[2 * i] : b2.x) * fin;
@@ -915,8 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < kCh; ++c) {
-              const int col = t.ct * kTN + colt(c);
+            for (int c = 0; c < 4; ++c) {
+              const int col = t.ct * kBN + colt(c);
               if (col >= p.ncols) continue;
               float o[32];
 #pragma unroll
@@ -935,8 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         release_slot(slot);
       } else {
-        static_assert(kPromote || kTN == 256, "one unit per tile: 256-column tiles");
-        const uint32_t buf = u % kNB;
+        const uint32_t buf = u & 1;
         const int slot = v % kRing;
         if (!wait_unit(buf, slot)) {
           ok = false;
@@ -949,8 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cp = 0; cp < 2; ++cp) {
           const int ca = sw ? cp : 2 * cp, cb = sw ? cp + 2 : 2 * cp + 1;
           uint32_t va[32], vb[32];
-          tmem_ld32(tl + buf * kTN + colt(ca), va);
-          tmem_ld32(tl + buf * kTN + colt(cb), vb);
+          tmem_ld32(tl + buf * kBN + colt(ca), va);
+          tmem_ld32(tl + buf * kBN + colt(cb), vb);
           tmem_wait_ld();
           if (sw) {
             if (row_ok) {
@@ -969,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < 2; ++half) {
             const uint32_t *vv = half ? vb : va;
             const int c = half ? cb : ca;
-            const int col = t.ct * kTN + colt(c);
+            const int col = t.ct * kBN + colt(c);
             if (!row_ok || col >= p.ncols) continue;
             float o[32];
 #pragma unroll
@@ -980,7 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             emit(col, o);
           }
         }
-        release_unit(buf);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
         ++u;
         release_slot(slot);
       }
@@ -1007,13 +725,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  // a pair: neither CTA frees its tensor memory or leaves while the other may
-  // still read its shared memory (MMAs) or count bytes on its barriers (loads)
-  if constexpr (kPair) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    if constexpr (kPair) tmem_dealloc_pair(tbase, kTmemCols);
-    else tmem_dealloc(tbase, kTmemCols);
+    tmem_dealloc(tbase, kTmemCols);
   }
 }
 
@@ -1029,11 +743,11 @@ int num_sms() {
   return g_num_sms;
 }
 
-template <int kElem, bool kBMN, bool kPromote, int kMode, int kCta, bool kSmall = false, int kTN = 256>
+template <int kElem, bool kBMN, bool kPromote, int kMode>
 static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmOut,
-                               const CUtensorMap &tmW, const GemmParams &p, int grid, cudaStream_t st) {
-  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode, kCta, kSmall, kTN>;
-  const size_t smem = gemm_smem_bytes<kCta, kMode, kTN>();
+                               const GemmParams &p, int grid, cudaStream_t st) {
+  auto kern = gmm_tc_kernel<kElem, kBMN, kPromote, kMode>;
+  const size_t smem = gemm_smem_bytes<kMode>();
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -1043,95 +757,35 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
     return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  if constexpr (kCta == 1) {
-    kern<<<grid, kThreads, smem, st>>>(tmA, tmB, tmOut, tmW, p);
-    return cudaGetLastError();
-  } else {
-    // clusters of two CTAs; as many pairs as can be resident at once (a
-    // persistent grid), never more than there are items
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = 2;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    static int max_pairs = 0;  // per instantiation
-    if (max_pairs == 0) {
-      cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = num_sms() / 2;
-      max_pairs = n;
-    }
-    const int pairs = grid < max_pairs ? grid : max_pairs;  // grid counts items here
-    if (pairs <= 0) return cudaErrorInvalidConfiguration;
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmOut, tmW, p);
-  }
+  kern<<<grid, kThreads, smem, st>>>(tmA, tmB, tmOut, p);
+  return cudaGetLastError();
 }
 
-template <int kCta>
-static cudaError_t launch_cta(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                              const CUtensorMap &tmOut, const CUtensorMap &tmW, const GemmParams &p, int grid,
-                              cudaStream_t st) {
+cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st) {
+  if (cfg.cta_pairs) return launch_gemm_pair(cfg, tmA, tmB, tmOut, p, grid, st);
+  if (cfg.tile_n != 256) return cudaErrorInvalidValue;
   if (cfg.mode == MODE_TGMM) {
     if (cfg.b_mn_major) return cudaErrorInvalidValue;
-    if (cfg.elem_bytes == 1 && cfg.promote)
-      return launch_inst<1, false, true, MODE_TGMM, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
-    if (cfg.elem_bytes == 2 && !cfg.promote)
-      return launch_inst<2, false, false, MODE_TGMM, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
+    if (cfg.elem_bytes == 1 && cfg.promote) return launch_inst<1, false, true, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
+    if (cfg.elem_bytes == 2 && !cfg.promote) return launch_inst<2, false, false, MODE_TGMM>(tmA, tmB, tmOut, p, grid, st);
     return cudaErrorInvalidValue;
   }
   if (cfg.mode == MODE_ROWS_BLK) {  // block-wise rhs scales: promoted fp8 only
     if (cfg.elem_bytes != 1 || !cfg.promote) return cudaErrorInvalidValue;
-    return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
-                          : launch_inst<1, false, true, MODE_ROWS_BLK, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
-  }
-  if constexpr (kCta == 2) {
-    if (cfg.tile_n == 128) {  // four 128-column TMEM buffers: promoted E4M3, K-major B
-      if (cfg.elem_bytes != 1 || !cfg.promote || cfg.b_mn_major) return cudaErrorInvalidValue;
-      if (cfg.mode == MODE_ROWS)
-        return launch_inst<1, false, true, MODE_ROWS, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
-      if (cfg.mode == MODE_TGMM)
-        return launch_inst<1, false, true, MODE_TGMM, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
-      if (cfg.mode == MODE_ROWS_BLK)
-        return launch_inst<1, false, true, MODE_ROWS_BLK, 2, false, 128>(tmA, tmB, tmOut, tmW, p, grid, st);
-      return cudaErrorInvalidValue;
-    }
-  }
-  if (cfg.tile_n != 256) return cudaErrorInvalidValue;
-  if constexpr (kCta == 1) {
-    if (p.small_rows > 0)  // promoted E4M3 row pass with small-group tiles (checked by launch_gemm)
-      return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS, 1, true>(tmA, tmB, tmOut, tmW, p, grid, st)
-                            : launch_inst<1, false, true, MODE_ROWS, 1, true>(tmA, tmB, tmOut, tmW, p, grid, st);
+    return cfg.b_mn_major ? launch_inst<1, true, true, MODE_ROWS_BLK>(tmA, tmB, tmOut, p, grid, st)
+                          : launch_inst<1, false, true, MODE_ROWS_BLK>(tmA, tmB, tmOut, p, grid, st);
   }
   if (cfg.elem_bytes == 1) {
     if (cfg.b_mn_major)
-      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
-                         : launch_inst<1, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
-    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
-                       : launch_inst<1, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
+      return cfg.promote ? launch_inst<1, true, true, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
+                         : launch_inst<1, true, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
+    return cfg.promote ? launch_inst<1, false, true, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
+                       : launch_inst<1, false, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
   }
   if (cfg.promote) return cudaErrorInvalidValue;
-  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st)
-                        : launch_inst<2, false, false, MODE_ROWS, kCta>(tmA, tmB, tmOut, tmW, p, grid, st);
-}
-
-// grid: CTAs for one-CTA tiles; for pairs (cfg.cta_pairs) the number of pair
-// items, capped at the resident pairs
-cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const CUtensorMap &tmOut, const CUtensorMap &tmW, const GemmParams &p, int grid,
-                        cudaStream_t st) {
-  if (p.small_rows > 0 && (cfg.cta_pairs || cfg.mode != MODE_ROWS || cfg.elem_bytes != 1 || !cfg.promote ||
-                           p.small_rows > kSmallN || p.ncols % kSmallCols || p.swiglu_f))
-    return cudaErrorInvalidValue;
-  if (cfg.tile_n == 128 && (!cfg.cta_pairs || p.swiglu_f)) return cudaErrorInvalidValue;
-  return cfg.cta_pairs ? launch_cta<2>(cfg, tmA, tmB, tmOut, tmW, p, grid, st)
-                       : launch_cta<1>(cfg, tmA, tmB, tmOut, tmW, p, grid, st);
+  return cfg.b_mn_major ? launch_inst<2, true, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st)
+                        : launch_inst<2, false, false, MODE_ROWS>(tmA, tmB, tmOut, p, grid, st);
 }
 
 }  // namespace gmm

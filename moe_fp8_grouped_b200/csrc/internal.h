@@ -113,10 +113,6 @@ struct GemmParams {
   int tg_rows_fastest;        // MODE_TGMM item order within a group: 1 = row tiles (dout
                               // columns) fastest, each lhs column tile reused by
                               // consecutive items; 0 = column tiles fastest
-  int small_rows;             // MODE_ROWS, promoted E4M3, one-CTA tiles: groups of 1 ..
-                              // small_rows (<= 64) rows take transposed tiles (the
-                              // weights as the 128-row operand, the group's rows as
-                              // 64 MMA columns); 0: every group takes 128-row tiles
   uint32_t *status;
   uint64_t wait_limit_ns;
 };
@@ -135,12 +131,13 @@ struct GemmConfig {
 int num_sms();
 
 // tmOut: the output as a TMA tensor (MODE_TGMM: dW [G*K, N], box 32 x 32);
-// unused by MODE_ROWS.  tmW: the weights as the 128-row operand of the
-// transposed small-group tiles (box 128 x 128 bytes, the same major-ness as
-// tmB); used only when p.small_rows > 0.  grid: CTAs (one-CTA tiles) or
-// items (pairs; the launch caps it at the pairs that fit on the GPU at once).
+// unused by MODE_ROWS.  grid: CTAs (one-CTA tiles) or items (pairs; the
+// launch caps it at the pairs that fit on the GPU at once).
 cudaError_t launch_gemm(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const CUtensorMap &tmOut, const CUtensorMap &tmW, const GemmParams &p, int grid,
-                        cudaStream_t st);
+                        const CUtensorMap &tmOut, const GemmParams &p, int grid, cudaStream_t st);
+
+// The CTA-pair kernels (gemm_pair.cu); launch_gemm dispatches to them.
+cudaError_t launch_gemm_pair(const GemmConfig &cfg, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                             const CUtensorMap &tmOut, const GemmParams &p, int items, cudaStream_t st);
 
 }  // namespace gmm

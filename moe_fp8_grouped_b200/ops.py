@@ -343,13 +343,12 @@ def gmm_set_wait_limit_ns(limit_ns: int):
 
 
 TILES = {"auto": B.TILES_AUTO, "one_cta": B.TILES_ONE_CTA, "cta_pairs": B.TILES_CTA_PAIRS,
-         "small_groups": B.TILES_SMALL_GROUPS, "cta_pairs_narrow": B.TILES_CTA_PAIRS_NARROW}
+         "cta_pairs_narrow": B.TILES_CTA_PAIRS_NARROW}
 
 
 def gmm_set_tiles(mode="auto"):
     """GEMM tile choice for the calls that follow: "auto", "one_cta" (128-row
     tiles), "cta_pairs" (256-row tiles over a two-CTA cluster) or
-    "small_groups" (transposed tiles for groups of at most 64 rows) or
     "cta_pairs_narrow" (CTA pairs; 256 x 128 tiles for the promoted passes
     with K-major weights)."""
     _check(B.lib().gmm_set_tiles(TILES[mode] if isinstance(mode, str) else int(mode)), "gmm_set_tiles")

@@ -1,16 +1,13 @@
-"""The GEMM passes on their other tiles, against the oracle and bit for bit
-against the plain one-CTA 128-row tile (every tile accumulates each output
-over the same contraction steps in the same order):
-
-- 256-row tiles shared by a pair of CTAs (a two-CTA cluster issuing M = 256
-  tensor-core MMAs), forced on the small ragged cases where the automatic
-  choice would take one-CTA tiles.  The cases put the pair tile's second
-  half past a group's end (odd 128-row tile counts, 1-row and 129-row
-  groups), leave rows unrouted, leave groups empty and use N not a multiple
-  of 256.
-- transposed small-group tiles (the weights as the 128-row MMA operand, a
-  group of at most 64 rows as 64 MMA columns) for such groups in the
-  promoted E4M3 forward and dlhs (tile mode "small_groups").
+"""The GEMM passes on tiles shared by a pair of CTAs (a two-CTA cluster
+issuing M = 256 tensor-core MMAs), 256 columns wide or, in mode
+"cta_pairs_narrow", 128 columns wide for the promoted passes with a K-major
+B operand; forced on the small ragged cases where the automatic choice would
+take one-CTA tiles.  Each pass is checked against the oracle and bit for bit
+against the one-CTA 128-row tile (every tile accumulates each output over the
+same contraction steps in the same order).  The cases put the pair tile's
+second half past a group's end (odd 128-row tile counts, 1-row and 129-row
+groups), leave rows unrouted, leave groups empty and use N not a multiple of
+256.
 """
 import numpy as np
 import pytest
@@ -196,91 +193,3 @@ def test_pairs_status_clean_and_max_groups(dev, mode):
     ref, ab = oracle.gmm_fwd(inp.lhs, oracle.Q_STATIC, inp.static_scale, qr, sr, inp.group_sizes, rows=rows)
     assert_close(pair[rows], ref, ab, "pair fwd, 1024 groups")
     assert torch.equal(pair, one)
-
-
-SMALL_CASES = {
-    # G, M, K, N, sizes: groups of 1, 2, 30, 33, 40, 63, 64 rows (small tiles) next to 65, 100, 128
-    "mixed": (12, 600, 384, 512, [1, 64, 65, 0, 2, 63, 128, 30, 0, 40, 33, 100]),
-    "n640": (4, 200, 256, 640, [5, 64, 0, 60]),   # N % 256 = 128; 71 rows unrouted
-    "all_small": (6, 300, 512, 256, [10, 20, 30, 40, 50, 64]),
-}
-
-
-def small_inputs(name):
-    G, M, K, N, sizes = SMALL_CASES[name]
-    return synth.small_case(G, M, K, N, seed=19, sizes=sizes)
-
-
-def auto_vs_plain(fn):
-    """fn() with small groups on transposed tiles, then on plain one-CTA
-    tiles."""
-    try:
-        gm.gmm_set_tiles("small_groups")
-        auto = fn()
-        gm.gmm_set_tiles("one_cta")
-        plain = fn()
-    finally:
-        gm.gmm_set_tiles("auto")
-    torch.cuda.synchronize()
-    return auto, plain
-
-
-@pytest.mark.parametrize("name", list(SMALL_CASES))
-@pytest.mark.parametrize("transpose", [False, True])
-@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_fwd_small_group_tiles(dev, name, transpose, out_dtype):
-    inp = small_inputs(name)
-    lhs, w, _, gs, _ = to_dev(inp, dev)
-    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
-    auto, plain = auto_vs_plain(lambda: gm.gmm_fwd(lhs, codes, scales, gs, rule="dynamic", transpose_rhs=transpose,
-                                                   out_dtype=out_dtype))
-    qr, sr = oracle.quantize_rhs(inp.w)
-    ref, ab = oracle.gmm_fwd(inp.lhs, oracle.Q_DYNAMIC, 0.0, qr, sr, inp.group_sizes)
-    assert_close(auto, ref, ab, f"small-tile fwd {name} t={transpose}")
-    assert torch.equal(auto, plain), f"small-tile fwd differs from the 128-row tile ({name} t={transpose})"
-    # a pre-quantized lhs takes the same tiles
-    ql, sl = gm.gmm_quantize(lhs, "dynamic", axis=1)
-    pre, _ = auto_vs_plain(lambda: gm.gmm_fwd(ql, codes, scales, gs, rule="dynamic", lhs_scales=sl,
-                                              transpose_rhs=transpose, out_dtype=out_dtype))
-    assert torch.equal(pre, auto)
-
-
-@pytest.mark.parametrize("name", list(SMALL_CASES))
-@pytest.mark.parametrize("transpose", [False, True])
-def test_dlhs_and_backward_small_group_tiles(dev, name, transpose):
-    inp = small_inputs(name)
-    lhs, w, dout, gs, _ = to_dev(inp, dev)
-    codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
-    auto, plain = auto_vs_plain(lambda: gm.gmm_dlhs(dout, codes, scales, gs, transpose_rhs=transpose,
-                                                    out_dtype=torch.float32))
-    qr, sr = oracle.quantize_rhs(inp.w)
-    ref, ab = oracle.gmm_dlhs(inp.dout, qr, sr, inp.group_sizes)
-    assert_close(auto, ref, ab, f"small-tile dlhs {name} t={transpose}")
-    assert torch.equal(auto, plain)
-    (dl, dw), _ = auto_vs_plain(lambda: gm.gmm_backward(lhs, dout, codes, scales, gs, rule="dynamic",
-                                                        transpose_rhs=transpose, dlhs_dtype=torch.float32))
-    assert torch.equal(dl, auto)
-
-
-def test_small_group_tiles_status_clean(dev):
-    """1024 groups (the maximum), most of 1 .. 64 rows, a few large: the item
-    prefix mixes both tile kinds; the device status stays clean."""
-    G, K, N = 1024, 256, 256
-    g = torch.Generator().manual_seed(20)
-    sizes = torch.randint(0, 65, (G,), generator=g)
-    sizes[[7, 300, 1000]] = torch.tensor([700, 129, 256])
-    M = int(sizes.sum()) + 50
-    inp = synth.small_case(G, M, K, N, seed=21, sizes=sizes.tolist())
-    lhs, w, _, gs, _ = to_dev(inp, dev)
-    codes, scales = gm.gmm_quantize_rhs(w)
-    ws = torch.empty(gm.gmm_workspace_bytes(0, M, K, N, G), dtype=torch.uint8, device=dev)
-    auto, plain = auto_vs_plain(lambda: gm.gmm_fwd(lhs, codes, scales, gs, rule="dynamic", ws=ws,
-                                                   out_dtype=torch.float32))
-    st, bits = gm.gmm_read_device_status(ws)
-    assert st == 0, (st, bits)
-    assert torch.equal(auto, plain)
-    offs = np.concatenate([[0], np.cumsum(sizes.numpy())])
-    rows = sorted({int(offs[i]) for i in (0, 5, 7, 8, 300, 600, 1000, 1023)} | {M - 1, M - 51})
-    qr, sr = oracle.quantize_rhs(inp.w)
-    ref, ab = oracle.gmm_fwd(inp.lhs, oracle.Q_DYNAMIC, 0.0, qr, sr, inp.group_sizes, rows=rows)
-    assert_close(auto[rows], ref, ab, "small-tile fwd, 1024 groups")
