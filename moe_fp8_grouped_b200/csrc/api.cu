@@ -405,11 +405,11 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   }
   const bool bmn = transpose_rhs == 0;  // [G, K, N]: N contiguous = MN-major B
   const uint32_t bke = 128 / elem;
+  const bool pairs = use_pairs(false, M, N, G);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, A, elem, K, M, K * elem, bke, 128)) return GMM_ERR_CUDA;
   // SwiGLU tiles take the gate rows and the up rows of a K-major rhs as two
   // 128-row boxes
-  const bool pairs = use_pairs(false, M, N, G);
   const int tn = tile_cols(pairs, elem == 1 && (dyn || blk), !bmn, F != 0);
   const bool okB = bmn ? make_map(&tmB, rhs.data, elem, N, static_cast<uint64_t>(G) * K, N * elem, bke, bke)
                        : make_map(&tmB, rhs.data, elem, K, static_cast<uint64_t>(G) * N, K * elem, bke,
