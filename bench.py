@@ -78,16 +78,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def tensor_peak(peaks, src, region_s: float, bf16_family: bool):
+def tensor_peak(peaks, src, region_s: float, bf16_family: bool, clocks=None):
     """The tensor peak a kernel timed inside a region of region_s seconds is
-    held to: the burst cuBLAS bf16 figure for regions under 2 s (the clock has
-    not settled under the power cap yet), the sustained one for longer regions;
-    x2 (the nominal dense fp8 / bf16 ratio, 4.5 / 2.25 PFLOP/s) for fp8."""
-    sustained = region_s >= 2.0
+    held to: the burst cuBLAS bf16 figure while the SM clock stays near its
+    maximum, the sustained (power-capped) one when the median SM clock sampled
+    during the region fell below 90 % of the maximum; without clock samples,
+    burst for regions under 2 s.  x2 (the nominal dense fp8 / bf16 ratio,
+    4.5 / 2.25 PFLOP/s) for fp8."""
+    mhz = clocks.get("sm_mhz") if clocks else None
+    mx = clocks.get("sm_max_mhz") if clocks else None
+    if mhz and mx:
+        sustained = mhz < 0.9 * mx
+        why = f"median SM clock {mhz:.0f} of {mx:.0f} MHz over the timed region ({region_s:.2f} s)"
+    else:
+        sustained = region_s >= 2.0
+        why = f"timed region {region_s:.2f} s, no clock samples"
     v = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * (1.0 if bf16_family else FP8_OVER_BF16)
     desc = (f"{src} bf16 {'sustained' if sustained else 'burst'} cuBLAS"
-            + ("" if bf16_family else f" x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)")
-            + f"; timed region {region_s:.2f} s")
+            + ("" if bf16_family else f" x {FP8_OVER_BF16} (nominal fp8/bf16 ratio)") + f"; {why}")
     return v, desc
 
 
@@ -377,7 +385,7 @@ def run_ours(args):
     value = job_tflops(flops_step, world, args.steps, ms)
 
     peaks, peak_src = load_peaks()
-    peak_tc, peak_tc_src = tensor_peak(peaks, peak_src, ms / 1e3, bf16_family)
+    peak_tc, peak_tc_src = tensor_peak(peaks, peak_src, ms / 1e3, bf16_family, clk)
     peak_bw = peaks["hbm_gbs"]
     bytes_pass = algorithmic_bytes(M, K, Np, G, G_ne, rule)
     passes = {}
@@ -673,7 +681,7 @@ def measure_forward_shapes(dev, names, calls, peaks, peak_src):
         G_ne = int((inp.group_sizes > 0).sum())
         flops = 2.0 * rows * w.K * w.N
         nbytes = algorithmic_bytes(w.M, w.K, w.N, w.G, G_ne, w.rule)["fwd"]
-        peak_tc, tc_src = tensor_peak(peaks, peak_src, sum(a.elapsed_time(b) for a, b in evs) / 1e3, False)
+        peak_tc, tc_src = tensor_peak(peaks, peak_src, sum(a.elapsed_time(b) for a, b in evs) / 1e3, False, clocks)
         floor_ms = max(flops / (peak_tc * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
 
         def figures(t_ms):

@@ -580,6 +580,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 16; ++i)
                   acc[c * 16 + i] = __ffma2_rn(make_float2(__uint_as_float(vv[2 * i]), __uint_as_float(vv[2 * i + 1])),
                                                rs2, acc[c * 16 + i]);
+              } else if (kBlkScales && !need_row) {
+                // block-wise rhs scales with a static lhs (s applied at the
+                // end): the column scale multiplies the unit directly; a loop
+                // of its own, so that no row-scale product is formed
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 c4 = *reinterpret_cast<const float4 *>(cs + colt(c) + 4 * i);
+                  acc[c * 16 + 2 * i] = __ffma2_rn(
+                      make_float2(__uint_as_float(vv[4 * i]), __uint_as_float(vv[4 * i + 1])),
+                      make_float2(c4.x, c4.y), acc[c * 16 + 2 * i]);
+                  acc[c * 16 + 2 * i + 1] = __ffma2_rn(
+                      make_float2(__uint_as_float(vv[4 * i + 2]), __uint_as_float(vv[4 * i + 3])),
+                      make_float2(c4.z, c4.w), acc[c * 16 + 2 * i + 1]);
+                }
               } else {
                 // tgmm with a dynamic lhs rule (lhs chunk scale along the
                 // columns k) or block-wise rhs scales (along the columns n)
