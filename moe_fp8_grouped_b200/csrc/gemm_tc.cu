@@ -26,6 +26,14 @@
 //   warps 4-11 epilogue: tcgen05.ld, scale, store.  Warp w reads TMEM lanes
 //              32 (w % 4) .. +31 (rows) and column half (w - 4) / 4.
 //
+// Promoted row tiles of at most 64 rows (small groups) run M = 64 MMAs: they
+// read half of the A stage from shared memory, which the weight stream of the
+// memory-bound shapes competes for (the static kernels keep M = 128: the
+// extra index arithmetic cost their epilogue more than it saved).  An M = 64 accumulator puts tile row r in
+// TMEM lane 32 (r / 16) + r % 16 and leaves lanes 16 .. 31 of each 32-lane
+// quarter untouched, so in those tiles only the first 16 lanes of each
+// epilogue warp hold rows.
+//
 // Scaling ("add static LHS scaling support for GMM v2 FWD", maxtext PR
 // #4735, review thread on the LhsRef docstring: the result is multiplied back
 // by the scale):
@@ -222,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBBoxes = kBMN ? 2 * kElem : 1;     // TMA boxes per B stage
   constexpr int kBBoxBytes = kBStage / kBBoxes;
   constexpr uint32_t kIdesc = instr_desc(kF16, kBMN);
+  constexpr uint32_t kIdesc64 = instr_desc(kF16, kBMN, 64);  // row tiles of <= 64 rows
   constexpr int kSt = stages_of<kMode>();
   constexpr int kRing = ring_of<kMode>();
 
@@ -368,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
           const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
+          const uint32_t idesc = (kPromote && !kTg && t.rend - t.r0 <= 64) ? kIdesc64 : kIdesc;
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
@@ -392,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
               const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
                                           : smem_desc_sw128(b0 + kk * 32, 16, 1024);
-              tc_mma<kF16>(d, adesc, bdesc, kIdesc, (unit_start && kk == 0) ? 0u : 1u);
+              tc_mma<kF16>(d, adesc, bdesc, idesc, (unit_start && kk == 0) ? 0u : 1u);
             }
             tc_commit(&empty[s]);
             if (kPromote || b == t.nblocks - 1) {
@@ -502,9 +512,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int col0 = t.ct * kBN + h * 128;
       int64_t orow;
       bool row_ok;
+      int trow = row;  // the tile row held by this thread's TMEM lane
       if constexpr (!kTg) {
-        orow = t.r0 + row;
-        row_ok = orow < t.rend;
+        const bool m64 = kPromote && t.rend - t.r0 <= 64;  // M = 64 accumulator layout
+        if (m64) trow = q * 16 + (lane & 15);
+        orow = t.r0 + trow;
+        row_ok = (!m64 || lane < 16) && orow < t.rend;
       } else {
         orow = static_cast<int64_t>(t.rt) * kBM + row;  // n
         row_ok = true;
@@ -560,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const float rs = need_row ? s_srow[slot * kBM + row] : 1.0f;
+          const float rs = need_row ? s_srow[slot * kBM + trow] : 1.0f;
           const float2 rs2 = make_float2(rs, rs);
           const float *cs = s_scol + slot * kBN;
 #pragma unroll

@@ -3,7 +3,8 @@
 Codes and scales are compared bit for bit; pass outputs element by element
 within 2e-3 * sum|a*b| (plus bf16 output rounding).  Cases span several
 tiles, ragged tails, empty groups, unrouted rows, N not a multiple of the
-256-wide tile, both rhs layouts and both output dtypes.  Each pass is run on
+256-wide tile, row tiles short enough for M = 64 MMAs, both rhs layouts and
+both output dtypes.  Each pass is run on
 its own (the pages' review found a bug where one pass's flag leaked into
 another: "Support quantization for tokamax gmm v2", maxtext PR #4451, review
 thread on the dlhs selection).
@@ -24,6 +25,9 @@ CASES = {
     "ragged": (5, 700, 384, 640, [1, 129, 0, 300, 200]),  # 70 unrouted rows, N % 256 = 128
     "g1": (1, 300, 256, 256, [300]),
     "big_group": (2, 1100, 512, 256, [1000, 100]),
+    # row tiles of 64, 16, 48, 64 (the tail of 192) and 63 rows run M = 64
+    # MMAs in the promoted passes; 65 rows one M = 128 tile; 32 rows unrouted
+    "short_tiles": (7, 480, 384, 512, [64, 65, 16, 0, 48, 192, 63]),
 }
 
 

@@ -26,6 +26,9 @@ CASES = {
     "odd_tiles": (3, 900, 256, 512, [129, 385, 300]),      # 2, 4, 3 row tiles: half-empty pair tiles
     "big_group": (2, 1100, 512, 256, [1000, 100]),
     "unrouted": (4, 1000, 256, 256, [10, 0, 250, 40]),     # 700 rows in no group
+    # one-CTA promoted tiles of <= 64 rows run M = 64 MMAs: compared bit for
+    # bit with the pair tiles' M = 256 MMAs
+    "short_tiles": (7, 480, 384, 512, [64, 65, 16, 0, 48, 192, 63]),
 }
 
 
