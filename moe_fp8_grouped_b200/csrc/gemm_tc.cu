@@ -22,7 +22,20 @@
 //              256-column accumulator buffers
 //   warp 2     scale loader: row / column scales of each TMEM unit into a
 //              shared-memory ring ahead of the epilogue
-//   warp 3     idle (gives its registers to the epilogue)
+//   warp 3     promoted kernels: second MMA issuer (idle otherwise, giving its
+//              registers to the epilogue)
+//
+// One thread cannot issue tcgen05.mma fast enough to keep the tensor core
+// busy once it also waits on the pipeline barriers (measured: ~2.2-3.3
+// PFLOP/s from one issuing thread, ~4.3 from two or three).  In the promoted
+// kernels every 128-long block is its own TMEM unit and units alternate
+// between the two accumulator buffers, so warp 1 issues the even units
+// (buffer 0) and warp 3 the odd ones (buffer 1): each unit is still
+// accumulated by one thread in contraction order, so the results do not
+// depend on the split.  Each issuer waits for its buffer to be released
+// before it waits for the unit's stage: units are released in order, so by
+// then every earlier use of that stage has completed and the stage barrier's
+// phase parity is unambiguous, whatever the stage count.
 //   warps 4-11 epilogue: tcgen05.ld, scale, store.  Warp w reads TMEM lanes
 //              32 (w % 4) .. +31 (rows) and column half (w - 4) / 4.
 //
@@ -282,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kEpiWarps);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, kPromote ? 2 : 1);  // one commit per MMA issuer
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sfull[i], 32);
       mbar_init(&sempty[i], kEpiWarps);
@@ -370,8 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // let every issued copy land before the CTA can exit
       for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
         mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
-    } else if (warp == 1) {
-      // ----------------------------------------------------- MMA issuer
+    } else if (warp == 1 || (kPromote && warp == 3)) {
+      // ---------------------------------------------------- MMA issuer(s)
+      // promoted kernels: warp 1 issues the even units, warp 3 the odd ones
+      const int par = warp == 3 ? 1 : 0;
       if (lane == 0) {
         int it = 0, u = 0;
         bool ok = true;
@@ -381,6 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
+            if (kPromote && (u & 1) != par) {  // the other issuer's unit
+              ++u;
+              continue;
+            }
             if (unit_start) {
               buf = u & 1;
               if (!mbar_wait(&tempty[buf], ((u >> 1) & 1) ^ 1, ctl)) {
