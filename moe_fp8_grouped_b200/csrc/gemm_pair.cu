@@ -237,6 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kNB = kTmemCols / kTN;              // TMEM accumulator buffers
   constexpr int kCh = kTN / 64;                     // 32-column chunks per epilogue thread
   constexpr int kRing = ring_of<kMode>();
+  // static E4M3 row tiles accumulate their even and odd blocks in the two
+  // TMEM buffers, as the one-CTA kernel does (bit-identical results)
+  constexpr bool kSplit = !kPromote && !kTg && kElem == 1;
   constexpr uint32_t kStageTx = kCta * (kAStage + kBS);  // bytes completing one stage (both CTAs)
 
   extern __shared__ uint8_t smem_raw[];
@@ -437,8 +440,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && leader) {
         int it = 0, u = 0;
         bool ok = true;
+        int nuse = 0;  // split tiles: tiles issued (buffer 1 only when a tile has two blocks or more)
+        int nuse1 = 0;
         for (int w = w0; ok && w < total; w += wstep) {
           const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
+          if constexpr (kSplit) {
+            // the same accumulation as the one-CTA static row tiles: even
+            // blocks into buffer 0, odd ones into buffer 1, summed by the
+            // epilogue
+            const bool two = t.nblocks > 1;
+            if (!mbar_wait(&tempty[0], (nuse & 1) ^ 1, ctl) || (two && !mbar_wait(&tempty[1], (nuse1 & 1) ^ 1, ctl))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int b = 0; b < t.nblocks; ++b, ++it) {
+              const int s = it % kSt;
+              if (!mbar_wait(&full[s], (it / kSt) & 1, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBS);
+              const uint32_t d = tbase + (b & 1) * kTN;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+                const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
+                                            : smem_desc_sw128(b0 + kk * 32, 16, 1024);
+                if constexpr (kPair) tc_mma_pair<kF16>(d, adesc, bdesc, kIdesc, (b < 2 && kk == 0) ? 0u : 1u);
+                else tc_mma<kF16>(d, adesc, bdesc, kIdesc, (b < 2 && kk == 0) ? 0u : 1u);
+              }
+              if constexpr (kPair) tc_commit_pair_both(&empty[s], 0x3);
+              else tc_commit(&empty[s]);
+            }
+            if (!ok) break;
+            if constexpr (kPair) tc_commit_pair_both(&tfull[0], 0x3);
+            else tc_commit(&tfull[0]);
+            ++nuse;
+            if (two) {
+              if constexpr (kPair) tc_commit_pair_both(&tfull[1], 0x3);
+              else tc_commit(&tfull[1]);
+              ++nuse1;
+            }
+            continue;
+          }
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
@@ -560,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t evict_first = kTg ? l2_policy_evict_first() : 0;  // dW is written once: keep operands in L2
     int nstore = 0;                                                     // tgmm stores issued by this warp
     int u = 0;  // TMEM units consumed
+    int n0 = 0, n1 = 0;  // split tiles: uses of buffers 0 and 1 consumed
     int v = 0;  // scale slots consumed
     bool ok = true;
     // waits for TMEM unit u (and its scale slot); the decision is uniform
@@ -736,6 +783,75 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 o[2 * i] = a.x * fin;
                 o[2 * i + 1] = a.y * fin;
+              }
+              emit(col, o);
+            }
+          }
+        }
+        release_slot(slot);
+      } else if constexpr (kSplit) {
+        static_assert(kTN == 256, "one pair of units per tile: 256-column tiles");
+        const bool two = t.nblocks > 1;
+        const int slot = v % kRing;
+        bool got = mbar_wait(&tfull[0], n0 & 1, ctl);
+        if (got && two) got = mbar_wait(&tfull[1], n1 & 1, ctl);
+        if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kRing) & 1, ctl);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float2 acc[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int bi = 0; bi < (two ? 2 : 1); ++bi) {
+#pragma unroll
+          for (int cp = 0; cp < 2; ++cp) {
+            uint32_t va[32], vb[32];
+            tmem_ld64(tl + bi * kTN + colt(2 * cp), va, vb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              acc[2 * cp * 16 + i] =
+                  __fadd2_rn(acc[2 * cp * 16 + i], make_float2(__uint_as_float(va[2 * i]), __uint_as_float(va[2 * i + 1])));
+              acc[(2 * cp + 1) * 16 + i] = __fadd2_rn(
+                  acc[(2 * cp + 1) * 16 + i], make_float2(__uint_as_float(vb[2 * i]), __uint_as_float(vb[2 * i + 1])));
+            }
+          }
+        }
+        release_unit(0);
+        if (two) release_unit(1);
+        ++n0;
+        if (two) ++n1;
+        if (row_ok) {
+          const float s0 = p.static_scale ? s_eff : 1.0f;
+          const float *cf = s_scol + slot * kBN;
+          if (sw) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const float *fg = cf + colt(c), *fu = cf + colt(c + 2);
+              float o[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 a = acc[c * 16 + i], b2 = acc[(c + 2) * 16 + i];
+                const float gs0 = need_col ? fg[2 * i] : 1.0f, gs1 = need_col ? fg[2 * i + 1] : 1.0f;
+                const float us0 = need_col ? fu[2 * i] : 1.0f, us1 = need_col ? fu[2 * i + 1] : 1.0f;
+                o[2 * i] = silu(a.x * s0 * gs0) * (b2.x * s0 * us0);
+                o[2 * i + 1] = silu(a.y * s0 * gs1) * (b2.y * s0 * us1);
+              }
+              emit(t.ct * 128 + h * 64 + c * 32, o);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int col = t.ct * kTN + colt(c);
+              if (col >= p.ncols) continue;
+              float o[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 a = acc[c * 16 + i];
+                o[2 * i] = a.x * s0 * (need_col ? cf[colt(c) + 2 * i] : 1.0f);
+                o[2 * i + 1] = a.y * s0 * (need_col ? cf[colt(c) + 2 * i + 1] : 1.0f);
               }
               emit(col, o);
             }

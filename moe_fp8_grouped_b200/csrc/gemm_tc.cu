@@ -82,15 +82,26 @@ constexpr int kEpiThreads = 256;
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 8;    // ring of per-unit scale slots (scale loader -> epilogue)
 constexpr int kNumBars = 32;      // mbarriers reserved in shared memory
+// Two MMA issuers (warps 1 and 3): the promoted kernels (one TMEM unit per
+// 128-long block, units alternating between the two buffers) and the static
+// E4M3 row passes (each tile's blocks split between the buffers, even blocks
+// in buffer 0, odd ones in buffer 1; the epilogue adds the two partial sums).
+// The bf16 family keeps one issuer and one accumulator per tile (its dlhs
+// measured slower split: the tile-end wait for both buffers is not paid back).
+template <int kElem, bool kPromote, int kMode>
+constexpr bool two_issuers() { return kPromote || (kElem == 1 && kMode != MODE_TGMM); }
+
 // Register split (setmaxnreg): the control warpgroup gives registers to the
 // two epilogue warpgroups.  Sum must not exceed the launch allocation
 // (registers per thread at launch x 384); launch_inst checks it.
-// The promote variants keep 128 accumulators per thread and get the larger
-// epilogue share.
-template <bool kPromote>
-constexpr int regs_ctl() { return kPromote ? 40 : 72; }
-template <bool kPromote>
-constexpr int regs_epi() { return kPromote ? 232 : 216; }
+// Kernels whose epilogue holds a thread's 128 accumulators in registers get
+// the larger epilogue share (the static row passes keep a little more for
+// their producer's SwiGLU box logic: fewer spills measured with 56 / 224 than
+// with 40 / 232).
+template <int kElem, bool kPromote, int kMode>
+constexpr int regs_ctl() { return kPromote ? 40 : (two_issuers<kElem, kPromote, kMode>() ? 56 : 72); }
+template <int kElem, bool kPromote, int kMode>
+constexpr int regs_epi() { return kPromote ? 232 : (two_issuers<kElem, kPromote, kMode>() ? 224 : 216); }
 
 // tgmm keeps 3 pipeline stages and uses the freed shared memory to stage its
 // output for TMA stores (one 4 KB block per epilogue warp)
@@ -245,6 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kIdesc = instr_desc(kF16, kBMN);
   constexpr uint32_t kIdesc64 = instr_desc(kF16, kBMN, 64);  // row tiles of <= 64 rows
   constexpr int kSt = stages_of<kMode>();
+  constexpr bool kTwo = two_issuers<kElem, kPromote, kMode>();
+  constexpr bool kSplit = kTwo && !kPromote;  // static row pass: a tile's blocks split between the buffers
+  static_assert(!kSplit || kSt % 2 == 0, "split tiles: each stage serves one issuer");
   constexpr int kRing = ring_of<kMode>();
 
   extern __shared__ uint8_t smem_raw[];
@@ -295,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kEpiWarps);
     }
-    mbar_init(drain, kPromote ? 2 : 1);  // one commit per MMA issuer
+    mbar_init(drain, kTwo ? 2 : 1);  // one commit per MMA issuer
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sfull[i], 32);
       mbar_init(&sempty[i], kEpiWarps);
@@ -327,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtl ctl_drain{p.wait_limit_ns, no_abort, p.status};
 
   if (warp < 4) {
-    setmaxnreg_dec<regs_ctl<kPromote>()>();
+    setmaxnreg_dec<regs_ctl<kElem, kPromote, kMode>()>();
     if (warp == 0 && lane == 0) {
       // ---------------------------------------------------- TMA producer
       int it = 0;
@@ -383,16 +397,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       // let every issued copy land before the CTA can exit
       for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
         mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
-    } else if (warp == 1 || (kPromote && warp == 3)) {
+    } else if (warp == 1 || (kTwo && warp == 3)) {
       // ---------------------------------------------------- MMA issuer(s)
-      // promoted kernels: warp 1 issues the even units, warp 3 the odd ones
+      // two issuers: warp 1 fills buffer 0 (the even units, or the even blocks
+      // of a split tile), warp 3 buffer 1
       const int par = warp == 3 ? 1 : 0;
       if (lane == 0) {
         int it = 0, u = 0;
+        int nuse = 0;  // split tiles: uses of this issuer's buffer
         bool ok = true;
+        auto issue = [&](int s, uint32_t d, uint32_t idesc, bool first) {
+          const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBStage);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
+                                        : smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            tc_mma<kF16>(d, adesc, bdesc, idesc, (first && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&empty[s]);
+        };
         for (int w = blockIdx.x; ok && w < total; w += gridDim.x) {
           const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
           const uint32_t idesc = (kPromote && !kTg && t.rend - t.r0 <= 64) ? kIdesc64 : kIdesc;
+          if constexpr (kSplit) {
+            // blocks b = par, par + 2, .. of the tile into buffer par
+            const bool mine = t.nblocks > par;
+            if (mine) {
+              if (!mbar_wait(&tempty[par], (nuse & 1) ^ 1, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            for (int b = 0; b < t.nblocks; ++b, ++it) {
+              if ((b & 1) != par) continue;
+              const int s = it % kSt;
+              if (!mbar_wait(&full[s], (it / kSt) & 1, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue(s, tbase + par * kBN, idesc, b == par);
+            }
+            if (!ok) break;
+            if (mine) {
+              tc_commit(&tfull[par]);
+              ++nuse;
+            }
+            continue;
+          }
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
@@ -414,16 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBStage);
-            const uint32_t d = tbase + buf * kBN;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
-              const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
-                                          : smem_desc_sw128(b0 + kk * 32, 16, 1024);
-              tc_mma<kF16>(d, adesc, bdesc, idesc, (unit_start && kk == 0) ? 0u : 1u);
-            }
-            tc_commit(&empty[s]);
+            issue(s, tbase + buf * kBN, idesc, unit_start);
             if (kPromote || b == t.nblocks - 1) {
               tc_commit(&tfull[buf]);
               ++u;
@@ -486,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       cp_async_wait_all();  // no copy in flight when the warp leaves
     }
   } else {
-    setmaxnreg_inc<regs_epi<kPromote>()>();
+    setmaxnreg_inc<regs_epi<kElem, kPromote, kMode>()>();
     // ---------------------------------------------------------- epilogue
     const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
     const int q = warp & 3, h = (warp - kEpiWarp0) >> 2;
@@ -508,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t evict_first = kTg ? l2_policy_evict_first() : 0;  // dW is written once: keep operands in L2
     int nstore = 0;                                                     // tgmm stores issued by this warp
     int u = 0;  // TMEM units consumed
+    int n0 = 0, n1 = 0;  // split tiles: uses of buffers 0 and 1 consumed
     int v = 0;  // scale slots consumed
     bool ok = true;
     // waits for TMEM unit u (and its scale slot); the decision is uniform
@@ -697,6 +743,81 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         release_slot(slot);
+      } else if constexpr (kSplit) {
+        // partial sums of the even blocks (buffer 0) and the odd ones (buffer
+        // 1): both into registers, the buffers released, then scale and store
+        const bool two = t.nblocks > 1;
+        const int slot = v % kRing;
+        bool got = mbar_wait(&tfull[0], n0 & 1, ctl);
+        if (got && two) got = mbar_wait(&tfull[1], n1 & 1, ctl);
+        if (got && use_ring) got = mbar_wait(&sfull[slot], (v / kRing) & 1, ctl);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float2 acc[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int bi = 0; bi < (two ? 2 : 1); ++bi) {
+#pragma unroll
+          for (int cp = 0; cp < 2; ++cp) {
+            // chunks 2 cp, 2 cp + 1: colt(2 cp + 1) = colt(2 cp) + 32
+            uint32_t va[32], vb[32];
+            tmem_ld64(tl + bi * kBN + colt(2 * cp), va, vb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              acc[2 * cp * 16 + i] =
+                  __fadd2_rn(acc[2 * cp * 16 + i], make_float2(__uint_as_float(va[2 * i]), __uint_as_float(va[2 * i + 1])));
+              acc[(2 * cp + 1) * 16 + i] = __fadd2_rn(
+                  acc[(2 * cp + 1) * 16 + i], make_float2(__uint_as_float(vb[2 * i]), __uint_as_float(vb[2 * i + 1])));
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&tempty[0]);
+          if (two) mbar_arrive(&tempty[1]);
+        }
+        ++n0;
+        if (two) ++n1;
+        if (row_ok) {
+          const float s0 = p.static_scale ? s_eff : 1.0f;
+          const float *cf = s_scol + slot * kBN;
+          if (sw) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const float *fg = cf + colt(c), *fu = cf + colt(c + 2);
+              float o[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 a = acc[c * 16 + i], b2 = acc[(c + 2) * 16 + i];
+                const float gs0 = need_col ? fg[2 * i] : 1.0f, gs1 = need_col ? fg[2 * i + 1] : 1.0f;
+                const float us0 = need_col ? fu[2 * i] : 1.0f, us1 = need_col ? fu[2 * i + 1] : 1.0f;
+                o[2 * i] = silu(a.x * s0 * gs0) * (b2.x * s0 * us0);
+                o[2 * i + 1] = silu(a.y * s0 * gs1) * (b2.y * s0 * us1);
+              }
+              emit(t.ct * 128 + h * 64 + c * 32, o);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int col = t.ct * kBN + colt(c);
+              if (col >= p.ncols) continue;
+              float o[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 a = acc[c * 16 + i];
+                o[2 * i] = a.x * s0 * (need_col ? cf[colt(c) + 2 * i] : 1.0f);
+                o[2 * i + 1] = a.y * s0 * (need_col ? cf[colt(c) + 2 * i + 1] : 1.0f);
+              }
+              emit(col, o);
+            }
+          }
+        }
+        release_slot(slot);
       } else {
         const uint32_t buf = u & 1;
         const int slot = v % kRing;
@@ -799,7 +920,7 @@ static cudaError_t launch_inst(const CUtensorMap &tmA, const CUtensorMap &tmB, c
   if (e != cudaSuccess) return e;
   // setmaxnreg.inc waits for registers the CTA owns: never launch a split that
   // does not fit the launch allocation
-  if (attr.numRegs * kThreads < regs_ctl<kPromote>() * 128 + regs_epi<kPromote>() * 256)
+  if (attr.numRegs * kThreads < regs_ctl<kElem, kPromote, kMode>() * 128 + regs_epi<kElem, kPromote, kMode>() * 256)
     return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
