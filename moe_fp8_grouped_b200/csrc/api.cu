@@ -14,17 +14,23 @@ namespace gmm {
 
 static uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 static int g_cta_pairs = GMM_TILES_AUTO;
-static constexpr bool kAutoPairs = false;  // the automatic choice takes one-CTA tiles
+// The automatic choice (measured on every workload, same box, 20-step runs):
+// CTA pairs for the E4M3 tgmm (2-5 % faster: half of the lhs chunk per SM)
+// and for the static E4M3 row passes when the groups average two row tiles
+// or more (Mixtral forward 1.54 -> 1.45 ms, EP-merged 0.068 -> 0.060 ms);
+// one-CTA tiles for the promoted row passes (pairs 8-60 % slower) and for the
+// bf16 family.
 
 // 256-row tiles over a CTA pair for the row passes when the groups average at
 // least two such tiles (a group's last pair tile is half empty when its
 // 128-row tile count is odd); for the tgmm when its rows do too and its dout
 // columns split into 256-wide pair tiles.
-static bool use_pairs(bool tgmm, int64_t M, int64_t N, int32_t G) {
+static bool use_pairs(bool tgmm, int64_t M, int64_t N, int32_t G, int elem, bool promoted) {
   if (g_cta_pairs == GMM_TILES_ONE_CTA) return false;
   if (tgmm && N % 256) return false;
   if (g_cta_pairs == GMM_TILES_CTA_PAIRS || g_cta_pairs == GMM_TILES_CTA_PAIRS_NARROW) return true;
-  return kAutoPairs && M >= 512 * static_cast<int64_t>(G);
+  if (elem != 1) return false;
+  return tgmm || (!promoted && M >= 256 * static_cast<int64_t>(G));
 }
 
 // 128-column pair tiles (four TMEM accumulator buffers) for the promoted E4M3
@@ -405,7 +411,7 @@ static gmm_status fwd_impl(gmm_operand lhs, gmm_operand rhs, int transpose_rhs, 
   }
   const bool bmn = transpose_rhs == 0;  // [G, K, N]: N contiguous = MN-major B
   const uint32_t bke = 128 / elem;
-  const bool pairs = use_pairs(false, M, N, G);
+  const bool pairs = use_pairs(false, M, N, G, elem, dyn || blk);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, A, elem, K, M, K * elem, bke, 128)) return GMM_ERR_CUDA;
   // SwiGLU tiles take the gate rows and the up rows of a K-major rhs as two
@@ -484,7 +490,7 @@ static gmm_status run_dlhs_gemm(const void *A, const float *A_scales, int elem, 
                                 int64_t N, void *dlhs, gmm_dtype out_dtype, cudaStream_t st) {
   const bool bmn = transpose_rhs != 0;  // [G, N, K]: K contiguous = MN-major B for dlhs
   const uint32_t bke = 128 / elem;
-  const bool pairs = use_pairs(false, M, K, G);
+  const bool pairs = use_pairs(false, M, K, G, elem, elem == 1);
   const int tn = tile_cols(pairs, elem == 1, !bmn, false);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, A, elem, N, M, N * elem, bke, 128)) return GMM_ERR_CUDA;
@@ -526,7 +532,7 @@ static gmm_status run_drhs_gemm(int elem, bool dyn, const float *static_scale, i
   // k (B = lhs^T chunks); the epilogue writes dW[g, k, n].  The chunk-major
   // operands [chunk][column][128] are 2-D tensors of 128-element lines: chunk
   // j's line of column c is row j * C + c, so every box is one contiguous block.
-  const bool pairs = use_pairs(true, M, N, G);
+  const bool pairs = use_pairs(true, M, N, G, elem, elem == 1);
   const int tn = tile_cols(pairs, elem == 1, true, false);
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, P.codes_b, elem, kBlk, static_cast<uint64_t>(cap) * N, kBlk * elem, bke, 128))

@@ -240,6 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // static E4M3 row tiles accumulate their even and odd blocks in the two
   // TMEM buffers, as the one-CTA kernel does (bit-identical results)
   constexpr bool kSplit = !kPromote && !kTg && kElem == 1;
+  static_assert(!kSplit || stages_of<kCta, kMode, kTN>() % 2 == 0, "split tiles: each stage serves one issuer");
+  // two MMA issuers: split static tiles, and promoted 256-column tiles (units
+  // alternate between the two TMEM buffers; each issuer waits for its buffer's
+  // release before the unit's stage, so the stage parities stay unambiguous)
+  constexpr bool kTwo = kSplit || (kPromote && kTN == 256);
   constexpr uint32_t kStageTx = kCta * (kAStage + kBS);  // bytes completing one stage (both CTAs)
 
   extern __shared__ uint8_t smem_raw[];
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kCta * kEpiWarps);  // a pair: the epilogue warps of both CTAs arrive on rank 0's
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, kTwo ? 2 : 1);  // one commit per MMA issuer
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sfull[i], 32);
       mbar_init(&sempty[i], kEpiWarps);
@@ -435,26 +440,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader)
         for (int i = (it > kSt ? it - kSt : 0); i < it; ++i)
           mbar_wait(&full[i % kSt], (i / kSt) & 1, ctl_drain);
-    } else if (warp == 1) {
-      // ----------------------------------------------------- MMA issuer
+    } else if (warp == 1 || (kTwo && warp == 3)) {
+      // ---------------------------------------------------- MMA issuer(s)
+      // two issuers (both in the leader CTA): warp 1 fills buffer 0 (even
+      // blocks of a split static tile, or even units), warp 3 buffer 1
+      const int par = warp == 3 ? 1 : 0;
       if (lane == 0 && leader) {
         int it = 0, u = 0;
         bool ok = true;
-        int nuse = 0;  // split tiles: tiles issued (buffer 1 only when a tile has two blocks or more)
-        int nuse1 = 0;
+        int nuse = 0;  // split tiles: tiles this issuer accumulated into its buffer
         for (int w = w0; ok && w < total; w += wstep) {
           const Item t = decode_item<kMode, kCta>(w, p, s_offs, s_tpre, s_ppre, tn, rank);
           if constexpr (kSplit) {
             // the same accumulation as the one-CTA static row tiles: even
             // blocks into buffer 0, odd ones into buffer 1, summed by the
             // epilogue
-            const bool two = t.nblocks > 1;
-            if (!mbar_wait(&tempty[0], (nuse & 1) ^ 1, ctl) || (two && !mbar_wait(&tempty[1], (nuse1 & 1) ^ 1, ctl))) {
-              ok = false;
-              break;
+            const bool mine = t.nblocks > par;
+            if (mine) {
+              if (!mbar_wait(&tempty[par], (nuse & 1) ^ 1, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
-            tc_fence_after();
             for (int b = 0; b < t.nblocks; ++b, ++it) {
+              if ((b & 1) != par) continue;
               const int s = it % kSt;
               if (!mbar_wait(&full[s], (it / kSt) & 1, ctl)) {
                 ok = false;
@@ -462,32 +472,33 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               tc_fence_after();
               const uint32_t a0 = smem_u32(sA + s * kAStage), b0 = smem_u32(sB + s * kBS);
-              const uint32_t d = tbase + (b & 1) * kTN;
+              const uint32_t d = tbase + par * kTN;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
                 const uint64_t bdesc = kBMN ? smem_desc_sw128(b0 + kk * kMmaK * 128, kBBoxBytes, 1024)
                                             : smem_desc_sw128(b0 + kk * 32, 16, 1024);
-                if constexpr (kPair) tc_mma_pair<kF16>(d, adesc, bdesc, kIdesc, (b < 2 && kk == 0) ? 0u : 1u);
-                else tc_mma<kF16>(d, adesc, bdesc, kIdesc, (b < 2 && kk == 0) ? 0u : 1u);
+                if constexpr (kPair) tc_mma_pair<kF16>(d, adesc, bdesc, kIdesc, (b == par && kk == 0) ? 0u : 1u);
+                else tc_mma<kF16>(d, adesc, bdesc, kIdesc, (b == par && kk == 0) ? 0u : 1u);
               }
               if constexpr (kPair) tc_commit_pair_both(&empty[s], 0x3);
               else tc_commit(&empty[s]);
             }
             if (!ok) break;
-            if constexpr (kPair) tc_commit_pair_both(&tfull[0], 0x3);
-            else tc_commit(&tfull[0]);
-            ++nuse;
-            if (two) {
-              if constexpr (kPair) tc_commit_pair_both(&tfull[1], 0x3);
-              else tc_commit(&tfull[1]);
-              ++nuse1;
+            if (mine) {
+              if constexpr (kPair) tc_commit_pair_both(&tfull[par], 0x3);
+              else tc_commit(&tfull[par]);
+              ++nuse;
             }
             continue;
           }
           uint32_t buf = 0;
           for (int b = 0; b < t.nblocks; ++b, ++it) {
             const bool unit_start = kPromote || b == 0;
+            if (kTwo && (u & 1) != par) {  // the other issuer's unit
+              ++u;
+              continue;
+            }
             if (unit_start) {
               buf = u % kNB;
               if (!mbar_wait(&tempty[buf], ((u / kNB) & 1) ^ 1, ctl)) {

@@ -1,10 +1,13 @@
 """The GEMM passes on tiles shared by a pair of CTAs (a two-CTA cluster
 issuing M = 256 tensor-core MMAs), 256 columns wide or, in mode
 "cta_pairs_narrow", 128 columns wide for the promoted passes with a K-major
-B operand; forced on the small ragged cases where the automatic choice would
-take one-CTA tiles.  Each pass is checked against the oracle and bit for bit
-against the one-CTA 128-row tile (every tile accumulates each output over the
-same contraction steps in the same order).  The cases put the pair tile's
+B operand, against one-CTA tiles, both forced (the automatic choice takes
+pairs for the E4M3 tgmm and for static E4M3 row passes whose groups average
+two row tiles or more).  Each pass is checked against the oracle and bit for
+bit against the one-CTA 128-row tile (every tile accumulates each output over
+the same contraction steps in the same order; static E4M3 row tiles in both
+variants sum their even and odd blocks in two accumulators and add the two
+at the end).  The cases put the pair tile's
 second half past a group's end (odd 128-row tile counts, 1-row and 129-row
 groups), leave rows unrouted, leave groups empty and use N not a multiple of
 256.
@@ -119,16 +122,18 @@ def test_drhs_and_backward_pairs(dev, mode, name, rule):
 
 
 @pytest.mark.parametrize("name", ["tiny", "odd_tiles", "unrouted"])
+@pytest.mark.parametrize("rule", ["static", "dynamic"])
 @pytest.mark.parametrize("transpose", [False, True])
 @pytest.mark.parametrize("mode", PAIR_MODES)
-def test_swiglu_pairs(dev, mode, name, transpose):
+def test_swiglu_pairs(dev, mode, name, rule, transpose):
     inp = case_inputs(name)
     lhs, w, _, gs, s = to_dev(inp, dev)
     codes, scales = gm.gmm_quantize_rhs(w, transpose_out=transpose)
-    one, pair = both_tiles(lambda: gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule="dynamic",
+    one, pair = both_tiles(lambda: gm.gmm_fwd_swiglu(lhs, codes, scales, gs, rule=rule,
+                                                     static_scale=s if rule == "static" else None,
                                                      transpose_rhs=transpose, out_dtype=torch.float32), mode)
     qr, sr = oracle.quantize_rhs(inp.w)
-    ref, terms = oracle.gmm_fwd_swiglu(inp.lhs, oracle.Q_DYNAMIC, inp.static_scale, qr, sr, inp.group_sizes)
+    ref, terms = oracle.gmm_fwd_swiglu(inp.lhs, rule_code(rule), inp.static_scale, qr, sr, inp.group_sizes)
     assert_within(pair, ref, swiglu_bound(torch.float32, terms, ref), f"pair swiglu {name}")
     assert torch.equal(pair, one)
 
