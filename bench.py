@@ -32,7 +32,15 @@ METRIC = "FP8 grouped-GEMM TFLOP/s (fwd, dlhs, drhs) and % of B200 dense FP8 pea
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
-GEMM_SRC = os.path.join(ROOT, "moe_fp8_grouped_b200", "csrc", "gemm_tc.cu")
+# the GEMM kernel sources a traffic record was captured from (one-CTA and pair tiles)
+GEMM_SRCS = [os.path.join(ROOT, "moe_fp8_grouped_b200", "csrc", f) for f in ("gemm_tc.cu", "gemm_pair.cu")]
+
+
+def gemm_src_hash() -> str:
+    h = hashlib.sha256()
+    for f in GEMM_SRCS:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -235,7 +243,7 @@ def traffic_record(kernel: str, key: str):
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
-        src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()[:16]
+        src_hash = gemm_src_hash()
         for r in rec.get(kernel, []):
             if r.get("gemm_src_sha256_16") == src_hash and r.get("workload_key") == key:
                 return r.get("bytes_per_launch")
