@@ -392,7 +392,10 @@ void gmm_set_wait_limit_ns(uint64_t limit_ns);
  * testing knob: every tile gives the same results bit for bit, each output
  * being accumulated over the same contraction steps in the same order).
  *   GMM_TILES_AUTO          (default) the tile this library measured fastest
- *                           for the call's shape and pass;
+ *                           for the call's shape and pass: CTA pairs for the
+ *                           E4M3 tgmm and for static E4M3 row passes whose
+ *                           groups average two 128-row tiles or more (M >=
+ *                           256 G), one-CTA tiles otherwise;
  *   GMM_TILES_ONE_CTA       128 x 256 tiles on one CTA;
  *   GMM_TILES_CTA_PAIRS     256 x 256 tiles over a pair of CTAs (a two-CTA
  *                           cluster sharing each M = 256 tensor-core MMA;
