@@ -3,11 +3,14 @@
 // the same three passes, the same roles per warp and the same scaling, with
 // each CTA holding 128 rows of every item's A tile and half of its B tile in
 // its own shared memory and its 128 rows of the accumulator in its own
-// tensor memory.  Rank 0 of the pair issues the MMAs; the loads of both CTAs
-// complete on rank 0's full barriers; rank 0 commits to both CTAs' barriers;
-// the epilogue warps of both CTAs release accumulators on rank 0's barriers.
-// Tile width kTN = 256, or 128 for the promoted E4M3 passes with a K-major B
-// operand (four accumulator buffers instead of two).
+// tensor memory.  Rank 0 of the pair issues the MMAs (from two threads, as
+// in gemm_tc.cu, for the static E4M3 row tiles and the promoted 256-column
+// tiles); the loads of both CTAs complete on rank 0's full barriers; rank 0
+// commits to both CTAs' barriers; the epilogue warps of both CTAs release
+// accumulators on rank 0's barriers.  Tile width kTN = 256, or 128 for the
+// promoted E4M3 passes with a K-major B operand (four accumulator buffers
+// instead of two).  The automatic tile choice takes these tiles for the E4M3
+// tgmm and the static E4M3 row passes with large groups.
 //
 // Passes and sources as in gemm_tc.cu: forward gmm ("FP8 Megablox for batch
 // split", maxtext PR #3770, Description; "Support quantization for tokamax

@@ -22,8 +22,9 @@
 //              256-column accumulator buffers
 //   warp 2     scale loader: row / column scales of each TMEM unit into a
 //              shared-memory ring ahead of the epilogue
-//   warp 3     promoted kernels: second MMA issuer (idle otherwise, giving its
-//              registers to the epilogue)
+//   warp 3     second MMA issuer (promoted kernels and static E4M3 row
+//              passes; idle in the bf16 family, giving its registers to the
+//              epilogue)
 //
 // One thread cannot issue tcgen05.mma fast enough to keep the tensor core
 // busy once it also waits on the pipeline barriers (measured: ~2.2-3.3
@@ -35,7 +36,8 @@
 // depend on the split.  Each issuer waits for its buffer to be released
 // before it waits for the unit's stage: units are released in order, so by
 // then every earlier use of that stage has completed and the stage barrier's
-// phase parity is unambiguous, whatever the stage count.
+// phase parity is unambiguous, whatever the stage count.  The static E4M3
+// row passes split each tile instead (see two_issuers below).
 //   warps 4-11 epilogue: tcgen05.ld, scale, store.  Warp w reads TMEM lanes
 //              32 (w % 4) .. +31 (rows) and column half (w - 4) / 4.
 //
