@@ -458,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the same accumulation as the one-CTA static row tiles: even
             // blocks into buffer 0, odd ones into buffer 1, summed by the
             // epilogue
+            // (every tile of a row pass has the same block count: see gemm_tc.cu)
             const bool mine = t.nblocks > par;
             if (mine) {
               if (!mbar_wait(&tempty[par], (nuse & 1) ^ 1, ctl)) {

@@ -423,7 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const Item t = decode_item<kMode>(w, p, s_offs, s_tpre, tn);
           const uint32_t idesc = (kPromote && !kTg && t.rend - t.r0 <= 64) ? kIdesc64 : kIdesc;
           if constexpr (kSplit) {
-            // blocks b = par, par + 2, .. of the tile into buffer par
+            // blocks b = par, par + 2, .. of the tile into buffer par.  Every
+            // tile of a row pass has the same block count, so either no tile
+            // uses buffer 1 (one block) or every tile uses both: an issuer's
+            // buffer release then always follows the previous tile's MMAs,
+            // which keeps its stage waits unambiguous
             const bool mine = t.nblocks > par;
             if (mine) {
               if (!mbar_wait(&tempty[par], (nuse & 1) ^ 1, ctl)) {
