@@ -32,6 +32,9 @@ CASES = {
     # one-CTA promoted tiles of <= 64 rows run M = 64 MMAs: compared bit for
     # bit with the pair tiles' M = 256 MMAs
     "short_tiles": (7, 480, 384, 512, [64, 65, 16, 0, 48, 192, 63]),
+    # K = 128: one contraction block per row tile (static E4M3 tiles fill
+    # only the first of their two accumulators)
+    "k128": (3, 600, 128, 256, [200, 0, 330]),
 }
 
 
