@@ -231,3 +231,37 @@ def test_fullsize_activation_codes_bit_exact(name):
         del ct, cs
     del inp
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["mixtral", "dsv3_up"])
+def test_fullsize_repeatable_and_tile_independent(name):
+    """Every output is accumulated in a fixed order (two MMA-issuing threads,
+    each unit or half tile owned by one of them), so repeated calls give the
+    same bits, and one-CTA tiles give the same bits as the automatic choice
+    (CTA pairs for the static forward and the tgmm here).  A race between the
+    issuers, the loads and the epilogue would show up as a difference."""
+    dev = torch.device("cuda:0")
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w, seed=1, device="cuda")
+    gs = inp.group_sizes.to(dev)
+    s = torch.tensor([inp.static_scale], dtype=torch.float32, device=dev)
+    sarg = s if w.rule == "static" else None
+    codes, scales = gm.gmm_quantize_rhs(inp.w)
+
+    def run():
+        out = gm.gmm_fwd(inp.lhs, codes, scales, gs, rule=w.rule, static_scale=sarg)
+        dl, dw = gm.gmm_backward(inp.lhs, inp.dout, codes, scales, gs, rule=w.rule, static_scale=sarg)
+        torch.cuda.synchronize()
+        return out, dl, dw
+
+    ref = run()
+    for label in ("repeat 1", "repeat 2", "one-CTA tiles"):
+        try:
+            if label == "one-CTA tiles":
+                gm.gmm_set_tiles("one_cta")
+            got = run()
+        finally:
+            gm.gmm_set_tiles("auto")
+        for what, a, b in zip(("fwd", "dlhs", "drhs"), ref, got):
+            assert torch.equal(a, b), f"{name} {what}: {label} differs"
+        del got
